@@ -1,0 +1,200 @@
+"""Double-precision CPU oracle for the memory-efficient activation path.
+
+TEST INFRASTRUCTURE ONLY.  The product (the CUDA library under
+``memory_efficient_activation_b200/`` and its binding) never imports this
+package.  It is used by ``tests/``, by ``__graft_entry__.smoke()`` and by the
+CPU-baseline leg of ``bench.py``; nothing else.
+
+The arithmetic lives in ``mea_oracle.c`` (plain C, libm, double precision,
+serial long-double reductions).  This module only builds it with gcc when the
+shared object is missing or older than the source, and marshals numpy arrays
+through ctypes.  Inputs are float64 arrays holding the exact stored values;
+outputs are float64 (exact results in double) plus the two rounding helpers
+that produce the value a correct bf16 / fp32 kernel output should be near.
+
+Sources (by page and section):
+
+* "Memory efficient Swish" (adeeplearner blog, 2021-05-17): Swish and its
+  save-input-only backward ("How is Swish implemented?", "How is the memory
+  efficient version Swish implemented?", "What makes this implementation save
+  GPU memory?").
+* "What activations cost, in memory and in arithmetic" (asifuddin.com,
+  problem B07), GIVEN: the activation family.
+
+Parity pins for every function here live in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mea_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# gcc command; keep -fno-fast-math / -ffp-contract=off so the double
+# arithmetic is the plain IEEE sequence written in the source.
+GCC_CMD = [
+    "gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC",
+    "-shared", "-Wall", "-Wextra", "-o", _LIB, _SRC, "-lm",
+]
+
+# The oracle's own activation numbering (mirrors the enum in mea_oracle.c).
+ACTS = {
+    "relu": 0,
+    "leaky_relu": 1,
+    "sigmoid": 2,
+    "tanh": 3,
+    "gelu_erf": 4,
+    "gelu_tanh": 5,
+    "swish": 6,
+}
+LAYOUTS = {"nchw": 0, "nhwc": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so from mea_oracle.c if needed; return its path."""
+    stale = (not os.path.exists(_LIB)
+             or os.path.getmtime(_LIB) < os.path.getmtime(_SRC))
+    if force or stale:
+        subprocess.run(GCC_CMD, check=True)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        d = ctypes.POINTER(ctypes.c_double)
+        i64 = ctypes.c_int64
+        lib.oracle_act_fwd.argtypes = [ctypes.c_int, d, d, i64, ctypes.c_double]
+        lib.oracle_act_fwd.restype = ctypes.c_int
+        lib.oracle_act_bwd.argtypes = [ctypes.c_int, d, d, d, i64, ctypes.c_double]
+        lib.oracle_act_bwd.restype = ctypes.c_int
+        lib.oracle_act_deriv.argtypes = [ctypes.c_int, d, d, i64, ctypes.c_double]
+        lib.oracle_act_deriv.restype = ctypes.c_int
+        lib.oracle_swish_dalpha.argtypes = [d, d, i64, ctypes.c_double]
+        lib.oracle_swish_dalpha.restype = ctypes.c_double
+        shp = ctypes.POINTER(ctypes.c_int64)
+        lib.oracle_affine_swish_fwd.argtypes = [ctypes.c_int, shp, d, d, d, d]
+        lib.oracle_affine_swish_fwd.restype = ctypes.c_int
+        lib.oracle_affine_swish_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d, d]
+        lib.oracle_affine_swish_bwd.restype = ctypes.c_int
+        lib.oracle_round_bf16.argtypes = [d, ctypes.POINTER(ctypes.c_uint16), i64]
+        lib.oracle_round_bf16.restype = None
+        lib.oracle_round_f32.argtypes = [d, ctypes.POINTER(ctypes.c_float), i64]
+        lib.oracle_round_f32.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, ctype=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def num_threads() -> int:
+    """OpenMP threads the elementwise loops use."""
+    return int(_load().oracle_num_threads())
+
+
+def act_fwd(act: str, x, param: float = 1.0) -> np.ndarray:
+    """y = f(x; param) in double.  param: alpha (Swish), slope (LeakyReLU)."""
+    x = _f64(x)
+    y = np.empty_like(x)
+    rc = _load().oracle_act_fwd(ACTS[act], _ptr(x), _ptr(y), x.size, float(param))
+    if rc:
+        raise ValueError(f"oracle_act_fwd({act}) failed: {rc}")
+    return y
+
+
+def act_bwd(act: str, x, dy, param: float = 1.0) -> np.ndarray:
+    """dx = dy * f'(x; param) in double, f' recomputed from x."""
+    x = _f64(x)
+    dy = _f64(dy)
+    if x.shape != dy.shape:
+        raise ValueError("x and dy shapes differ")
+    dx = np.empty_like(x)
+    rc = _load().oracle_act_bwd(ACTS[act], _ptr(x), _ptr(dy), _ptr(dx), x.size, float(param))
+    if rc:
+        raise ValueError(f"oracle_act_bwd({act}) failed: {rc}")
+    return dx
+
+
+def act_deriv(act: str, x, param: float = 1.0) -> np.ndarray:
+    """f'(x; param) in double."""
+    x = _f64(x)
+    d = np.empty_like(x)
+    rc = _load().oracle_act_deriv(ACTS[act], _ptr(x), _ptr(d), x.size, float(param))
+    if rc:
+        raise ValueError(f"oracle_act_deriv({act}) failed: {rc}")
+    return d
+
+
+def swish_dalpha(x, dy, alpha: float) -> float:
+    """d alpha = sum dy x^2 s (1 - s), serial long-double sum."""
+    x = _f64(x)
+    dy = _f64(dy)
+    return float(_load().oracle_swish_dalpha(_ptr(x), _ptr(dy), x.size, float(alpha)))
+
+
+def _shape4(shape) -> np.ndarray:
+    s = np.ascontiguousarray(np.asarray(shape, dtype=np.int64))
+    if s.shape != (4,):
+        raise ValueError("shape must be (N, C, H, W)")
+    return s
+
+
+def affine_swish_fwd(layout: str, shape, x, gamma, beta) -> np.ndarray:
+    """y = z Sigmoid(z), z = gamma_c x + beta_c; shape is (N, C, H, W)."""
+    s = _shape4(shape)
+    x, gamma, beta = _f64(x), _f64(gamma), _f64(beta)
+    y = np.empty_like(x)
+    rc = _load().oracle_affine_swish_fwd(LAYOUTS[layout], _ptr(s, ctypes.c_int64),
+                                         _ptr(x), _ptr(gamma), _ptr(beta), _ptr(y))
+    if rc:
+        raise ValueError(f"oracle_affine_swish_fwd failed: {rc}")
+    return y
+
+
+def affine_swish_bwd(layout: str, shape, x, dy, gamma, beta):
+    """Returns (dx, dgamma, dbeta) in double."""
+    s = _shape4(shape)
+    x, dy, gamma, beta = _f64(x), _f64(dy), _f64(gamma), _f64(beta)
+    dx = np.empty_like(x)
+    C = int(s[1])
+    dg = np.empty(C, dtype=np.float64)
+    db = np.empty(C, dtype=np.float64)
+    rc = _load().oracle_affine_swish_bwd(LAYOUTS[layout], _ptr(s, ctypes.c_int64),
+                                         _ptr(x), _ptr(dy), _ptr(gamma), _ptr(beta),
+                                         _ptr(dx), _ptr(dg), _ptr(db))
+    if rc:
+        raise ValueError(f"oracle_affine_swish_bwd failed: {rc}")
+    return dx, dg, db
+
+
+def round_bf16(v) -> np.ndarray:
+    """Nearest bf16 (ties to even) of each double, as uint16 bit patterns."""
+    v = _f64(v)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_round_bf16(_ptr(v), _ptr(out, ctypes.c_uint16), v.size)
+    return out
+
+
+def round_f32(v) -> np.ndarray:
+    """Nearest binary32 (ties to even) of each double."""
+    v = _f64(v)
+    out = np.empty(v.shape, dtype=np.float32)
+    _load().oracle_round_f32(_ptr(v), _ptr(out, ctypes.c_float), v.size)
+    return out

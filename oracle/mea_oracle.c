@@ -1,0 +1,380 @@
+/*
+ * mea_oracle.c -- plain, slow, double-precision CPU oracle for the
+ * memory-efficient activation path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product (the CUDA library and its
+ * Python binding) links, loads or calls this file.  Only the test-suite, the
+ * smoke check and the CPU-baseline leg of the benchmark use it.  It shares no
+ * code, header, constant or helper with the CUDA path.
+ *
+ * Every function takes its inputs as exact doubles (the caller widens the
+ * stored bf16 / fp32 values, which is exact) and returns the mathematically
+ * defined result evaluated in double with libm.  Comparison against a GPU
+ * result happens after rounding the double result to the output storage type
+ * (oracle_round_bf16 / oracle_round_f32 below).
+ *
+ * Sources, by page and section:
+ *  - "Memory efficient Swish" (adeeplearner blog, 2021-05-17), sections
+ *    "What is a Swish activation function?" and "How is Swish implemented?":
+ *    Swish(x) = x * Sigmoid(alpha x), Sigmoid(v) = 1 / (1 + e^-v).
+ *  - same page, "How is the memory efficient version Swish implemented?" and
+ *    "What makes this implementation save GPU memory?": the forward keeps only
+ *    x, the backward recomputes the sigmoid from x and returns
+ *    dy * s * (1 + x (1 - s)) at alpha = 1 (product-rule derivation, with
+ *    e^-x / (1 + e^-x) rewritten as 1 - Sigmoid(x)).
+ *  - "What activations cost, in memory and in arithmetic" (asifuddin.com,
+ *    problem B07), GIVEN: the activation family ReLU, LeakyReLU, sigmoid,
+ *    tanh, GELU (erf) and GELU (tanh approximation).  The page names them
+ *    only; the definitions used here are the standard ones.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - alpha is one scalar per tensor; the derivative in x generalises by the
+ *    chain rule to s + alpha x s sigma(-alpha x); d alpha is the derivative of
+ *    sum(dy * y) in alpha, i.e. sum(dy * x^2 * s * sigma(-alpha x)).
+ *  - 1 - Sigmoid(v) is evaluated as Sigmoid(-v) (the same value, without the
+ *    cancellation that 1 - s suffers when s is close to 1).
+ *  - ReLU'(0) = 0 and LeakyReLU'(0) = slope (the derivative is the predicate
+ *    x > 0).  A NaN input fails that predicate.
+ *  - GELU-tanh uses the published constants sqrt(2/pi) and 0.044715
+ *    (Hendrycks and Gimpel, 2016); 1 + tanh(u) is evaluated as 2 Sigmoid(2u).
+ *  - Fused affine + Swish: z = gamma_c x + beta_c, y = z Sigmoid(z) (alpha 1),
+ *    channel c = i mod C for NHWC and (i / (H W)) mod C for NCHW.
+ *
+ * Reductions (d alpha, d gamma, d beta) are serial sums in index order in
+ * long double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Activation ids of this oracle (its own numbering; the Python wrapper maps
+ * activation names onto it). */
+enum {
+    OR_RELU = 0,
+    OR_LEAKY_RELU = 1,
+    OR_SIGMOID = 2,
+    OR_TANH = 3,
+    OR_GELU_ERF = 4,
+    OR_GELU_TANH = 5,
+    OR_SWISH = 6,
+    OR_NUM_ACTS = 7
+};
+
+enum { OR_NCHW = 0, OR_NHWC = 1 };
+
+/* ---------------------------------------------------------------- sigmoid */
+
+/* Sigmoid(v) = 1 / (1 + e^-v).  For v < 0 the equal form e^v / (1 + e^v) is
+ * used so that e^-v never overflows; both forms are the definition. */
+static double sigm(double v)
+{
+    if (v != v) return v;
+    if (v >= 0.0) return 1.0 / (1.0 + exp(-v));
+    double e = exp(v);
+    return e / (1.0 + e);
+}
+
+/* ------------------------------------------------------------------ Swish */
+
+static double swish_f(double x, double alpha)
+{
+    return x * sigm(alpha * x);
+}
+
+/* d/dx [x Sigmoid(alpha x)] = s + alpha x s (1 - s), with (1 - s) taken as
+ * Sigmoid(-alpha x). */
+static double swish_df(double x, double alpha)
+{
+    double z = alpha * x;
+    double s = sigm(z);
+    return s + z * s * sigm(-z);
+}
+
+/* d/dalpha [x Sigmoid(alpha x)] = x^2 s (1 - s). */
+static double swish_dalpha_term(double x, double alpha)
+{
+    double z = alpha * x;
+    return x * x * sigm(z) * sigm(-z);
+}
+
+/* ------------------------------------------------------------ the family */
+
+static double relu_f(double x)
+{
+    if (x != x) return x;
+    return x > 0.0 ? x : 0.0;
+}
+
+static double relu_df(double x)
+{
+    return x > 0.0 ? 1.0 : 0.0;
+}
+
+static double leaky_f(double x, double slope)
+{
+    return x > 0.0 ? x : slope * x;
+}
+
+static double leaky_df(double x, double slope)
+{
+    return x > 0.0 ? 1.0 : slope;
+}
+
+static double sigmoid_f(double x)
+{
+    return sigm(x);
+}
+
+/* Sigmoid' = s (1 - s) = Sigmoid(x) Sigmoid(-x). */
+static double sigmoid_df(double x)
+{
+    return sigm(x) * sigm(-x);
+}
+
+static double tanh_f(double x)
+{
+    return tanh(x);
+}
+
+/* tanh' = 1 - tanh^2 = 4 Sigmoid(2x) Sigmoid(-2x) (no cancellation). */
+static double tanh_df(double x)
+{
+    return 4.0 * sigm(2.0 * x) * sigm(-2.0 * x);
+}
+
+/* Standard normal CDF Phi(x) = erfc(-x / sqrt 2) / 2 and density phi(x). */
+static double std_normal_cdf(double x)
+{
+    return 0.5 * erfc(-x / sqrt(2.0));
+}
+
+static double std_normal_pdf(double x)
+{
+    return exp(-0.5 * x * x) / sqrt(2.0 * M_PI);
+}
+
+/* GELU (erf form): x Phi(x). */
+static double gelu_erf_f(double x)
+{
+    return x * std_normal_cdf(x);
+}
+
+/* d/dx [x Phi(x)] = Phi(x) + x phi(x). */
+static double gelu_erf_df(double x)
+{
+    return std_normal_cdf(x) + x * std_normal_pdf(x);
+}
+
+/* GELU (tanh approximation): x (1 + tanh u) / 2 = x Sigmoid(2u),
+ * u = sqrt(2/pi) (x + 0.044715 x^3). */
+static const double GELU_K0 = 0.7978845608028654;   /* sqrt(2 / pi) */
+static const double GELU_K1 = 0.044715;
+
+static double gelu_tanh_u(double x)
+{
+    return GELU_K0 * (x + GELU_K1 * x * x * x);
+}
+
+static double gelu_tanh_f(double x)
+{
+    return x * sigm(2.0 * gelu_tanh_u(x));
+}
+
+/* d/dx [x Sigmoid(2u)] = Sigmoid(2u) + x 2u' Sigmoid(2u) Sigmoid(-2u),
+ * u' = sqrt(2/pi) (1 + 3 * 0.044715 x^2). */
+static double gelu_tanh_df(double x)
+{
+    double v = 2.0 * gelu_tanh_u(x);
+    double dv = 2.0 * GELU_K0 * (1.0 + 3.0 * GELU_K1 * x * x);
+    double s = sigm(v);
+    return s + x * dv * s * sigm(-v);
+}
+
+static double act_f(int act, double x, double param)
+{
+    switch (act) {
+    case OR_RELU: return relu_f(x);
+    case OR_LEAKY_RELU: return leaky_f(x, param);
+    case OR_SIGMOID: return sigmoid_f(x);
+    case OR_TANH: return tanh_f(x);
+    case OR_GELU_ERF: return gelu_erf_f(x);
+    case OR_GELU_TANH: return gelu_tanh_f(x);
+    case OR_SWISH: return swish_f(x, param);
+    }
+    return NAN;
+}
+
+static double act_df(int act, double x, double param)
+{
+    switch (act) {
+    case OR_RELU: return relu_df(x);
+    case OR_LEAKY_RELU: return leaky_df(x, param);
+    case OR_SIGMOID: return sigmoid_df(x);
+    case OR_TANH: return tanh_df(x);
+    case OR_GELU_ERF: return gelu_erf_df(x);
+    case OR_GELU_TANH: return gelu_tanh_df(x);
+    case OR_SWISH: return swish_df(x, param);
+    }
+    return NAN;
+}
+
+/* ------------------------------------------------------- exported: family */
+
+/* y[i] = f(x[i]; param).  param is alpha for Swish, the slope for
+ * LeakyReLU, ignored otherwise.  Returns 0, or -1 for an unknown act. */
+int oracle_act_fwd(int act, const double *x, double *y, int64_t n, double param)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || n < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) y[i] = act_f(act, x[i], param);
+    return 0;
+}
+
+/* dx[i] = dy[i] * f'(x[i]; param), with f' recomputed from x alone. */
+int oracle_act_bwd(int act, const double *x, const double *dy, double *dx,
+                   int64_t n, double param)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || n < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) dx[i] = dy[i] * act_df(act, x[i], param);
+    return 0;
+}
+
+/* The derivative alone (dy = 1), for closed-form and finite-difference
+ * checks. */
+int oracle_act_deriv(int act, const double *x, double *d, int64_t n, double param)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) d[i] = act_df(act, x[i], param);
+    return 0;
+}
+
+/* d alpha = sum_i dy_i x_i^2 s_i (1 - s_i), serial, index order, long
+ * double accumulator. */
+double oracle_swish_dalpha(const double *x, const double *dy, int64_t n, double alpha)
+{
+    long double acc = 0.0L;
+    for (int64_t i = 0; i < n; ++i)
+        acc += (long double)(dy[i] * swish_dalpha_term(x[i], alpha));
+    return (double)acc;
+}
+
+/* ------------------------------------------------ exported: affine + Swish */
+
+static int64_t channel_of(int layout, const int64_t shape[4], int64_t i)
+{
+    int64_t C = shape[1], HW = shape[2] * shape[3];
+    if (layout == OR_NHWC) return i % C;
+    return (i / HW) % C;
+}
+
+/* y = z Sigmoid(z), z = gamma_c x + beta_c; shape = {N, C, H, W} in both
+ * layouts (the layout says how the flat index maps to a channel). */
+int oracle_affine_swish_fwd(int layout, const int64_t shape[4], const double *x,
+                            const double *gamma, const double *beta, double *y)
+{
+    if (layout != OR_NCHW && layout != OR_NHWC) return -1;
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        double z = gamma[c] * x[i] + beta[c];
+        y[i] = z * sigm(z);
+    }
+    return 0;
+}
+
+/* dz = dy (s + z s (1 - s)); dx = gamma_c dz; dgamma_c = sum dz x;
+ * dbeta_c = sum dz (serial, index order, long double). */
+int oracle_affine_swish_bwd(int layout, const int64_t shape[4], const double *x,
+                            const double *dy, const double *gamma, const double *beta,
+                            double *dx, double *dgamma, double *dbeta)
+{
+    if (layout != OR_NCHW && layout != OR_NHWC) return -1;
+    int64_t C = shape[1];
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+    long double *acc_g = (long double *)calloc((size_t)(C > 0 ? C : 1), sizeof(long double));
+    long double *acc_b = (long double *)calloc((size_t)(C > 0 ? C : 1), sizeof(long double));
+    if (!acc_g || !acc_b) { free(acc_g); free(acc_b); return -2; }
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        double z = gamma[c] * x[i] + beta[c];
+        double s = sigm(z);
+        double dz = dy[i] * (s + z * s * sigm(-z));
+        dx[i] = gamma[c] * dz;
+        acc_g[c] += (long double)(dz * x[i]);
+        acc_b[c] += (long double)dz;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        dgamma[c] = (double)acc_g[c];
+        dbeta[c] = (double)acc_b[c];
+    }
+    free(acc_g);
+    free(acc_b);
+    return 0;
+}
+
+/* ------------------------------------------------------ storage rounding */
+
+/* Round a double to the nearest bfloat16 (1 sign bit, 8 exponent bits with
+ * bias 127, 7 stored mantissa bits), ties to even, and return its bit
+ * pattern.  Written from the format's definition: find the spacing of
+ * representable values around |v| (2^(e-7) in the binade [2^e, 2^(e+1)),
+ * 2^-133 in the subnormal range), round |v| / spacing to an integer with
+ * ties to even, and encode.  Values at or beyond the rounding boundary above
+ * the largest finite bf16 become infinity. */
+static uint16_t bf16_from_double(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (v != v) return (uint16_t)(sign | 0x7fc0u);
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7f80u);
+    int e2;
+    frexp(a, &e2);          /* a in [2^(e2-1), 2^e2) */
+    int e = e2 - 1;
+    if (e < -126) e = -126; /* subnormals share the spacing of the lowest binade */
+    double spacing = ldexp(1.0, e - 7);
+    double q = nearbyint(a / spacing);   /* default rounding: ties to even */
+    double r = q * spacing;
+    double max_finite = ldexp(255.0, 120); /* (2 - 2^-7) * 2^127 */
+    if (r > max_finite) return (uint16_t)(sign | 0x7f80u);
+    if (r == 0.0) return sign;
+    int re2;
+    frexp(r, &re2);
+    int re = re2 - 1;
+    if (re < -126) {
+        /* subnormal: value = m * 2^-133, m in 1..127 */
+        uint16_t m = (uint16_t)ldexp(r, 133);
+        return (uint16_t)(sign | m);
+    }
+    uint16_t m = (uint16_t)(ldexp(r, 7 - re) - 128.0); /* stored mantissa 0..127 */
+    uint16_t ex = (uint16_t)(re + 127);
+    return (uint16_t)(sign | (ex << 7) | m);
+}
+
+void oracle_round_bf16(const double *v, uint16_t *out, int64_t n)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = bf16_from_double(v[i]);
+}
+
+/* Round to binary32 with ties to even (C's conversion in the default
+ * rounding mode). */
+void oracle_round_f32(const double *v, float *out, int64_t n)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = (float)v[i];
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
