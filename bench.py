@@ -1,0 +1,454 @@
+"""Benchmark: Swish forward + save-input-only backward, bf16 storage / fp32
+math, on the transformer-scale activation [8, 2048, 4096] (67,108,864
+elements), the configuration the headline metric is quoted on.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = mea_act_fwd (read x, write y) + mea_act_bwd (read x and dy,
+write dx) over one batch: 10 algorithmic bytes per element, 671,088,640 bytes
+per step.  Each rank processes its own full-size batch (weak scaling, no
+data-path collective); under torchrun the elapsed time is the max over ranks.
+Inputs are resident in HBM when the timed region starts; the per-step working
+set (x, y, dy, dx = 536 MB) is larger than the 126 MB L2, so no flush is
+needed between steps.
+
+Rank 0 prints one JSON line.  Besides the device-timed value it reports the
+end-to-end number through the same public API with host buffers (pinned
+host -> device copies of x and dy, device -> host copies of y and dx inside
+the timed region), the dominant kernel's roofline fraction from CUDA events
+on its own stream, the SM clocks sampled during the timed region, and the
+CPU oracle's throughput on a bounded sample (the baseline, not the target).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import memory_efficient_activation_b200 as mea  # noqa: E402
+from memory_efficient_activation_b200 import accounting, synthetic  # noqa: E402
+
+METRIC = "Swish fwd+bwd GB/s and % of B200 HBM roofline at 67M bf16 elements"
+WORKLOAD = "swish_bf16_8x2048x4096"
+SHAPE = (8, 2048, 4096)
+DTYPE = "bf16"
+FALLBACK_HBM_GBS = 6650.0
+DOMINANT_KERNEL = "act_kernel<Swish, Bf16, MODE 1> (mea_act_bwd)"
+
+
+# ----------------------------------------------------------------- helpers
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, ws, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(v: float, ws: int) -> float:
+    if ws <= 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "memory_efficient_activation_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+        if e.get("source_hash") != _source_hash():
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class _ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+               (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+               (0x100, "display_clock_setting")]
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].isdigit():
+                    idx = int(ids[device_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in self.REASONS:
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ our arm
+
+def _inputs(rank: int):
+    w = synthetic.swish_bf16_transformer(seed=1 + 1000 * rank, shape=SHAPE)
+    return w
+
+
+def run_ours(args, rank, ws, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = _inputs(rank)
+    n = w.n
+    x = w.x.to(dev)
+    dy = w.dy.to(dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mea.act_fwd("swish", x, 1.0, out=y)
+        mea.act_bwd("swish", x, dy, 1.0, out=dx)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # Timed region: K steps, per-kernel events on the launching stream.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    with _ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            ev[k][0].record(stream)
+            mea.act_fwd("swish", x, 1.0, out=y)
+            ev[k][1].record(stream)
+            mea.act_bwd("swish", x, dy, 1.0, out=dx)
+            ev[k][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    _barrier(ws)
+    elapsed_ms = _max_over_ranks(start.elapsed_time(end), ws)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    fwd_ms = _max_over_ranks(fwd_ms, ws)
+    bwd_ms = _max_over_ranks(bwd_ms, ws)
+
+    step_bytes = accounting.step_bytes(n, DTYPE)
+    ms_per_step = elapsed_ms / args.steps
+    value = ws * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # End to end through the public API with host buffers.
+    e2e = run_e2e(args, rank, ws, local, w)
+
+    peak, peak_kind = _peaks()
+    bwd_bytes = accounting.bwd_bytes(n, DTYPE)
+    achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+    roofline = {
+        "kernel": DOMINANT_KERNEL,
+        "bound": "hbm",
+        "achieved": round(achieved, 1),
+        "peak": peak,
+        "peak_kind": f"{peak_kind} (copy bandwidth, burst)",
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": _traffic("swish_bf16_bwd"),
+        "algorithmic_bytes_per_launch": bwd_bytes,
+        "fwd_ms": round(fwd_ms, 5),
+        "bwd_ms": round(bwd_ms, 5),
+        "fwd_frac": round(accounting.fwd_bytes(n, DTYPE) / (fwd_ms * 1e-3) / 1e9 / peak, 4),
+        "step_frac": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+    }
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": DTYPE,
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD,
+            "shape": list(SHAPE),
+            "elements_per_gpu": n,
+            "alpha": 1.0,
+            "bytes_per_step_per_gpu": step_bytes,
+            "x_dist": "N(0,1)", "dy_dist": "N(0,1)",
+            "l2": "inputs larger than L2 (536 MB working set per step vs 126 MB L2); no flush",
+            "parallelism": f"replicas x{ws} (independent shards, no data-path collective)",
+            "pct_of_hbm_roofline": round(100 * value / ws / peak, 2),
+            "saved_bytes_per_layer": accounting.saved_bytes_per_layer(n, DTYPE),
+            "saved_bytes_per_layer_naive": accounting.saved_bytes_per_layer(n, DTYPE, naive=True),
+        },
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    return out
+
+
+def run_e2e(args, rank, ws, local, w):
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    hx = w.x.contiguous().pin_memory()
+    hdy = w.dy.contiguous().pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    x = torch.empty_like(hx, device=dev)
+    dy = torch.empty_like(hx, device=dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        x.copy_(hx, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        mea.act_fwd("swish", x, 1.0, out=y)
+        mea.act_bwd("swish", x, dy, 1.0, out=dx)
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    ms = _max_over_ranks(s.elapsed_time(e), ws)
+    nbytes = accounting.step_bytes(w.n, DTYPE)
+    return {
+        "value": round(ws * nbytes * steps / (ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "h2d_bytes_per_step": 2 * accounting.tensor_bytes(w.n, DTYPE),
+        "d2h_bytes_per_step": 2 * accounting.tensor_bytes(w.n, DTYPE),
+        "steps": steps,
+        "ms_per_step": round(ms / steps, 4),
+    }
+
+
+# ------------------------------------------------- oracle (CPU) baseline
+
+def _oracle_step(oracle, xd, gd):
+    y = oracle.act_fwd("swish", xd, 1.0)
+    dx = oracle.act_bwd("swish", xd, gd, 1.0)
+    oracle.round_bf16(y)
+    oracle.round_bf16(dx)
+
+
+def cpu_baseline(w, budget_s: float = 12.0):
+    """The double-precision oracle (as it stands, OpenMP over the host cores)
+    on the same workload: forward + backward + rounding of y and dx to bf16,
+    repeated over the full 67M-element batch until about budget_s seconds of
+    work; GB/s under the same 10 bytes/element accounting."""
+    import oracle
+    xd = w.x.reshape(-1).double().numpy()
+    gd = w.dy.reshape(-1).double().numpy()
+    reps, t_total = 0, 0.0
+    while t_total < budget_s and reps < 50:
+        t0 = time.perf_counter()
+        _oracle_step(oracle, xd, gd)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    n = w.n
+    return {
+        "value": round(reps * accounting.step_bytes(n, DTYPE) / t_total / 1e9, 3),
+        "unit": "GB/s",
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": f"{reps} x full {n}-element batch (fwd + bwd + bf16 rounding), {t_total:.1f} s",
+    }
+
+
+def run_reference(args, rank, ws):
+    """The reference arm: the CPU oracle on bounded samples of the same
+    workload, one sample per step, sized so warm-up plus steps take about
+    args.ref_seconds."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    w = _inputs(0)
+    xs = w.x.reshape(-1)
+    gs = w.dy.reshape(-1)
+    probe = 1 << 20
+    xd, gd = xs[:probe].double().numpy(), gs[:probe].double().numpy()
+    t0 = time.perf_counter()
+    _oracle_step(oracle, xd, gd)
+    per_elem = (time.perf_counter() - t0) / probe
+    total_steps = args.steps + args.warmup
+    sample = int(args.ref_seconds / max(total_steps, 1) / max(per_elem, 1e-12))
+    sample = max(1 << 12, min(sample, w.n))
+    xd, gd = xs[:sample].double().numpy(), gs[:sample].double().numpy()
+    for _ in range(args.warmup):
+        _oracle_step(oracle, xd, gd)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(oracle, xd, gd)
+    dt = time.perf_counter() - t0
+    nbytes = accounting.step_bytes(sample, DTYPE)
+    value = round(args.steps * nbytes / dt / 1e9, 4)
+    cb = {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+          "sample": f"first {sample} of {w.n} elements per step (fwd + bwd + bf16 rounding)"}
+    del np
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * dt / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "shape": list(SHAPE), "sample_elements": sample},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        out = run_reference(args, rank, ws)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    rank, ws, local = _dist()
+    out = run_ours(args, rank, ws, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,205 @@
+/*
+ * mea.h -- C ABI of the memory-efficient activation library (libmea.so).
+ *
+ * The library implements save-input-only elementwise activations on NVIDIA
+ * B200 (sm_100a): the forward writes y = f(x) and keeps nothing else; the
+ * backward recomputes what it needs from the saved input x in the same pass
+ * and writes dx = dy * f'(x) (plus d alpha for a learnable Swish alpha, or
+ * d gamma / d beta for the fused per-channel affine + Swish).
+ *
+ * Sources, by page and section:
+ *  - "Memory efficient Swish" (adeeplearner blog, 2021-05-17):
+ *      "What is a Swish activation function?" / "How is Swish implemented?"
+ *        Swish(x) = x * Sigmoid(alpha x), Sigmoid(v) = 1 / (1 + e^-v);
+ *      "How is the memory efficient version Swish implemented?" and
+ *      "What makes this implementation save GPU memory?"
+ *        the forward saves only the input; the backward recomputes the
+ *        sigmoid from it: dx = dy * s * (1 + x (1 - s)) at alpha = 1.
+ *  - "What activations cost, in memory and in arithmetic" (asifuddin.com,
+ *    problem B07), GIVEN: the family ReLU, LeakyReLU, sigmoid, tanh, GELU
+ *    (erf) and GELU (tanh approximation); SOLUTION: elementwise work is bound
+ *    by memory bandwidth (about c/4 FLOP per byte in bf16).
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named x, dy, y, dx, gamma, beta, dgamma, dbeta, param_dev,
+ *    dparam_dev and workspace are DEVICE pointers (memory the GPU can load
+ *    and store, e.g. from cudaMalloc or a PyTorch CUDA tensor).  The shape
+ *    array is a HOST pointer.  The caller owns every buffer; the library
+ *    allocates nothing and keeps no pointer after the call returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Argument validation is synchronous; a launch
+ *    failure is reported as MEA_ERR_CUDA (from cudaGetLastError).  No kernel
+ *    traps or asserts; no call synchronises the device.
+ *  - Storage dtypes: MEA_F32 (IEEE binary32) and MEA_BF16 (bfloat16).  All
+ *    arithmetic is fp32 on the widened values; bf16 results are rounded to
+ *    nearest even.  Reductions accumulate in fp64 and return fp32.
+ *  - Layout: tensors are dense and contiguous.  Pointers that are not
+ *    16-byte aligned, and element counts that are not a multiple of the
+ *    vector width, take a scalar path; that is never an error.
+ *  - n = 0 (or a zero in shape) is a no-op that returns MEA_OK.
+ *  - Results are bitwise deterministic for a given input, shape and dtype
+ *    (reductions run on a grid fixed by the element count and sum in a fixed
+ *    order), independent of the stream, the run and the GPU's SM count.
+ */
+#ifndef MEA_H
+#define MEA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MEA_API __attribute__((visibility("default")))
+#else
+#define MEA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the runtime's and the driver's stream handle type). */
+typedef struct CUstream_st *mea_stream_t;
+
+/* Activation functions.  Definitions (problem B07 names them; the
+ * definitions are the standard ones; Swish is from the Swish page):
+ *   MEA_RELU        max(x, 0);            derivative: 1 if x > 0 else 0
+ *   MEA_LEAKY_RELU  x > 0 ? x : slope x;  derivative: 1 if x > 0 else slope
+ *   MEA_SIGMOID     1 / (1 + e^-x);       derivative: s (1 - s)
+ *   MEA_TANH        tanh x;               derivative: 1 - tanh^2 x
+ *   MEA_GELU_ERF    x Phi(x), Phi the standard normal CDF;
+ *                   derivative: Phi(x) + x phi(x)
+ *   MEA_GELU_TANH   x (1 + tanh u) / 2, u = sqrt(2/pi) (x + 0.044715 x^3)
+ *   MEA_SWISH       x Sigmoid(alpha x);   derivative: s + alpha x s (1 - s),
+ *                   s = Sigmoid(alpha x); d alpha = sum dy x^2 s (1 - s)   */
+typedef enum {
+    MEA_RELU = 0,
+    MEA_LEAKY_RELU = 1,
+    MEA_SIGMOID = 2,
+    MEA_TANH = 3,
+    MEA_GELU_ERF = 4,
+    MEA_GELU_TANH = 5,
+    MEA_SWISH = 6
+} mea_act_t;
+
+typedef enum { MEA_F32 = 0, MEA_BF16 = 1 } mea_dtype_t;
+
+/* Memory order of a 4-D activation whose logical shape is {N, C, H, W}. */
+typedef enum { MEA_NCHW = 0, MEA_NHWC = 1 } mea_layout_t;
+
+typedef enum {
+    MEA_OK = 0,
+    MEA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, overlap */
+    MEA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve */
+    MEA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    MEA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
+} mea_status_t;
+
+/* Forward: y[i] = f(x[i]) for i < n.
+ *   act, dtype   activation and storage dtype of x and y.
+ *   x            device, n elements, read only.  This is the one tensor the
+ *                caller keeps for the backward.
+ *   y            device, n elements, written.  Must not overlap x (x is the
+ *                saved tensor): any overlap returns MEA_ERR_INVALID_ARG.
+ *   n            element count, >= 0.
+ *   param        alpha for MEA_SWISH, slope for MEA_LEAKY_RELU, ignored
+ *                otherwise.
+ *   param_dev    optional device pointer to one float; when non-NULL it is
+ *                read on the device and replaces `param` (a learnable alpha
+ *                that lives on the GPU).
+ *   stream       CUDA stream the kernel is queued on.
+ * Source: the Swish page's forward (section "How is the memory efficient
+ * version Swish implemented?"), generalised to the family of problem B07. */
+MEA_API mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y,
+                         int64_t n, float param, const float *param_dev,
+                         mea_stream_t stream);
+
+/* Bytes of device workspace mea_act_bwd needs: 0 unless want_dparam is
+ * non-zero (d alpha of MEA_SWISH), in which case it is a small function of n
+ * (at most 256 + 8 * 1184 bytes).  Pure host arithmetic; no CUDA call. */
+MEA_API size_t mea_act_bwd_workspace_bytes(mea_act_t act, int64_t n, int want_dparam);
+
+/* Backward with recompute: dx[i] = dy[i] * f'(x[i]) for i < n, f' evaluated
+ * from x alone (nothing but x was saved).
+ *   x, dy        device, n elements each, read only.
+ *   dx           device, n elements, written.  May be the same pointer as
+ *                dy or as x (each element is read before it is written); a
+ *                partial overlap returns MEA_ERR_INVALID_ARG.
+ *   param,
+ *   param_dev    as in mea_act_fwd.
+ *   dparam_dev   optional device pointer to one float.  When non-NULL (only
+ *                for MEA_SWISH, else MEA_ERR_UNSUPPORTED) it is OVERWRITTEN
+ *                with d alpha = sum_i dy_i x_i^2 s_i (1 - s_i), fp64
+ *                accumulation in a fixed order, rounded to fp32.
+ *   workspace,
+ *   ws_bytes     device scratch of at least mea_act_bwd_workspace_bytes()
+ *                bytes, 16-byte aligned, when dparam_dev is non-NULL (else
+ *                ignored).  Its first 4 bytes are a completion counter that
+ *                must be zero before the first use (zero-fill the buffer
+ *                once); every call returns the counter to zero when its
+ *                kernel completes, so the buffer can be reused without
+ *                clearing.  Calls that share a workspace must not run
+ *                concurrently on the GPU.
+ * Source: the Swish page, sections "How is the memory efficient version
+ * Swish implemented?" and "What makes this implementation save GPU memory?";
+ * d alpha is the derivative of sum(dy * Swish) in alpha. */
+MEA_API mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const void *dy,
+                         void *dx, int64_t n, float param, const float *param_dev,
+                         float *dparam_dev, void *workspace, size_t ws_bytes,
+                         mea_stream_t stream);
+
+/* Bytes of device workspace mea_affine_swish_bwd needs for this dtype,
+ * layout and logical shape {N, C, H, W} (host pointer).  Pure host
+ * arithmetic; returns 0 for an invalid request. */
+MEA_API size_t mea_affine_swish_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout,
+                                            const int64_t shape[4]);
+
+/* Fused per-channel affine + Swish forward: z = gamma_c x + beta_c,
+ * y = z Sigmoid(z).
+ *   shape        host array {N, C, H, W} (logical dims, all >= 0).
+ *   layout       MEA_NHWC: channel of flat index i is i mod C;
+ *                MEA_NCHW: channel is (i / (H W)) mod C.
+ *   x, y         device, N*C*H*W elements of `dtype`; y must not overlap x.
+ *   gamma, beta  device fp32[C], read only.
+ * Source: the save-input-only Swish of the Swish page applied after a
+ * per-channel affine (the op that precedes Swish in EfficientNet blocks). */
+MEA_API mea_status_t mea_affine_swish_fwd(mea_dtype_t dtype, mea_layout_t layout,
+                                  const int64_t shape[4], const void *x,
+                                  const float *gamma, const float *beta, void *y,
+                                  mea_stream_t stream);
+
+/* Fused per-channel affine + Swish backward: recomputes z from x and
+ *   dz = dy (s + z s (1 - s)), s = Sigmoid(z);
+ *   dx = gamma_c dz;  dgamma_c = sum dz x;  dbeta_c = sum dz
+ * (sums over all N*H*W positions of channel c, fp64 accumulation in a fixed
+ * order, rounded to fp32).
+ *   x, dy        device, read only; dx device, written (may equal dy or x
+ *                exactly, no partial overlap).
+ *   gamma, beta  device fp32[C], read only.
+ *   dgamma,
+ *   dbeta        device fp32[C], OVERWRITTEN (not accumulated).
+ *   workspace    device scratch of at least
+ *                mea_affine_swish_bwd_workspace_bytes() bytes, 16-byte
+ *                aligned, with the same completion-counter rule as the
+ *                workspace of mea_act_bwd (zero-fill once; each call leaves
+ *                the counter at zero; no concurrent sharing). */
+MEA_API mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout,
+                                  const int64_t shape[4], const void *x, const void *dy,
+                                  const float *gamma, const float *beta, void *dx,
+                                  float *dgamma, float *dbeta, void *workspace,
+                                  size_t ws_bytes, mea_stream_t stream);
+
+/* Static description of a status code. */
+MEA_API const char *mea_status_string(mea_status_t status);
+
+/* Detail of the most recent failing call on this host thread (which
+ * argument, which CUDA error); "" if none.  Valid until the next call. */
+MEA_API const char *mea_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+MEA_API int mea_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEA_H */

@@ -1,1 +1,280 @@
-"""Memory-efficient elementwise activations for B200 (placeholder; binding follows)."""
+"""Memory-efficient elementwise activations for NVIDIA B200 (sm_100a).
+
+The forward of every activation writes y = f(x) and keeps only x; the backward
+recomputes what it needs from x in the same pass ("Memory efficient Swish",
+sections "How is the memory efficient version Swish implemented?" and "What
+makes this implementation save GPU memory?").  All arithmetic runs in the
+CUDA kernels of libmea.so, reached through its C ABI (include/mea.h).  This
+module only marshals PyTorch CUDA tensors (device memory and the current
+stream) into those calls; PyTorch is plumbing here, not the compute path.
+
+Functions (the C ABI's names without the ``mea_`` prefix):
+    act_fwd, act_bwd, affine_swish_fwd, affine_swish_bwd,
+    act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes
+Autograd / modules:
+    ActivationFunction, MemoryEfficientActivation, MemoryEfficientSwish,
+    AffineSwishFunction, MemoryEfficientAffineSwish
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import torch
+
+from . import _capi
+from ._capi import ACT_IDS, LAYOUT_IDS, MeaError
+
+__all__ = [
+    "act_fwd", "act_bwd", "affine_swish_fwd", "affine_swish_bwd",
+    "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
+    "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
+    "AffineSwishFunction", "MemoryEfficientAffineSwish", "MeaError", "ACTIVATIONS",
+]
+
+ACTIVATIONS = tuple(ACT_IDS)
+_DTYPES = {torch.float32: _capi.MEA_F32, torch.bfloat16: _capi.MEA_BF16}
+
+
+def _dtype_id(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.float32 or torch.bfloat16") from None
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _act_id(act: str) -> int:
+    try:
+        return ACT_IDS[act]
+    except KeyError:
+        raise ValueError(f"unknown activation {act!r}; one of {ACTIVATIONS}") from None
+
+
+# ------------------------------------------------------------- workspaces
+
+class _WorkspacePool:
+    """Zero-filled reduction workspaces, one per (device, stream).  The
+    kernels return the completion counter to zero, so a buffer is zeroed only
+    when it is created or grown."""
+
+    def __init__(self):
+        self._lock = threading.Lock()
+        self._bufs = {}
+
+    def get(self, device: torch.device, stream: int, nbytes: int) -> torch.Tensor:
+        key = (device.index, stream)
+        with self._lock:
+            buf = self._bufs.get(key)
+            if buf is None or buf.numel() < nbytes:
+                buf = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
+                self._bufs[key] = buf
+            return buf
+
+
+_pool = _WorkspacePool()
+
+
+def act_bwd_workspace_bytes(act: str, n: int, want_dparam: bool) -> int:
+    return int(_capi.lib().mea_act_bwd_workspace_bytes(_act_id(act), int(n), int(bool(want_dparam))))
+
+
+def affine_swish_bwd_workspace_bytes(dtype: torch.dtype, layout: str, shape_nchw) -> int:
+    return int(_capi.lib().mea_affine_swish_bwd_workspace_bytes(
+        _DTYPES[dtype], LAYOUT_IDS[layout], _capi.shape4(shape_nchw)))
+
+
+# ------------------------------------------------------------ entry points
+
+def act_fwd(act: str, x: torch.Tensor, param: float = 1.0, param_dev: torch.Tensor | None = None,
+            out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = f(x).  param: alpha (Swish) or slope (LeakyReLU); param_dev: an
+    optional one-element fp32 CUDA tensor read on the device instead."""
+    _need_cuda(x)
+    y = torch.empty_like(x) if out is None else out
+    _need_cuda(y)
+    if param_dev is not None:
+        _need_cuda(param_dev)
+    st = _capi.lib().mea_act_fwd(_act_id(act), _dtype_id(x), x.data_ptr(), y.data_ptr(), x.numel(),
+                                  float(param), _ptr(param_dev), _stream(x))
+    _capi.check("mea_act_fwd", st)
+    return y
+
+
+def act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, param: float = 1.0,
+            param_dev: torch.Tensor | None = None, dparam: torch.Tensor | None = None,
+            out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """dx = dy * f'(x), f' recomputed from x.  If dparam (a one-element fp32
+    CUDA tensor) is given, it is overwritten with d alpha (Swish only)."""
+    _need_cuda(x, dy)
+    if dy.dtype != x.dtype or dy.shape != x.shape:
+        raise ValueError("dy must match x in dtype and shape")
+    dx = torch.empty_like(x) if out is None else out
+    _need_cuda(dx)
+    ws_ptr, ws_bytes = None, 0
+    if dparam is not None:
+        _need_cuda(dparam)
+        ws_bytes = act_bwd_workspace_bytes(act, x.numel(), True)
+        ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), ws_bytes)
+        ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+    if param_dev is not None:
+        _need_cuda(param_dev)
+    st = _capi.lib().mea_act_bwd(_act_id(act), _dtype_id(x), x.data_ptr(), dy.data_ptr(), dx.data_ptr(),
+                                  x.numel(), float(param), _ptr(param_dev), _ptr(dparam), ws_ptr, ws_bytes,
+                                  _stream(x))
+    _capi.check("mea_act_bwd", st)
+    return dx
+
+
+def _affine_shape(x: torch.Tensor, layout: str):
+    if x.dim() != 4:
+        raise ValueError("affine + Swish takes a 4-D tensor")
+    if layout == "nhwc":
+        N, H, W, C = x.shape
+    elif layout == "nchw":
+        N, C, H, W = x.shape
+    else:
+        raise ValueError(f"layout must be 'nchw' or 'nhwc', not {layout!r}")
+    return (N, C, H, W)
+
+
+def affine_swish_fwd(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, layout: str = "nhwc",
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = z Sigmoid(z), z = gamma_c x + beta_c.  x is (N, H, W, C) for
+    'nhwc' or (N, C, H, W) for 'nchw'; gamma and beta are fp32 [C]."""
+    _need_cuda(x, gamma, beta)
+    shape = _affine_shape(x, layout)
+    y = torch.empty_like(x) if out is None else out
+    _need_cuda(y)
+    st = _capi.lib().mea_affine_swish_fwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
+                                           gamma.data_ptr(), beta.data_ptr(), y.data_ptr(), _stream(x))
+    _capi.check("mea_affine_swish_fwd", st)
+    return y
+
+
+def affine_swish_bwd(x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+                     layout: str = "nhwc", out: torch.Tensor | None = None,
+                     dgamma: torch.Tensor | None = None, dbeta: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None):
+    """Returns (dx, dgamma, dbeta); z and the sigmoid are recomputed from x."""
+    _need_cuda(x, dy, gamma, beta)
+    if dy.dtype != x.dtype or dy.shape != x.shape:
+        raise ValueError("dy must match x in dtype and shape")
+    shape = _affine_shape(x, layout)
+    C = shape[1]
+    dx = torch.empty_like(x) if out is None else out
+    dg = torch.empty(C, dtype=torch.float32, device=x.device) if dgamma is None else dgamma
+    db = torch.empty(C, dtype=torch.float32, device=x.device) if dbeta is None else dbeta
+    _need_cuda(dx, dg, db)
+    need = affine_swish_bwd_workspace_bytes(x.dtype, layout, shape)
+    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    st = _capi.lib().mea_affine_swish_bwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
+                                           dy.data_ptr(), gamma.data_ptr(), beta.data_ptr(), dx.data_ptr(),
+                                           dg.data_ptr(), db.data_ptr(), ws.data_ptr(),
+                                           ws.numel() * ws.element_size(), _stream(x))
+    _capi.check("mea_affine_swish_bwd", st)
+    return dx, dg, db
+
+
+# ---------------------------------------------------------------- autograd
+
+class ActivationFunction(torch.autograd.Function):
+    """Save-input-only autograd function: ctx keeps x (and alpha), nothing else."""
+
+    @staticmethod
+    def forward(ctx, x, act: str, param: float, alpha: torch.Tensor | None):
+        x = x.contiguous()
+        y = act_fwd(act, x, param, param_dev=alpha)
+        ctx.act, ctx.param = act, param
+        if alpha is None:
+            ctx.save_for_backward(x)
+        else:
+            ctx.save_for_backward(x, alpha)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        saved = ctx.saved_tensors
+        x = saved[0]
+        alpha = saved[1] if len(saved) > 1 else None
+        dy = dy.contiguous()
+        want = alpha is not None and ctx.needs_input_grad[3]
+        dalpha = torch.empty(1, dtype=torch.float32, device=x.device) if want else None
+        dx = act_bwd(ctx.act, x, dy, ctx.param, param_dev=alpha, dparam=dalpha)
+        return dx, None, None, (dalpha.view_as(alpha) if want else None)
+
+
+class MemoryEfficientActivation(torch.nn.Module):
+    """An activation of the family whose backward recomputes from x."""
+
+    def __init__(self, act: str = "swish", param: float | None = None):
+        super().__init__()
+        _act_id(act)
+        self.act = act
+        self.param = (0.01 if act == "leaky_relu" else 1.0) if param is None else float(param)
+
+    def forward(self, x):
+        return ActivationFunction.apply(x, self.act, self.param, None)
+
+
+class MemoryEfficientSwish(torch.nn.Module):
+    """Swish x * Sigmoid(alpha x); alpha fixed (default 1) or learnable."""
+
+    def __init__(self, alpha: float = 1.0, learnable: bool = False):
+        super().__init__()
+        if learnable:
+            self.alpha = torch.nn.Parameter(torch.tensor([float(alpha)], dtype=torch.float32))
+        else:
+            self.register_buffer("alpha", None)
+            self.alpha_value = float(alpha)
+
+    def forward(self, x):
+        if self.alpha is not None:
+            return ActivationFunction.apply(x, "swish", 1.0, self.alpha)
+        return ActivationFunction.apply(x, "swish", self.alpha_value, None)
+
+
+class AffineSwishFunction(torch.autograd.Function):
+    """Fused per-channel affine + Swish that saves only x (and gamma, beta)."""
+
+    @staticmethod
+    def forward(ctx, x, gamma, beta, layout: str):
+        x = x.contiguous()
+        y = affine_swish_fwd(x, gamma, beta, layout)
+        ctx.layout = layout
+        ctx.save_for_backward(x, gamma, beta)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, gamma, beta = ctx.saved_tensors
+        dx, dg, db = affine_swish_bwd(x, dy.contiguous(), gamma, beta, ctx.layout)
+        return dx, dg, db, None
+
+
+class MemoryEfficientAffineSwish(torch.nn.Module):
+    """y = z Sigmoid(z), z = gamma_c x + beta_c, with learnable fp32 gamma, beta."""
+
+    def __init__(self, channels: int, layout: str = "nhwc"):
+        super().__init__()
+        self.layout = layout
+        self.gamma = torch.nn.Parameter(torch.ones(channels, dtype=torch.float32))
+        self.beta = torch.nn.Parameter(torch.zeros(channels, dtype=torch.float32))
+
+    def forward(self, x):
+        return AffineSwishFunction.apply(x, self.gamma, self.beta, self.layout)

@@ -1,0 +1,88 @@
+"""ctypes declarations of the C ABI in include/mea.h (libmea.so).
+
+Marshalling only: this module loads the shared library that sits next to it
+and declares argument and result types.  There is no fallback: if the library
+is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
+
+# Enumerations of include/mea.h.
+MEA_RELU, MEA_LEAKY_RELU, MEA_SIGMOID, MEA_TANH, MEA_GELU_ERF, MEA_GELU_TANH, MEA_SWISH = range(7)
+MEA_F32, MEA_BF16 = 0, 1
+MEA_NCHW, MEA_NHWC = 0, 1
+MEA_OK, MEA_ERR_INVALID_ARG, MEA_ERR_UNSUPPORTED, MEA_ERR_WORKSPACE, MEA_ERR_CUDA = range(5)
+
+ACT_IDS = {
+    "relu": MEA_RELU,
+    "leaky_relu": MEA_LEAKY_RELU,
+    "sigmoid": MEA_SIGMOID,
+    "tanh": MEA_TANH,
+    "gelu_erf": MEA_GELU_ERF,
+    "gelu_tanh": MEA_GELU_TANH,
+    "swish": MEA_SWISH,
+}
+LAYOUT_IDS = {"nchw": MEA_NCHW, "nhwc": MEA_NHWC}
+
+# Every symbol the header declares, with (restype, argtypes).
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_f = ctypes.c_float
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_shape = ctypes.POINTER(ctypes.c_int64)
+SIGNATURES = {
+    "mea_act_fwd": (_i, [_i, _i, _vp, _vp, _i64, _f, _vp, _vp]),
+    "mea_act_bwd_workspace_bytes": (_sz, [_i, _i64, _i]),
+    "mea_act_bwd": (_i, [_i, _i, _vp, _vp, _vp, _i64, _f, _vp, _vp, _vp, _sz, _vp]),
+    "mea_affine_swish_bwd_workspace_bytes": (_sz, [_i, _i, _shape]),
+    "mea_affine_swish_fwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp]),
+    "mea_affine_swish_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mea_status_string": (ctypes.c_char_p, [_i]),
+    "mea_last_error": (ctypes.c_char_p, []),
+    "mea_version": (_i, []),
+}
+
+_lib = None
+
+
+class MeaError(RuntimeError):
+    """A libmea call returned a status other than MEA_OK."""
+
+    def __init__(self, fn: str, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status}: {detail}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmea.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with `python -m memory_efficient_activation_b200.build` "
+                "(the activation path runs only in its CUDA kernels)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def check(fn: str, status: int) -> None:
+    if status != MEA_OK:
+        detail = lib().mea_last_error().decode(errors="replace")
+        raise MeaError(fn, status, detail or lib().mea_status_string(status).decode())
+
+
+def shape4(shape) -> ctypes.Array:
+    vals = [int(v) for v in shape]
+    if len(vals) != 4:
+        raise ValueError("shape must have four entries (N, C, H, W)")
+    return (ctypes.c_int64 * 4)(*vals)

@@ -1,0 +1,213 @@
+// mea_act.cu -- streaming kernels of the save-input-only activation family.
+//
+// One template serves every activation, dtype and pass:
+//   MODE 0  forward:            y  = f(x)
+//   MODE 1  backward:           dx = dy f'(x), f' recomputed from x
+//   MODE 2  backward + d alpha: as MODE 1, plus sum dy x^2 s (1 - s) (Swish)
+//
+// The work is HBM-bound (problem B07 of "What activations cost, in memory and
+// in arithmetic": about c/4 FLOP per byte), so the kernel is built around the
+// memory system: 16-byte vector loads through the non-coherent path without
+// L1 allocation, kUnroll independent vectors in flight per thread (2 kUnroll
+// in the backward), a grid-stride loop over a grid sized to the resident
+// capacity of the GPU (a multiple of the SM count), and stores straight from
+// registers.  Pointers that are not 16-byte aligned take the scalar loop of
+// the same kernel; so does the ragged tail of n mod V elements.
+//
+// The d alpha reduction is deterministic: its grid is a function of n only,
+// each thread accumulates fp32 vector sums into an fp64 register, blocks
+// reduce through a fixed xor-butterfly, every block writes one fp64 partial,
+// and the last block to finish (found with an atomic ticket, no waiting)
+// adds the partials in index order and writes the fp32 result.  The ticket
+// wraps back to zero, so the workspace is left as it was found.
+#include "mea_device.cuh"
+#include "mea_internal.h"
+#include "mea_math.cuh"
+
+#include <cstdint>
+#include <type_traits>
+
+namespace mea {
+
+// Writes this block's partial; the last block to arrive sums all partials in
+// index order and stores the fp32 result.  No block ever waits.
+__device__ __forceinline__ void finish_reduction(double acc, float *out, void *ws)
+{
+    __shared__ double red[32];
+    unsigned int *ticket = static_cast<unsigned int *>(ws);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
+
+    double b = block_sum(acc, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = b;
+    if (!last_block_done(ticket)) return;
+    double v = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) v += __ldcg(partials + i);
+    double total = block_sum(v, red);
+    if (threadIdx.x == 0) *out = (float)total;
+}
+
+// ------------------------------------------------------------ the kernel
+
+template <class A, typename T, int MODE>
+__global__ void __launch_bounds__(kThreads)
+act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__restrict__ out, int64_t n,
+           int vec_ok, float param, const float *__restrict__ param_dev, float *__restrict__ dparam,
+           void *__restrict__ ws)
+{
+    using S = Store<T>;
+    constexpr int V = S::V;
+    constexpr bool P = S::P;
+    const Coef k = A::coef(param_dev ? __ldg(param_dev) : param);
+    const int64_t nvec = vec_ok ? n / V : 0;
+    const int tid = threadIdx.x;
+    const int64_t tile = (int64_t)kThreads * kUnroll;
+    const int64_t gstride = (int64_t)gridDim.x * tile;
+    double acc = 0.0;
+
+    for (int64_t base = (int64_t)blockIdx.x * tile + tid; base < nvec; base += gstride) {
+        uint4 xv[kUnroll], gv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kThreads;
+            if (i < nvec) {
+                xv[u] = ld_nc_v4(static_cast<const uint4 *>(x) + i);
+                if constexpr (MODE != 0) gv[u] = ld_nc_v4(static_cast<const uint4 *>(dy) + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kThreads;
+            if (i < nvec) {
+                float xf[V], gf[V], of[V], tf[V];
+                S::unpack(xv[u], xf);
+                if constexpr (MODE != 0) S::unpack(gv[u], gf);
+                bool tail = false;
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    if constexpr (MODE == 0)
+                        of[j] = A::template f<P>(xf[j], k, tail);
+                    else if constexpr (MODE == 1)
+                        of[j] = A::template df<P>(xf[j], gf[j], k, tail);
+                    else
+                        of[j] = A::template df_da<P>(xf[j], gf[j], k, tail, tf[j]);
+                }
+                if (tail) {
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        if (A::is_tail(xf[j], k)) {
+                            if constexpr (MODE == 0)
+                                of[j] = A::template f_tail<P>(xf[j], k);
+                            else if constexpr (MODE == 1)
+                                of[j] = A::template df_tail<P>(xf[j], gf[j], k);
+                            else
+                                of[j] = A::template df_da_tail<P>(xf[j], gf[j], k, tf[j]);
+                        }
+                    }
+                }
+                st_v4(static_cast<uint4 *>(out) + i, S::pack(of));
+                if constexpr (MODE == 2) acc += (double)tree_sum<V>(tf);
+            }
+        }
+    }
+
+    // Scalar loop: the n mod V tail of the vector path, or every element when
+    // a pointer is not 16-byte aligned.
+    for (int64_t i = nvec * V + (int64_t)blockIdx.x * kThreads + tid; i < n;
+         i += (int64_t)gridDim.x * kThreads) {
+        const float xi = S::load1(x, i);
+        bool tail = false;
+        float o, term = 0.f;
+        if constexpr (MODE == 0) {
+            o = A::template f<P>(xi, k, tail);
+            if (tail) o = A::template f_tail<P>(xi, k);
+        } else {
+            const float gi = S::load1(dy, i);
+            if constexpr (MODE == 1) {
+                o = A::template df<P>(xi, gi, k, tail);
+                if (tail) o = A::template df_tail<P>(xi, gi, k);
+            } else {
+                o = A::template df_da<P>(xi, gi, k, tail, term);
+                if (tail) o = A::template df_da_tail<P>(xi, gi, k, term);
+            }
+        }
+        S::store1(out, i, o);
+        if constexpr (MODE == 2) acc += (double)term;
+    }
+
+    if constexpr (MODE == 2) finish_reduction(acc, dparam, ws);
+}
+
+// ------------------------------------------------------------ launchers
+
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+            c = 148;
+        cached[dev] = c;
+    }
+    return cached[dev];
+}
+
+template <class A, typename T, int MODE>
+struct KernelTag {};
+
+template <class A, typename T, int MODE>
+static cudaError_t launch_one(const ActLaunch &a)
+{
+    constexpr int V = Store<T>::V;
+    auto kernel = act_kernel<A, T, MODE>;
+    uintptr_t align = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
+    if (MODE != 0) align |= reinterpret_cast<uintptr_t>(a.dy);
+    const int vec_ok = (align & 15u) == 0;
+    int grid;
+    if (MODE == 2) {
+        grid = red_grid(a.n);
+    } else {
+        const int64_t units = vec_ok ? (a.n / V + (int64_t)kThreads * kUnroll - 1) / ((int64_t)kThreads * kUnroll)
+                                     : (a.n + kThreads - 1) / kThreads;
+        const int64_t cap = (int64_t)sm_count() * resident_blocks<KernelTag<A, T, MODE>>(kernel, kThreads);
+        int64_t g = units < cap ? units : cap;
+        if (g < 1) g = 1;
+        grid = (int)g;
+    }
+    kernel<<<grid, kThreads, 0, a.stream>>>(a.x, a.dy, a.out, a.n, vec_ok, a.param, a.param_dev, a.dparam,
+                                            a.workspace);
+    return cudaGetLastError();
+}
+
+template <class A, int MODE>
+static cudaError_t by_dtype(const ActLaunch &a)
+{
+    return a.dtype == kBF16 ? launch_one<A, Bf16, MODE>(a) : launch_one<A, float, MODE>(a);
+}
+
+template <int MODE>
+static cudaError_t by_act(const ActLaunch &a)
+{
+    switch (a.act) {
+    case 0: return by_dtype<ReLU, MODE>(a);
+    case 1: return by_dtype<LeakyReLU, MODE>(a);
+    case 2: return by_dtype<Sigmoid, MODE>(a);
+    case 3: return by_dtype<Tanh, MODE>(a);
+    case 4: return by_dtype<GeluErf, MODE>(a);
+    case 5: return by_dtype<GeluTanh, MODE>(a);
+    case 6: return by_dtype<Swish, MODE>(a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_act_fwd(const ActLaunch &a) { return by_act<0>(a); }
+
+cudaError_t launch_act_bwd(const ActLaunch &a)
+{
+    if (a.dparam) return by_dtype<Swish, 2>(a);   // the C-ABI admits d alpha for Swish only
+    return by_act<1>(a);
+}
+
+}  // namespace mea

@@ -1,0 +1,253 @@
+// mea_capi.cu -- the C ABI of include/mea.h: argument validation, error
+// reporting and dispatch to the kernel launchers.  Host code only.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "../../include/mea.h"
+#include "mea_internal.h"
+
+namespace {
+
+thread_local char g_err[512];
+
+void clear_error() { g_err[0] = '\0'; }
+
+mea_status_t fail(mea_status_t st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+bool valid_act(int a) { return a >= MEA_RELU && a <= MEA_SWISH; }
+bool valid_dtype(int d) { return d == MEA_F32 || d == MEA_BF16; }
+size_t dtype_bytes(int d) { return d == MEA_BF16 ? 2 : 4; }
+
+// Largest element count whose byte size and index arithmetic stay in range.
+constexpr int64_t kMaxElems = (int64_t)1 << 60;
+
+// [a, a + na) and [b, b + nb) share at least one byte.
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+// Identical ranges are allowed (each element is read before it is written);
+// any other overlap is not.
+bool partial_overlap(const void *a, const void *b, size_t bytes)
+{
+    return a != b && overlaps(a, bytes, b, bytes);
+}
+
+mea_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(MEA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+mea_status_t check_shape(const int64_t *shape, int64_t *n)
+{
+    if (!shape) return fail(MEA_ERR_INVALID_ARG, "shape is NULL");
+    int64_t prod = 1;
+    for (int i = 0; i < 4; ++i) {
+        if (shape[i] < 0) return fail(MEA_ERR_INVALID_ARG, "shape[%d] = %lld is negative", i, (long long)shape[i]);
+        if (shape[i] > 0 && prod > kMaxElems / shape[i])
+            return fail(MEA_ERR_INVALID_ARG, "shape has more than 2^60 elements");
+        prod *= shape[i];
+    }
+    *n = prod;
+    return MEA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mea_status_string(mea_status_t status)
+{
+    switch (status) {
+    case MEA_OK: return "success";
+    case MEA_ERR_INVALID_ARG: return "invalid argument";
+    case MEA_ERR_UNSUPPORTED: return "unsupported request";
+    case MEA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MEA_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char *mea_last_error(void) { return g_err; }
+
+int mea_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y, int64_t n, float param,
+                         const float *param_dev, mea_stream_t stream)
+{
+    clear_error();
+    if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    if (n < 0 || n > kMaxElems) return fail(MEA_ERR_INVALID_ARG, "n = %lld out of range", (long long)n);
+    if (n == 0) return MEA_OK;
+    if (!x || !y) return fail(MEA_ERR_INVALID_ARG, "x or y is NULL");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (overlaps(x, bytes, y, bytes))
+        return fail(MEA_ERR_INVALID_ARG, "y overlaps x (x is the saved tensor; the forward keeps it intact)");
+    mea::ActLaunch l{};
+    l.act = act;
+    l.dtype = dtype;
+    l.x = x;
+    l.out = y;
+    l.n = n;
+    l.param = param;
+    l.param_dev = param_dev;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_act_fwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_act_fwd launch");
+}
+
+size_t mea_act_bwd_workspace_bytes(mea_act_t act, int64_t n, int want_dparam)
+{
+    (void)act;
+    if (!want_dparam || n < 0) return 0;
+    return mea::kWsHeader + sizeof(double) * (size_t)mea::red_grid(n);
+}
+
+mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const void *dy, void *dx, int64_t n,
+                         float param, const float *param_dev, float *dparam_dev, void *workspace,
+                         size_t ws_bytes, mea_stream_t stream)
+{
+    clear_error();
+    if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    if (n < 0 || n > kMaxElems) return fail(MEA_ERR_INVALID_ARG, "n = %lld out of range", (long long)n);
+    if (dparam_dev && act != MEA_SWISH)
+        return fail(MEA_ERR_UNSUPPORTED, "a parameter gradient exists only for MEA_SWISH (d alpha)");
+    if (dparam_dev) {
+        const size_t need = mea_act_bwd_workspace_bytes(act, n, 1);
+        if (!workspace || ws_bytes < need)
+            return fail(MEA_ERR_WORKSPACE, "d alpha needs %zu bytes of workspace, got %zu%s", need, ws_bytes,
+                        workspace ? "" : " (NULL)");
+        if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+            return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    }
+    if (n == 0 && !dparam_dev) return MEA_OK;
+    if (n > 0 && (!x || !dy || !dx)) return fail(MEA_ERR_INVALID_ARG, "x, dy or dx is NULL");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (n > 0 && (partial_overlap(dx, dy, bytes) || partial_overlap(dx, x, bytes)))
+        return fail(MEA_ERR_INVALID_ARG, "dx partially overlaps x or dy (only exact aliasing is allowed)");
+    mea::ActLaunch l{};
+    l.act = act;
+    l.dtype = dtype;
+    l.x = x;
+    l.dy = dy;
+    l.out = dx;
+    l.n = n;
+    l.param = param;
+    l.param_dev = param_dev;
+    l.dparam = dparam_dev;
+    l.workspace = workspace;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_act_bwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_act_bwd launch");
+}
+
+size_t mea_affine_swish_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4])
+{
+    int64_t n = 0;
+    if (!valid_dtype(dtype) || (layout != MEA_NCHW && layout != MEA_NHWC)) return 0;
+    char saved[sizeof(g_err)];
+    __builtin_memcpy(saved, g_err, sizeof(g_err));
+    const bool ok = check_shape(shape, &n) == MEA_OK;
+    __builtin_memcpy(g_err, saved, sizeof(g_err));
+    if (!ok) return 0;
+    return mea::affine_bwd_workspace_bytes(dtype, layout, shape[0], shape[1], shape[2], shape[3]);
+}
+
+mea_status_t mea_affine_swish_fwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
+                                  const float *gamma, const float *beta, void *y, mea_stream_t stream)
+{
+    clear_error();
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    if (layout != MEA_NCHW && layout != MEA_NHWC)
+        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", (int)layout);
+    int64_t n = 0;
+    mea_status_t st = check_shape(shape, &n);
+    if (st != MEA_OK) return st;
+    if (n == 0) return MEA_OK;
+    if (!x || !y || !gamma || !beta) return fail(MEA_ERR_INVALID_ARG, "x, y, gamma or beta is NULL");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (overlaps(x, bytes, y, bytes))
+        return fail(MEA_ERR_INVALID_ARG, "y overlaps x (x is the saved tensor; the forward keeps it intact)");
+    mea::AffineLaunch l{};
+    l.dtype = dtype;
+    l.layout = layout;
+    l.N = shape[0];
+    l.C = shape[1];
+    l.H = shape[2];
+    l.W = shape[3];
+    l.x = x;
+    l.gamma = gamma;
+    l.beta = beta;
+    l.out = y;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_affine_fwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_fwd launch");
+}
+
+mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
+                                  const void *dy, const float *gamma, const float *beta, void *dx, float *dgamma,
+                                  float *dbeta, void *workspace, size_t ws_bytes, mea_stream_t stream)
+{
+    clear_error();
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    if (layout != MEA_NCHW && layout != MEA_NHWC)
+        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", (int)layout);
+    int64_t n = 0;
+    mea_status_t st = check_shape(shape, &n);
+    if (st != MEA_OK) return st;
+    if (shape[1] == 0) return MEA_OK;                 // no channels: nothing to write
+    if (!dgamma || !dbeta || !gamma || !beta)
+        return fail(MEA_ERR_INVALID_ARG, "gamma, beta, dgamma or dbeta is NULL");
+    if (n > 0 && (!x || !dy || !dx)) return fail(MEA_ERR_INVALID_ARG, "x, dy or dx is NULL");
+    const size_t need = mea_affine_swish_bwd_workspace_bytes(dtype, layout, shape);
+    if (!workspace || ws_bytes < need)
+        return fail(MEA_ERR_WORKSPACE, "affine backward needs %zu bytes of workspace, got %zu%s", need, ws_bytes,
+                    workspace ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+        return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (n > 0 && (partial_overlap(dx, dy, bytes) || partial_overlap(dx, x, bytes)))
+        return fail(MEA_ERR_INVALID_ARG, "dx partially overlaps x or dy (only exact aliasing is allowed)");
+    const size_t cbytes = (size_t)shape[1] * sizeof(float);
+    if (overlaps(dgamma, cbytes, dbeta, cbytes)) return fail(MEA_ERR_INVALID_ARG, "dgamma overlaps dbeta");
+    if (n == 0) {
+        // An empty batch still defines the parameter gradients: zero.
+        cudaError_t e = cudaMemsetAsync(dgamma, 0, cbytes, reinterpret_cast<cudaStream_t>(stream));
+        if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, cbytes, reinterpret_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_bwd zero fill");
+    }
+    mea::AffineLaunch l{};
+    l.dtype = dtype;
+    l.layout = layout;
+    l.N = shape[0];
+    l.C = shape[1];
+    l.H = shape[2];
+    l.W = shape[3];
+    l.x = x;
+    l.dy = dy;
+    l.gamma = gamma;
+    l.beta = beta;
+    l.out = dx;
+    l.dgamma = dgamma;
+    l.dbeta = dbeta;
+    l.workspace = workspace;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_affine_bwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_bwd launch");
+}
+
+}  // extern "C"

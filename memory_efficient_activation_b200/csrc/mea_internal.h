@@ -1,0 +1,87 @@
+// mea_internal.h -- launchers shared between the C-ABI layer and the kernels.
+// Not installed; the public interface is include/mea.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mea {
+
+// Storage dtype and activation ids follow include/mea.h.
+enum Dtype { kF32 = 0, kBF16 = 1 };
+
+constexpr int kThreads = 256;          // threads per block of the streaming kernels
+constexpr int kUnroll = 4;             // 16-byte vectors per thread per iteration
+constexpr int kRedGridMax = 1184;      // 148 SMs x 8: cap of the reduction grid
+constexpr int64_t kRedElemsPerBlock = 8192;
+constexpr size_t kWsHeader = 256;      // ticket counter lives in the first 256 bytes
+
+// Reduction grid of the d alpha backward: a function of n only, so the sum
+// order (and hence the bits of the result) never depends on the device.
+inline int red_grid(int64_t n)
+{
+    int64_t g = (n + kRedElemsPerBlock - 1) / kRedElemsPerBlock;
+    if (g < 1) g = 1;
+    if (g > kRedGridMax) g = kRedGridMax;
+    return (int)g;
+}
+
+struct ActLaunch {
+    int act;                 // mea_act_t
+    int dtype;               // Dtype
+    const void *x;
+    const void *dy;          // backward only
+    void *out;               // y or dx
+    int64_t n;
+    float param;
+    const float *param_dev;  // nullable
+    float *dparam;           // nullable (Swish d alpha)
+    void *workspace;         // ticket + fp64 partials when dparam is set
+    cudaStream_t stream;
+};
+
+// Returns a cudaError_t from the launch (cudaSuccess on success).
+cudaError_t launch_act_fwd(const ActLaunch &a);
+cudaError_t launch_act_bwd(const ActLaunch &a);
+
+struct AffineLaunch {
+    int dtype;
+    int layout;              // mea_layout_t
+    int64_t N, C, H, W;
+    const void *x;
+    const void *dy;
+    const float *gamma;
+    const float *beta;
+    void *out;
+    float *dgamma;
+    float *dbeta;
+    void *workspace;
+    cudaStream_t stream;
+};
+
+size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
+cudaError_t launch_affine_fwd(const AffineLaunch &a);
+cudaError_t launch_affine_bwd(const AffineLaunch &a);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Resident blocks per SM of one kernel instantiation at `threads` threads
+// per block.  The Tag type gives every instantiation its own cache (kernels
+// of one template share a function-pointer type).  Every GPU this library
+// targets is a B200, so the value does not vary between devices.
+template <class Tag, typename K>
+int resident_blocks(K kernel, int threads)
+{
+    static int blocks = 0;
+    if (blocks == 0) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, 0) != cudaSuccess || b <= 0)
+            b = 1;
+        blocks = b;
+    }
+    return blocks;
+}
+
+}  // namespace mea

@@ -1,0 +1,464 @@
+// mea_math.cuh -- fp32 device arithmetic of the activation family.
+//
+// Each activation is a struct with the forward value f(x) and the backward
+// product dy * f'(x), both recomputed from x alone (the save-input-only
+// contract of "Memory efficient Swish", sections "How is the memory efficient
+// version Swish implemented?" and "What makes this implementation save GPU
+// memory?").  The family is the one costed in "What activations cost, in
+// memory and in arithmetic" (problem B07, GIVEN); definitions are standard.
+//
+// Sigmoid primitive.  Sigmoid(v) = 1 / (1 + E) with E = e^-v = 2^t,
+// t = -v log2(e), evaluated with the PTX instructions ex2.approx.ftz.f32 and
+// rcp.approx.ftz.f32 (two MUFU operations).  1 - Sigmoid(v) is taken as
+// E * s where v > 0 and as 1 - s where v <= 0, so neither branch cancels.
+//
+// Precision modes (template flag P):
+//  - P = false (bf16 storage): t is one fp32 product.  Its rounding moves E
+//    by at most |t| 2^-24 ln 2 relative (< 2^-12 for |t| <= 126), far below
+//    half a bf16 ulp.
+//  - P = true (fp32 storage): t = x * (c_hi + c_lo) is carried as a
+//    float-float pair and E is corrected by (1 + t_lo ln 2), which removes
+//    the argument-rounding error that would otherwise reach ~1e-5 at
+//    |t| ~ 126.  GELU-tanh forms its cubic argument in fp64 for the same
+//    reason.
+//
+// Deep tails.  Where E > 2^126 the sigmoid itself would be subnormal and the
+// .ftz instructions would flush it, although x * Sigmoid(alpha x) is still a
+// normal number for alpha x down to about -103.  Those elements (flagged by
+// the main path through `tail`) are recomputed from 2^(64 - t), which stays
+// normal, and the result is scaled by 2^-64 at the end.
+#pragma once
+
+#include <stdint.h>
+
+namespace mea {
+
+constexpr float kLn2f = 0.693147180559945309f;
+constexpr float kLog2eHi = 1.44269502162933349609375f;      // fp32(log2 e)
+constexpr float kLog2eLo = 1.9259629911266174681e-08f;      // log2 e - kLog2eHi
+constexpr double kLog2eD = 1.4426950408889634074;
+constexpr float kTailT = 124.0f;       // main path used while t <= this (margin below 126)
+constexpr float kCorrMax = 192.0f;     // |t| beyond which E is 0 or inf anyway
+constexpr float kTwoM64 = 5.42101086242752217e-20f;          // 2^-64
+constexpr float kBig = 3.0e38f;
+
+__device__ __forceinline__ float ex2_ftz(float t)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
+    return r;
+}
+
+__device__ __forceinline__ float rcp_ftz(float v)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// Multiplicative correction 2^t_lo ~ 1 + t_lo ln 2 for a float-float t.
+__device__ __forceinline__ float corr(float t_hi, float t_lo)
+{
+    float c = fmaf(t_lo, kLn2f, 1.0f);
+    return fabsf(t_hi) < kCorrMax ? c : 1.0f;
+}
+
+// Low part of x * (c_hi + c_lo) given t_hi = x * c_hi.
+__device__ __forceinline__ float prod_lo(float x, float c_hi, float c_lo, float t_hi)
+{
+    return fmaf(x, c_lo, fmaf(x, c_hi, -t_hi));
+}
+
+// Per-launch constants, built on the device from the scalar parameter.
+struct Coef {
+    float p;      // alpha (Swish) or slope (LeakyReLU)
+    float c_hi;   // exponent coefficient (fp32 head)
+    float c_lo;   // exponent coefficient (tail)
+};
+
+// Float-float value of m * log2(e) for an fp32 m.
+__device__ __forceinline__ void scaled_log2e(float m, float &hi, float &lo)
+{
+    hi = m * kLog2eHi;
+    lo = fmaf(m, kLog2eLo, fmaf(m, kLog2eHi, -hi));
+}
+
+// ------------------------------------------------------------------ ReLU
+struct ReLU {
+    static __device__ __forceinline__ Coef coef(float) { return Coef{0.f, 0.f, 0.f}; }
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &, bool &)
+    {
+        return x > 0.f ? x : (x != x ? x : 0.f);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &) { return x; }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &, bool &)
+    {
+        return dy * (x > 0.f ? 1.f : 0.f);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float, float dy, const Coef &) { return dy; }
+    static __device__ __forceinline__ bool is_tail(float, const Coef &) { return false; }
+};
+
+// ------------------------------------------------------------- LeakyReLU
+struct LeakyReLU {
+    static __device__ __forceinline__ Coef coef(float slope) { return Coef{slope, 0.f, 0.f}; }
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &k, bool &)
+    {
+        return x > 0.f ? x : k.p * x;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &) { return x; }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &k, bool &)
+    {
+        return dy * (x > 0.f ? 1.f : k.p);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float, float dy, const Coef &) { return dy; }
+    static __device__ __forceinline__ bool is_tail(float, const Coef &) { return false; }
+};
+
+// -------------------------------------------------------------- Sigmoid
+// t = -x log2 e; s = 1 / (1 + 2^t).
+struct Sigmoid {
+    static __device__ __forceinline__ Coef coef(float)
+    {
+        Coef k;
+        k.p = 1.f;
+        scaled_log2e(-1.f, k.c_hi, k.c_lo);
+        return k;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float expo(float x, const Coef &k, float &t)
+    {
+        t = x * k.c_hi;
+        float E = ex2_ftz(t);
+        if (P) E *= corr(t, prod_lo(x, k.c_hi, k.c_lo, t));
+        return E;
+    }
+    // 2^(64 - t): the sigmoid scaled by 2^64 in the tail (t > 126).
+    template <bool P>
+    static __device__ __forceinline__ float tail_s64(float x, const Coef &k)
+    {
+        float t = x * k.c_hi;
+        float s64 = ex2_ftz(64.f - t);
+        if (P) s64 *= corr(t, -prod_lo(x, k.c_hi, k.c_lo, t));
+        return s64;
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &k) { return x * k.c_hi > kTailT; }
+
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &k, bool &tail)
+    {
+        float t;
+        float E = expo<P>(x, k, t);
+        tail |= t > kTailT;
+        return rcp_ftz(1.f + E);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &k)
+    {
+        return tail_s64<P>(x, k) * kTwoM64;
+    }
+    // dx = dy s (1 - s)
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &k, bool &tail)
+    {
+        float t;
+        float E = expo<P>(x, k, t);
+        tail |= t > kTailT;
+        float s = rcp_ftz(1.f + E);
+        float sm = x > 0.f ? E * s : 1.f - s;
+        return dy * (s * sm);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
+    {
+        return (dy * tail_s64<P>(x, k)) * kTwoM64;   // 1 - s = 1 there
+    }
+};
+
+// ----------------------------------------------------------------- Tanh
+// Forward: CUDA's tanhf.  Backward: 1 - tanh^2 x = 4 Sigmoid(2|x|)
+// Sigmoid(-2|x|) = 4 E s with E = 2^t, t = -2|x| log2 e (t <= 0), s = 1/(1+E).
+struct Tanh {
+    static __device__ __forceinline__ Coef coef(float)
+    {
+        Coef k;
+        k.p = 1.f;
+        scaled_log2e(-2.f, k.c_hi, k.c_lo);
+        return k;
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &k)
+    {
+        return fabsf(x) * k.c_hi < -120.f;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &, bool &)
+    {
+        return tanhf(x);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &) { return tanhf(x); }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &k, bool &tail)
+    {
+        float a = fabsf(x);
+        float t = a * k.c_hi;
+        float E = ex2_ftz(t);
+        if (P) E *= corr(t, prod_lo(a, k.c_hi, k.c_lo, t));
+        tail |= t < -120.f;
+        float s = rcp_ftz(1.f + E);
+        return dy * ((4.f * E) * s);
+    }
+    // t < -120: s = 1, 4E = 2^(t + 2) may be subnormal; use 2^(t + 66) 2^-64.
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
+    {
+        float a = fabsf(x);
+        float t = a * k.c_hi;
+        float e64 = ex2_ftz(t + 66.f);
+        if (P) e64 *= corr(t, prod_lo(a, k.c_hi, k.c_lo, t));
+        return (dy * e64) * kTwoM64;
+    }
+};
+
+// ------------------------------------------------------------- GELU-erf
+// y = x Phi(x), Phi(x) = erfc(-x / sqrt 2) / 2 (CUDA's erfcf); backward
+// Phi(x) + x phi(x), phi(x) = e^(-x^2 / 2) / sqrt(2 pi) (CUDA's expf).
+// Precise mode carries -x / sqrt 2 and x^2 as float-float pairs and applies
+// the first-order corrections d erfc = -(2 / sqrt pi) e^(-w^2) dw and
+// e^(-l/2) ~ 1 - l/2.
+struct GeluErf {
+    static constexpr float kNegRsqrt2Hi = -0.707106769084930419921875f;
+    static constexpr float kNegRsqrt2Lo = -1.2101617104478969362e-08f;
+    static constexpr float kTwoRsqrtPi = 1.12837916709551257f;     // 2 / sqrt(pi)
+    static constexpr float kRsqrt2Pi = 0.398942280401432678f;      // 1 / sqrt(2 pi)
+
+    static __device__ __forceinline__ Coef coef(float) { return Coef{1.f, 0.f, 0.f}; }
+    static __device__ __forceinline__ bool is_tail(float, const Coef &) { return false; }
+
+    // returns erfc(-x / sqrt 2) and sets g = e^(-x^2 / 2)
+    template <bool P>
+    static __device__ __forceinline__ float erfc_and_gauss(float x, float &g)
+    {
+        float w = x * kNegRsqrt2Hi;
+        float ec = erfcf(w);
+        float h = x * x;
+        g = expf(-0.5f * h);
+        if (P) {
+            float l = fmaf(x, x, -h);
+            l = h < kBig ? l : 0.f;
+            g *= fmaf(-0.5f, l, 1.f);
+            float wl = fmaf(x, kNegRsqrt2Lo, fmaf(x, kNegRsqrt2Hi, -w));
+            ec = fmaf(-kTwoRsqrtPi * wl, g, ec);
+        }
+        return ec;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &, bool &)
+    {
+        float g;
+        float ec = erfc_and_gauss<P>(x, g);
+        return (0.5f * x) * ec;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &k)
+    {
+        bool t = false;
+        return f<P>(x, k, t);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &, bool &)
+    {
+        float g;
+        float ec = erfc_and_gauss<P>(x, g);
+        float d = fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
+        return dy * d;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
+    {
+        bool t = false;
+        return df<P>(x, dy, k, t);
+    }
+};
+
+// ------------------------------------------------------------ GELU-tanh
+// y = x Sigmoid(v), v = 2u = x (k1 + k3 x^2), k1 = 2 sqrt(2/pi),
+// k3 = 2 sqrt(2/pi) 0.044715 (Hendrycks and Gimpel's constants).
+// t = -v log2 e = x (c1 + c3 x^2).  Backward:
+// Sigmoid(v) + x v' Sigmoid(v) Sigmoid(-v), v' = k1 + 3 k3 x^2.
+struct GeluTanh {
+    static constexpr double kK1 = 1.5957691216057307;            // 2 sqrt(2/pi)
+    static constexpr double kK3 = 1.5957691216057307 * 0.044715;
+    static constexpr float kK1f = (float)kK1;
+    static constexpr float kK3x3f = (float)(3.0 * kK3);
+    static constexpr float kC1f = (float)(-kK1 * kLog2eD);
+    static constexpr float kC3f = (float)(-kK3 * kLog2eD);
+    static constexpr double kC1d = -kK1 * kLog2eD;
+    static constexpr double kC3d = -kK3 * kLog2eD;
+
+    static __device__ __forceinline__ Coef coef(float) { return Coef{1.f, 0.f, 0.f}; }
+
+    template <bool P>
+    static __device__ __forceinline__ float expo_arg(float x, float &t_lo)
+    {
+        if (P) {
+            double xd = (double)x;
+            double td = xd * fma(kC3d, xd * xd, kC1d);
+            float t = (float)td;
+            t_lo = (float)(td - (double)t);
+            return t;
+        }
+        t_lo = 0.f;
+        return x * fmaf(kC3f, x * x, kC1f);
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &)
+    {
+        float tl;
+        return expo_arg<false>(x, tl) > kTailT;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &, bool &tail)
+    {
+        float tl;
+        float t = expo_arg<P>(x, tl);
+        float E = ex2_ftz(t);
+        if (P) E *= corr(t, tl);
+        tail |= t > kTailT;
+        return x * rcp_ftz(1.f + E);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float s64_tail(float x)
+    {
+        float tl;
+        float t = expo_arg<P>(x, tl);
+        float s64 = ex2_ftz(64.f - t);
+        if (P) s64 *= corr(t, -tl);
+        return s64;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &)
+    {
+        return (x * s64_tail<P>(x)) * kTwoM64;
+    }
+    // x v', clamped so that it times a zero sigmoid factor stays 0
+    static __device__ __forceinline__ float xdv(float x)
+    {
+        float q = x * fmaf(kK3x3f, x * x, kK1f);
+        return fmaxf(fminf(q, kBig), -kBig);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &, bool &tail)
+    {
+        float tl;
+        float t = expo_arg<P>(x, tl);
+        float E = ex2_ftz(t);
+        if (P) E *= corr(t, tl);
+        tail |= t > kTailT;
+        float s = rcp_ftz(1.f + E);
+        float sm = x > 0.f ? E * s : 1.f - s;
+        float q = xdv(x);
+        return dy * fmaf(q * s, sm, s);
+    }
+    // v << 0: Sigmoid(-v) = 1, f' = s (1 + x v')
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &)
+    {
+        float q = xdv(x);
+        return ((dy * s64_tail<P>(x)) * (1.f + q)) * kTwoM64;
+    }
+};
+
+// ---------------------------------------------------------------- Swish
+// y = x Sigmoid(z), z = alpha x; t = x c, c = -alpha log2 e (float-float).
+// dx = dy (s + z s Sigmoid(-z)); d alpha term = dy x^2 s Sigmoid(-z).
+struct Swish {
+    static __device__ __forceinline__ Coef coef(float alpha)
+    {
+        Coef k;
+        k.p = alpha;
+        scaled_log2e(-alpha, k.c_hi, k.c_lo);
+        return k;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float expo(float x, const Coef &k, float &t)
+    {
+        t = x * k.c_hi;
+        float E = ex2_ftz(t);
+        if (P) E *= corr(t, prod_lo(x, k.c_hi, k.c_lo, t));
+        return E;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float tail_s64(float x, const Coef &k)
+    {
+        float t = x * k.c_hi;
+        float s64 = ex2_ftz(64.f - t);
+        if (P) s64 *= corr(t, -prod_lo(x, k.c_hi, k.c_lo, t));
+        return s64;
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &k) { return x * k.c_hi > kTailT; }
+
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const Coef &k, bool &tail)
+    {
+        float t;
+        float E = expo<P>(x, k, t);
+        tail |= t > kTailT;
+        return x * rcp_ftz(1.f + E);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const Coef &k)
+    {
+        return (x * tail_s64<P>(x, k)) * kTwoM64;
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &k, bool &tail)
+    {
+        float t;
+        float E = expo<P>(x, k, t);
+        tail |= t > kTailT;
+        float s = rcp_ftz(1.f + E);
+        float z = k.p * x;
+        float sm = z > 0.f ? E * s : 1.f - s;
+        z = fminf(z, kBig);
+        return dy * fmaf(z * s, sm, s);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
+    {
+        float z = fmaxf(k.p * x, -kBig);
+        return ((dy * tail_s64<P>(x, k)) * (1.f + z)) * kTwoM64;
+    }
+    // Backward plus the d alpha term dy x^2 s (1 - s).
+    template <bool P>
+    static __device__ __forceinline__ float df_da(float x, float dy, const Coef &k, bool &tail,
+                                                  float &term)
+    {
+        float t;
+        float E = expo<P>(x, k, t);
+        tail |= t > kTailT;
+        float s = rcp_ftz(1.f + E);
+        float z = k.p * x;
+        float sm = z > 0.f ? E * s : 1.f - s;
+        term = (((x * s) * sm) * x) * dy;
+        z = fminf(z, kBig);
+        return dy * fmaf(z * s, sm, s);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float df_da_tail(float x, float dy, const Coef &k, float &term)
+    {
+        float s64 = tail_s64<P>(x, k);
+        float z = fmaxf(k.p * x, -kBig);
+        term = (((x * s64) * x) * dy) * kTwoM64;
+        return ((dy * s64) * (1.f + z)) * kTwoM64;
+    }
+};
+
+}  // namespace mea

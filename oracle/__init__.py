@@ -79,12 +79,14 @@ def _load():
         lib.oracle_act_bwd.restype = ctypes.c_int
         lib.oracle_act_deriv.argtypes = [ctypes.c_int, d, d, i64, ctypes.c_double]
         lib.oracle_act_deriv.restype = ctypes.c_int
+        lib.oracle_act_bwd_scale.argtypes = [ctypes.c_int, d, d, d, i64, ctypes.c_double]
+        lib.oracle_act_bwd_scale.restype = ctypes.c_int
         lib.oracle_swish_dalpha.argtypes = [d, d, i64, ctypes.c_double]
         lib.oracle_swish_dalpha.restype = ctypes.c_double
         shp = ctypes.POINTER(ctypes.c_int64)
         lib.oracle_affine_swish_fwd.argtypes = [ctypes.c_int, shp, d, d, d, d]
         lib.oracle_affine_swish_fwd.restype = ctypes.c_int
-        lib.oracle_affine_swish_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d, d]
+        lib.oracle_affine_swish_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d, d, d]
         lib.oracle_affine_swish_bwd.restype = ctypes.c_int
         lib.oracle_round_bf16.argtypes = [d, ctypes.POINTER(ctypes.c_uint16), i64]
         lib.oracle_round_bf16.restype = None
@@ -132,6 +134,19 @@ def act_bwd(act: str, x, dy, param: float = 1.0) -> np.ndarray:
     return dx
 
 
+def act_bwd_scale(act: str, x, dy, param: float = 1.0) -> np.ndarray:
+    """|dy| times the sum of the absolute terms of f'(x): the scale the error
+    of a finite-precision dx is proportional to (equals |dx| where f' has a
+    single term)."""
+    x = _f64(x)
+    dy = _f64(dy)
+    m = np.empty_like(x)
+    rc = _load().oracle_act_bwd_scale(ACTS[act], _ptr(x), _ptr(dy), _ptr(m), x.size, float(param))
+    if rc:
+        raise ValueError(f"oracle_act_bwd_scale({act}) failed: {rc}")
+    return m
+
+
 def act_deriv(act: str, x, param: float = 1.0) -> np.ndarray:
     """f'(x; param) in double."""
     x = _f64(x)
@@ -168,20 +183,23 @@ def affine_swish_fwd(layout: str, shape, x, gamma, beta) -> np.ndarray:
     return y
 
 
-def affine_swish_bwd(layout: str, shape, x, dy, gamma, beta):
-    """Returns (dx, dgamma, dbeta) in double."""
+def affine_swish_bwd(layout: str, shape, x, dy, gamma, beta, with_scale: bool = False):
+    """Returns (dx, dgamma, dbeta) in double, plus the condition scale of dx
+    when with_scale is set."""
     s = _shape4(shape)
     x, dy, gamma, beta = _f64(x), _f64(dy), _f64(gamma), _f64(beta)
     dx = np.empty_like(x)
     C = int(s[1])
     dg = np.empty(C, dtype=np.float64)
     db = np.empty(C, dtype=np.float64)
+    scale = np.empty_like(x) if with_scale else None
     rc = _load().oracle_affine_swish_bwd(LAYOUTS[layout], _ptr(s, ctypes.c_int64),
                                          _ptr(x), _ptr(dy), _ptr(gamma), _ptr(beta),
-                                         _ptr(dx), _ptr(dg), _ptr(db))
+                                         _ptr(dx), _ptr(dg), _ptr(db),
+                                         _ptr(scale) if with_scale else None)
     if rc:
         raise ValueError(f"oracle_affine_swish_bwd failed: {rc}")
-    return dx, dg, db
+    return (dx, dg, db, scale) if with_scale else (dx, dg, db)
 
 
 def round_bf16(v) -> np.ndarray:

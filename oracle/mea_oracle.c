@@ -252,6 +252,41 @@ int oracle_act_deriv(int act, const double *x, double *d, int64_t n, double para
     return 0;
 }
 
+/* Condition scale of the backward product dx = dy f'(x): |dy| times the sum
+ * of the absolute values of the terms f' is made of.  Where f' is a sum
+ * whose terms cancel (Swish and both GELUs near the zero of f'), the error
+ * of any finite-precision evaluation is proportional to this scale rather
+ * than to |dx|; elsewhere it equals |dx|.  Used by the tests to state the
+ * fp32 tolerance as |g - r| <= 1e-5 max(|r|, scale). */
+static double act_df_abs_terms(int act, double x, double param)
+{
+    switch (act) {
+    case OR_SWISH: {
+        double z = param * x, s = sigm(z);
+        return s + fabs(z) * s * sigm(-z);
+    }
+    case OR_GELU_ERF:
+        return std_normal_cdf(x) + fabs(x) * std_normal_pdf(x);
+    case OR_GELU_TANH: {
+        double v = 2.0 * gelu_tanh_u(x);
+        double dv = 2.0 * GELU_K0 * (1.0 + 3.0 * GELU_K1 * x * x);
+        double s = sigm(v);
+        return s + fabs(x * dv) * s * sigm(-v);
+    }
+    default:
+        return fabs(act_df(act, x, param));
+    }
+}
+
+int oracle_act_bwd_scale(int act, const double *x, const double *dy, double *m,
+                         int64_t n, double param)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || n < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) m[i] = fabs(dy[i]) * act_df_abs_terms(act, x[i], param);
+    return 0;
+}
+
 /* d alpha = sum_i dy_i x_i^2 s_i (1 - s_i), serial, index order, long
  * double accumulator. */
 double oracle_swish_dalpha(const double *x, const double *dy, int64_t n, double alpha)
@@ -288,10 +323,11 @@ int oracle_affine_swish_fwd(int layout, const int64_t shape[4], const double *x,
 }
 
 /* dz = dy (s + z s (1 - s)); dx = gamma_c dz; dgamma_c = sum dz x;
- * dbeta_c = sum dz (serial, index order, long double). */
+ * dbeta_c = sum dz (serial, index order, long double).  dx_scale, when not
+ * NULL, receives the condition scale of each dx (see oracle_act_bwd_scale). */
 int oracle_affine_swish_bwd(int layout, const int64_t shape[4], const double *x,
                             const double *dy, const double *gamma, const double *beta,
-                            double *dx, double *dgamma, double *dbeta)
+                            double *dx, double *dgamma, double *dbeta, double *dx_scale)
 {
     if (layout != OR_NCHW && layout != OR_NHWC) return -1;
     int64_t C = shape[1];
@@ -305,6 +341,8 @@ int oracle_affine_swish_bwd(int layout, const int64_t shape[4], const double *x,
         double s = sigm(z);
         double dz = dy[i] * (s + z * s * sigm(-z));
         dx[i] = gamma[c] * dz;
+        if (dx_scale)   /* condition scale of dx (see oracle_act_bwd_scale) */
+            dx_scale[i] = fabs(gamma[c] * dy[i]) * (s + fabs(z) * s * sigm(-z));
         acc_g[c] += (long double)(dz * x[i]);
         acc_b[c] += (long double)dz;
     }

@@ -1,0 +1,107 @@
+"""Comparison rules between GPU outputs and the oracle (test helpers).
+
+bf16 outputs: the ordered-integer distance between the GPU's bit pattern and
+the oracle's double result rounded to nearest-even bf16 is at most 1 (+0 and
+-0 count as equal; NaN matches NaN).
+
+fp32 outputs: |g - r| <= 1e-5 * max(|r|, m), where r is the oracle's double
+result and m the condition scale of the output (for a backward product, |dy|
+times the sum of the absolute terms of f'; for a forward, |r| itself).  This
+is the fp32 bound "max relative error 1e-5" read per element, with the
+denominator taken from the terms where f' cancels near its zero.
+
+Both: results whose exact value is below the smallest normal, 2^-126, may be
+flushed; they pass when |g - r| <= floor (2^-126 unless a caller scales it,
+e.g. by |dy| for a backward product).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TINY = 2.0 ** -126
+F32_TOL = 1e-5
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to(torch.float64).cpu().numpy().ravel()
+
+
+def _ordered(bits: np.ndarray) -> np.ndarray:
+    b = bits.astype(np.int64)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None) -> dict:
+    g_bits = bf16_bits(gpu)
+    ref = np.asarray(ref, dtype=np.float64).ravel()
+    r_bits = oracle.round_bf16(ref)
+    dist = np.abs(_ordered(g_bits) - _ordered(r_bits))
+    g = bits_to_f64(g_bits)
+    fl = TINY if floor is None else np.asarray(floor, dtype=np.float64).ravel()
+    with np.errstate(invalid="ignore"):
+        nan_ok = np.isnan(g) & np.isnan(ref)
+        tiny_ok = (np.abs(ref) < TINY) & (np.abs(g - ref) <= fl)
+    ok = (dist <= 1) | nan_ok | tiny_ok
+    bad = np.flatnonzero(~ok)
+    return {
+        "n": ref.size,
+        "bad": bad.size,
+        "max_ulp": int(dist[~(nan_ok | tiny_ok)].max(initial=0)),
+        "exact_frac": float(np.mean(dist == 0)) if ref.size else 1.0,
+        "first_bad": [(int(i), float(ref[i]), float(g[i]), int(dist[i])) for i in bad[:8]],
+    }
+
+
+def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F32_TOL) -> dict:
+    g = to_f64(gpu)
+    ref = np.asarray(ref, dtype=np.float64).ravel()
+    denom = np.abs(ref) if scale is None else np.maximum(np.abs(ref), np.asarray(scale).ravel())
+    fl = TINY if floor is None else np.asarray(floor, dtype=np.float64).ravel()
+    with np.errstate(invalid="ignore", divide="ignore"):
+        err = np.abs(g - ref)
+        nan_ok = np.isnan(g) & np.isnan(ref)
+        same = g == ref
+        tiny_ok = (np.abs(ref) < TINY) & (err <= fl)
+        ok = (err <= tol * denom) | nan_ok | same | tiny_ok
+        rel = np.where(denom > 0, err / denom, 0.0)
+        pure = np.where(np.abs(ref) >= TINY, err / np.abs(ref), 0.0)
+    bad = np.flatnonzero(~ok)
+    sel = ~(nan_ok | same | tiny_ok)
+    return {
+        "n": ref.size,
+        "bad": bad.size,
+        "max_rel": float(np.nanmax(rel[sel], initial=0.0)),
+        "max_pure_rel": float(np.nanmax(pure[sel], initial=0.0)),
+        "pure_over_tol": int(np.sum(pure[sel] > tol)),
+        "first_bad": [(int(i), float(ref[i]), float(g[i])) for i in bad[:8]],
+    }
+
+
+def assert_bf16(gpu, ref, floor=None, what=""):
+    r = bf16_report(gpu, ref, floor)
+    assert r["bad"] == 0, f"{what}: {r}"
+    return r
+
+
+def assert_f32(gpu, ref, scale=None, floor=None, what="", tol=F32_TOL):
+    r = f32_report(gpu, ref, scale, floor, tol)
+    assert r["bad"] == 0, f"{what}: {r}"
+    return r
+
+
+def check(dtype: str, gpu, ref, scale=None, floor=None, what=""):
+    if dtype == "bf16":
+        return assert_bf16(gpu, ref, floor, what)
+    return assert_f32(gpu, ref, scale, floor, what)

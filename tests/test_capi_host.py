@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library loads, exports every function include/mea.h declares with the
+enumerations the binding uses, and rejects invalid calls synchronously with
+the documented status codes before any CUDA call.  Pointer arguments here
+are fake addresses: every call below is refused during validation.
+"""
+import os
+import re
+
+import pytest
+
+from memory_efficient_activation_b200 import _capi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mea.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _capi.lib()
+
+
+def _header_functions():
+    src = open(HEADER).read()
+    return re.findall(r"MEA_API\s+[\w\s\*]+?\b(mea_\w+)\s*\(", src)
+
+
+def _header_enum(name):
+    src = open(HEADER).read()
+    return {k: int(v) for k, v in re.findall(r"\b(" + name + r"\w*)\s*=\s*(\d+)", src)}
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _header_functions()
+    assert len(declared) == 9, declared
+    for fn in declared:
+        assert hasattr(lib, fn), fn
+        assert fn in _capi.SIGNATURES, fn
+    assert set(_capi.SIGNATURES) == set(declared)
+
+
+def test_enums_match_header():
+    acts = _header_enum("MEA_")
+    for name, val in [("MEA_RELU", _capi.MEA_RELU), ("MEA_LEAKY_RELU", _capi.MEA_LEAKY_RELU),
+                      ("MEA_SIGMOID", _capi.MEA_SIGMOID), ("MEA_TANH", _capi.MEA_TANH),
+                      ("MEA_GELU_ERF", _capi.MEA_GELU_ERF), ("MEA_GELU_TANH", _capi.MEA_GELU_TANH),
+                      ("MEA_SWISH", _capi.MEA_SWISH), ("MEA_F32", _capi.MEA_F32), ("MEA_BF16", _capi.MEA_BF16),
+                      ("MEA_NCHW", _capi.MEA_NCHW), ("MEA_NHWC", _capi.MEA_NHWC), ("MEA_OK", _capi.MEA_OK),
+                      ("MEA_ERR_INVALID_ARG", _capi.MEA_ERR_INVALID_ARG),
+                      ("MEA_ERR_UNSUPPORTED", _capi.MEA_ERR_UNSUPPORTED),
+                      ("MEA_ERR_WORKSPACE", _capi.MEA_ERR_WORKSPACE), ("MEA_ERR_CUDA", _capi.MEA_ERR_CUDA)]:
+        assert acts[name] == val, name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.mea_version() == 10000
+    for st in range(5):
+        assert lib.mea_status_string(st)
+    assert lib.mea_status_string(99) == b"unknown status"
+
+
+X, Y, G, D = 0x100000, 0x200000, 0x300000, 0x400000
+
+
+def test_fwd_validation(lib):
+    f = lib.mea_act_fwd
+    assert f(7, 1, X, Y, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b"act" in lib.mea_last_error()
+    assert f(-1, 1, X, Y, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 2, X, Y, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 1, X, Y, -1, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 1, None, Y, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 1, X, None, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    # y may not overlap x at all (x is the saved tensor)
+    assert f(6, 1, X, X, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 1, X, X + 18, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(6, 0, X, X + 36, 10, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    # n = 0 is a no-op, even with NULL pointers
+    assert f(6, 1, None, None, 0, 1.0, None, None) == _capi.MEA_OK
+    assert lib.mea_last_error() == b""
+
+
+def test_bwd_validation(lib):
+    b = lib.mea_act_bwd
+    ok_ws = lib.mea_act_bwd_workspace_bytes(6, 1000, 1)
+    assert b(6, 1, X, G, D, -5, 1.0, None, None, None, 0, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b(6, 1, X, None, D, 5, 1.0, None, None, None, 0, None) == _capi.MEA_ERR_INVALID_ARG
+    # d alpha only for Swish
+    assert b(0, 1, X, G, D, 5, 1.0, None, 0x500000, 0x600000, ok_ws, None) == _capi.MEA_ERR_UNSUPPORTED
+    # workspace missing / small / misaligned
+    assert b(6, 1, X, G, D, 1000, 1.0, None, 0x500000, None, ok_ws, None) == _capi.MEA_ERR_WORKSPACE
+    assert b(6, 1, X, G, D, 1000, 1.0, None, 0x500000, 0x600000, ok_ws - 1, None) == _capi.MEA_ERR_WORKSPACE
+    assert b(6, 1, X, G, D, 1000, 1.0, None, 0x500000, 0x600008, ok_ws, None) == _capi.MEA_ERR_WORKSPACE
+    # partial overlap of dx with dy or x is refused; exact aliasing is not checked here
+    assert b(6, 1, X, G, G + 2, 100, 1.0, None, None, None, 0, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b(6, 1, X, G, X + 64, 100, 1.0, None, None, None, 0, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b(6, 1, None, None, None, 0, 1.0, None, None, None, 0, None) == _capi.MEA_OK
+
+
+def test_workspace_sizes(lib):
+    w = lib.mea_act_bwd_workspace_bytes
+    assert w(6, 1000, 0) == 0
+    assert w(6, 0, 1) == 256 + 8
+    assert w(6, 8192, 1) == 256 + 8
+    assert w(6, 8193, 1) == 256 + 16
+    assert w(6, 1 << 40, 1) == 256 + 8 * 1184
+    aw = lib.mea_affine_swish_bwd_workspace_bytes
+    assert aw(1, 1, _capi.shape4((128, 144, 56, 56))) >= 256 + 16 * 144
+    assert aw(1, 0, _capi.shape4((64, 32, 112, 112))) >= 256 + 16 * 32
+    assert aw(1, 1, _capi.shape4((1, -1, 1, 1))) == 0
+    assert aw(1, 5, _capi.shape4((1, 1, 1, 1))) == 0
+    assert aw(3, 1, _capi.shape4((1, 1, 1, 1))) == 0
+
+
+def test_affine_validation(lib):
+    s = _capi.shape4((2, 16, 3, 3))
+    fw = lib.mea_affine_swish_fwd
+    assert fw(1, 2, s, X, G, D, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fw(1, 1, None, X, G, D, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fw(1, 1, _capi.shape4((2, -16, 3, 3)), X, G, D, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fw(1, 1, s, X, None, D, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fw(1, 1, s, X, G, D, X + 2, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fw(1, 1, _capi.shape4((0, 16, 3, 3)), None, None, None, None, None) == _capi.MEA_OK
+    bw = lib.mea_affine_swish_bwd
+    need = lib.mea_affine_swish_bwd_workspace_bytes(1, 1, s)
+    assert bw(1, 1, s, X, G, 0x700000, 0x710000, D, 0x720000, 0x730000, None, need, None) \
+        == _capi.MEA_ERR_WORKSPACE
+    assert bw(1, 1, s, X, G, 0x700000, 0x710000, D, 0x720000, 0x730000, 0x800000, need - 8, None) \
+        == _capi.MEA_ERR_WORKSPACE
+    assert bw(1, 1, s, X, G, 0x700000, 0x710000, D, 0x720000, 0x720010, 0x800000, need, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    assert bw(1, 1, s, X, G, None, 0x710000, D, 0x720000, 0x730000, 0x800000, need, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import memory_efficient_activation_b200 as mea
+    with pytest.raises(ValueError):
+        mea.act_fwd("swish", torch.zeros(4))
+    with pytest.raises(ValueError):
+        mea.act_fwd("softplus", torch.zeros(4))

@@ -196,3 +196,21 @@ def test_swish_nan_propagates():
     assert np.isnan(y[0]) and not np.isnan(y[1])
     dx = oracle.act_bwd("swish", x, np.ones(2))
     assert np.isnan(dx[0]) and not np.isnan(dx[1])
+
+
+@pytest.mark.parametrize("act", ["swish", "gelu_erf", "gelu_tanh", "sigmoid", "tanh", "relu", "leaky_relu"])
+def test_bwd_scale_bounds_and_equalities(act):
+    # The condition scale is |dy| times the sum of |terms| of f': never below
+    # |dx|, equal to it wherever the terms share a sign (x >= 0 here for all
+    # members), and strictly above it where they cancel.
+    x = np.linspace(-8.0, 8.0, 3201)
+    dy = synthetic.normal_f64(x.size, 1.0, 17, 1)
+    p = 0.01 if act == "leaky_relu" else 1.0
+    m = oracle.act_bwd_scale(act, x, dy, p)
+    dx = np.abs(oracle.act_bwd(act, x, dy, p))
+    assert np.all(m >= dx * (1 - 1e-15))
+    pos = x >= 0
+    np.testing.assert_allclose(m[pos], dx[pos], rtol=1e-14, atol=0)
+    if act in ("swish", "gelu_erf", "gelu_tanh"):
+        # at the zero of f' the scale stays finite and positive
+        assert np.all(m[(x < -0.5) & (x > -2.0)] > 0.1 * np.abs(dy[(x < -0.5) & (x > -2.0)]))
