@@ -157,9 +157,9 @@ __device__ __forceinline__ double block_sum(double v, double *red)
 __device__ __forceinline__ bool last_block_done(unsigned int *ticket)
 {
     __shared__ int is_last;
+    __threadfence();          // every thread's partial stores are visible device-wide
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
         unsigned int t = atomicInc(ticket, gridDim.x - 1);
         is_last = (t == gridDim.x - 1);
     }

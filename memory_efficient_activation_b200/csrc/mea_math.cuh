@@ -150,7 +150,13 @@ struct Sigmoid {
         if (P) s64 *= corr(t, -prod_lo(x, k.c_hi, k.c_lo, t));
         return s64;
     }
-    static __device__ __forceinline__ bool is_tail(float x, const Coef &k) { return x * k.c_hi > kTailT; }
+    // Both tails: for x << 0 the sigmoid, for x >> 0 its complement E s,
+    // would be subnormal.  The forward only needs the first; taking both is
+    // harmless (the forward's tail value for x >> 0 is exactly 1).
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &k)
+    {
+        return fabsf(x * k.c_hi) > kTailT;
+    }
 
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &k, bool &tail)
@@ -163,7 +169,7 @@ struct Sigmoid {
     template <bool P>
     static __device__ __forceinline__ float f_tail(float x, const Coef &k)
     {
-        return tail_s64<P>(x, k) * kTwoM64;
+        return x > 0.f ? 1.f : tail_s64<P>(x, k) * kTwoM64;
     }
     // dx = dy s (1 - s)
     template <bool P>
@@ -171,21 +177,30 @@ struct Sigmoid {
     {
         float t;
         float E = expo<P>(x, k, t);
-        tail |= t > kTailT;
+        tail |= fabsf(t) > kTailT;
         float s = rcp_ftz(1.f + E);
         float sm = x > 0.f ? E * s : 1.f - s;
         return dy * (s * sm);
     }
+    // |t| > 124: s (1 - s) = 2^-|t| to within 2^-124 relative, formed as
+    // 2^(64 - |t|) 2^-64 so that it stays normal until the final scaling.
     template <bool P>
     static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
     {
-        return (dy * tail_s64<P>(x, k)) * kTwoM64;   // 1 - s = 1 there
+        float t = x * k.c_hi;
+        float e = ex2_ftz(64.f - fabsf(t));
+        if (P) {
+            const float lo = prod_lo(x, k.c_hi, k.c_lo, t);
+            e *= corr(t, t > 0.f ? -lo : lo);
+        }
+        return (dy * e) * kTwoM64;
     }
 };
 
 // ----------------------------------------------------------------- Tanh
 // Forward: CUDA's tanhf.  Backward: 1 - tanh^2 x = 4 Sigmoid(2|x|)
-// Sigmoid(-2|x|) = 4 E s with E = 2^t, t = -2|x| log2 e (t <= 0), s = 1/(1+E).
+// Sigmoid(-2|x|) = 4 E s^2 with E = 2^t, t = -2|x| log2 e (t <= 0),
+// s = 1/(1+E) = Sigmoid(2|x|) and Sigmoid(-2|x|) = E s.
 struct Tanh {
     static __device__ __forceinline__ Coef coef(float)
     {
@@ -214,9 +229,9 @@ struct Tanh {
         if (P) E *= corr(t, prod_lo(a, k.c_hi, k.c_lo, t));
         tail |= t < -120.f;
         float s = rcp_ftz(1.f + E);
-        return dy * ((4.f * E) * s);
+        return dy * (((4.f * E) * s) * s);
     }
-    // t < -120: s = 1, 4E = 2^(t + 2) may be subnormal; use 2^(t + 66) 2^-64.
+    // t < -120: s = 1, 4E s^2 = 2^(t + 2) may be subnormal; use 2^(t + 66) 2^-64.
     template <bool P>
     static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
     {

@@ -12,7 +12,11 @@ denominator taken from the terms where f' cancels near its zero.
 
 Both: results whose exact value is below the smallest normal, 2^-126, may be
 flushed; they pass when |g - r| <= floor (2^-126 unless a caller scales it,
-e.g. by |dy| for a backward product).
+e.g. by |dy| for a backward product).  A bf16 backward output whose ulp test
+fails also passes when it meets the fp32 rule against its condition scale:
+that happens only where f' nearly vanishes and its argument was formed in
+fp32 (the fused affine's z = gamma x + beta), so the exact result is smaller
+than the rounding of the fp32 intermediates allows to resolve.
 """
 from __future__ import annotations
 
@@ -43,7 +47,7 @@ def _ordered(bits: np.ndarray) -> np.ndarray:
     return np.where(b & 0x8000, -mag, mag)
 
 
-def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None) -> dict:
+def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None, scale=None) -> dict:
     g_bits = bf16_bits(gpu)
     ref = np.asarray(ref, dtype=np.float64).ravel()
     r_bits = oracle.round_bf16(ref)
@@ -53,12 +57,18 @@ def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None) -> dict:
     with np.errstate(invalid="ignore"):
         nan_ok = np.isnan(g) & np.isnan(ref)
         tiny_ok = (np.abs(ref) < TINY) & (np.abs(g - ref) <= fl)
-    ok = (dist <= 1) | nan_ok | tiny_ok
+        # Near the zero of f' (where the terms of f' cancel) the fp32
+        # arithmetic behind a bf16 output is held to the fp32 rule instead:
+        # |g - r| <= 1e-5 * condition scale.
+        cond_ok = np.zeros_like(nan_ok) if scale is None else \
+            np.abs(g - ref) <= F32_TOL * np.asarray(scale, dtype=np.float64).ravel()
+    ok = (dist <= 1) | nan_ok | tiny_ok | cond_ok
     bad = np.flatnonzero(~ok)
     return {
         "n": ref.size,
         "bad": bad.size,
         "max_ulp": int(dist[~(nan_ok | tiny_ok)].max(initial=0)),
+        "cond_only": int(np.sum(cond_ok & (dist > 1))),
         "exact_frac": float(np.mean(dist == 0)) if ref.size else 1.0,
         "first_bad": [(int(i), float(ref[i]), float(g[i]), int(dist[i])) for i in bad[:8]],
     }
@@ -89,8 +99,8 @@ def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F
     }
 
 
-def assert_bf16(gpu, ref, floor=None, what=""):
-    r = bf16_report(gpu, ref, floor)
+def assert_bf16(gpu, ref, floor=None, what="", scale=None):
+    r = bf16_report(gpu, ref, floor, scale)
     assert r["bad"] == 0, f"{what}: {r}"
     return r
 
@@ -101,7 +111,10 @@ def assert_f32(gpu, ref, scale=None, floor=None, what="", tol=F32_TOL):
     return r
 
 
-def check(dtype: str, gpu, ref, scale=None, floor=None, what=""):
+def check(dtype: str, gpu, ref, scale=None, floor=None, what="", bf16_cond=False):
+    """bf16 outputs use the condition-scale alternative only when bf16_cond is
+    set (outputs whose argument was formed in fp32, e.g. the fused affine);
+    activations applied to bf16 inputs are held to the plain 1-ulp rule."""
     if dtype == "bf16":
-        return assert_bf16(gpu, ref, floor, what)
+        return assert_bf16(gpu, ref, floor, what, scale if bf16_cond else None)
     return assert_f32(gpu, ref, scale, floor, what)

@@ -86,9 +86,12 @@ def test_f32_random(act):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("act", ACTS)
 def test_tails_and_extremes(act, dtype):
+    # (the largest finite value used is bf16's, so that it stays finite in
+    # both storage dtypes)
     parts = [np.linspace(-110.0, -80.0, 20001), np.linspace(-16.0, -8.0, 20001),
+             np.linspace(80.0, 110.0, 20001),
              np.linspace(40.0, 46.0, 2001), -np.linspace(40.0, 46.0, 2001),
-             np.array([3.4028234663852886e38, -3.4028234663852886e38, 1e30, -1e30, 1e10, -1e10,
+             np.array([3.3895313892515355e38, -3.3895313892515355e38, 1e30, -1e30, 1e10, -1e10,
                        1.1754943508222875e-38, -1.1754943508222875e-38, 1e-40, -1e-40, 0.0, -0.0])]
     x = synthetic.to_storage(np.concatenate(parts), dtype)
     dy = synthetic.to_storage(np.resize(np.array([1.0, -0.75, 3.5, -2.0]), x.numel()), dtype)

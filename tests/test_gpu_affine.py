@@ -58,7 +58,8 @@ def test_affine_small_shapes(dtype, layout, shape):
     rdx, rdg, rdb, scale = oracle.affine_swish_bwd(layout, nchw, xd, gd, g.double().numpy(),
                                                    b.double().numpy(), with_scale=True)
     check(dtype, y.cpu(), ry, what="affine fwd")
-    check(dtype, dx.cpu(), rdx, scale=scale, floor=TINY * np.maximum(1, np.abs(gd)), what="affine dx")
+    check(dtype, dx.cpu(), rdx, scale=scale, floor=TINY * np.maximum(1, np.abs(gd)), what="affine dx",
+          bf16_cond=True)
     # channel sums: fp32 results within 1e-5 relative, with an absolute
     # allowance of 1e-7 of the sum of |terms| for channels that cancel
     N, C, H, W = nchw
@@ -81,7 +82,7 @@ def test_affine_nhwc_full_workload():
     nchw = w.extra["nchw_shape"]
     xd, gd = to_f64(w.x), to_f64(w.dy)
     gg, bb = w.extra["gamma"].double().numpy(), w.extra["beta"].double().numpy()
-    rdx, rdg, rdb = oracle.affine_swish_bwd("nhwc", nchw, xd, gd, gg, bb)
+    rdx, rdg, rdb, scale = oracle.affine_swish_bwd("nhwc", nchw, xd, gd, gg, bb, with_scale=True)
     # 1e-5 relative per channel, plus 1e-8 of the channel's sum of |terms|
     # for a channel whose 401,408 terms happen to cancel to a small total.
     C = nchw[1]
@@ -98,7 +99,8 @@ def test_affine_nhwc_full_workload():
     idx_t = torch.from_numpy(idx).cuda()
     ry = oracle.affine_swish_fwd("nhwc", nchw, xd, gg, bb)
     check("bf16", y.view(-1)[idx_t].cpu(), ry[idx], what="nhwc fwd sampled")
-    check("bf16", dx.view(-1)[idx_t].cpu(), rdx[idx], what="nhwc dx sampled")
+    check("bf16", dx.view(-1)[idx_t].cpu(), rdx[idx], scale=scale[idx], what="nhwc dx sampled",
+          bf16_cond=True)
 
 
 def test_affine_deterministic_and_counter_reset():
@@ -140,8 +142,8 @@ def test_affine_module_autograd():
     y.backward(dy.cuda())
     torch.cuda.synchronize()
     xd, gd = to_f64(x), to_f64(dy)
-    rdx, rdg, rdb = oracle.affine_swish_bwd("nhwc", (4, 144, 8, 8), xd, gd, g.double().numpy(),
-                                            b.double().numpy())
-    check("bf16", xc.grad.cpu(), rdx, what="module dx")
+    rdx, rdg, rdb, scale = oracle.affine_swish_bwd("nhwc", (4, 144, 8, 8), xd, gd, g.double().numpy(),
+                                                   b.double().numpy(), with_scale=True)
+    check("bf16", xc.grad.cpu(), rdx, scale=scale, what="module dx", bf16_cond=True)
     assert np.allclose(m.gamma.grad.cpu().double().numpy(), rdg, rtol=1e-5, atol=1e-6)
     assert np.allclose(m.beta.grad.cpu().double().numpy(), rdb, rtol=1e-5, atol=1e-6)
