@@ -188,6 +188,34 @@ MEA_API mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout
                                   float *dgamma, float *dbeta, void *workspace,
                                   size_t ws_bytes, mea_stream_t stream);
 
+/* Backward with d alpha that allocates nothing and takes no workspace.
+ * No counterpart on the pages: this is a library convenience, not part of
+ * the method.  It computes exactly what mea_act_bwd computes (same kernel,
+ * same fixed reduction order, bitwise the same dx and d alpha) for callers
+ * that cannot allocate device memory for the reduction scratch -- code whose
+ * device memory is handed out entirely by another allocator (a framework's
+ * caching allocator or a fixed memory plan), and latency-sensitive paths
+ * that cannot accept the synchronisation cudaFree (and possibly cudaMalloc)
+ * brings.  The scratch is a fixed 9,728-byte array in the library's device
+ * code, present on every GPU that loads the library until the process exits.
+ *   Arguments as for mea_act_bwd, without workspace / ws_bytes.  With
+ *   dparam_dev NULL it is a plain backward (no scratch is used).
+ *   Every element count is served (the reduction grid is capped so that its
+ *   scratch fits the array); a request needing more scratch than the array
+ *   holds would be refused with MEA_ERR_WORKSPACE.
+ *   The first call on a device (with that device current) looks up the
+ *   array's device address with cudaGetSymbolAddress; make that first call
+ *   before any stream capture.  Every call clears the array's completion
+ *   counter with cudaMemsetAsync on `stream` and then launches the kernel;
+ *   it calls no cudaMalloc, cudaFree or other allocating routine.
+ *   All calls on a device share the one array: calls whose kernels may run
+ *   at the same time on the GPU (unordered streams) race and must not be
+ *   issued; calls ordered on one stream are safe. */
+MEA_API mea_status_t mea_act_bwd_dparam_noalloc(mea_act_t act, mea_dtype_t dtype, const void *x,
+                                                const void *dy, void *dx, int64_t n, float param,
+                                                const float *param_dev, float *dparam_dev,
+                                                mea_stream_t stream);
+
 /* Static description of a status code. */
 MEA_API const char *mea_status_string(mea_status_t status);
 

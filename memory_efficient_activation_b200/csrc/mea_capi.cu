@@ -66,6 +66,10 @@ mea_status_t check_shape(const int64_t *shape, int64_t *n)
 
 }  // namespace
 
+namespace mea {
+void set_last_error_detail(const char *detail) { snprintf(g_err, sizeof(g_err), "%s", detail); }
+}  // namespace mea
+
 extern "C" {
 
 const char *mea_status_string(mea_status_t status)

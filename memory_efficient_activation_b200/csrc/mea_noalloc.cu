@@ -1,0 +1,107 @@
+// mea_noalloc.cu -- the Swish backward with d alpha, with its reduction
+// scratch taken from a fixed array in the library instead of a caller buffer.
+//
+// Who needs it: callers that cannot call cudaMalloc / cudaFree for the small
+// reduction workspace.  Examples are code whose device memory is handed out
+// entirely by another allocator (a framework's caching allocator or a fixed
+// memory plan that must not be bypassed), and latency-sensitive paths that
+// cannot accept the device-wide synchronisation cudaFree implies (and that
+// cudaMalloc may imply).  This entry point allocates nothing: the scratch is
+// a file-scope __device__ array of kNoAllocScratchBytes bytes, created when
+// the library's device code is loaded on a GPU and held until the process
+// exits.
+//
+// Host code cannot use the array's name as a device address (on the host it
+// names a host-side stand-in), so the device address is looked up with
+// cudaGetSymbolAddress once per device, with that device current, on the
+// first call made while it is current; that first call should come before
+// any stream capture.  The array is shared by every call on a device and
+// keeps whatever the last call left in it; the completion counter at its
+// start is cleared (cudaMemsetAsync on the caller's stream) before every
+// launch.  Calls whose kernels overlap on the GPU (different streams, no
+// ordering between them) race on the array and must not be issued.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/mea.h"
+#include "mea_internal.h"
+
+// Header (completion counter) plus one fp64 partial per block of the
+// largest reduction grid: enough for every element count (9,728 bytes).
+static constexpr size_t kNoAllocScratchBytes = mea::kWsHeader + sizeof(double) * mea::kRedGridMax;
+
+static __device__ __align__(256) unsigned char g_dalpha_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch on the current device (looked up once).
+cudaError_t scratch_for_current_device(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_dalpha_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+namespace mea {
+// Records the detail string mea_last_error returns (defined with the rest of
+// the C ABI in mea_capi.cu).
+void set_last_error_detail(const char *detail);
+}  // namespace mea
+
+extern "C" mea_status_t mea_act_bwd_dparam_noalloc(mea_act_t act, mea_dtype_t dtype, const void *x,
+                                                   const void *dy, void *dx, int64_t n, float param,
+                                                   const float *param_dev, float *dparam_dev,
+                                                   mea_stream_t stream)
+{
+    // Without d alpha there is no reduction and no scratch: a plain backward.
+    if (!dparam_dev)
+        return mea_act_bwd(act, dtype, x, dy, dx, n, param, param_dev, nullptr, nullptr, 0, stream);
+    void *scratch = nullptr;
+    cudaError_t e = scratch_for_current_device(&scratch);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "looking up the fixed d alpha scratch: %s (%s)", cudaGetErrorName(e),
+                 cudaGetErrorString(e));
+        mea::set_last_error_detail(msg);
+        return MEA_ERR_CUDA;
+    }
+    // A negative n, an activation without a parameter gradient, or a
+    // reduction needing more scratch than the fixed array holds (not
+    // reachable with the capped grid) is refused by the regular entry point,
+    // which reports the scratch's real size, before anything is queued.  Any
+    // other invalid argument is refused by it after the counter clear below,
+    // which is harmless (it only touches the library's own array).
+    if (n < 0 || act != MEA_SWISH || mea_act_bwd_workspace_bytes(act, n, 1) > kNoAllocScratchBytes)
+        return mea_act_bwd(act, dtype, x, dy, dx, n, param, param_dev, dparam_dev, scratch,
+                           kNoAllocScratchBytes, stream);
+    // The completion counter must start at zero.
+    e = cudaMemsetAsync(scratch, 0, mea::kWsHeader, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "clearing the fixed d alpha scratch: %s (%s)", cudaGetErrorName(e),
+                 cudaGetErrorString(e));
+        mea::set_last_error_detail(msg);
+        return MEA_ERR_CUDA;
+    }
+    return mea_act_bwd(act, dtype, x, dy, dx, n, param, param_dev, dparam_dev, scratch, kNoAllocScratchBytes,
+                       stream);
+}
