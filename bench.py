@@ -72,10 +72,8 @@ def _barrier(ws):
 def _max_over_ranks(v: float, ws: int) -> float:
     if ws <= 1:
         return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from memory_efficient_activation_b200 import dist as mdist
+    return mdist.max_over_ranks(v, device="cuda")
 
 
 def _peaks():
@@ -422,6 +420,111 @@ def run_reference(args, rank, ws):
     }
 
 
+# --------------------------------------- secondary workloads (not the headline)
+
+def _time_ops(ops, steps, warmup, stream):
+    """ops: list of (name, fn, algorithmic_bytes).  Runs warmup then `steps`
+    rounds of all ops in order, with CUDA events around every op on the
+    launching stream; returns {name: mean ms} and the total elapsed ms."""
+    for _ in range(warmup):
+        for _, fn, _ in ops:
+            fn()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record(stream)
+        for j, (_, fn, _) in enumerate(ops):
+            fn()
+            ev[k][j + 1].record(stream)
+    torch.cuda.synchronize()
+    per = {name: statistics.mean(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(steps))
+           for j, (name, _, _) in enumerate(ops)}
+    total = sum(ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps))
+    return per, total
+
+
+def run_secondary(args):
+    """Per-kernel GB/s and roofline fractions for the other configurations
+    (activation family, EfficientNet-like fp32 maps with d alpha, fused
+    affine + Swish NHWC, the L2-resident 1M fp32 case).  Diagnostics: the
+    headline line is the default run."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = _peaks()
+    ops = []
+    keep = []
+    wl = args.workload
+    if wl == "family_bf16":
+        w = synthetic.family_bf16("swish")
+        x, dy = w.x.to(dev), w.dy.to(dev)
+        y, dx = torch.empty_like(x), torch.empty_like(x)
+        keep += [x, dy, y, dx]
+        n = w.n
+        for act in synthetic.ACTIVATIONS:
+            p = 0.01 if act == "leaky_relu" else 1.0
+            ops.append((f"{act}_fwd", lambda a=act, p=p: mea.act_fwd(a, x, p, out=y), accounting.fwd_bytes(n, "bf16")))
+            ops.append((f"{act}_bwd", lambda a=act, p=p: mea.act_bwd(a, x, dy, p, out=dx),
+                        accounting.bwd_bytes(n, "bf16")))
+    elif wl == "effnet_f32_dalpha":
+        for i in range(len(synthetic.EFFNET_B0_SHAPES)):
+            w = synthetic.effnet_swish_f32(i)
+            x, dy = w.x.to(dev), w.dy.to(dev)
+            y, dx = torch.empty_like(x), torch.empty_like(x)
+            a = torch.tensor([w.param], dtype=torch.float32, device=dev)
+            d = torch.empty(1, dtype=torch.float32, device=dev)
+            keep += [x, dy, y, dx, a, d]
+            tag = "x".join(map(str, w.x.shape))
+            ops.append((f"{tag}_fwd", lambda x=x, y=y, a=a: mea.act_fwd("swish", x, 0.0, param_dev=a, out=y),
+                        accounting.fwd_bytes(w.n, "f32")))
+            ops.append((f"{tag}_bwd_dalpha",
+                        lambda x=x, dy=dy, dx=dx, a=a, d=d: mea.act_bwd("swish", x, dy, 0.0, param_dev=a, dparam=d,
+                                                                        out=dx),
+                        accounting.bwd_bytes(w.n, "f32")))
+    elif wl == "affine_nhwc_bf16":
+        w = synthetic.affine_swish_nhwc()
+        x, dy = w.x.to(dev), w.dy.to(dev)
+        g, b = w.extra["gamma"].to(dev), w.extra["beta"].to(dev)
+        y, dx = torch.empty_like(x), torch.empty_like(x)
+        C = g.numel()
+        dg = torch.empty(C, device=dev)
+        db = torch.empty(C, device=dev)
+        keep += [x, dy, g, b, y, dx, dg, db]
+        ops.append(("affine_fwd", lambda: mea.affine_swish_fwd(x, g, b, "nhwc", out=y),
+                    accounting.affine_fwd_bytes(w.n, "bf16", C)))
+        ops.append(("affine_bwd", lambda: mea.affine_swish_bwd(x, dy, g, b, "nhwc", out=dx, dgamma=dg, dbeta=db),
+                    accounting.affine_bwd_bytes(w.n, "bf16", C)))
+    elif wl == "swish_f32_1m":
+        w = synthetic.swish_f32_1m()
+        x, dy = w.x.to(dev), w.dy.to(dev)
+        y, dx = torch.empty_like(x), torch.empty_like(x)
+        keep += [x, dy, y, dx]
+        ops.append(("fwd", lambda: mea.act_fwd("swish", x, out=y), accounting.fwd_bytes(w.n, "f32")))
+        ops.append(("bwd", lambda: mea.act_bwd("swish", x, dy, out=dx), accounting.bwd_bytes(w.n, "f32")))
+    else:
+        raise SystemExit(f"unknown workload {wl}")
+    with _ClockSampler(0) as clk:
+        per, total = _time_ops(ops, args.steps, args.warmup, stream)
+    tot_bytes = sum(b for _, _, b in ops)
+    out = {
+        "workload": wl,
+        "value": round(tot_bytes * args.steps / (total * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "peak": peak,
+        "peak_kind": peak_kind,
+        "ops": {name: {"ms": round(per[name], 5), "GB/s": round(b / (per[name] * 1e-3) / 1e9, 1),
+                       "frac": round(b / (per[name] * 1e-3) / 1e9 / peak, 4), "bytes": b}
+                for name, _, b in ops},
+        "clocks": clk.summary(),
+    }
+    if wl == "swish_f32_1m":
+        out["note"] = "21 MB of traffic per step fits in the 126 MB L2: an L2-resident figure, not HBM bandwidth"
+    del keep
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,6 +535,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="swish_bf16",
+                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16", "swish_f32_1m"],
+                    help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -442,6 +548,10 @@ def main(argv=None):
         out = run_reference(args, rank, ws)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return 0
+
+    if args.workload != "swish_bf16":
+        print(json.dumps(run_secondary(args)), flush=True)
         return 0
 
     rank, ws, local = _dist()

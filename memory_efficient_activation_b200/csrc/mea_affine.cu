@@ -9,16 +9,14 @@
 // section "What makes this implementation save GPU memory?", applied to the
 // affine + Swish pair that EfficientNet-style blocks run back to back).
 //
-// NHWC fast path (C a multiple of the 16-byte vector width, aligned
-// pointers): a block has a multiple of G = C / V threads, so the grid-stride
-// step is a multiple of G and every thread keeps the same V channels for the
-// whole loop.  Its gamma / beta live in registers and its dgamma / dbeta
-// partial sums in fp64 registers (fp32 inside one unrolled step).  The block
-// folds its threads' sums per channel through shared memory in a fixed
-// order and writes one fp64 partial per channel; the last block to finish
-// (atomic ticket, no waiting) adds the per-block partials in block order.
-// The backward grid is fixed by the shape, so the result is bitwise
-// reproducible on any device.
+// NHWC fast path (C a multiple of 4, aligned pointers): a block is a
+// multiple of G = C / 4 threads, so every thread keeps the same 4 channels,
+// with gamma / beta in registers.  The forward handles one tile per block.
+// The backward runs a fixed grid (a function of the shape) that walks the
+// tiles with register prefetch, keeps fp64 per-channel sums per thread,
+// folds them per block in row order and writes one row of fp64 partials per
+// block; a second kernel adds each channel's column in block order.  So
+// dgamma / dbeta are bitwise reproducible on any device.
 //
 // Plane path (NCHW, and NHWC shapes the fast path does not take): block
 // (c, s) owns channel c and the s-th slice of the batch; for NCHW it streams
@@ -33,22 +31,25 @@
 namespace mea {
 
 constexpr int kAffUnroll = 4;
-constexpr int kNhwcMaxThreads = 640;
-constexpr int kAffGridMax = 148;         // NHWC backward blocks (fixed, not device-derived)
+constexpr int kNhwcMaxThreads = 512;
+constexpr int kNhwcTargetThreads = 256;
+constexpr int kColsumThreads = 256;
+constexpr int kNhwcBwdGridCap = 888;     // 148 x 6
 constexpr int kPlaneThreads = 256;
 constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks
 
-// Threads per NHWC block: lcm(G, 32) times the largest m that keeps it within
-// kNhwcMaxThreads, where G = C / V is the number of channel groups.  Returns
-// 0 when lcm(G, 32) itself is too large (the NHWC fast path is then not
-// taken), so a block is always whole warps and a multiple of G.
+// Threads per NHWC block: lcm(G, 32) times the largest m that keeps it at
+// or below kNhwcTargetThreads (at least one lcm), where G = C / V is the
+// number of channel groups.  A block is then whole warps and a multiple of
+// G, so every thread of a block keeps the same V channels.  Returns 0 when
+// lcm(G, 32) exceeds kNhwcMaxThreads (the NHWC fast path is then not taken).
 static int nhwc_threads(int groups)
 {
     int a = groups, b = 32;
     while (b) { int t = a % b; a = b; b = t; }
     const long lcm = (long)groups / a * 32;
     if (lcm > kNhwcMaxThreads) return 0;
-    long m = kNhwcMaxThreads / lcm;
+    long m = kNhwcTargetThreads / lcm;
     if (m < 1) m = 1;
     return (int)(lcm * m);
 }
@@ -63,121 +64,229 @@ static int plane_slices(int64_t N, int64_t C)
 
 // ------------------------------------------------------------ NHWC fast
 
-template <typename T, int MODE>
+// Load units of the NHWC kernels: VE elements per thread per access (bf16:
+// 4 elements in 8 bytes or 8 in 16; fp32: 4 in 16 bytes).  Fewer channels
+// per thread keep the per-thread gamma / beta / partial-sum registers small,
+// which is what sets the occupancy of these kernels.
+template <typename T, int VE>
+struct Unit;
+
+template <>
+struct Unit<Bf16, 8> {
+    using W = uint4;
+    static constexpr bool P = false;
+    static __device__ __forceinline__ W load(const void *p, int64_t i) { return ld_nc_v4(static_cast<const uint4 *>(p) + i); }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const W &w) { st_v4(static_cast<uint4 *>(p) + i, w); }
+    static __device__ __forceinline__ void unpack(const W &w, float (&f)[8]) { Store<Bf16>::unpack(w, f); }
+    static __device__ __forceinline__ W pack(const float (&f)[8]) { return Store<Bf16>::pack(f); }
+};
+
+template <>
+struct Unit<Bf16, 4> {
+    using W = uint2;
+    static constexpr bool P = false;
+    static __device__ __forceinline__ W load(const void *p, int64_t i)
+    {
+        W r;
+        asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y)
+            : "l"(static_cast<const uint2 *>(p) + i));
+        return r;
+    }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const W &w)
+    {
+        asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(static_cast<uint2 *>(p) + i), "r"(w.x), "r"(w.y)
+                     : "memory");
+    }
+    static __device__ __forceinline__ void unpack(const W &w, float (&f)[4])
+    {
+        f[0] = __uint_as_float(w.x << 16);
+        f[1] = __uint_as_float(w.x & 0xffff0000u);
+        f[2] = __uint_as_float(w.y << 16);
+        f[3] = __uint_as_float(w.y & 0xffff0000u);
+    }
+    static __device__ __forceinline__ W pack(const float (&f)[4])
+    {
+        return make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+    }
+};
+
+template <>
+struct Unit<float, 4> {
+    using W = uint4;
+    static constexpr bool P = true;
+    static __device__ __forceinline__ W load(const void *p, int64_t i) { return ld_nc_v4(static_cast<const uint4 *>(p) + i); }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const W &w) { st_v4(static_cast<uint4 *>(p) + i, w); }
+    static __device__ __forceinline__ void unpack(const W &w, float (&f)[4]) { Store<float>::unpack(w, f); }
+    static __device__ __forceinline__ W pack(const float (&f)[4]) { return Store<float>::pack(f); }
+};
+
+// Forward: one tile of blockDim.x * U units per block (as the plain
+// activation kernels), y = z Sigmoid(z), z = gamma_c x + beta_c.
+template <typename T, int U, int VE>
 __global__ void __launch_bounds__(kNhwcMaxThreads)
-affine_nhwc_kernel(const void *__restrict__ x, const void *__restrict__ dy, const float *__restrict__ gamma,
-                   const float *__restrict__ beta, void *__restrict__ out, int64_t nvec, int groups, int C,
-                   float *__restrict__ dgamma, float *__restrict__ dbeta, void *__restrict__ ws)
+affine_nhwc_fwd_kernel(const void *__restrict__ x, const float *__restrict__ gamma, const float *__restrict__ beta,
+                       void *__restrict__ out, int64_t nunits, int groups)
 {
-    using S = Store<T>;
-    constexpr int V = S::V;
-    constexpr bool P = S::P;
+    using L = Unit<T, VE>;
+    constexpr bool P = L::P;
     const int tid = threadIdx.x;
     const int g = tid % groups;
     const Coef k = Swish::coef(1.f);
-    float ga[V], be[V];
+    float ga[VE], be[VE];
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-        ga[j] = __ldg(gamma + g * V + j);
-        be[j] = __ldg(beta + g * V + j);
+    for (int j = 0; j < VE; ++j) {
+        ga[j] = __ldg(gamma + g * VE + j);
+        be[j] = __ldg(beta + g * VE + j);
     }
-    // MODE 1: this thread's fp64 dgamma / dbeta sums live in shared memory,
-    // acc[(kind * V + j) * blockDim.x + tid], which frees 2 V fp64 registers.
-    extern __shared__ double acc[];
-    if constexpr (MODE == 1) {
+    const int64_t base = (int64_t)blockIdx.x * blockDim.x * U + tid;
+    typename L::W xv[U];
 #pragma unroll
-        for (int j = 0; j < 2 * V; ++j) acc[j * blockDim.x + tid] = 0.0;
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) xv[u] = L::load(x, i);
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) {
+            float xf[VE], of[VE];
+            L::unpack(xv[u], xf);
+            bool tail = false;
+#pragma unroll
+            for (int j = 0; j < VE; ++j) of[j] = Swish::f<P>(fmaf(ga[j], xf[j], be[j]), k, tail);
+            if (tail) {
+#pragma unroll
+                for (int j = 0; j < VE; ++j) {
+                    const float z = fmaf(ga[j], xf[j], be[j]);
+                    if (Swish::is_tail(z, k)) of[j] = Swish::f_tail<P>(z, k);
+                }
+            }
+            L::store(out, i, L::pack(of));
+        }
+    }
+}
 
-    const int64_t step = (int64_t)blockDim.x * kAffUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * step + tid; base < nvec; base += (int64_t)gridDim.x * step) {
-        uint4 xv[kAffUnroll], gv[kAffUnroll];
+// Backward: a fixed grid of blocks (a function of the shape only) walks the
+// tiles of blockDim.x * U units with a grid stride, loading the next tile's
+// x and dy before working on the current one.  Each thread keeps the same VE
+// channels throughout; its dz x and dz sums go from fp32 per tile into fp64
+// registers.  At the end the block folds its threads' sums per channel in
+// row order (fp64, through shared memory) and writes one row of partials:
+//   partials[blockIdx.x * 2C + kind * C + c],  kind 0 = dgamma, 1 = dbeta.
+template <typename T, int U, int VE>
+__global__ void __launch_bounds__(kNhwcMaxThreads)
+affine_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, const float *__restrict__ gamma,
+                       const float *__restrict__ beta, void *__restrict__ dx, int64_t nunits, int groups, int C,
+                       double *__restrict__ partials)
+{
+    using L = Unit<T, VE>;
+    constexpr bool P = L::P;
+    const int tid = threadIdx.x;
+    const int g = tid % groups;
+    const Coef k = Swish::coef(1.f);
+    float ga[VE], be[VE];
 #pragma unroll
-        for (int u = 0; u < kAffUnroll; ++u) {
-            const int64_t i = base + (int64_t)u * blockDim.x;
-            if (i < nvec) {
-                xv[u] = ld_nc_v4(static_cast<const uint4 *>(x) + i);
-                if constexpr (MODE == 1) gv[u] = ld_nc_v4(static_cast<const uint4 *>(dy) + i);
+    for (int j = 0; j < VE; ++j) {
+        ga[j] = __ldg(gamma + g * VE + j);
+        be[j] = __ldg(beta + g * VE + j);
+    }
+    double ag[VE], ab[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) ag[j] = ab[j] = 0.0;
+    const int64_t tile = (int64_t)blockDim.x * U;
+    const int64_t stride = (int64_t)gridDim.x * tile;
+    int64_t base = (int64_t)blockIdx.x * tile + tid;
+    typename L::W xv[U], gv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) {
+            xv[u] = L::load(x, i);
+            gv[u] = L::load(dy, i);
+        }
+    }
+    for (; base < nunits; base += stride) {
+        typename L::W xn[U], gn[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + stride + (int64_t)u * blockDim.x;
+            if (i < nunits) {
+                xn[u] = L::load(x, i);
+                gn[u] = L::load(dy, i);
             }
         }
-        float sg[V], sb[V];
+        float sg[VE], sb[VE];
 #pragma unroll
-        for (int j = 0; j < V; ++j) sg[j] = sb[j] = 0.f;
+        for (int j = 0; j < VE; ++j) sg[j] = sb[j] = 0.f;
 #pragma unroll
-        for (int u = 0; u < kAffUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t i = base + (int64_t)u * blockDim.x;
-            if (i < nvec) {
-                float xf[V], gf[V], zf[V], of[V];
-                S::unpack(xv[u], xf);
-                if constexpr (MODE == 1) S::unpack(gv[u], gf);
+            if (i < nunits) {
+                float xf[VE], gf[VE], of[VE];
+                L::unpack(xv[u], xf);
+                L::unpack(gv[u], gf);
                 bool tail = false;
 #pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    zf[j] = fmaf(ga[j], xf[j], be[j]);
-                    if constexpr (MODE == 0)
-                        of[j] = Swish::f<P>(zf[j], k, tail);
-                    else
-                        of[j] = Swish::df<P>(zf[j], gf[j], k, tail);   // dz
-                }
+                for (int j = 0; j < VE; ++j) of[j] = Swish::df<P>(fmaf(ga[j], xf[j], be[j]), gf[j], k, tail);
                 if (tail) {
 #pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        if (Swish::is_tail(zf[j], k)) {
-                            if constexpr (MODE == 0)
-                                of[j] = Swish::f_tail<P>(zf[j], k);
-                            else
-                                of[j] = Swish::df_tail<P>(zf[j], gf[j], k);
-                        }
+                    for (int j = 0; j < VE; ++j) {
+                        const float z = fmaf(ga[j], xf[j], be[j]);
+                        if (Swish::is_tail(z, k)) of[j] = Swish::df_tail<P>(z, gf[j], k);
                     }
                 }
-                if constexpr (MODE == 1) {
 #pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        sg[j] = fmaf(of[j], xf[j], sg[j]);
-                        sb[j] += of[j];
-                        of[j] = ga[j] * of[j];
-                    }
+                for (int j = 0; j < VE; ++j) {
+                    sg[j] = fmaf(of[j], xf[j], sg[j]);   // dz x
+                    sb[j] += of[j];                      // dz
+                    of[j] = ga[j] * of[j];               // dx
                 }
-                st_v4(static_cast<uint4 *>(out) + i, S::pack(of));
+                L::store(dx, i, L::pack(of));
             }
         }
-        if constexpr (MODE == 1) {
 #pragma unroll
-            for (int j = 0; j < V; ++j) {
-                acc[j * blockDim.x + tid] += (double)sg[j];
-                acc[(V + j) * blockDim.x + tid] += (double)sb[j];
-            }
+        for (int j = 0; j < VE; ++j) {
+            ag[j] += (double)sg[j];
+            ab[j] += (double)sb[j];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            xv[u] = xn[u];
+            gv[u] = gn[u];
         }
     }
-    if constexpr (MODE == 0) return;
-
-    // Fold the rows of threads that share a channel group, in row order.
-    unsigned int *ticket = static_cast<unsigned int *>(ws);
-    double *partials = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
-    const int rows = blockDim.x / groups;
+    extern __shared__ double red[];   // 2 VE * blockDim.x doubles
+#pragma unroll
+    for (int j = 0; j < VE; ++j) {
+        red[j * blockDim.x + tid] = ag[j];
+        red[(VE + j) * blockDim.x + tid] = ab[j];
+    }
     __syncthreads();
+    const int rows = blockDim.x / groups;
     for (int o = tid; o < 2 * C; o += blockDim.x) {
         const int kind = o / C, c = o % C;
-        const int cg = c / V, cj = c % V;
-        const double *col = acc + (kind * V + cj) * blockDim.x + cg;
+        const double *col = red + (kind * VE + c % VE) * blockDim.x + c / VE;
         double s = 0.0;
         for (int r = 0; r < rows; ++r) s += col[r * groups];
-        partials[(int64_t)o * gridDim.x + blockIdx.x] = s;
+        partials[(int64_t)blockIdx.x * 2 * C + o] = s;
     }
-    if (!last_block_done(ticket)) return;
+}
 
-    // Last block: output o (kind * C + c) is the sum over blocks in order;
-    // one warp per output, lanes take blocks lane, lane + 32, ... and meet in
-    // a fixed butterfly.
-    const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    for (int o = warp; o < 2 * C; o += nwarps) {
-        double s = 0.0;
-        for (int b = lane; b < (int)gridDim.x; b += 32) s += __ldcg(partials + (int64_t)o * gridDim.x + b);
-        s = warp_sum(s);
-        if (lane == 0) {
-            if (o < C) dgamma[o] = (float)s;
-            else dbeta[o - C] = (float)s;
-        }
+// Output o (kind * C + c) = sum over the nb rows of partials, column o, in
+// fp64: thread t adds rows t, t + kColsumThreads, ... in order, then a fixed
+// block-wide tree.  One block per output.
+__global__ void __launch_bounds__(kColsumThreads)
+affine_colsum_kernel(const double *__restrict__ partials, int nb, int C, float *__restrict__ dgamma,
+                     float *__restrict__ dbeta)
+{
+    __shared__ double red[32];
+    const int o = blockIdx.x;
+    double s = 0.0;
+    for (int b = threadIdx.x; b < nb; b += kColsumThreads) s += partials[(int64_t)b * 2 * C + o];
+    s = block_sum(s, red);
+    if (threadIdx.x == 0) {
+        if (o < C) dgamma[o] = (float)s;
+        else dbeta[o - C] = (float)s;
     }
 }
 
@@ -263,25 +372,44 @@ affine_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, con
 
 // ------------------------------------------------------------ launchers
 
+// NHWC launch shape per storage dtype: elements per thread access (VE) and
+// accesses per thread (U) for the forward and the backward (measured on B200
+// at [128, 56, 56, 144] bf16 against 8 / 16-byte units, 1-16 accesses,
+// tile-per-block and fixed-grid backward variants).
+template <typename T>
+struct NhwcCfg;
+template <>
+struct NhwcCfg<Bf16> {
+    static constexpr int VE = 4, U_FWD = 16, U_BWD = 2;
+};
+template <>
+struct NhwcCfg<float> {
+    static constexpr int VE = 4, U_FWD = 8, U_BWD = 2;
+};
+
 template <typename T>
 static bool nhwc_fast(const AffineLaunch &a)
 {
-    constexpr int V = Store<T>::V;
+    constexpr int VE = NhwcCfg<T>::VE;
+    constexpr int bytes = VE * (sizeof(T) == 4 ? 4 : 2);
     uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
     if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
-    return a.layout == 1 && a.C % V == 0 && (a.C / V) <= 1024 && nhwc_threads((int)(a.C / V)) > 0 &&
-           (al & 15u) == 0;
+    return a.layout == 1 && a.C % VE == 0 && nhwc_threads((int)(a.C / VE)) > 0 && (al % bytes) == 0;
 }
 
-template <typename T>
-static int nhwc_bwd_grid(const AffineLaunch &a, int threads)
+static int64_t nhwc_blocks(int64_t nunits, int threads, int U)
 {
-    constexpr int V = Store<T>::V;
-    const int64_t nvec = a.N * a.C * a.H * a.W / V;
-    int64_t g = (nvec + (int64_t)threads * kAffUnroll - 1) / ((int64_t)threads * kAffUnroll);
-    if (g > kAffGridMax) g = kAffGridMax;
-    if (g < 1) g = 1;
-    return (int)g;
+    const int64_t per = (int64_t)threads * U;
+    const int64_t nb = (nunits + per - 1) / per;
+    return nb < 1 ? 1 : nb;
+}
+
+// Backward grid: one block per tile up to kNhwcBwdGridCap blocks (a function
+// of the shape only, so the summation order is fixed).
+static int nhwc_bwd_grid(int64_t nunits, int threads, int U)
+{
+    const int64_t nb = nhwc_blocks(nunits, threads, U);
+    return (int)(nb < kNhwcBwdGridCap ? nb : kNhwcBwdGridCap);
 }
 
 template <typename T, int MODE>
@@ -291,28 +419,34 @@ static cudaError_t launch_affine(const AffineLaunch &a)
     const int64_t HW = a.H * a.W;
     const int64_t n = a.N * a.C * HW;
     if (nhwc_fast<T>(a)) {
-        const int groups = (int)(a.C / V);
+        constexpr int VE = NhwcCfg<T>::VE;
+        const int groups = (int)(a.C / VE);
         const int threads = nhwc_threads(groups);
-        auto kernel = affine_nhwc_kernel<T, MODE>;
-        const int64_t nvec = n / V;
-        int grid;
-        size_t smem = 0;
-        if (MODE == 1) {
-            grid = nhwc_bwd_grid<T>(a, threads);
-            smem = sizeof(double) * 2 * V * threads;
-            if (smem > 48 * 1024) {
-                cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-                if (e != cudaSuccess) return e;
-            }
-        } else {
-            int b = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, 0) != cudaSuccess || b < 1) b = 1;
-            int64_t units = (nvec + (int64_t)threads * kAffUnroll - 1) / ((int64_t)threads * kAffUnroll);
-            int64_t cap = (int64_t)sm_count() * b;
-            grid = (int)(units < cap ? (units < 1 ? 1 : units) : cap);
+        const int64_t nunits = n / VE;
+        if (MODE == 0) {
+            constexpr int U = NhwcCfg<T>::U_FWD;
+            const int64_t nb = nhwc_blocks(nunits, threads, U);
+            if (nb > 0x7fffffff) return cudaErrorInvalidConfiguration;
+            affine_nhwc_fwd_kernel<T, U, VE><<<(unsigned)nb, threads, 0, a.stream>>>(a.x, a.gamma, a.beta, a.out,
+                                                                                      nunits, groups);
+            return cudaGetLastError();
         }
-        kernel<<<grid, threads, smem, a.stream>>>(a.x, a.dy, a.gamma, a.beta, a.out, nvec, groups, (int)a.C,
-                                                  a.dgamma, a.dbeta, a.workspace);
+        constexpr int U = NhwcCfg<T>::U_BWD;
+        auto kernel = affine_nhwc_bwd_kernel<T, U, VE>;
+        const int nb = nhwc_bwd_grid(nunits, threads, U);
+        double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+        const size_t smem = sizeof(double) * 2 * VE * threads;
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             (int)cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess && smem > 48 * 1024)
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kernel<<<(unsigned)nb, threads, smem, a.stream>>>(a.x, a.dy, a.gamma, a.beta, a.out, nunits, groups,
+                                                          (int)a.C, partials);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        affine_colsum_kernel<<<(unsigned)(2 * a.C), kColsumThreads, 0, a.stream>>>(partials, nb, (int)a.C, a.dgamma,
+                                                                                  a.dbeta);
         return cudaGetLastError();
     }
     uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
@@ -334,15 +468,13 @@ size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, i
 {
     // Mirrors the launch decision; pointer alignment is not known here, so
     // the larger of the two layouts' needs is returned for NHWC.
-    const int V = dtype == kBF16 ? 8 : 4;
+    const int VE = dtype == kBF16 ? NhwcCfg<Bf16>::VE : NhwcCfg<float>::VE;
+    const int U = dtype == kBF16 ? NhwcCfg<Bf16>::U_BWD : NhwcCfg<float>::U_BWD;
     size_t plane = kWsHeader + sizeof(double) * 2 * (size_t)C * (size_t)plane_slices(N, C);
-    if (layout == 1 && C % V == 0 && C / V <= 1024 && nhwc_threads((int)(C / V)) > 0) {
-        const int threads = nhwc_threads((int)(C / V));
-        const int64_t nvec = N * C * H * W / V;
-        int64_t g = (nvec + (int64_t)threads * kAffUnroll - 1) / ((int64_t)threads * kAffUnroll);
-        if (g > kAffGridMax) g = kAffGridMax;
-        if (g < 1) g = 1;
-        size_t fast = kWsHeader + sizeof(double) * 2 * (size_t)C * (size_t)g;
+    if (layout == 1 && C % VE == 0 && nhwc_threads((int)(C / VE)) > 0) {
+        const int threads = nhwc_threads((int)(C / VE));
+        const int64_t nunits = N * C * H * W / VE;
+        size_t fast = kWsHeader + sizeof(double) * 2 * (size_t)C * (size_t)nhwc_bwd_grid(nunits, threads, U);
         return fast > plane ? fast : plane;
     }
     return plane;

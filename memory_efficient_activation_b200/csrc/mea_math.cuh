@@ -244,63 +244,131 @@ struct Tanh {
 };
 
 // ------------------------------------------------------------- GELU-erf
-// y = x Phi(x), Phi(x) = erfc(-x / sqrt 2) / 2 (CUDA's erfcf); backward
-// Phi(x) + x phi(x), phi(x) = e^(-x^2 / 2) / sqrt(2 pi) (CUDA's expf).
-// Precise mode carries -x / sqrt 2 and x^2 as float-float pairs and applies
-// the first-order corrections d erfc = -(2 / sqrt pi) e^(-w^2) dw and
-// e^(-l/2) ~ 1 - l/2.
+// y = x Phi(x), Phi(x) = erfc(w) / 2 with w = -x / sqrt 2; backward
+// Phi(x) + x phi(x), phi(x) = e^(-w^2) / sqrt(2 pi).
+//
+// fp32 storage (P = true): CUDA's erfcf and expf, with -x / sqrt 2 and x^2
+// carried as float-float pairs and the first-order corrections
+// d erfc = -(2 / sqrt pi) e^(-w^2) dw and e^(-l/2) ~ 1 - l/2.
+//
+// bf16 storage (P = false): the Chebyshev-fitted approximation of erfc from
+// Press, Teukolsky, Vetterling and Flannery, "Numerical Recipes in C", 2nd
+// ed., section 6.2 (fractional error below 1.2e-7 for every argument):
+//   erfc(|w|) = t exp(-w^2 + P(t)),  t = 1 / (1 + |w| / 2),
+//   P a degree-9 polynomial in t;  erfc(w) = 2 - erfc(|w|) for w < 0.
+// It costs one reciprocal and one exponential on the MUFU pipe plus a
+// Horner chain, instead of the library's erfcf.  Where the exponential would
+// be subnormal (-w^2 + P(t) < -124 ln 2, i.e. x below about -13.1) but
+// x Phi(x) is still normal, the element is recomputed with the exponentials
+// scaled by 2^64.
 struct GeluErf {
     static constexpr float kNegRsqrt2Hi = -0.707106769084930419921875f;
     static constexpr float kNegRsqrt2Lo = -1.2101617104478969362e-08f;
     static constexpr float kTwoRsqrtPi = 1.12837916709551257f;     // 2 / sqrt(pi)
     static constexpr float kRsqrt2Pi = 0.398942280401432678f;      // 1 / sqrt(2 pi)
+    static constexpr float kLog2ef = 1.44269504088896340736f;
 
     static __device__ __forceinline__ Coef coef(float) { return Coef{1.f, 0.f, 0.f}; }
-    static __device__ __forceinline__ bool is_tail(float, const Coef &) { return false; }
 
-    // returns erfc(-x / sqrt 2) and sets g = e^(-x^2 / 2)
-    template <bool P>
-    static __device__ __forceinline__ float erfc_and_gauss(float x, float &g)
+    // Chebyshev approximation pieces for a = |w|: t, and u = (-a^2 + P(t)) log2 e.
+    static __device__ __forceinline__ float nr_parts(float a, float &t)
+    {
+        t = rcp_ftz(fmaf(0.5f, a, 1.0f));
+        float p = 0.17087277f;
+        p = fmaf(p, t, -0.82215223f);
+        p = fmaf(p, t, 1.48851587f);
+        p = fmaf(p, t, -1.13520398f);
+        p = fmaf(p, t, 0.27886807f);
+        p = fmaf(p, t, -0.18628806f);
+        p = fmaf(p, t, 0.09678418f);
+        p = fmaf(p, t, 0.37409196f);
+        p = fmaf(p, t, 1.00002368f);
+        p = fmaf(p, t, -1.26551223f);
+        return fmaf(-a, a, p) * kLog2ef;
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &)
+    {
+        if (!(x < 0.f)) return false;
+        float t;
+        return nr_parts(x * kNegRsqrt2Hi, t) < -kTailT;
+    }
+
+    // returns erfc(-x / sqrt 2) and sets g = e^(-x^2 / 2) (accurate path)
+    static __device__ __forceinline__ float erfc_and_gauss_precise(float x, float &g)
     {
         float w = x * kNegRsqrt2Hi;
         float ec = erfcf(w);
         float h = x * x;
         g = expf(-0.5f * h);
-        if (P) {
-            float l = fmaf(x, x, -h);
-            l = h < kBig ? l : 0.f;
-            g *= fmaf(-0.5f, l, 1.f);
-            float wl = fmaf(x, kNegRsqrt2Lo, fmaf(x, kNegRsqrt2Hi, -w));
-            ec = fmaf(-kTwoRsqrtPi * wl, g, ec);
-        }
-        return ec;
+        float l = fmaf(x, x, -h);
+        l = h < kBig ? l : 0.f;
+        g *= fmaf(-0.5f, l, 1.f);
+        float wl = fmaf(x, kNegRsqrt2Lo, fmaf(x, kNegRsqrt2Hi, -w));
+        return fmaf(-kTwoRsqrtPi * wl, g, ec);
     }
     template <bool P>
-    static __device__ __forceinline__ float f(float x, const Coef &, bool &)
+    static __device__ __forceinline__ float f(float x, const Coef &, bool &tail)
     {
-        float g;
-        float ec = erfc_and_gauss<P>(x, g);
-        return (0.5f * x) * ec;
+        if constexpr (P) {
+            float g;
+            float ec = erfc_and_gauss_precise(x, g);
+            return (0.5f * x) * ec;
+        } else {
+            const float w = x * kNegRsqrt2Hi;
+            float t;
+            const float u = nr_parts(fabsf(w), t);
+            tail |= (u < -kTailT) && (x < 0.f);
+            const float ans = t * ex2_ftz(u);
+            const float ec = w >= 0.f ? ans : 2.f - ans;
+            return (0.5f * x) * ec;
+        }
     }
     template <bool P>
     static __device__ __forceinline__ float f_tail(float x, const Coef &k)
     {
-        bool t = false;
-        return f<P>(x, k, t);
+        if constexpr (P) {
+            bool t = false;
+            return f<P>(x, k, t);
+        } else {
+            // x << 0: w > 0, erfc(w) = t 2^u with u < -124; scale by 2^64
+            const float w = x * kNegRsqrt2Hi;
+            float t;
+            const float u = nr_parts(w, t);
+            return (((0.5f * x) * t) * ex2_ftz(u + 64.f)) * kTwoM64;
+        }
     }
     template <bool P>
-    static __device__ __forceinline__ float df(float x, float dy, const Coef &, bool &)
+    static __device__ __forceinline__ float df(float x, float dy, const Coef &, bool &tail)
     {
-        float g;
-        float ec = erfc_and_gauss<P>(x, g);
-        float d = fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
-        return dy * d;
+        if constexpr (P) {
+            float g;
+            float ec = erfc_and_gauss_precise(x, g);
+            return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
+        } else {
+            const float w = x * kNegRsqrt2Hi;
+            float t;
+            const float u = nr_parts(fabsf(w), t);
+            tail |= (u < -kTailT) && (x < 0.f);
+            const float ans = t * ex2_ftz(u);
+            const float ec = w >= 0.f ? ans : 2.f - ans;
+            const float g = ex2_ftz(-(w * w) * kLog2ef);
+            return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
+        }
     }
     template <bool P>
     static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
     {
-        bool t = false;
-        return df<P>(x, dy, k, t);
+        if constexpr (P) {
+            bool t = false;
+            return df<P>(x, dy, k, t);
+        } else {
+            const float w = x * kNegRsqrt2Hi;
+            float t;
+            const float u = nr_parts(w, t);
+            const float e64 = ex2_ftz(u + 64.f);                       // erfc(w) / t, scaled
+            const float g64 = ex2_ftz(fmaf(-(w * w), kLog2ef, 64.f));  // e^(-w^2), scaled
+            return (dy * fmaf(x * kRsqrt2Pi, g64, (0.5f * t) * e64)) * kTwoM64;
+        }
     }
 };
 

@@ -145,5 +145,9 @@ def test_affine_module_autograd():
     rdx, rdg, rdb, scale = oracle.affine_swish_bwd("nhwc", (4, 144, 8, 8), xd, gd, g.double().numpy(),
                                                    b.double().numpy(), with_scale=True)
     check("bf16", xc.grad.cpu(), rdx, scale=scale, what="module dx", bf16_cond=True)
-    assert np.allclose(m.gamma.grad.cpu().double().numpy(), rdg, rtol=1e-5, atol=1e-6)
-    assert np.allclose(m.beta.grad.cpu().double().numpy(), rdb, rtol=1e-5, atol=1e-6)
+    ch = np.arange(xd.size) % 144
+    dz = rdx / g.double().numpy()[ch]
+    tg = np.bincount(ch, np.abs(dz * xd), minlength=144)
+    tb = np.bincount(ch, np.abs(dz), minlength=144)
+    assert np.all(np.abs(m.gamma.grad.cpu().double().numpy() - rdg) <= _sum_tol(rdg, tg))
+    assert np.all(np.abs(m.beta.grad.cpu().double().numpy() - rdb) <= _sum_tol(rdb, tb))
