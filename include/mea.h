@@ -115,7 +115,7 @@ MEA_API mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x
 
 /* Bytes of device workspace mea_act_bwd needs: 0 unless want_dparam is
  * non-zero (d alpha of MEA_SWISH), in which case it is a small function of n
- * (at most 256 + 8 * 1184 bytes).  Pure host arithmetic; no CUDA call. */
+ * (at most 256 + 8 * 444 = 3,808 bytes).  Pure host arithmetic; no CUDA call. */
 MEA_API size_t mea_act_bwd_workspace_bytes(mea_act_t act, int64_t n, int want_dparam);
 
 /* Backward with recompute: dx[i] = dy[i] * f'(x[i]) for i < n, f' evaluated
@@ -196,7 +196,7 @@ MEA_API mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout
  * device memory is handed out entirely by another allocator (a framework's
  * caching allocator or a fixed memory plan), and latency-sensitive paths
  * that cannot accept the synchronisation cudaFree (and possibly cudaMalloc)
- * brings.  The scratch is a fixed 9,728-byte array in the library's device
+ * brings.  The scratch is a fixed 3,808-byte array in the library's device
  * code, present on every GPU that loads the library until the process exits.
  *   Arguments as for mea_act_bwd, without workspace / ws_bytes.  With
  *   dparam_dev NULL it is a plain backward (no scratch is used).

@@ -53,7 +53,7 @@ __device__ __forceinline__ void finish_reduction(double acc, float *out, void *w
 // ------------------------------------------------------------ the kernel
 
 template <class A, typename T, int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, MODE == 2 ? 3 : 1)
 act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__restrict__ out, int64_t n,
            int vec_ok, float param, const float *__restrict__ param_dev, float *__restrict__ dparam,
            void *__restrict__ ws)
@@ -65,7 +65,6 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
     const int64_t nvec = vec_ok ? n / V : 0;
     const int tid = threadIdx.x;
     const int64_t tile = (int64_t)kThreads * kUnroll;
-    const int64_t gstride = (int64_t)gridDim.x * tile;
     double acc = 0.0;
 
     if constexpr (MODE != 2) {
@@ -90,12 +89,22 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
                 S::unpack(xv[u], xf);
                 if constexpr (MODE != 0) S::unpack(gv[u], gf);
                 bool tail = false;
+                if constexpr (HasPairs<A, P>::value) {
 #pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    if constexpr (MODE == 0)
-                        of[j] = A::template f<P>(xf[j], k, tail);
-                    else
-                        of[j] = A::template df<P>(xf[j], gf[j], k, tail);
+                    for (int j = 0; j < V; j += 2) {
+                        if constexpr (MODE == 0)
+                            A::f2(xf[j], xf[j + 1], k, tail, of[j], of[j + 1]);
+                        else
+                            A::df2(xf[j], xf[j + 1], gf[j], gf[j + 1], k, tail, of[j], of[j + 1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        if constexpr (MODE == 0)
+                            of[j] = A::template f<P>(xf[j], k, tail);
+                        else
+                            of[j] = A::template df<P>(xf[j], gf[j], k, tail);
+                    }
                 }
                 if (tail) {
 #pragma unroll
@@ -112,21 +121,36 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
             }
         }
     } else {
-        // d alpha: grid-stride over a grid fixed by n, so that every
-        // element's place in the summation order is fixed too.
-        for (int64_t base = (int64_t)blockIdx.x * tile + tid; base < nvec; base += gstride) {
-            uint4 xv[kUnroll], gv[kUnroll];
+        // d alpha: grid-stride over a grid fixed by n (one resident wave on a
+        // B200), so that every element's place in the summation order is
+        // fixed too.  The next iteration's x and dy are loaded before the
+        // current one is worked on.
+        constexpr int R = kRedUnroll;
+        const int64_t rtile = (int64_t)kThreads * R;
+        const int64_t rstride = (int64_t)gridDim.x * rtile;
+        int64_t rb = (int64_t)blockIdx.x * rtile + tid;
+        uint4 xv[R], gv[R];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t i = base + (int64_t)u * kThreads;
+        for (int u = 0; u < R; ++u) {
+            const int64_t i = rb + (int64_t)u * kThreads;
+            if (i < nvec) {
+                xv[u] = ld_nc_v4(static_cast<const uint4 *>(x) + i);
+                gv[u] = ld_nc_v4(static_cast<const uint4 *>(dy) + i);
+            }
+        }
+        for (; rb < nvec; rb += rstride) {
+            uint4 xn[R], gn[R];
+#pragma unroll
+            for (int u = 0; u < R; ++u) {
+                const int64_t i = rb + rstride + (int64_t)u * kThreads;
                 if (i < nvec) {
-                    xv[u] = ld_nc_v4(static_cast<const uint4 *>(x) + i);
-                    gv[u] = ld_nc_v4(static_cast<const uint4 *>(dy) + i);
+                    xn[u] = ld_nc_v4(static_cast<const uint4 *>(x) + i);
+                    gn[u] = ld_nc_v4(static_cast<const uint4 *>(dy) + i);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t i = base + (int64_t)u * kThreads;
+            for (int u = 0; u < R; ++u) {
+                const int64_t i = rb + (int64_t)u * kThreads;
                 if (i < nvec) {
                     float xf[V], gf[V], of[V], tf[V];
                     S::unpack(xv[u], xf);
@@ -142,6 +166,11 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
                     st_v4(static_cast<uint4 *>(out) + i, S::pack(of));
                     acc += (double)tree_sum<V>(tf);
                 }
+            }
+#pragma unroll
+            for (int u = 0; u < R; ++u) {
+                xv[u] = xn[u];
+                gv[u] = gn[u];
             }
         }
     }

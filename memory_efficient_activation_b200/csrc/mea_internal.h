@@ -13,18 +13,23 @@ enum Dtype { kF32 = 0, kBF16 = 1 };
 
 constexpr int kThreads = 256;          // threads per block of the streaming kernels
 constexpr int kUnroll = 4;             // 16-byte vectors per thread per iteration
-constexpr int kRedGridMax = 1184;      // 148 SMs x 8: cap of the reduction grid
+constexpr int kRedGridMax = 444;       // 148 SMs x 3 resident blocks: one wave on a B200
+constexpr int kRedUnroll = 2;          // vectors per thread per iteration of the d alpha loop
 constexpr int64_t kRedElemsPerBlock = 8192;
 constexpr size_t kWsHeader = 256;      // ticket counter lives in the first 256 bytes
 
 // Reduction grid of the d alpha backward: a function of n only, so the sum
 // order (and hence the bits of the result) never depends on the device.
+// With u = ceil(n / kRedElemsPerBlock) work units and k = ceil(u /
+// kRedGridMax) units per block, the grid is ceil(u / k): every block gets k
+// units (the last ones possibly one fewer), so no block is left with a
+// partly empty last pass.
 inline int red_grid(int64_t n)
 {
-    int64_t g = (n + kRedElemsPerBlock - 1) / kRedElemsPerBlock;
-    if (g < 1) g = 1;
-    if (g > kRedGridMax) g = kRedGridMax;
-    return (int)g;
+    int64_t u = (n + kRedElemsPerBlock - 1) / kRedElemsPerBlock;
+    if (u < 1) u = 1;
+    const int64_t k = (u + kRedGridMax - 1) / kRedGridMax;
+    return (int)((u + k - 1) / k);
 }
 
 struct ActLaunch {

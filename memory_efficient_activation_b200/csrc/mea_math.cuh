@@ -56,6 +56,37 @@ __device__ __forceinline__ float rcp_ftz(float v)
     return r;
 }
 
+// Two fp32 values in one 64-bit register pair, for the packed .f32x2
+// arithmetic of sm_100 (one instruction, two IEEE results with the same
+// rounding as the scalar instruction).  Used where a kernel is bound by
+// instruction issue rather than by memory.
+struct F2 {
+    unsigned long long v;
+};
+__device__ __forceinline__ F2 pk(float lo, float hi)
+{
+    F2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk(F2 a, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ F2 sp2(float c) { return pk(c, c); }
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c)
+{
+    F2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return r;
+}
+__device__ __forceinline__ F2 mul2(F2 a, F2 b)
+{
+    F2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
+
 // Multiplicative correction 2^t_lo ~ 1 + t_lo ln 2 for a float-float t.
 __device__ __forceinline__ float corr(float t_hi, float t_lo)
 {
@@ -68,6 +99,13 @@ __device__ __forceinline__ float prod_lo(float x, float c_hi, float c_lo, float 
 {
     return fmaf(x, c_lo, fmaf(x, c_hi, -t_hi));
 }
+
+// Activations that provide pairwise (packed .f32x2) versions of f and df for
+// a precision mode specialise this to true.
+template <class A, bool P>
+struct HasPairs {
+    static constexpr bool value = false;
+};
 
 // Per-launch constants, built on the device from the scalar parameter.
 struct Coef {
@@ -306,6 +344,63 @@ struct GeluErf {
         float wl = fmaf(x, kNegRsqrt2Lo, fmaf(x, kNegRsqrt2Hi, -w));
         return fmaf(-kTwoRsqrtPi * wl, g, ec);
     }
+    // Pairwise bf16-mode forward and backward: the same operations in the
+    // same order as f / df below (bitwise the same results), with the
+    // multiply-add chains on packed pairs and the two MUFU operations scalar.
+    static __device__ __forceinline__ void nr_parts2(F2 x, float &w0, float &w1, F2 &t, F2 &u)
+    {
+        const F2 w = mul2(x, sp2(kNegRsqrt2Hi));
+        upk(w, w0, w1);
+        const F2 a = pk(fabsf(w0), fabsf(w1));
+        float d0, d1;
+        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
+        t = pk(rcp_ftz(d0), rcp_ftz(d1));
+        F2 p = sp2(0.17087277f);
+        p = fma2(p, t, sp2(-0.82215223f));
+        p = fma2(p, t, sp2(1.48851587f));
+        p = fma2(p, t, sp2(-1.13520398f));
+        p = fma2(p, t, sp2(0.27886807f));
+        p = fma2(p, t, sp2(-0.18628806f));
+        p = fma2(p, t, sp2(0.09678418f));
+        p = fma2(p, t, sp2(0.37409196f));
+        p = fma2(p, t, sp2(1.00002368f));
+        p = fma2(p, t, sp2(-1.26551223f));
+        u = mul2(fma2(pk(-fabsf(w0), -fabsf(w1)), a, p), sp2(kLog2ef));
+    }
+    static __device__ __forceinline__ F2 erfc2(float w0, float w1, F2 t, float u0, float u1)
+    {
+        float a0, a1;
+        upk(mul2(t, pk(ex2_ftz(u0), ex2_ftz(u1))), a0, a1);
+        return pk(w0 >= 0.f ? a0 : 2.f - a0, w1 >= 0.f ? a1 : 2.f - a1);
+    }
+    static __device__ __forceinline__ void f2(float x0, float x1, const Coef &, bool &tail, float &o0, float &o1)
+    {
+        const F2 x = pk(x0, x1);
+        float w0, w1, u0, u1;
+        F2 t, u;
+        nr_parts2(x, w0, w1, t, u);
+        upk(u, u0, u1);
+        tail |= ((u0 < -kTailT) && (x0 < 0.f)) || ((u1 < -kTailT) && (x1 < 0.f));
+        upk(mul2(mul2(sp2(0.5f), x), erfc2(w0, w1, t, u0, u1)), o0, o1);
+    }
+    static __device__ __forceinline__ void df2(float x0, float x1, float dy0, float dy1, const Coef &, bool &tail,
+                                               float &o0, float &o1)
+    {
+        const F2 x = pk(x0, x1);
+        float w0, w1, u0, u1;
+        F2 t, u;
+        nr_parts2(x, w0, w1, t, u);
+        upk(u, u0, u1);
+        tail |= ((u0 < -kTailT) && (x0 < 0.f)) || ((u1 < -kTailT) && (x1 < 0.f));
+        const F2 ec = erfc2(w0, w1, t, u0, u1);
+        const F2 w = pk(w0, w1);
+        float v0, v1;
+        upk(mul2(mul2(w, w), sp2(-kLog2ef)), v0, v1);
+        const F2 g = pk(ex2_ftz(v0), ex2_ftz(v1));
+        const F2 d = fma2(mul2(x, sp2(kRsqrt2Pi)), g, mul2(sp2(0.5f), ec));
+        upk(mul2(pk(dy0, dy1), d), o0, o1);
+    }
+
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &, bool &tail)
     {
@@ -370,6 +465,11 @@ struct GeluErf {
             return (dy * fmaf(x * kRsqrt2Pi, g64, (0.5f * t) * e64)) * kTwoM64;
         }
     }
+};
+
+template <>
+struct HasPairs<GeluErf, false> {
+    static constexpr bool value = true;
 };
 
 // ------------------------------------------------------------ GELU-tanh

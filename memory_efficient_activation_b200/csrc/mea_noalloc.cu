@@ -30,7 +30,7 @@
 #include "mea_internal.h"
 
 // Header (completion counter) plus one fp64 partial per block of the
-// largest reduction grid: enough for every element count (9,728 bytes).
+// largest reduction grid: enough for every element count (3,808 bytes).
 static constexpr size_t kNoAllocScratchBytes = mea::kWsHeader + sizeof(double) * mea::kRedGridMax;
 
 static __device__ __align__(256) unsigned char g_dalpha_scratch[kNoAllocScratchBytes];
