@@ -61,6 +61,7 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
     using S = Store<T>;
     constexpr int V = S::V;
     constexpr bool P = S::P;
+    pdl_wait();
     const Coef k = A::coef(param_dev ? __ldg(param_dev) : param);
     const int64_t nvec = vec_ok ? n / V : 0;
     const int tid = threadIdx.x;
@@ -175,6 +176,8 @@ act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__rest
         }
     }
 
+    pdl_trigger();
+
     // Scalar loop: the n mod V tail of the vector path, or every element when
     // a pointer is not 16-byte aligned.
     for (int64_t i = nvec * V + (int64_t)blockIdx.x * kThreads + tid; i < n;
@@ -245,9 +248,8 @@ static cudaError_t launch_one(const ActLaunch &a)
     if (g < 1) g = 1;
     if (g > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const int grid = (int)g;
-    kernel<<<grid, kThreads, 0, a.stream>>>(a.x, a.dy, a.out, a.n, vec_ok, a.param, a.param_dev, a.dparam,
-                                            a.workspace);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kThreads), 0, a.stream, a.x, a.dy, a.out, a.n, vec_ok,
+                      a.param, a.param_dev, a.dparam, a.workspace);
 }
 
 template <class A, int MODE>

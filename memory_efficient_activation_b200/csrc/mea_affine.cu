@@ -30,7 +30,6 @@
 
 namespace mea {
 
-constexpr int kAffUnroll = 4;
 constexpr int kNhwcMaxThreads = 512;
 constexpr int kNhwcTargetThreads = 256;
 constexpr int kColsumThreads = 256;
@@ -132,6 +131,7 @@ affine_nhwc_fwd_kernel(const void *__restrict__ x, const float *__restrict__ gam
     const int tid = threadIdx.x;
     const int g = tid % groups;
     const Coef k = Swish::coef(1.f);
+    pdl_wait();
     float ga[VE], be[VE];
 #pragma unroll
     for (int j = 0; j < VE; ++j) {
@@ -164,6 +164,7 @@ affine_nhwc_fwd_kernel(const void *__restrict__ x, const float *__restrict__ gam
             L::store(out, i, L::pack(of));
         }
     }
+    pdl_trigger();
 }
 
 // Backward: a fixed grid of blocks (a function of the shape only) walks the
@@ -184,6 +185,7 @@ affine_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, 
     const int tid = threadIdx.x;
     const int g = tid % groups;
     const Coef k = Swish::coef(1.f);
+    pdl_wait();
     float ga[VE], be[VE];
 #pragma unroll
     for (int j = 0; j < VE; ++j) {
@@ -255,6 +257,7 @@ affine_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, 
             gv[u] = gn[u];
         }
     }
+    pdl_trigger();
     extern __shared__ double red[];   // 2 VE * blockDim.x doubles
 #pragma unroll
     for (int j = 0; j < VE; ++j) {
@@ -281,6 +284,8 @@ affine_colsum_kernel(const double *__restrict__ partials, int nb, int C, float *
 {
     __shared__ double red[32];
     const int o = blockIdx.x;
+    pdl_wait();
+    pdl_trigger();
     double s = 0.0;
     for (int b = threadIdx.x; b < nb; b += kColsumThreads) s += partials[(int64_t)b * 2 * C + o];
     s = block_sum(s, red);
@@ -305,6 +310,7 @@ affine_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, con
     const int64_t c = blockIdx.x / slices;
     const int s = blockIdx.x % slices;
     const int64_t n0 = (int64_t)s * N / slices, n1 = (int64_t)(s + 1) * N / slices;
+    pdl_wait();
     const float ga = __ldg(gamma + c), be = __ldg(beta + c);
     const Coef k = Swish::coef(1.f);
     double ag = 0.0, ab = 0.0;
@@ -350,6 +356,7 @@ affine_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, con
             S::store1(out, i, o);
         }
     }
+    pdl_trigger();
     if constexpr (MODE == 0) return;
 
     __shared__ double red[32];
@@ -427,9 +434,8 @@ static cudaError_t launch_affine(const AffineLaunch &a)
             constexpr int U = NhwcCfg<T>::U_FWD;
             const int64_t nb = nhwc_blocks(nunits, threads, U);
             if (nb > 0x7fffffff) return cudaErrorInvalidConfiguration;
-            affine_nhwc_fwd_kernel<T, U, VE><<<(unsigned)nb, threads, 0, a.stream>>>(a.x, a.gamma, a.beta, a.out,
-                                                                                      nunits, groups);
-            return cudaGetLastError();
+            return launch_pdl(affine_nhwc_fwd_kernel<T, U, VE>, dim3((unsigned)nb), dim3(threads), 0, a.stream, a.x,
+                              a.gamma, a.beta, a.out, nunits, groups);
         }
         constexpr int U = NhwcCfg<T>::U_BWD;
         auto kernel = affine_nhwc_bwd_kernel<T, U, VE>;
@@ -441,13 +447,11 @@ static cudaError_t launch_affine(const AffineLaunch &a)
         if (e == cudaSuccess && smem > 48 * 1024)
             e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kernel<<<(unsigned)nb, threads, smem, a.stream>>>(a.x, a.dy, a.gamma, a.beta, a.out, nunits, groups,
-                                                          (int)a.C, partials);
-        e = cudaGetLastError();
+        e = launch_pdl(kernel, dim3((unsigned)nb), dim3(threads), smem, a.stream, a.x, a.dy, a.gamma, a.beta, a.out,
+                       nunits, groups, (int)a.C, partials);
         if (e != cudaSuccess) return e;
-        affine_colsum_kernel<<<(unsigned)(2 * a.C), kColsumThreads, 0, a.stream>>>(partials, nb, (int)a.C, a.dgamma,
-                                                                                  a.dbeta);
-        return cudaGetLastError();
+        return launch_pdl(affine_colsum_kernel, dim3((unsigned)(2 * a.C)), dim3(kColsumThreads), 0, a.stream,
+                          partials, nb, (int)a.C, a.dgamma, a.dbeta);
     }
     uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
     if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
@@ -456,12 +460,12 @@ static cudaError_t launch_affine(const AffineLaunch &a)
     const int64_t grid = a.C * slices;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     if (a.layout == 1)
-        affine_plane_kernel<T, MODE, true><<<(unsigned)grid, kPlaneThreads, 0, a.stream>>>(
-            a.x, a.dy, a.gamma, a.beta, a.out, a.N, a.C, HW, slices, vec_ok, a.dgamma, a.dbeta, a.workspace);
-    else
-        affine_plane_kernel<T, MODE, false><<<(unsigned)grid, kPlaneThreads, 0, a.stream>>>(
-            a.x, a.dy, a.gamma, a.beta, a.out, a.N, a.C, HW, slices, vec_ok, a.dgamma, a.dbeta, a.workspace);
-    return cudaGetLastError();
+        return launch_pdl(affine_plane_kernel<T, MODE, true>, dim3((unsigned)grid), dim3(kPlaneThreads), 0, a.stream,
+                          a.x, a.dy, a.gamma, a.beta, a.out, a.N, a.C, HW, slices, vec_ok, a.dgamma, a.dbeta,
+                          a.workspace);
+    return launch_pdl(affine_plane_kernel<T, MODE, false>, dim3((unsigned)grid), dim3(kPlaneThreads), 0, a.stream,
+                      a.x, a.dy, a.gamma, a.beta, a.out, a.N, a.C, HW, slices, vec_ok, a.dgamma, a.dbeta,
+                      a.workspace);
 }
 
 size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W)

@@ -9,6 +9,19 @@
 
 namespace mea {
 
+// ------------------------------------------------- programmatic dependence
+//
+// Every kernel of the library is launched with programmatic stream
+// serialisation (see launch_pdl in mea_internal.h): the next kernel on the
+// stream may be scheduled while this one drains.  pdl_wait() must come
+// before the first access to memory a preceding kernel may write; it returns
+// once every preceding grid on the stream has completed and its memory is
+// visible (and at once when the launch carried no such dependence).
+// pdl_trigger() tells the hardware that the dependent grid may start
+// launching; it does not weaken pdl_wait() in the dependent.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------- memory helpers
 
 // 16-byte load through the non-coherent (read-only) path, not allocated in

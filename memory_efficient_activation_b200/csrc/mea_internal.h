@@ -69,6 +69,26 @@ size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, i
 cudaError_t launch_affine_fwd(const AffineLaunch &a);
 cudaError_t launch_affine_bwd(const AffineLaunch &a);
 
+// Launch with programmatic stream serialisation: the kernel may begin while
+// the previous kernel on the stream drains, and waits (pdl_wait) before it
+// touches memory.  Returns the launch's cudaError_t.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
