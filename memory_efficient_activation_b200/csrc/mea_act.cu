@@ -53,7 +53,7 @@ __device__ __forceinline__ void finish_reduction(double acc, float *out, void *w
 // ------------------------------------------------------------ the kernel
 
 template <class A, typename T, int MODE>
-__global__ void __launch_bounds__(kThreads, MODE == 2 ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, MODE == 2 ? 3 : 4)
 act_kernel(const void *__restrict__ x, const void *__restrict__ dy, void *__restrict__ out, int64_t n,
            int vec_ok, float param, const float *__restrict__ param_dev, float *__restrict__ dparam,
            void *__restrict__ ws)
