@@ -536,6 +536,8 @@ def run_secondary(args):
                                                                                dgamma=q[0], dbeta=q[1], workspace=ws)
                                    for s, q, ws in zip(sets, gr, wss)],
                     accounting.affine_bwd_bytes(w.n, "bf16", C)))
+    elif wl == "memory_study":
+        return run_memory_study(args)
     elif wl == "swish_f32_1m":
         w = synthetic.swish_f32_1m()
         sets = clones([w.x, w.dy, w.x, w.x], 1)       # L2-resident on purpose
@@ -571,6 +573,80 @@ def run_secondary(args):
     return out
 
 
+class _PlainSwish(torch.nn.Module):
+    """The plain autograd Swish of the pages' first listing: x * sigmoid(alpha x)
+    built from PyTorch ops, which keeps every intermediate for the backward.
+    Comparator only."""
+
+    def __init__(self, alpha=1.0):
+        super().__init__()
+        self.alpha = alpha
+
+    def forward(self, x):
+        return x * torch.sigmoid(self.alpha * x)
+
+
+def run_memory_study(args, layers: int = 32, shape=SHAPE):
+    """Peak memory and step time of an L-layer stack at [8, 2048, 4096] bf16 with
+    the plain autograd Swish versus the save-input-only Swish, in two stacks:
+    activations only, and Linear(d, d) + Swish blocks (a transformer-style MLP
+    path).  Re-measures, on synthetic data, the memory the Swish page's
+    "How much GPU memory is saved?" section reports for EfficientNets."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = shape[-1]
+    x0 = synthetic.normal(accounting.elements(shape), 1.0, 7, synthetic.STREAM_X, "bf16").view(shape).to(dev)
+    res = {}
+    for stack in ("activations", "linear_swish"):
+        for impl in ("plain", "save_input_only"):
+            torch.manual_seed(0)
+            mods = []
+            for _ in range(layers):
+                if stack == "linear_swish":
+                    mods.append(torch.nn.Linear(d, d, bias=False, device=dev, dtype=torch.bfloat16))
+                mods.append(_PlainSwish() if impl == "plain" else mea.MemoryEfficientSwish())
+            net = torch.nn.Sequential(*mods)
+            for p in net.parameters():
+                p.requires_grad_(True)
+
+            def step():
+                x = x0.detach().requires_grad_(True)
+                y = net(x)
+                y.backward(torch.ones_like(y))
+                return x.grad
+
+            step()
+            torch.cuda.synchronize()
+            for p in net.parameters():
+                p.grad = None
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats(dev)
+            base = torch.cuda.memory_allocated(dev)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            reps = max(1, min(args.steps, 5))
+            for _ in range(reps):
+                step()
+                for p in net.parameters():
+                    p.grad = None
+            s1.record()
+            torch.cuda.synchronize()
+            res[f"{stack}/{impl}"] = {
+                "peak_GB": round((torch.cuda.max_memory_allocated(dev) - base) / 1e9, 3),
+                "ms_per_fwd_bwd": round(s0.elapsed_time(s1) / reps, 3),
+            }
+            del net, mods
+            torch.cuda.empty_cache()
+    for stack in ("activations", "linear_swish"):
+        a, b = res[f"{stack}/plain"], res[f"{stack}/save_input_only"]
+        res[f"{stack}/saved_GB"] = round(a["peak_GB"] - b["peak_GB"], 3)
+        res[f"{stack}/saved_fraction"] = round(1 - b["peak_GB"] / a["peak_GB"], 4)
+    return {"workload": "memory_study", "layers": layers, "shape": list(shape), "dtype": "bf16",
+            "per_layer_tensor_MB": round(accounting.tensor_bytes(accounting.elements(shape), "bf16") / 1e6, 1),
+            "note": "peak = max_memory_allocated above the memory held before the step (inputs, weights)",
+            "results": res}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -584,7 +660,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="swish_bf16",
-                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16", "swish_f32_1m"],
+                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16", "swish_f32_1m",
+                             "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:
