@@ -88,6 +88,15 @@ def _load():
         lib.oracle_affine_swish_fwd.restype = ctypes.c_int
         lib.oracle_affine_swish_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d, d, d]
         lib.oracle_affine_swish_bwd.restype = ctypes.c_int
+        lib.oracle_affine_act_fwd.argtypes = [ctypes.c_int, ctypes.c_int, shp, d, d, d, ctypes.c_double, d]
+        lib.oracle_affine_act_fwd.restype = ctypes.c_int
+        lib.oracle_affine_act_bwd.argtypes = [ctypes.c_int, ctypes.c_int, shp, d, d, d, d, ctypes.c_double,
+                                              d, d, d, d]
+        lib.oracle_affine_act_bwd.restype = ctypes.c_int
+        lib.oracle_swish_channel_fwd.argtypes = [ctypes.c_int, shp, d, d, d]
+        lib.oracle_swish_channel_fwd.restype = ctypes.c_int
+        lib.oracle_swish_channel_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d]
+        lib.oracle_swish_channel_bwd.restype = ctypes.c_int
         lib.oracle_round_bf16.argtypes = [d, ctypes.POINTER(ctypes.c_uint16), i64]
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_f32.argtypes = [d, ctypes.POINTER(ctypes.c_float), i64]
@@ -200,6 +209,60 @@ def affine_swish_bwd(layout: str, shape, x, dy, gamma, beta, with_scale: bool = 
     if rc:
         raise ValueError(f"oracle_affine_swish_bwd failed: {rc}")
     return (dx, dg, db, scale) if with_scale else (dx, dg, db)
+
+
+def affine_act_fwd(act: str, layout: str, shape, x, gamma, beta, param: float = 1.0) -> np.ndarray:
+    """y = f(gamma_c x + beta_c; param); shape is (N, C, H, W)."""
+    s = _shape4(shape)
+    x, gamma, beta = _f64(x), _f64(gamma), _f64(beta)
+    y = np.empty_like(x)
+    rc = _load().oracle_affine_act_fwd(ACTS[act], LAYOUTS[layout], _ptr(s, ctypes.c_int64), _ptr(x),
+                                       _ptr(gamma), _ptr(beta), float(param), _ptr(y))
+    if rc:
+        raise ValueError(f"oracle_affine_act_fwd failed: {rc}")
+    return y
+
+
+def affine_act_bwd(act: str, layout: str, shape, x, dy, gamma, beta, param: float = 1.0):
+    """Returns (dx, dgamma, dbeta, dx condition scale) in double."""
+    s = _shape4(shape)
+    x, dy, gamma, beta = _f64(x), _f64(dy), _f64(gamma), _f64(beta)
+    C = int(s[1])
+    dx = np.empty_like(x)
+    scale = np.empty_like(x)
+    dg = np.empty(C, dtype=np.float64)
+    db = np.empty(C, dtype=np.float64)
+    rc = _load().oracle_affine_act_bwd(ACTS[act], LAYOUTS[layout], _ptr(s, ctypes.c_int64), _ptr(x), _ptr(dy),
+                                       _ptr(gamma), _ptr(beta), float(param), _ptr(dx), _ptr(dg), _ptr(db),
+                                       _ptr(scale))
+    if rc:
+        raise ValueError(f"oracle_affine_act_bwd failed: {rc}")
+    return dx, dg, db, scale
+
+
+def swish_channel_fwd(layout: str, shape, x, alpha) -> np.ndarray:
+    """y = x Sigmoid(alpha_c x); shape is (N, C, H, W)."""
+    s = _shape4(shape)
+    x, alpha = _f64(x), _f64(alpha)
+    y = np.empty_like(x)
+    rc = _load().oracle_swish_channel_fwd(LAYOUTS[layout], _ptr(s, ctypes.c_int64), _ptr(x), _ptr(alpha), _ptr(y))
+    if rc:
+        raise ValueError(f"oracle_swish_channel_fwd failed: {rc}")
+    return y
+
+
+def swish_channel_bwd(layout: str, shape, x, dy, alpha):
+    """Returns (dx, dalpha per channel, dx condition scale) in double."""
+    s = _shape4(shape)
+    x, dy, alpha = _f64(x), _f64(dy), _f64(alpha)
+    dx = np.empty_like(x)
+    scale = np.empty_like(x)
+    da = np.empty(int(s[1]), dtype=np.float64)
+    rc = _load().oracle_swish_channel_bwd(LAYOUTS[layout], _ptr(s, ctypes.c_int64), _ptr(x), _ptr(dy),
+                                          _ptr(alpha), _ptr(dx), _ptr(da), _ptr(scale))
+    if rc:
+        raise ValueError(f"oracle_swish_channel_bwd failed: {rc}")
+    return dx, da, scale
 
 
 def round_bf16(v) -> np.ndarray:

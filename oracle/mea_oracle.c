@@ -355,6 +355,87 @@ int oracle_affine_swish_bwd(int layout, const int64_t shape[4], const double *x,
     return 0;
 }
 
+/* ------------------------------------ exported: per-channel family (NEXT) */
+
+/* Per-channel affine followed by any activation of the family:
+ * z = gamma_c x + beta_c, y = f(z; param).  The affine + Swish functions above
+ * are the case act = Swish, param = 1. */
+int oracle_affine_act_fwd(int act, int layout, const int64_t shape[4], const double *x,
+                          const double *gamma, const double *beta, double param, double *y)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || (layout != OR_NCHW && layout != OR_NHWC)) return -1;
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        y[i] = act_f(act, gamma[c] * x[i] + beta[c], param);
+    }
+    return 0;
+}
+
+/* dz = dy f'(z); dx = gamma_c dz; dgamma_c = sum dz x; dbeta_c = sum dz
+ * (serial, index order, long double).  dx_scale (nullable) receives
+ * |gamma_c| times the condition scale of dy f'(z) (see oracle_act_bwd_scale). */
+int oracle_affine_act_bwd(int act, int layout, const int64_t shape[4], const double *x,
+                          const double *dy, const double *gamma, const double *beta, double param,
+                          double *dx, double *dgamma, double *dbeta, double *dx_scale)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || (layout != OR_NCHW && layout != OR_NHWC)) return -1;
+    int64_t C = shape[1];
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+    long double *acc_g = (long double *)calloc((size_t)(C > 0 ? C : 1), sizeof(long double));
+    long double *acc_b = (long double *)calloc((size_t)(C > 0 ? C : 1), sizeof(long double));
+    if (!acc_g || !acc_b) { free(acc_g); free(acc_b); return -2; }
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        double z = gamma[c] * x[i] + beta[c];
+        double dz = dy[i] * act_df(act, z, param);
+        dx[i] = gamma[c] * dz;
+        if (dx_scale) dx_scale[i] = fabs(gamma[c] * dy[i]) * act_df_abs_terms(act, z, param);
+        acc_g[c] += (long double)(dz * x[i]);
+        acc_b[c] += (long double)dz;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        dgamma[c] = (double)acc_g[c];
+        dbeta[c] = (double)acc_b[c];
+    }
+    free(acc_g);
+    free(acc_b);
+    return 0;
+}
+
+/* Swish with one alpha per channel: y = x Sigmoid(alpha_c x). */
+int oracle_swish_channel_fwd(int layout, const int64_t shape[4], const double *x,
+                             const double *alpha, double *y)
+{
+    if (layout != OR_NCHW && layout != OR_NHWC) return -1;
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) y[i] = swish_f(x[i], alpha[channel_of(layout, shape, i)]);
+    return 0;
+}
+
+/* dx = dy Swish'(x; alpha_c); dalpha_c = sum over channel c of
+ * dy x^2 s (1 - s) (serial, index order, long double).  dx_scale as above. */
+int oracle_swish_channel_bwd(int layout, const int64_t shape[4], const double *x, const double *dy,
+                             const double *alpha, double *dx, double *dalpha, double *dx_scale)
+{
+    if (layout != OR_NCHW && layout != OR_NHWC) return -1;
+    int64_t C = shape[1];
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+    long double *acc = (long double *)calloc((size_t)(C > 0 ? C : 1), sizeof(long double));
+    if (!acc) return -2;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        dx[i] = dy[i] * swish_df(x[i], alpha[c]);
+        if (dx_scale) dx_scale[i] = fabs(dy[i]) * act_df_abs_terms(OR_SWISH, x[i], alpha[c]);
+        acc[c] += (long double)(dy[i] * swish_dalpha_term(x[i], alpha[c]));
+    }
+    for (int64_t c = 0; c < C; ++c) dalpha[c] = (double)acc[c];
+    free(acc);
+    return 0;
+}
+
 /* ------------------------------------------------------ storage rounding */
 
 /* Round a double to the nearest bfloat16 (1 sign bit, 8 exponent bits with
