@@ -482,7 +482,9 @@ def _sets_for(nbytes: int) -> int:
 def run_secondary(args):
     """Per-kernel GB/s and roofline fractions for the other configurations
     (activation family, EfficientNet-like fp32 maps with d alpha, fused
-    affine + Swish NHWC, the L2-resident 1M fp32 case).  Diagnostics: the
+    affine + Swish NHWC, fused affine + every activation NHWC, Swish with a
+    per-channel alpha on EfficientNet-like maps, the L2-resident 1M fp32
+    case).  Diagnostics: the
     headline line is the default run."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -515,11 +517,11 @@ def run_secondary(args):
             wss = [torch.zeros(mea.act_bwd_workspace_bytes("swish", w.n, True), dtype=torch.uint8, device=dev)
                    for _ in range(k)]
             tag = "x".join(map(str, w.x.shape))
-            ops.append((f"{tag}_fwd", [lambda b=b: mea.act_fwd("swish", b[0], 0.0, param_dev=a, out=b[2])
+            ops.append((f"{tag}_fwd", [lambda b=b, a=a: mea.act_fwd("swish", b[0], 0.0, param_dev=a, out=b[2])
                                        for b in sets], accounting.fwd_bytes(w.n, "f32")))
             ops.append((f"{tag}_bwd_dalpha",
-                        [lambda b=b, d=d, ws=ws: mea.act_bwd("swish", b[0], b[1], 0.0, param_dev=a, dparam=d, out=b[3],
-                                                             workspace=ws)
+                        [lambda b=b, d=d, ws=ws, a=a: mea.act_bwd("swish", b[0], b[1], 0.0, param_dev=a, dparam=d,
+                                                                  out=b[3], workspace=ws)
                          for b, d, ws in zip(sets, ds, wss)], accounting.bwd_bytes(w.n, "f32")))
     elif wl == "affine_nhwc_bf16":
         w = synthetic.affine_swish_nhwc()
@@ -536,6 +538,41 @@ def run_secondary(args):
                                                                                dgamma=q[0], dbeta=q[1], workspace=ws)
                                    for s, q, ws in zip(sets, gr, wss)],
                     accounting.affine_bwd_bytes(w.n, "bf16", C)))
+    elif wl == "affine_family_nhwc_bf16":
+        w = synthetic.affine_act_nhwc("swish")
+        C = w.extra["gamma"].numel()
+        k = _sets_for(accounting.affine_bwd_bytes(w.n, "bf16", C))
+        g, b_ = w.extra["gamma"].to(dev), w.extra["beta"].to(dev)
+        sets = clones([w.x, w.dy, w.x, w.x], k)
+        gr = [(torch.empty(C, device=dev), torch.empty(C, device=dev)) for _ in range(k)]
+        need = mea.affine_act_bwd_workspace_bytes(torch.bfloat16, "nhwc", w.extra["nchw_shape"])
+        wss = [torch.zeros(need, dtype=torch.uint8, device=dev) for _ in range(k)]
+        for act in synthetic.ACTIVATIONS:
+            p = 0.01 if act == "leaky_relu" else 1.0
+            ops.append((f"{act}_fwd", [lambda a=act, p=p, s=s: mea.affine_act_fwd(a, s[0], g, b_, p, "nhwc", out=s[2])
+                                       for s in sets], accounting.affine_fwd_bytes(w.n, "bf16", C)))
+            ops.append((f"{act}_bwd", [lambda a=act, p=p, s=s, q=q, ws=ws:
+                                       mea.affine_act_bwd(a, s[0], s[1], g, b_, p, "nhwc", out=s[3], dgamma=q[0],
+                                                          dbeta=q[1], workspace=ws)
+                                       for s, q, ws in zip(sets, gr, wss)],
+                        accounting.affine_bwd_bytes(w.n, "bf16", C)))
+    elif wl == "swish_channel_f32":
+        for i in range(len(synthetic.EFFNET_B0_SHAPES)):
+            w = synthetic.swish_channel_nchw(seed=8 + i, shape=synthetic.EFFNET_B0_SHAPES[i])
+            C = w.extra["alpha"].numel()
+            k = _sets_for(accounting.channel_swish_bwd_bytes(w.n, "f32", C))
+            a = w.extra["alpha"].to(dev)
+            sets = clones([w.x, w.dy, w.x, w.x], k)
+            ds = [torch.empty(C, dtype=torch.float32, device=dev) for _ in range(k)]
+            need = mea.swish_channel_bwd_workspace_bytes(torch.float32, "nchw", w.extra["nchw_shape"])
+            wss = [torch.zeros(need, dtype=torch.uint8, device=dev) for _ in range(k)]
+            tag = "x".join(map(str, w.x.shape))
+            ops.append((f"{tag}_fwd", [lambda b=b, a=a: mea.swish_channel_fwd(b[0], a, "nchw", out=b[2])
+                                       for b in sets], accounting.channel_swish_fwd_bytes(w.n, "f32", C)))
+            ops.append((f"{tag}_bwd_dalpha",
+                        [lambda b=b, d=d, ws=ws, a=a: mea.swish_channel_bwd(b[0], b[1], a, "nchw", out=b[3], dalpha=d,
+                                                                            workspace=ws)
+                         for b, d, ws in zip(sets, ds, wss)], accounting.channel_swish_bwd_bytes(w.n, "f32", C)))
     elif wl == "memory_study":
         return run_memory_study(args)
     elif wl == "swish_f32_1m":
@@ -660,8 +697,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="swish_bf16",
-                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16", "swish_f32_1m",
-                             "memory_study"],
+                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
+                             "affine_family_nhwc_bf16", "swish_channel_f32", "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:

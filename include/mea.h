@@ -4,8 +4,9 @@
  * The library implements save-input-only elementwise activations on NVIDIA
  * B200 (sm_100a): the forward writes y = f(x) and keeps nothing else; the
  * backward recomputes what it needs from the saved input x in the same pass
- * and writes dx = dy * f'(x) (plus d alpha for a learnable Swish alpha, or
- * d gamma / d beta for the fused per-channel affine + Swish).
+ * and writes dx = dy * f'(x) (plus d alpha for a learnable Swish alpha,
+ * scalar or one per channel, or d gamma / d beta for the fused per-channel
+ * affine + activation).
  *
  * Sources, by page and section:
  *  - "Memory efficient Swish" (adeeplearner blog, 2021-05-17):
@@ -187,6 +188,68 @@ MEA_API mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout
                                   const float *gamma, const float *beta, void *dx,
                                   float *dgamma, float *dbeta, void *workspace,
                                   size_t ws_bytes, mea_stream_t stream);
+
+/* Bytes of device workspace mea_affine_act_bwd needs (the same for every
+ * activation; equal to mea_affine_swish_bwd_workspace_bytes).  Pure host
+ * arithmetic; returns 0 for an invalid request. */
+MEA_API size_t mea_affine_act_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout,
+                                                  const int64_t shape[4]);
+
+/* Fused per-channel affine + any activation of the family, forward:
+ * z = gamma_c x + beta_c, y = f(z), f as in mea_act_t with `param` (slope
+ * of MEA_LEAKY_RELU, alpha of MEA_SWISH; ignored otherwise).
+ *   Arguments otherwise as in mea_affine_swish_fwd; mea_affine_swish_fwd is
+ *   this call with act = MEA_SWISH and param = 1.
+ * Source: the save-input-only scheme of the Swish page ("What makes this
+ * implementation save GPU memory?") applied to the per-channel affine that
+ * precedes the activation, for the family of problem B07. */
+MEA_API mea_status_t mea_affine_act_fwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t layout,
+                                        const int64_t shape[4], const void *x, const float *gamma,
+                                        const float *beta, float param, void *y,
+                                        mea_stream_t stream);
+
+/* Fused per-channel affine + activation, backward: recomputes z from x and
+ *   dz = dy f'(z);  dx = gamma_c dz;  dgamma_c = sum dz x;  dbeta_c = sum dz
+ * (sums over all N*H*W positions of channel c, fp64 accumulation in a fixed
+ * order, rounded to fp32; dgamma and dbeta are OVERWRITTEN).
+ *   Arguments otherwise as in mea_affine_swish_bwd (workspace of at least
+ *   mea_affine_act_bwd_workspace_bytes() bytes, same counter rule). */
+MEA_API mea_status_t mea_affine_act_bwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t layout,
+                                        const int64_t shape[4], const void *x, const void *dy,
+                                        const float *gamma, const float *beta, float param,
+                                        void *dx, float *dgamma, float *dbeta, void *workspace,
+                                        size_t ws_bytes, mea_stream_t stream);
+
+/* Bytes of device workspace mea_swish_channel_bwd needs.  Pure host
+ * arithmetic; returns 0 for an invalid request. */
+MEA_API size_t mea_swish_channel_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout,
+                                                     const int64_t shape[4]);
+
+/* Swish with one learnable alpha per channel, forward:
+ * y = x Sigmoid(alpha_c x).
+ *   shape, layout  as in mea_affine_swish_fwd (channel of each element).
+ *   x, y           device, N*C*H*W elements of `dtype`; y must not overlap x.
+ *   alpha          device fp32[C], read only.
+ * Source: the Swish page's learnable alpha ("What is a Swish activation
+ * function?"), one value per channel. */
+MEA_API mea_status_t mea_swish_channel_fwd(mea_dtype_t dtype, mea_layout_t layout,
+                                           const int64_t shape[4], const void *x,
+                                           const float *alpha, void *y, mea_stream_t stream);
+
+/* Swish with a per-channel alpha, backward (recompute from x alone):
+ *   s = Sigmoid(alpha_c x);  dx = dy (s + alpha_c x s (1 - s));
+ *   dalpha_c = sum dy x^2 s (1 - s)   (over the N*H*W positions of channel
+ *   c, fp64 accumulation in a fixed order, rounded to fp32, OVERWRITTEN).
+ *   x, dy     device, read only; dx device, written (may equal dy or x
+ *             exactly, no partial overlap).
+ *   alpha     device fp32[C]; dalpha device fp32[C].
+ *   workspace device scratch of at least mea_swish_channel_bwd_workspace_bytes()
+ *             bytes, 16-byte aligned, with the completion-counter rule of
+ *             mea_act_bwd. */
+MEA_API mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layout,
+                                           const int64_t shape[4], const void *x, const void *dy,
+                                           const float *alpha, void *dx, float *dalpha,
+                                           void *workspace, size_t ws_bytes, mea_stream_t stream);
 
 /* Backward with d alpha that allocates nothing and takes no workspace.
  * No counterpart on the pages: this is a library convenience, not part of

@@ -10,10 +10,14 @@ stream) into those calls; PyTorch is plumbing here, not the compute path.
 
 Functions (the C ABI's names without the ``mea_`` prefix):
     act_fwd, act_bwd, affine_swish_fwd, affine_swish_bwd,
-    act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes
+    affine_act_fwd, affine_act_bwd, swish_channel_fwd, swish_channel_bwd,
+    act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes,
+    affine_act_bwd_workspace_bytes, swish_channel_bwd_workspace_bytes
 Autograd / modules:
     ActivationFunction, MemoryEfficientActivation, MemoryEfficientSwish,
-    AffineSwishFunction, MemoryEfficientAffineSwish
+    AffineSwishFunction, MemoryEfficientAffineSwish,
+    AffineActFunction, MemoryEfficientAffineActivation,
+    SwishChannelFunction, MemoryEfficientChannelSwish
 """
 from __future__ import annotations
 
@@ -27,9 +31,13 @@ from ._capi import ACT_IDS, LAYOUT_IDS, MeaError
 
 __all__ = [
     "act_fwd", "act_bwd", "affine_swish_fwd", "affine_swish_bwd",
+    "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
     "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
+    "affine_act_bwd_workspace_bytes", "swish_channel_bwd_workspace_bytes",
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
-    "AffineSwishFunction", "MemoryEfficientAffineSwish", "MeaError", "ACTIVATIONS",
+    "AffineSwishFunction", "MemoryEfficientAffineSwish",
+    "AffineActFunction", "MemoryEfficientAffineActivation",
+    "SwishChannelFunction", "MemoryEfficientChannelSwish", "MeaError", "ACTIVATIONS",
 ]
 
 ACTIVATIONS = tuple(ACT_IDS)
@@ -99,6 +107,16 @@ def affine_swish_bwd_workspace_bytes(dtype: torch.dtype, layout: str, shape_nchw
         _DTYPES[dtype], LAYOUT_IDS[layout], _capi.shape4(shape_nchw)))
 
 
+def affine_act_bwd_workspace_bytes(dtype: torch.dtype, layout: str, shape_nchw) -> int:
+    return int(_capi.lib().mea_affine_act_bwd_workspace_bytes(
+        _DTYPES[dtype], LAYOUT_IDS[layout], _capi.shape4(shape_nchw)))
+
+
+def swish_channel_bwd_workspace_bytes(dtype: torch.dtype, layout: str, shape_nchw) -> int:
+    return int(_capi.lib().mea_swish_channel_bwd_workspace_bytes(
+        _DTYPES[dtype], LAYOUT_IDS[layout], _capi.shape4(shape_nchw)))
+
+
 # ------------------------------------------------------------ entry points
 
 def act_fwd(act: str, x: torch.Tensor, param: float = 1.0, param_dev: torch.Tensor | None = None,
@@ -143,7 +161,7 @@ def act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, param: float = 1.0,
 
 def _affine_shape(x: torch.Tensor, layout: str):
     if x.dim() != 4:
-        raise ValueError("affine + Swish takes a 4-D tensor")
+        raise ValueError("per-channel operations take a 4-D tensor")
     if layout == "nhwc":
         N, H, W, C = x.shape
     elif layout == "nchw":
@@ -153,12 +171,20 @@ def _affine_shape(x: torch.Tensor, layout: str):
     return (N, C, H, W)
 
 
+def _chan_params(C: int, *ps):
+    for p in ps:
+        _need_cuda(p)
+        if p.dtype != torch.float32 or p.numel() != C:
+            raise ValueError(f"per-channel parameters must be fp32 with {C} elements")
+
+
 def affine_swish_fwd(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, layout: str = "nhwc",
                      out: torch.Tensor | None = None) -> torch.Tensor:
     """y = z Sigmoid(z), z = gamma_c x + beta_c.  x is (N, H, W, C) for
     'nhwc' or (N, C, H, W) for 'nchw'; gamma and beta are fp32 [C]."""
-    _need_cuda(x, gamma, beta)
+    _need_cuda(x)
     shape = _affine_shape(x, layout)
+    _chan_params(shape[1], gamma, beta)
     y = torch.empty_like(x) if out is None else out
     _need_cuda(y)
     st = _capi.lib().mea_affine_swish_fwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
@@ -172,11 +198,12 @@ def affine_swish_bwd(x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, bet
                      dgamma: torch.Tensor | None = None, dbeta: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None):
     """Returns (dx, dgamma, dbeta); z and the sigmoid are recomputed from x."""
-    _need_cuda(x, dy, gamma, beta)
+    _need_cuda(x, dy)
     if dy.dtype != x.dtype or dy.shape != x.shape:
         raise ValueError("dy must match x in dtype and shape")
     shape = _affine_shape(x, layout)
     C = shape[1]
+    _chan_params(C, gamma, beta)
     dx = torch.empty_like(x) if out is None else out
     dg = torch.empty(C, dtype=torch.float32, device=x.device) if dgamma is None else dgamma
     db = torch.empty(C, dtype=torch.float32, device=x.device) if dbeta is None else dbeta
@@ -189,6 +216,83 @@ def affine_swish_bwd(x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, bet
                                            ws.numel() * ws.element_size(), _stream(x))
     _capi.check("mea_affine_swish_bwd", st)
     return dx, dg, db
+
+
+def affine_act_fwd(act: str, x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, param: float = 1.0,
+                   layout: str = "nhwc", out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = f(z), z = gamma_c x + beta_c, f any activation of the family
+    (param: LeakyReLU slope or Swish alpha)."""
+    _need_cuda(x)
+    shape = _affine_shape(x, layout)
+    _chan_params(shape[1], gamma, beta)
+    y = torch.empty_like(x) if out is None else out
+    _need_cuda(y)
+    st = _capi.lib().mea_affine_act_fwd(_act_id(act), _dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape),
+                                         x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), float(param),
+                                         y.data_ptr(), _stream(x))
+    _capi.check("mea_affine_act_fwd", st)
+    return y
+
+
+def affine_act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+                   param: float = 1.0, layout: str = "nhwc", out: torch.Tensor | None = None,
+                   dgamma: torch.Tensor | None = None, dbeta: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None):
+    """Returns (dx, dgamma, dbeta); z and f'(z) are recomputed from x."""
+    _need_cuda(x, dy)
+    if dy.dtype != x.dtype or dy.shape != x.shape:
+        raise ValueError("dy must match x in dtype and shape")
+    shape = _affine_shape(x, layout)
+    C = shape[1]
+    _chan_params(C, gamma, beta)
+    dx = torch.empty_like(x) if out is None else out
+    dg = torch.empty(C, dtype=torch.float32, device=x.device) if dgamma is None else dgamma
+    db = torch.empty(C, dtype=torch.float32, device=x.device) if dbeta is None else dbeta
+    _need_cuda(dx, dg, db)
+    need = affine_act_bwd_workspace_bytes(x.dtype, layout, shape)
+    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    st = _capi.lib().mea_affine_act_bwd(_act_id(act), _dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape),
+                                         x.data_ptr(), dy.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                         float(param), dx.data_ptr(), dg.data_ptr(), db.data_ptr(), ws.data_ptr(),
+                                         ws.numel() * ws.element_size(), _stream(x))
+    _capi.check("mea_affine_act_bwd", st)
+    return dx, dg, db
+
+
+def swish_channel_fwd(x: torch.Tensor, alpha: torch.Tensor, layout: str = "nchw",
+                      out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = x Sigmoid(alpha_c x), alpha fp32 [C]."""
+    _need_cuda(x)
+    shape = _affine_shape(x, layout)
+    _chan_params(shape[1], alpha)
+    y = torch.empty_like(x) if out is None else out
+    _need_cuda(y)
+    st = _capi.lib().mea_swish_channel_fwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
+                                            alpha.data_ptr(), y.data_ptr(), _stream(x))
+    _capi.check("mea_swish_channel_fwd", st)
+    return y
+
+
+def swish_channel_bwd(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, layout: str = "nchw",
+                      out: torch.Tensor | None = None, dalpha: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None):
+    """Returns (dx, dalpha); the sigmoid is recomputed from x."""
+    _need_cuda(x, dy)
+    if dy.dtype != x.dtype or dy.shape != x.shape:
+        raise ValueError("dy must match x in dtype and shape")
+    shape = _affine_shape(x, layout)
+    C = shape[1]
+    _chan_params(C, alpha)
+    dx = torch.empty_like(x) if out is None else out
+    da = torch.empty(C, dtype=torch.float32, device=x.device) if dalpha is None else dalpha
+    _need_cuda(dx, da)
+    need = swish_channel_bwd_workspace_bytes(x.dtype, layout, shape)
+    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    st = _capi.lib().mea_swish_channel_bwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
+                                            dy.data_ptr(), alpha.data_ptr(), dx.data_ptr(), da.data_ptr(),
+                                            ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
+    _capi.check("mea_swish_channel_bwd", st)
+    return dx, da
 
 
 # ---------------------------------------------------------------- autograd
@@ -278,3 +382,67 @@ class MemoryEfficientAffineSwish(torch.nn.Module):
 
     def forward(self, x):
         return AffineSwishFunction.apply(x, self.gamma, self.beta, self.layout)
+
+
+class AffineActFunction(torch.autograd.Function):
+    """Fused per-channel affine + activation that saves only x (and gamma, beta)."""
+
+    @staticmethod
+    def forward(ctx, x, gamma, beta, act: str, param: float, layout: str):
+        x = x.contiguous()
+        y = affine_act_fwd(act, x, gamma, beta, param, layout)
+        ctx.act, ctx.param, ctx.layout = act, param, layout
+        ctx.save_for_backward(x, gamma, beta)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, gamma, beta = ctx.saved_tensors
+        dx, dg, db = affine_act_bwd(ctx.act, x, dy.contiguous(), gamma, beta, ctx.param, ctx.layout)
+        return dx, dg, db, None, None, None
+
+
+class MemoryEfficientAffineActivation(torch.nn.Module):
+    """y = f(gamma_c x + beta_c) for any activation of the family, with
+    learnable fp32 gamma, beta (a folded batch norm or a per-channel scale)."""
+
+    def __init__(self, channels: int, act: str = "swish", param: float | None = None, layout: str = "nhwc"):
+        super().__init__()
+        _act_id(act)
+        self.act, self.layout = act, layout
+        self.param = (0.01 if act == "leaky_relu" else 1.0) if param is None else float(param)
+        self.gamma = torch.nn.Parameter(torch.ones(channels, dtype=torch.float32))
+        self.beta = torch.nn.Parameter(torch.zeros(channels, dtype=torch.float32))
+
+    def forward(self, x):
+        return AffineActFunction.apply(x, self.gamma, self.beta, self.act, self.param, self.layout)
+
+
+class SwishChannelFunction(torch.autograd.Function):
+    """Swish with one alpha per channel that saves only x (and alpha)."""
+
+    @staticmethod
+    def forward(ctx, x, alpha, layout: str):
+        x = x.contiguous()
+        y = swish_channel_fwd(x, alpha, layout)
+        ctx.layout = layout
+        ctx.save_for_backward(x, alpha)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, alpha = ctx.saved_tensors
+        dx, da = swish_channel_bwd(x, dy.contiguous(), alpha, ctx.layout)
+        return dx, (da if ctx.needs_input_grad[1] else None), None
+
+
+class MemoryEfficientChannelSwish(torch.nn.Module):
+    """Swish x Sigmoid(alpha_c x) with a learnable fp32 alpha per channel."""
+
+    def __init__(self, channels: int, alpha: float = 1.0, layout: str = "nchw"):
+        super().__init__()
+        self.layout = layout
+        self.alpha = torch.nn.Parameter(torch.full((channels,), float(alpha), dtype=torch.float32))
+
+    def forward(self, x):
+        return SwishChannelFunction.apply(x, self.alpha, self.layout)

@@ -59,14 +59,25 @@ def step_bytes(n: int, dtype: str) -> int:
 
 
 def affine_fwd_bytes(n: int, dtype: str, channels: int) -> int:
-    """Fused affine + Swish forward: x in, y out, plus gamma and beta (fp32)."""
+    """Fused affine + activation forward: x in, y out, plus gamma and beta (fp32)."""
     return 2 * tensor_bytes(n, dtype) + 2 * 4 * channels
 
 
 def affine_bwd_bytes(n: int, dtype: str, channels: int) -> int:
-    """Fused affine + Swish backward: x, dy in, dx out, gamma, beta in,
+    """Fused affine + activation backward: x, dy in, dx out, gamma, beta in,
     dgamma, dbeta out (fp32)."""
     return 3 * tensor_bytes(n, dtype) + 4 * 4 * channels
+
+
+def channel_swish_fwd_bytes(n: int, dtype: str, channels: int) -> int:
+    """Swish with a per-channel alpha, forward: x in, y out, alpha in (fp32)."""
+    return 2 * tensor_bytes(n, dtype) + 4 * channels
+
+
+def channel_swish_bwd_bytes(n: int, dtype: str, channels: int) -> int:
+    """Swish with a per-channel alpha, backward: x, dy in, dx out, alpha in,
+    dalpha out (fp32)."""
+    return 3 * tensor_bytes(n, dtype) + 2 * 4 * channels
 
 
 def saved_bytes_per_layer(n: int, dtype: str, naive: bool = False) -> int:

@@ -64,6 +64,114 @@ mea_status_t check_shape(const int64_t *shape, int64_t *n)
     return MEA_OK;
 }
 
+// Shared by the per-channel entry points.
+size_t chan_ws_bytes(int kind, int dtype, int layout, const int64_t *shape)
+{
+    int64_t n = 0;
+    if (!valid_dtype(dtype) || (layout != MEA_NCHW && layout != MEA_NHWC)) return 0;
+    char saved[sizeof(g_err)];
+    __builtin_memcpy(saved, g_err, sizeof(g_err));
+    const bool ok = check_shape(shape, &n) == MEA_OK;
+    __builtin_memcpy(g_err, saved, sizeof(g_err));
+    if (!ok) return 0;
+    return kind == 0 ? mea::affine_bwd_workspace_bytes(dtype, layout, shape[0], shape[1], shape[2], shape[3])
+                     : mea::channel_swish_bwd_workspace_bytes(dtype, layout, shape[0], shape[1], shape[2], shape[3]);
+}
+
+// kind 0: affine + activation (p0 = gamma, p1 = beta); kind 1: Swish with a
+// per-channel alpha (p0 = alpha).
+mea_status_t chan_fwd(int kind, const char *name, int act, int dtype, int layout, const int64_t *shape,
+                      const void *x, const float *p0, const float *p1, float param, void *y, mea_stream_t stream)
+{
+    clear_error();
+    if (kind == 0 && !valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", dtype);
+    if (layout != MEA_NCHW && layout != MEA_NHWC)
+        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", layout);
+    int64_t n = 0;
+    mea_status_t st = check_shape(shape, &n);
+    if (st != MEA_OK) return st;
+    if (n == 0) return MEA_OK;
+    if (!x || !y || !p0 || (kind == 0 && !p1))
+        return fail(MEA_ERR_INVALID_ARG, kind == 0 ? "x, y, gamma or beta is NULL" : "x, y or alpha is NULL");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (overlaps(x, bytes, y, bytes))
+        return fail(MEA_ERR_INVALID_ARG, "y overlaps x (x is the saved tensor; the forward keeps it intact)");
+    mea::AffineLaunch l{};
+    l.act = act;
+    l.param = param;
+    l.dtype = dtype;
+    l.layout = layout;
+    l.N = shape[0];
+    l.C = shape[1];
+    l.H = shape[2];
+    l.W = shape[3];
+    l.x = x;
+    l.gamma = p0;
+    l.beta = p1;
+    l.out = y;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = kind == 0 ? mea::launch_affine_fwd(l) : mea::launch_channel_swish_fwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, name);
+}
+
+mea_status_t chan_bwd(int kind, const char *name, int act, int dtype, int layout, const int64_t *shape,
+                      const void *x, const void *dy, const float *p0, const float *p1, float param, void *dx,
+                      float *d0, float *d1, void *workspace, size_t ws_bytes, mea_stream_t stream)
+{
+    clear_error();
+    if (kind == 0 && !valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", dtype);
+    if (layout != MEA_NCHW && layout != MEA_NHWC)
+        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", layout);
+    int64_t n = 0;
+    mea_status_t st = check_shape(shape, &n);
+    if (st != MEA_OK) return st;
+    if (shape[1] == 0) return MEA_OK;                 // no channels: nothing to write
+    if (kind == 0 && (!d0 || !d1 || !p0 || !p1))
+        return fail(MEA_ERR_INVALID_ARG, "gamma, beta, dgamma or dbeta is NULL");
+    if (kind == 1 && (!d0 || !p0)) return fail(MEA_ERR_INVALID_ARG, "alpha or dalpha is NULL");
+    if (n > 0 && (!x || !dy || !dx)) return fail(MEA_ERR_INVALID_ARG, "x, dy or dx is NULL");
+    const size_t need = chan_ws_bytes(kind, dtype, layout, shape);
+    if (!workspace || ws_bytes < need)
+        return fail(MEA_ERR_WORKSPACE, "%s needs %zu bytes of workspace, got %zu%s", name, need, ws_bytes,
+                    workspace ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+        return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    const size_t bytes = (size_t)n * dtype_bytes(dtype);
+    if (n > 0 && (partial_overlap(dx, dy, bytes) || partial_overlap(dx, x, bytes)))
+        return fail(MEA_ERR_INVALID_ARG, "dx partially overlaps x or dy (only exact aliasing is allowed)");
+    const size_t cbytes = (size_t)shape[1] * sizeof(float);
+    if (kind == 0 && overlaps(d0, cbytes, d1, cbytes)) return fail(MEA_ERR_INVALID_ARG, "dgamma overlaps dbeta");
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (n == 0) {
+        // An empty batch still defines the parameter gradients: zero.
+        cudaError_t e = cudaMemsetAsync(d0, 0, cbytes, s);
+        if (e == cudaSuccess && kind == 0) e = cudaMemsetAsync(d1, 0, cbytes, s);
+        return e == cudaSuccess ? MEA_OK : cuda_fail(e, name);
+    }
+    mea::AffineLaunch l{};
+    l.act = act;
+    l.param = param;
+    l.dtype = dtype;
+    l.layout = layout;
+    l.N = shape[0];
+    l.C = shape[1];
+    l.H = shape[2];
+    l.W = shape[3];
+    l.x = x;
+    l.dy = dy;
+    l.gamma = p0;
+    l.beta = p1;
+    l.out = dx;
+    l.dgamma = d0;
+    l.dbeta = d1;
+    l.workspace = workspace;
+    l.stream = s;
+    cudaError_t e = kind == 0 ? mea::launch_affine_bwd(l) : mea::launch_channel_swish_bwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, name);
+}
+
 }  // namespace
 
 namespace mea {
@@ -86,7 +194,7 @@ const char *mea_status_string(mea_status_t status)
 
 const char *mea_last_error(void) { return g_err; }
 
-int mea_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+int mea_version(void) { return 1 * 10000 + 1 * 100 + 0; }
 
 mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y, int64_t n, float param,
                          const float *param_dev, mea_stream_t stream)
@@ -161,97 +269,61 @@ mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const 
 
 size_t mea_affine_swish_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4])
 {
-    int64_t n = 0;
-    if (!valid_dtype(dtype) || (layout != MEA_NCHW && layout != MEA_NHWC)) return 0;
-    char saved[sizeof(g_err)];
-    __builtin_memcpy(saved, g_err, sizeof(g_err));
-    const bool ok = check_shape(shape, &n) == MEA_OK;
-    __builtin_memcpy(g_err, saved, sizeof(g_err));
-    if (!ok) return 0;
-    return mea::affine_bwd_workspace_bytes(dtype, layout, shape[0], shape[1], shape[2], shape[3]);
+    return chan_ws_bytes(0, dtype, layout, shape);
 }
 
 mea_status_t mea_affine_swish_fwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
                                   const float *gamma, const float *beta, void *y, mea_stream_t stream)
 {
-    clear_error();
-    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
-    if (layout != MEA_NCHW && layout != MEA_NHWC)
-        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", (int)layout);
-    int64_t n = 0;
-    mea_status_t st = check_shape(shape, &n);
-    if (st != MEA_OK) return st;
-    if (n == 0) return MEA_OK;
-    if (!x || !y || !gamma || !beta) return fail(MEA_ERR_INVALID_ARG, "x, y, gamma or beta is NULL");
-    const size_t bytes = (size_t)n * dtype_bytes(dtype);
-    if (overlaps(x, bytes, y, bytes))
-        return fail(MEA_ERR_INVALID_ARG, "y overlaps x (x is the saved tensor; the forward keeps it intact)");
-    mea::AffineLaunch l{};
-    l.dtype = dtype;
-    l.layout = layout;
-    l.N = shape[0];
-    l.C = shape[1];
-    l.H = shape[2];
-    l.W = shape[3];
-    l.x = x;
-    l.gamma = gamma;
-    l.beta = beta;
-    l.out = y;
-    l.stream = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = mea::launch_affine_fwd(l);
-    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_fwd launch");
+    return chan_fwd(0, "mea_affine_swish_fwd", MEA_SWISH, dtype, layout, shape, x, gamma, beta, 1.f, y, stream);
 }
 
 mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
                                   const void *dy, const float *gamma, const float *beta, void *dx, float *dgamma,
                                   float *dbeta, void *workspace, size_t ws_bytes, mea_stream_t stream)
 {
-    clear_error();
-    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
-    if (layout != MEA_NCHW && layout != MEA_NHWC)
-        return fail(MEA_ERR_INVALID_ARG, "layout = %d is not a mea_layout_t", (int)layout);
-    int64_t n = 0;
-    mea_status_t st = check_shape(shape, &n);
-    if (st != MEA_OK) return st;
-    if (shape[1] == 0) return MEA_OK;                 // no channels: nothing to write
-    if (!dgamma || !dbeta || !gamma || !beta)
-        return fail(MEA_ERR_INVALID_ARG, "gamma, beta, dgamma or dbeta is NULL");
-    if (n > 0 && (!x || !dy || !dx)) return fail(MEA_ERR_INVALID_ARG, "x, dy or dx is NULL");
-    const size_t need = mea_affine_swish_bwd_workspace_bytes(dtype, layout, shape);
-    if (!workspace || ws_bytes < need)
-        return fail(MEA_ERR_WORKSPACE, "affine backward needs %zu bytes of workspace, got %zu%s", need, ws_bytes,
-                    workspace ? "" : " (NULL)");
-    if (reinterpret_cast<uintptr_t>(workspace) & 15u)
-        return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
-    const size_t bytes = (size_t)n * dtype_bytes(dtype);
-    if (n > 0 && (partial_overlap(dx, dy, bytes) || partial_overlap(dx, x, bytes)))
-        return fail(MEA_ERR_INVALID_ARG, "dx partially overlaps x or dy (only exact aliasing is allowed)");
-    const size_t cbytes = (size_t)shape[1] * sizeof(float);
-    if (overlaps(dgamma, cbytes, dbeta, cbytes)) return fail(MEA_ERR_INVALID_ARG, "dgamma overlaps dbeta");
-    if (n == 0) {
-        // An empty batch still defines the parameter gradients: zero.
-        cudaError_t e = cudaMemsetAsync(dgamma, 0, cbytes, reinterpret_cast<cudaStream_t>(stream));
-        if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, cbytes, reinterpret_cast<cudaStream_t>(stream));
-        return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_bwd zero fill");
-    }
-    mea::AffineLaunch l{};
-    l.dtype = dtype;
-    l.layout = layout;
-    l.N = shape[0];
-    l.C = shape[1];
-    l.H = shape[2];
-    l.W = shape[3];
-    l.x = x;
-    l.dy = dy;
-    l.gamma = gamma;
-    l.beta = beta;
-    l.out = dx;
-    l.dgamma = dgamma;
-    l.dbeta = dbeta;
-    l.workspace = workspace;
-    l.stream = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = mea::launch_affine_bwd(l);
-    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_affine_swish_bwd launch");
+    return chan_bwd(0, "mea_affine_swish_bwd", MEA_SWISH, dtype, layout, shape, x, dy, gamma, beta, 1.f, dx, dgamma,
+                    dbeta, workspace, ws_bytes, stream);
+}
+
+size_t mea_affine_act_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4])
+{
+    return chan_ws_bytes(0, dtype, layout, shape);
+}
+
+mea_status_t mea_affine_act_fwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4],
+                                const void *x, const float *gamma, const float *beta, float param, void *y,
+                                mea_stream_t stream)
+{
+    return chan_fwd(0, "mea_affine_act_fwd", act, dtype, layout, shape, x, gamma, beta, param, y, stream);
+}
+
+mea_status_t mea_affine_act_bwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4],
+                                const void *x, const void *dy, const float *gamma, const float *beta, float param,
+                                void *dx, float *dgamma, float *dbeta, void *workspace, size_t ws_bytes,
+                                mea_stream_t stream)
+{
+    return chan_bwd(0, "mea_affine_act_bwd", act, dtype, layout, shape, x, dy, gamma, beta, param, dx, dgamma, dbeta,
+                    workspace, ws_bytes, stream);
+}
+
+size_t mea_swish_channel_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4])
+{
+    return chan_ws_bytes(1, dtype, layout, shape);
+}
+
+mea_status_t mea_swish_channel_fwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
+                                   const float *alpha, void *y, mea_stream_t stream)
+{
+    return chan_fwd(1, "mea_swish_channel_fwd", MEA_SWISH, dtype, layout, shape, x, alpha, nullptr, 1.f, y, stream);
+}
+
+mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
+                                   const void *dy, const float *alpha, void *dx, float *dalpha, void *workspace,
+                                   size_t ws_bytes, mea_stream_t stream)
+{
+    return chan_bwd(1, "mea_swish_channel_bwd", MEA_SWISH, dtype, layout, shape, x, dy, alpha, nullptr, 1.f, dx,
+                    dalpha, nullptr, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

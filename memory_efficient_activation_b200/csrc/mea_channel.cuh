@@ -1,0 +1,505 @@
+// mea_channel.cuh -- per-channel elementwise kernels (fused affine + any
+// activation; Swish with one alpha per channel), forward and backward.
+//
+// A per-channel operation Op supplies the arithmetic; the kernels here supply
+// the data movement and the deterministic per-channel reductions.  Op has:
+//   NR                     reductions per channel (affine: dgamma, dbeta;
+//                          channel alpha: dalpha)
+//   K  kcoef(ChanArgs)     constants shared by every channel
+//   Ch load(ChanArgs, c)   constants of channel c
+//   f<P>, f_tail<P>, is_tail      forward value, deep-tail recompute, test
+//   bwd<P>(x, dy, ..., o, t)      backward main path -> raw results o, t
+//   bwd_tail<P>(...)              deep-tail recompute of o, t
+//   finish(x, o, t, ch, acc[NR])  dx, and adds the channel's reduction terms
+//
+// Only x is kept between the passes; the backward recomputes everything from
+// it (the save-input-only idea of "Memory efficient Swish", section "What
+// makes this implementation save GPU memory?", applied to the per-channel op
+// that precedes the activation in EfficientNet-style blocks).
+//
+// NHWC fast path (C a multiple of 4, aligned pointers): a block is a
+// multiple of G = C / 4 threads, so every thread keeps the same 4 channels,
+// with their constants in registers.  The forward handles one tile per block.
+// The backward runs a fixed grid (a function of the shape) that walks the
+// tiles with register prefetch, keeps fp64 per-channel sums per thread,
+// folds them per block in row order and writes one row of fp64 partials per
+// block; a second kernel adds each channel's column in block order.  So the
+// reductions are bitwise reproducible on any device.
+//
+// Plane path (NCHW, and NHWC shapes the fast path does not take): block
+// (c, s) owns channel c and the s-th slice of the batch; for NCHW it streams
+// the contiguous H W planes of that channel (16-byte vectors when H W is a
+// multiple of the vector width and the pointers are aligned), and the last
+// block to finish (atomic ticket) adds the per-block partials in order.
+#pragma once
+
+#include <cstdint>
+
+#include "mea_device.cuh"
+#include "mea_internal.h"
+#include "mea_math.cuh"
+
+namespace mea {
+
+constexpr int kNhwcMaxThreads = 512;
+constexpr int kNhwcTargetThreads = 256;
+constexpr int kColsumThreads = 256;
+constexpr int kNhwcBwdGridCap = 888;     // 148 x 6
+// Register cap of the NHWC backward.  Registers are allocated per warp in
+// granules of 8 per thread, so with 288-thread blocks (C = 144: lcm(36, 32))
+// 72 registers keep three blocks resident per SM and 56 keep four.
+#ifndef MEA_NHWC_BWD_MAXREGS
+#define MEA_NHWC_BWD_MAXREGS 72
+#endif
+constexpr int kNhwcBwdMaxRegs = MEA_NHWC_BWD_MAXREGS;
+constexpr int kPlaneThreads = 256;
+constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks
+
+// Parameter arrays and scalar of a per-channel operation (device pointers).
+struct ChanArgs {
+    const float *p0;   // gamma (affine) or alpha (channel Swish), [C]
+    const float *p1;   // beta (affine), [C]; unused otherwise
+    float scalar;      // activation parameter (LeakyReLU slope, Swish alpha)
+};
+
+// Threads per NHWC block: lcm(G, 32) times the largest m that keeps it at
+// or below kNhwcTargetThreads (at least one lcm), where G = C / 4 is the
+// number of channel groups.  A block is then whole warps and a multiple of
+// G, so every thread of a block keeps the same channels.  Returns 0 when
+// lcm(G, 32) exceeds kNhwcMaxThreads (the NHWC fast path is then not taken).
+inline int nhwc_threads(int groups)
+{
+    int a = groups, b = 32;
+    while (b) {
+        int t = a % b;
+        a = b;
+        b = t;
+    }
+    const long lcm = (long)groups / a * 32;
+    if (lcm > kNhwcMaxThreads) return 0;
+    long m = kNhwcTargetThreads / lcm;
+    if (m < 1) m = 1;
+    return (int)(lcm * m);
+}
+
+inline int plane_slices(int64_t N, int64_t C)
+{
+    int64_t s = (kPlaneBlocksTarget + C - 1) / C;
+    if (s > N) s = N;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+// ------------------------------------------------------------ load units
+
+// VE elements per thread per access (bf16: 4 elements in 8 bytes; fp32: 4 in
+// 16 bytes).  Few channels per thread keep the per-thread constants and
+// partial sums in few registers, which is what sets the occupancy here.
+template <typename T, int VE>
+struct Unit;
+
+template <>
+struct Unit<Bf16, 4> {
+    using W = uint2;
+    static constexpr bool P = false;
+    static __device__ __forceinline__ W load(const void *p, int64_t i)
+    {
+        W r;
+        asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+            : "=r"(r.x), "=r"(r.y)
+            : "l"(static_cast<const uint2 *>(p) + i));
+        return r;
+    }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const W &w)
+    {
+        asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(static_cast<uint2 *>(p) + i), "r"(w.x), "r"(w.y)
+                     : "memory");
+    }
+    static __device__ __forceinline__ void unpack(const W &w, float (&f)[4])
+    {
+        f[0] = __uint_as_float(w.x << 16);
+        f[1] = __uint_as_float(w.x & 0xffff0000u);
+        f[2] = __uint_as_float(w.y << 16);
+        f[3] = __uint_as_float(w.y & 0xffff0000u);
+    }
+    static __device__ __forceinline__ W pack(const float (&f)[4])
+    {
+        return make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+    }
+};
+
+template <>
+struct Unit<float, 4> {
+    using W = uint4;
+    static constexpr bool P = true;
+    static __device__ __forceinline__ W load(const void *p, int64_t i) { return ld_nc_v4(static_cast<const uint4 *>(p) + i); }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const W &w) { st_v4(static_cast<uint4 *>(p) + i, w); }
+    static __device__ __forceinline__ void unpack(const W &w, float (&f)[4]) { Store<float>::unpack(w, f); }
+    static __device__ __forceinline__ W pack(const float (&f)[4]) { return Store<float>::pack(f); }
+};
+
+// NHWC launch shape per storage dtype: elements per thread access (VE) and
+// accesses per thread (U) for the forward and the backward (measured on B200
+// at [128, 56, 56, 144] bf16 against 8 / 16-byte units, 1-16 accesses,
+// tile-per-block and fixed-grid backward variants).
+template <typename T>
+struct NhwcCfg;
+#ifndef MEA_NHWC_BWD_U
+#define MEA_NHWC_BWD_U 2
+#endif
+template <>
+struct NhwcCfg<Bf16> {
+    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U;
+};
+template <>
+struct NhwcCfg<float> {
+    static constexpr int VE = 4, U_FWD = 8, U_BWD = MEA_NHWC_BWD_U;
+};
+
+// ------------------------------------------------------------ NHWC kernels
+
+// Forward: one tile of blockDim.x * U units per block (as the plain
+// activation kernels).
+template <class Op, typename T, int U, int VE>
+__global__ void __launch_bounds__(kNhwcMaxThreads)
+chan_nhwc_fwd_kernel(const void *__restrict__ x, ChanArgs ca, void *__restrict__ out, int64_t nunits, int groups)
+{
+    using L = Unit<T, VE>;
+    constexpr bool P = L::P;
+    const int tid = threadIdx.x;
+    const int g = tid % groups;
+    pdl_wait();
+    const typename Op::K k = Op::kcoef(ca);
+    typename Op::Ch ch[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) ch[j] = Op::load(ca, g * VE + j);
+    const int64_t base = (int64_t)blockIdx.x * blockDim.x * U + tid;
+    typename L::W xv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) xv[u] = L::load(x, i);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) {
+            float xf[VE], of[VE];
+            L::unpack(xv[u], xf);
+            bool tail = false;
+#pragma unroll
+            for (int j = 0; j < VE; ++j) of[j] = Op::template f<P>(xf[j], k, ch[j], tail);
+            if (tail) {
+#pragma unroll
+                for (int j = 0; j < VE; ++j)
+                    if (Op::is_tail(xf[j], k, ch[j])) of[j] = Op::template f_tail<P>(xf[j], k, ch[j]);
+            }
+            L::store(out, i, L::pack(of));
+        }
+    }
+    pdl_trigger();
+}
+
+// Backward: a fixed grid of blocks (a function of the shape only) walks the
+// tiles of blockDim.x * U units with a grid stride, loading the next tile's
+// x and dy before working on the current one.  Each thread keeps the same VE
+// channels throughout; its reduction terms go from fp32 per tile into fp64
+// registers.  At the end the block folds its threads' sums per channel in
+// row order (fp64, through shared memory) and writes one row of partials:
+//   partials[blockIdx.x * NR C + r * C + c].
+template <class Op, typename T, int U, int VE>
+__global__ void __maxnreg__(kNhwcBwdMaxRegs)
+chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca, void *__restrict__ dx,
+                     int64_t nunits, int groups, int C, double *__restrict__ partials)
+{
+    using L = Unit<T, VE>;
+    constexpr bool P = L::P;
+    constexpr int NR = Op::NR;
+    const int tid = threadIdx.x;
+    const int g = tid % groups;
+    pdl_wait();
+    const typename Op::K k = Op::kcoef(ca);
+    typename Op::Ch ch[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) ch[j] = Op::load(ca, g * VE + j);
+    // fp64 running sums, one slot per (reduction, channel of the thread,
+    // thread): each thread owns its slots, so no synchronisation until the
+    // fold.  Kept in shared memory rather than registers, which leaves room
+    // for four blocks of 288 threads per SM.
+    extern __shared__ double acc[];   // NR VE * blockDim.x doubles
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int j = 0; j < VE; ++j) acc[(r * VE + j) * blockDim.x + tid] = 0.0;
+    const int64_t tile = (int64_t)blockDim.x * U;
+    const int64_t stride = (int64_t)gridDim.x * tile;
+    int64_t base = (int64_t)blockIdx.x * tile + tid;
+    typename L::W xv[U], gv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + (int64_t)u * blockDim.x;
+        if (i < nunits) {
+            xv[u] = L::load(x, i);
+            gv[u] = L::load(dy, i);
+        }
+    }
+    for (; base < nunits; base += stride) {
+        typename L::W xn[U], gn[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + stride + (int64_t)u * blockDim.x;
+            if (i < nunits) {
+                xn[u] = L::load(x, i);
+                gn[u] = L::load(dy, i);
+            }
+        }
+        float accf[VE][NR];
+#pragma unroll
+        for (int j = 0; j < VE; ++j)
+#pragma unroll
+            for (int r = 0; r < NR; ++r) accf[j][r] = 0.f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + (int64_t)u * blockDim.x;
+            if (i < nunits) {
+                float xf[VE], gf[VE], o[VE], t[VE], of[VE];
+                L::unpack(xv[u], xf);
+                L::unpack(gv[u], gf);
+                bool tail = false;
+#pragma unroll
+                for (int j = 0; j < VE; ++j) Op::template bwd<P>(xf[j], gf[j], k, ch[j], tail, o[j], t[j]);
+                if (tail) {
+#pragma unroll
+                    for (int j = 0; j < VE; ++j)
+                        if (Op::is_tail(xf[j], k, ch[j])) Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], t[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < VE; ++j) of[j] = Op::finish(xf[j], o[j], t[j], ch[j], accf[j]);
+                L::store(dx, i, L::pack(of));
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int j = 0; j < VE; ++j) acc[(r * VE + j) * blockDim.x + tid] += (double)accf[j][r];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            xv[u] = xn[u];
+            gv[u] = gn[u];
+        }
+    }
+    pdl_trigger();
+    __syncthreads();
+    const double *red = acc;
+    const int rows = blockDim.x / groups;
+    for (int o = tid; o < NR * C; o += blockDim.x) {
+        const int r = o / C, c = o % C;
+        const double *col = red + (r * VE + c % VE) * blockDim.x + c / VE;
+        double s = 0.0;
+        for (int q = 0; q < rows; ++q) s += col[q * groups];
+        partials[(int64_t)blockIdx.x * NR * C + o] = s;
+    }
+}
+
+// Output o (r * C + c) = sum over the nb rows of partials, column o, in
+// fp64: thread t adds rows t, t + kColsumThreads, ... in order, then a fixed
+// block-wide tree.  One block per output; r = 0 goes to out0, r = 1 to out1.
+template <int NR>
+__global__ void __launch_bounds__(kColsumThreads)
+chan_colsum_kernel(const double *__restrict__ partials, int nb, int C, float *__restrict__ out0,
+                   float *__restrict__ out1)
+{
+    __shared__ double red[32];
+    const int o = blockIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    double s = 0.0;
+    for (int b = threadIdx.x; b < nb; b += kColsumThreads) s += partials[(int64_t)b * NR * C + o];
+    s = block_sum(s, red);
+    if (threadIdx.x == 0) {
+        if (o < C) out0[o] = (float)s;
+        else out1[o - C] = (float)s;
+    }
+}
+
+// ------------------------------------------------------------ plane path
+
+template <class Op, typename T, int MODE, bool NHWC>
+__global__ void __launch_bounds__(kPlaneThreads)
+chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca, void *__restrict__ out,
+                  int64_t N, int64_t C, int64_t HW, int slices, int vec_ok, float *__restrict__ out0,
+                  float *__restrict__ out1, void *__restrict__ ws)
+{
+    using S = Store<T>;
+    constexpr int V = S::V;
+    constexpr bool P = S::P;
+    constexpr int NR = Op::NR;
+    const int64_t c = blockIdx.x / slices;
+    const int s = blockIdx.x % slices;
+    const int64_t n0 = (int64_t)s * N / slices, n1 = (int64_t)(s + 1) * N / slices;
+    pdl_wait();
+    const typename Op::K k = Op::kcoef(ca);
+    const typename Op::Ch ch = Op::load(ca, (int)c);
+    double acc[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) acc[r] = 0.0;
+
+    auto one = [&](float xi, float gi, float &res) {
+        bool tail = false;
+        if constexpr (MODE == 0) {
+            res = Op::template f<P>(xi, k, ch, tail);
+            if (tail) res = Op::template f_tail<P>(xi, k, ch);
+        } else {
+            float o, t;
+            Op::template bwd<P>(xi, gi, k, ch, tail, o, t);
+            if (tail) Op::template bwd_tail<P>(xi, gi, k, ch, o, t);
+            float tmp[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) tmp[r] = 0.f;
+            res = Op::finish(xi, o, t, ch, tmp);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) acc[r] += (double)tmp[r];
+        }
+    };
+
+    if (!NHWC && vec_ok) {
+        // NCHW planes are contiguous and each starts on a 16-byte boundary.
+        const int64_t hwv = HW / V;
+        const int64_t total = (n1 - n0) * hwv;
+        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
+            const int64_t n = n0 + q / hwv;
+            const int64_t vi = (n * C + c) * hwv + q % hwv;
+            float xf[V], gf[V], of[V];
+            S::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+            if constexpr (MODE == 1) S::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vi), gf);
+#pragma unroll
+            for (int j = 0; j < V; ++j) one(xf[j], MODE == 1 ? gf[j] : 0.f, of[j]);
+            st_v4(static_cast<uint4 *>(out) + vi, S::pack(of));
+        }
+    } else {
+        const int64_t total = (n1 - n0) * HW;
+        for (int64_t p = threadIdx.x; p < total; p += blockDim.x) {
+            const int64_t n = n0 + p / HW, hw = p % HW;
+            const int64_t i = NHWC ? (n * HW + hw) * C + c : (n * C + c) * HW + hw;
+            const float xi = S::load1(x, i);
+            const float gi = MODE == 1 ? S::load1(dy, i) : 0.f;
+            float o;
+            one(xi, gi, o);
+            S::store1(out, i, o);
+        }
+    }
+    pdl_trigger();
+    if constexpr (MODE == 0) {
+        return;
+    } else {
+        __shared__ double red[32];
+        unsigned int *ticket = static_cast<unsigned int *>(ws);
+        double *partials = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            const double b = block_sum(acc[r], red);
+            if (threadIdx.x == 0) partials[(r * C + c) * slices + s] = b;
+        }
+        if (!last_block_done(ticket)) return;
+        for (int64_t o = threadIdx.x; o < NR * C; o += blockDim.x) {
+            double t = 0.0;
+            for (int q = 0; q < slices; ++q) t += __ldcg(partials + o * slices + q);
+            if (o < C) out0[o] = (float)t;
+            else out1[o - C] = (float)t;
+        }
+    }
+}
+
+// ------------------------------------------------------------ launchers
+
+inline int64_t nhwc_blocks(int64_t nunits, int threads, int U)
+{
+    const int64_t per = (int64_t)threads * U;
+    const int64_t nb = (nunits + per - 1) / per;
+    return nb < 1 ? 1 : nb;
+}
+
+// Backward grid: one block per tile up to kNhwcBwdGridCap blocks (a function
+// of the shape only, so the summation order is fixed).
+inline int nhwc_bwd_grid(int64_t nunits, int threads, int U)
+{
+    const int64_t nb = nhwc_blocks(nunits, threads, U);
+    return (int)(nb < kNhwcBwdGridCap ? nb : kNhwcBwdGridCap);
+}
+
+template <typename T>
+inline bool nhwc_fast(const AffineLaunch &a)
+{
+    constexpr int VE = NhwcCfg<T>::VE;
+    constexpr int bytes = VE * (sizeof(T) == 4 ? 4 : 2);
+    uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
+    if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
+    return a.layout == 1 && a.C % VE == 0 && nhwc_threads((int)(a.C / VE)) > 0 && (al % bytes) == 0;
+}
+
+// Workspace of the backward of a per-channel operation with nr reductions:
+// the larger of the NHWC fast path's and the plane path's needs (pointer
+// alignment, which decides between them, is not known here).
+inline size_t chan_bwd_workspace_bytes(int nr, int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W)
+{
+    const int VE = dtype == kBF16 ? NhwcCfg<Bf16>::VE : NhwcCfg<float>::VE;
+    const int U = dtype == kBF16 ? NhwcCfg<Bf16>::U_BWD : NhwcCfg<float>::U_BWD;
+    size_t plane = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)plane_slices(N, C);
+    if (layout == 1 && C % VE == 0 && nhwc_threads((int)(C / VE)) > 0) {
+        const int threads = nhwc_threads((int)(C / VE));
+        const int64_t nunits = N * C * H * W / VE;
+        size_t fast = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)nhwc_bwd_grid(nunits, threads, U);
+        return fast > plane ? fast : plane;
+    }
+    return plane;
+}
+
+template <class Op, typename T, int MODE>
+cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out0, float *out1)
+{
+    constexpr int V = Store<T>::V;
+    constexpr int NR = Op::NR;
+    const int64_t HW = a.H * a.W;
+    const int64_t n = a.N * a.C * HW;
+    if (nhwc_fast<T>(a)) {
+        constexpr int VE = NhwcCfg<T>::VE;
+        const int groups = (int)(a.C / VE);
+        const int threads = nhwc_threads(groups);
+        const int64_t nunits = n / VE;
+        if (MODE == 0) {
+            constexpr int U = NhwcCfg<T>::U_FWD;
+            const int64_t nb = nhwc_blocks(nunits, threads, U);
+            if (nb > 0x7fffffff) return cudaErrorInvalidConfiguration;
+            return launch_pdl(chan_nhwc_fwd_kernel<Op, T, U, VE>, dim3((unsigned)nb), dim3(threads), 0, a.stream, a.x,
+                              ca, a.out, nunits, groups);
+        }
+        constexpr int U = NhwcCfg<T>::U_BWD;
+        auto kernel = chan_nhwc_bwd_kernel<Op, T, U, VE>;
+        const int nb = nhwc_bwd_grid(nunits, threads, U);
+        double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+        const size_t smem = sizeof(double) * NR * VE * threads;
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             (int)cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess && smem > 48 * 1024)
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(kernel, dim3((unsigned)nb), dim3(threads), smem, a.stream, a.x, a.dy, ca, a.out, nunits, groups,
+                       (int)a.C, partials);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(chan_colsum_kernel<NR>, dim3((unsigned)(NR * a.C)), dim3(kColsumThreads), 0, a.stream,
+                          partials, nb, (int)a.C, out0, out1);
+    }
+    uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
+    if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
+    const int vec_ok = a.layout == 0 && HW % V == 0 && (al & 15u) == 0;
+    const int slices = plane_slices(a.N, a.C);
+    const int64_t grid = a.C * slices;
+    if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (a.layout == 1)
+        return launch_pdl(chan_plane_kernel<Op, T, MODE, true>, dim3((unsigned)grid), dim3(kPlaneThreads), 0,
+                          a.stream, a.x, a.dy, ca, a.out, a.N, a.C, HW, slices, vec_ok, out0, out1, a.workspace);
+    return launch_pdl(chan_plane_kernel<Op, T, MODE, false>, dim3((unsigned)grid), dim3(kPlaneThreads), 0, a.stream,
+                      a.x, a.dy, ca, a.out, a.N, a.C, HW, slices, vec_ok, out0, out1, a.workspace);
+}
+
+}  // namespace mea

@@ -1,0 +1,73 @@
+// mea_channel_alpha.cu -- Swish with one learnable alpha per channel:
+//
+//   y = x Sigmoid(alpha_c x)
+//   dx = dy (s + alpha_c x s Sigmoid(-alpha_c x)),  s = Sigmoid(alpha_c x)
+//   dalpha_c = sum dy x^2 s Sigmoid(-alpha_c x)   (over all N H W positions)
+//
+// The per-channel generalisation of the scalar learnable alpha (the Swish
+// page's module carries alpha; its gradient in alpha is the derivative of
+// sum(dy Swish) in alpha).  Data movement and the deterministic reductions
+// are the per-channel kernels of mea_channel.cuh; this file supplies the
+// arithmetic (ChannelSwishOp) and the dispatch over storage dtype.
+#include "mea_channel.cuh"
+
+namespace mea {
+
+struct ChannelSwishOp {
+    static constexpr int NR = 1;   // dalpha
+    struct K {
+    };
+    using Ch = Coef;               // Swish constants of the channel's alpha
+    static __device__ __forceinline__ K kcoef(const ChanArgs &) { return K{}; }
+    static __device__ __forceinline__ Ch load(const ChanArgs &a, int c) { return Swish::coef(__ldg(a.p0 + c)); }
+
+    template <bool P>
+    static __device__ __forceinline__ float f(float x, const K &, const Ch &h, bool &tail)
+    {
+        return Swish::f<P>(x, h, tail);
+    }
+    template <bool P>
+    static __device__ __forceinline__ float f_tail(float x, const K &, const Ch &h)
+    {
+        return Swish::f_tail<P>(x, h);
+    }
+    static __device__ __forceinline__ bool is_tail(float x, const K &, const Ch &h) { return Swish::is_tail(x, h); }
+    // o = dx, t = d alpha term
+    template <bool P>
+    static __device__ __forceinline__ void bwd(float x, float dy, const K &, const Ch &h, bool &tail, float &o,
+                                               float &t)
+    {
+        o = Swish::df_da<P>(x, dy, h, tail, t);
+    }
+    template <bool P>
+    static __device__ __forceinline__ void bwd_tail(float x, float dy, const K &, const Ch &h, float &o, float &t)
+    {
+        o = Swish::df_da_tail<P>(x, dy, h, t);
+    }
+    static __device__ __forceinline__ float finish(float, float o, float t, const Ch &, float (&acc)[NR])
+    {
+        acc[0] += t;
+        return o;
+    }
+};
+
+size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W)
+{
+    return chan_bwd_workspace_bytes(ChannelSwishOp::NR, dtype, layout, N, C, H, W);
+}
+
+cudaError_t launch_channel_swish_fwd(const AffineLaunch &a)
+{
+    const ChanArgs ca{a.gamma, nullptr, 1.f};
+    return a.dtype == kBF16 ? launch_channel<ChannelSwishOp, Bf16, 0>(a, ca, nullptr, nullptr)
+                            : launch_channel<ChannelSwishOp, float, 0>(a, ca, nullptr, nullptr);
+}
+
+cudaError_t launch_channel_swish_bwd(const AffineLaunch &a)
+{
+    const ChanArgs ca{a.gamma, nullptr, 1.f};
+    return a.dtype == kBF16 ? launch_channel<ChannelSwishOp, Bf16, 1>(a, ca, a.dgamma, nullptr)
+                            : launch_channel<ChannelSwishOp, float, 1>(a, ca, a.dgamma, nullptr);
+}
+
+}  // namespace mea

@@ -171,3 +171,26 @@ def affine_swish_nchw(seed: int = 5, shape=(64, 144, 56, 56), dtype: str = "bf16
                     normal(n, 1.0, seed, STREAM_DY, dtype).view(shape),
                     1.0, {"gamma": gamma, "beta": beta, "layout": "nchw",
                           "nchw_shape": (N, C, H, W)})
+
+
+def affine_act_nhwc(act: str, seed: int = 6, shape=AFFINE_NHWC_SHAPE, dtype: str = "bf16") -> Workload:
+    """Fused per-channel affine + any activation of the family, NHWC, with the
+    distributions of the affine + Swish recipe (LeakyReLU slope 0.01, Swish
+    alpha 1)."""
+    w = affine_swish_nhwc(seed=seed, shape=shape, dtype=dtype)
+    w.name = w.name.replace("affine_swish", f"affine_{act}")
+    w.act = act
+    w.param = 0.01 if act == "leaky_relu" else 1.0
+    return w
+
+
+def swish_channel_nchw(seed: int = 7, shape=(64, 144, 56, 56), dtype: str = "f32") -> Workload:
+    """Swish with a learnable alpha per channel, NCHW (N, C, H, W), x ~ N(0, 1.5^2),
+    dy ~ N(0, 1), alpha_c ~ U(0.5, 2) (fp32, one draw per channel)."""
+    N, C, H, W = shape
+    n = N * C * H * W
+    alpha = torch.from_numpy(uniform_f64(C, 0.5, 2.0, seed, STREAM_PARAM)).to(torch.float32)
+    return Workload(f"swish_channel_nchw_{'x'.join(map(str, shape))}", "swish_channel", dtype,
+                    normal(n, 1.5, seed, STREAM_X, dtype).view(shape),
+                    normal(n, 1.0, seed, STREAM_DY, dtype).view(shape),
+                    1.0, {"alpha": alpha, "layout": "nchw", "nchw_shape": (N, C, H, W)})

@@ -47,7 +47,9 @@ def _ordered(bits: np.ndarray) -> np.ndarray:
     return np.where(b & 0x8000, -mag, mag)
 
 
-def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None, scale=None) -> dict:
+def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None, scale=None, alt=None) -> dict:
+    """alt: optional (ref2, scale2) -- an element also passes when it meets
+    the same rule against ref2 (see check)."""
     g_bits = bf16_bits(gpu)
     ref = np.asarray(ref, dtype=np.float64).ravel()
     r_bits = oracle.round_bf16(ref)
@@ -63,10 +65,16 @@ def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None, scale=None) -> d
         cond_ok = np.zeros_like(nan_ok) if scale is None else \
             np.abs(g - ref) <= F32_TOL * np.asarray(scale, dtype=np.float64).ravel()
     ok = (dist <= 1) | nan_ok | tiny_ok | cond_ok
+    alt_ok = np.zeros_like(ok)
+    if alt is not None:
+        alt_ok = bf16_report(gpu, alt[0], floor, alt[1] if scale is not None else None)["ok"]
+        ok = ok | alt_ok
     bad = np.flatnonzero(~ok)
     return {
         "n": ref.size,
         "bad": bad.size,
+        "ok": ok,
+        "alt_only": int(np.sum(alt_ok & ~((dist <= 1) | nan_ok | tiny_ok | cond_ok))),
         "max_ulp": int(dist[~(nan_ok | tiny_ok)].max(initial=0)),
         "cond_only": int(np.sum(cond_ok & (dist > 1))),
         "exact_frac": float(np.mean(dist == 0)) if ref.size else 1.0,
@@ -74,7 +82,7 @@ def bf16_report(gpu: torch.Tensor, ref: np.ndarray, floor=None, scale=None) -> d
     }
 
 
-def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F32_TOL) -> dict:
+def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F32_TOL, alt=None) -> dict:
     g = to_f64(gpu)
     ref = np.asarray(ref, dtype=np.float64).ravel()
     denom = np.abs(ref) if scale is None else np.maximum(np.abs(ref), np.asarray(scale).ravel())
@@ -87,11 +95,16 @@ def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F
         ok = (err <= tol * denom) | nan_ok | same | tiny_ok
         rel = np.where(denom > 0, err / denom, 0.0)
         pure = np.where(np.abs(ref) >= TINY, err / np.abs(ref), 0.0)
+    base_ok = ok
+    if alt is not None:
+        ok = ok | f32_report(gpu, alt[0], alt[1], floor, tol)["ok"]
     bad = np.flatnonzero(~ok)
     sel = ~(nan_ok | same | tiny_ok)
     return {
         "n": ref.size,
         "bad": bad.size,
+        "ok": ok,
+        "alt_only": int(np.sum(ok & ~base_ok)),
         "max_rel": float(np.nanmax(rel[sel], initial=0.0)),
         "max_pure_rel": float(np.nanmax(pure[sel], initial=0.0)),
         "pure_over_tol": int(np.sum(pure[sel] > tol)),
@@ -99,22 +112,33 @@ def f32_report(gpu: torch.Tensor, ref: np.ndarray, scale=None, floor=None, tol=F
     }
 
 
-def assert_bf16(gpu, ref, floor=None, what="", scale=None):
-    r = bf16_report(gpu, ref, floor, scale)
-    assert r["bad"] == 0, f"{what}: {r}"
+def _shown(r):
+    return {k: v for k, v in r.items() if k != "ok"}
+
+
+def assert_bf16(gpu, ref, floor=None, what="", scale=None, alt=None):
+    r = bf16_report(gpu, ref, floor, scale, alt)
+    assert r["bad"] == 0, f"{what}: {_shown(r)}"
     return r
 
 
-def assert_f32(gpu, ref, scale=None, floor=None, what="", tol=F32_TOL):
-    r = f32_report(gpu, ref, scale, floor, tol)
-    assert r["bad"] == 0, f"{what}: {r}"
+def assert_f32(gpu, ref, scale=None, floor=None, what="", tol=F32_TOL, alt=None):
+    r = f32_report(gpu, ref, scale, floor, tol, alt)
+    assert r["bad"] == 0, f"{what}: {_shown(r)}"
     return r
 
 
-def check(dtype: str, gpu, ref, scale=None, floor=None, what="", bf16_cond=False):
+def check(dtype: str, gpu, ref, scale=None, floor=None, what="", bf16_cond=False, alt=None):
     """bf16 outputs use the condition-scale alternative only when bf16_cond is
     set (outputs whose argument was formed in fp32, e.g. the fused affine);
-    activations applied to bf16 inputs are held to the plain 1-ulp rule."""
+    activations applied to bf16 inputs are held to the plain 1-ulp rule.
+
+    alt = (ref2, scale2): an element also passes when it meets the same rule
+    against ref2.  The fused affine passes the oracle's result at z rounded
+    once to fp32: z = gamma x + beta is an fp32 intermediate of the kernel,
+    and where f is steep relative to its value (GELU-tanh's cubic in the
+    deep negative tail) that one rounding alone moves f(z) by more than
+    1e-5 relative; the kernel is then held to 1e-5 of f at the rounded z."""
     if dtype == "bf16":
-        return assert_bf16(gpu, ref, floor, what, scale if bf16_cond else None)
-    return assert_f32(gpu, ref, scale, floor, what)
+        return assert_bf16(gpu, ref, floor, what, scale if bf16_cond else None, alt)
+    return assert_f32(gpu, ref, scale, floor, what, alt=alt)

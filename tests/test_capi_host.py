@@ -34,7 +34,7 @@ def _header_enum(name):
 
 def test_every_declared_symbol_is_exported(lib):
     declared = _header_functions()
-    assert len(declared) == 10, declared
+    assert len(declared) == 16, declared
     for fn in declared:
         assert hasattr(lib, fn), fn
         assert fn in _capi.SIGNATURES, fn
@@ -55,7 +55,7 @@ def test_enums_match_header():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.mea_version() == 10000
+    assert lib.mea_version() == 10100
     for st in range(5):
         assert lib.mea_status_string(st)
     assert lib.mea_status_string(99) == b"unknown status"
@@ -142,3 +142,37 @@ def test_binding_refuses_cpu_tensors():
         mea.act_fwd("swish", torch.zeros(4))
     with pytest.raises(ValueError):
         mea.act_fwd("softplus", torch.zeros(4))
+
+
+def test_affine_act_and_channel_validation(lib):
+    s = _capi.shape4((2, 16, 3, 3))
+    fa = lib.mea_affine_act_fwd
+    assert fa(7, 1, 1, s, X, G, D, 1.0, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b"act" in lib.mea_last_error()
+    assert fa(0, 1, 1, s, X, G, None, 1.0, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fa(0, 1, 1, s, X, G, D, 1.0, X + 4, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fa(0, 1, 1, _capi.shape4((0, 16, 3, 3)), None, None, None, 1.0, None, None) == _capi.MEA_OK
+    ba = lib.mea_affine_act_bwd
+    need = lib.mea_affine_act_bwd_workspace_bytes(1, 1, s)
+    assert need == lib.mea_affine_swish_bwd_workspace_bytes(1, 1, s)
+    assert ba(9, 1, 1, s, X, G, 0x700000, 0x710000, 0.1, D, 0x720000, 0x730000, 0x800000, need, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    assert ba(1, 1, 1, s, X, G, 0x700000, 0x710000, 0.1, D, 0x720000, 0x730000, 0x800008, need, None) \
+        == _capi.MEA_ERR_WORKSPACE
+    assert ba(1, 1, 1, s, X, G, 0x700000, 0x710000, 0.1, D, 0x720000, None, 0x800000, need, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    # zero channels: nothing to write, even without buffers
+    assert ba(1, 1, 1, _capi.shape4((2, 0, 3, 3)), None, None, None, None, 0.1, None, None, None, None, 0,
+              None) == _capi.MEA_OK
+    fc = lib.mea_swish_channel_fwd
+    assert fc(1, 1, s, X, None, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fc(1, 3, s, X, G, Y, None) == _capi.MEA_ERR_INVALID_ARG
+    assert fc(1, 1, s, X, G, X, None) == _capi.MEA_ERR_INVALID_ARG
+    bc = lib.mea_swish_channel_bwd
+    cneed = lib.mea_swish_channel_bwd_workspace_bytes(1, 1, s)
+    # one reduction per channel instead of two: a smaller workspace
+    assert 256 + 8 * 16 <= cneed < need
+    assert bc(1, 1, s, X, G, 0x700000, D, None, 0x800000, cneed, None) == _capi.MEA_ERR_INVALID_ARG
+    assert bc(1, 1, s, X, G, 0x700000, D, 0x720000, 0x800000, cneed - 1, None) == _capi.MEA_ERR_WORKSPACE
+    assert bc(1, 1, s, X, G, 0x700000, G + 2, 0x720000, 0x800000, cneed, None) == _capi.MEA_ERR_INVALID_ARG
+    assert lib.mea_swish_channel_bwd_workspace_bytes(1, 1, _capi.shape4((1, -2, 1, 1))) == 0
