@@ -38,9 +38,14 @@
  *    16-byte aligned, and element counts that are not a multiple of the
  *    vector width, take a scalar path; that is never an error.
  *  - n = 0 (or a zero in shape) is a no-op that returns MEA_OK.
- *  - Results are bitwise deterministic for a given input, shape and dtype
- *    (reductions run on a grid fixed by the element count and sum in a fixed
- *    order), independent of the stream, the run and the GPU's SM count.
+ *  - Results are bitwise deterministic for a given input, shape, dtype and
+ *    pointer alignment class (16-byte aligned or not: it selects the kernel
+ *    path): reductions run on a grid fixed by the shape and sum in a fixed
+ *    order, independent of the stream, the run and the GPU's SM count.
+ *  - Workspaces: the first 4 bytes are a completion counter (see
+ *    mea_act_bwd); bytes 4..7 are an error word that a kernel sets non-zero
+ *    if one of its bounded waits on shared-memory barriers expires (which
+ *    does not happen in correct operation); results are then undefined.
  */
 #ifndef MEA_H
 #define MEA_H

@@ -7,6 +7,7 @@
 #include <cstdio>
 
 #include "../../include/mea.h"
+#include "mea_channel_api.h"
 #include "mea_internal.h"
 
 namespace {

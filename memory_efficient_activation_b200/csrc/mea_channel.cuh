@@ -35,9 +35,11 @@
 
 #include <cstdint>
 
+#include "mea_channel_api.h"
 #include "mea_device.cuh"
 #include "mea_internal.h"
 #include "mea_math.cuh"
+#include "mea_pipe.cuh"
 
 namespace mea {
 
@@ -147,13 +149,14 @@ struct NhwcCfg;
 #ifndef MEA_NHWC_BWD_U
 #define MEA_NHWC_BWD_U 2
 #endif
+// U_PIPE: units per consumer thread per tile of the pipelined backward.
 template <>
 struct NhwcCfg<Bf16> {
-    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U;
+    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U, U_PIPE = 4;
 };
 template <>
 struct NhwcCfg<float> {
-    static constexpr int VE = 4, U_FWD = 8, U_BWD = MEA_NHWC_BWD_U;
+    static constexpr int VE = 4, U_FWD = 8, U_BWD = MEA_NHWC_BWD_U, U_PIPE = 2;
 };
 
 // ------------------------------------------------------------ NHWC kernels
@@ -301,6 +304,172 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
     }
 }
 
+// Backward, pipelined: the same work split and summation order as
+// chan_nhwc_bwd_kernel (block b owns tiles b, b + grid, ...; fp32 sums per
+// tile, fp64 per thread, one row of fp64 partials per block), but the x and
+// dy tiles reach shared memory by 1-D bulk copies (cp.async.bulk) that one
+// producer thread keeps `stages` tiles ahead, so the bytes in flight no
+// longer cost registers.  Warp 0 is the producer; warps 1.. are consumers
+// (blockDim.x - 32 of them, a multiple of the G = C / VE channel groups, so
+// every consumer thread keeps the same VE channels).  A consumer copies its
+// UT units of the tile from shared memory to registers, releases the stage
+// (one arrival per warp on the stage's `empty` barrier), computes, and
+// stores dx to global memory directly.  The partial tile at the end (fewer
+// than a tile's units) is done with plain loads by the block that owns its
+// index.  Waits are bounded: one that expires sets err[0] and the kernel
+// finishes without computing further tiles.
+//
+// Shared memory: [0, 256) barriers; then NR VE * consumers fp64 running sums;
+// then `stages` x {x tile, dy tile}.
+constexpr int kPipeMaxStages = 8;
+constexpr int kPipeHeader = 256;
+// 64 registers: three blocks of 288 + 32 threads (C = 144) per SM.
+constexpr int kPipeMaxRegs = 64;
+
+template <class Op, typename T, int VE, int UT>
+__global__ void __maxnreg__(kPipeMaxRegs)
+chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca,
+                          void *__restrict__ dx, int64_t nunits, int groups, int C, int stages,
+                          double *__restrict__ partials, unsigned int *__restrict__ err)
+{
+    using L = Unit<T, VE>;
+    using W = typename L::W;
+    constexpr bool P = L::P;
+    constexpr int NR = Op::NR;
+    constexpr int UB = sizeof(W);
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + kPipeMaxStages;
+    const int consumers = blockDim.x - 32;
+    double *acc = reinterpret_cast<double *>(smem + kPipeHeader);
+    const size_t acc_bytes = ((size_t)NR * VE * consumers * sizeof(double) + 127) & ~(size_t)127;
+    unsigned char *buf = smem + kPipeHeader + acc_bytes;
+    const int64_t tile_units = (int64_t)consumers * UT;
+    const uint32_t tile_bytes = (uint32_t)(tile_units * UB);
+    const int64_t ntiles = nunits / tile_units;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(smem_addr(full + s), 1);
+            mbar_init(smem_addr(empty + s), consumers / 32);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+    pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int it = 0;
+            for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+                const int s = it % stages;
+                if (it >= stages && !mbar_wait(smem_addr(empty + s), ((it / stages) & 1) ^ 1)) {
+                    atomicExch(err, 1u);
+                    break;
+                }
+                const uint32_t fb = smem_addr(full + s);
+                mbar_arrive_expect_tx(fb, 2 * tile_bytes);
+                unsigned char *bx = buf + (size_t)s * 2 * tile_bytes;
+                bulk_load(smem_addr(bx), static_cast<const unsigned char *>(x) + t * tile_bytes, tile_bytes, fb);
+                bulk_load(smem_addr(bx + tile_bytes), static_cast<const unsigned char *>(dy) + t * tile_bytes,
+                          tile_bytes, fb);
+            }
+            // Every issued copy lands before the block may exit.
+            for (int j = it > stages ? it - stages : 0; j < it; ++j)
+                if (!mbar_wait(smem_addr(full + j % stages), (j / stages) & 1)) atomicExch(err, 1u);
+        }
+        return;
+    }
+
+    const int ct = threadIdx.x - 32;
+    const int g = ct % groups;
+    const typename Op::K k = Op::kcoef(ca);
+    typename Op::Ch ch[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) ch[j] = Op::load(ca, g * VE + j);
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int j = 0; j < VE; ++j) acc[(r * VE + j) * consumers + ct] = 0.0;
+
+    auto work = [&](const W (&xv)[UT], const W (&gv)[UT], int64_t base, int64_t limit) {
+        float accf[VE][NR];
+#pragma unroll
+        for (int j = 0; j < VE; ++j)
+#pragma unroll
+            for (int r = 0; r < NR; ++r) accf[j][r] = 0.f;
+#pragma unroll
+        for (int u = 0; u < UT; ++u) {
+            const int64_t i = base + (int64_t)u * consumers;
+            if (i < limit) {
+                float xf[VE], gf[VE], o[VE], tt[VE], of[VE];
+                L::unpack(xv[u], xf);
+                L::unpack(gv[u], gf);
+                bool tail = false;
+#pragma unroll
+                for (int j = 0; j < VE; ++j) Op::template bwd<P>(xf[j], gf[j], k, ch[j], tail, o[j], tt[j]);
+                if (tail) {
+#pragma unroll
+                    for (int j = 0; j < VE; ++j)
+                        if (Op::is_tail(xf[j], k, ch[j]))
+                            Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < VE; ++j) of[j] = Op::finish(xf[j], o[j], tt[j], ch[j], accf[j]);
+                L::store(dx, i, L::pack(of));
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int j = 0; j < VE; ++j) acc[(r * VE + j) * consumers + ct] += (double)accf[j][r];
+    };
+
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+        const int s = it % stages;
+        if (!mbar_wait(smem_addr(full + s), (it / stages) & 1)) {
+            atomicExch(err, 1u);
+            break;
+        }
+        const unsigned char *bx = buf + (size_t)s * 2 * tile_bytes;
+        W xv[UT], gv[UT];
+#pragma unroll
+        for (int u = 0; u < UT; ++u) {
+            xv[u] = reinterpret_cast<const W *>(bx)[u * consumers + ct];
+            gv[u] = reinterpret_cast<const W *>(bx + tile_bytes)[u * consumers + ct];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(empty + s));
+        work(xv, gv, t * tile_units + ct, nunits);
+    }
+    // The partial tile at the end, if any, belongs to block ntiles % grid.
+    if (ntiles * tile_units < nunits && blockIdx.x == ntiles % gridDim.x) {
+        const int64_t base = ntiles * tile_units + ct;
+        W xv[UT], gv[UT];
+#pragma unroll
+        for (int u = 0; u < UT; ++u) {
+            const int64_t i = base + (int64_t)u * consumers;
+            if (i < nunits) {
+                xv[u] = L::load(x, i);
+                gv[u] = L::load(dy, i);
+            }
+        }
+        work(xv, gv, base, nunits);
+    }
+    pdl_trigger();
+    named_sync(1, consumers);
+    const int rows = consumers / groups;
+    for (int o = ct; o < NR * C; o += consumers) {
+        const int r = o / C, c = o % C;
+        const double *col = acc + (r * VE + c % VE) * consumers + c / VE;
+        double sum = 0.0;
+        for (int q = 0; q < rows; ++q) sum += col[q * groups];
+        partials[(int64_t)blockIdx.x * NR * C + o] = sum;
+    }
+}
+
 // Output o (r * C + c) = sum over the nb rows of partials, column o, in
 // fp64: thread t adds rows t, t + kColsumThreads, ... in order, then a fixed
 // block-wide tree.  One block per output; r = 0 goes to out0, r = 1 to out1.
@@ -437,6 +606,35 @@ inline bool nhwc_fast(const AffineLaunch &a)
     return a.layout == 1 && a.C % VE == 0 && nhwc_threads((int)(a.C / VE)) > 0 && (al % bytes) == 0;
 }
 
+// Pipelined backward: shared memory per block is held to kPipeSmemBudget so
+// that three blocks fit an SM (228 KB, 1 KB of it reserved per block), and
+// the grid is at most kPipeGrid blocks (one wave of three per SM on a B200;
+// a constant, so the summation order does not depend on the device).
+constexpr int kPipeSmemBudget = 75 * 1024;
+constexpr int kPipeGrid = 444;
+
+struct PipeShape {
+    int stages;          // 0: the pipelined kernel is not used
+    int grid;
+    size_t smem;
+};
+
+template <typename T>
+inline PipeShape pipe_shape(int nr, int64_t nunits, int consumers)
+{
+    constexpr int VE = NhwcCfg<T>::VE, UT = NhwcCfg<T>::U_PIPE;
+    constexpr int UB = VE * (sizeof(T) == 4 ? 4 : 2);
+    const size_t acc = ((size_t)nr * VE * consumers * sizeof(double) + 127) & ~(size_t)127;
+    const size_t tile = (size_t)consumers * UT * UB;
+    const long room = (long)kPipeSmemBudget - kPipeHeader - (long)acc;
+    long stages = room > 0 ? room / (long)(2 * tile) : 0;
+    if (stages > kPipeMaxStages) stages = kPipeMaxStages;
+    if (stages < 2) return PipeShape{0, 0, 0};
+    const int64_t ntiles = nunits / ((int64_t)consumers * UT);
+    const int64_t grid = ntiles < 1 ? 1 : (ntiles < kPipeGrid ? ntiles : kPipeGrid);
+    return PipeShape{(int)stages, (int)grid, kPipeHeader + acc + (size_t)stages * 2 * tile};
+}
+
 // Workspace of the backward of a per-channel operation with nr reductions:
 // the larger of the NHWC fast path's and the plane path's needs (pointer
 // alignment, which decides between them, is not known here).
@@ -448,7 +646,11 @@ inline size_t chan_bwd_workspace_bytes(int nr, int dtype, int layout, int64_t N,
     if (layout == 1 && C % VE == 0 && nhwc_threads((int)(C / VE)) > 0) {
         const int threads = nhwc_threads((int)(C / VE));
         const int64_t nunits = N * C * H * W / VE;
-        size_t fast = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)nhwc_bwd_grid(nunits, threads, U);
+        const int reg_rows = nhwc_bwd_grid(nunits, threads, U);
+        const int pipe_rows = dtype == kBF16 ? pipe_shape<Bf16>(nr, nunits, threads).grid
+                                             : pipe_shape<float>(nr, nunits, threads).grid;
+        const int rows = reg_rows > pipe_rows ? reg_rows : pipe_rows;
+        size_t fast = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)rows;
         return fast > plane ? fast : plane;
     }
     return plane;
@@ -473,18 +675,35 @@ cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out
             return launch_pdl(chan_nhwc_fwd_kernel<Op, T, U, VE>, dim3((unsigned)nb), dim3(threads), 0, a.stream, a.x,
                               ca, a.out, nunits, groups);
         }
-        constexpr int U = NhwcCfg<T>::U_BWD;
-        auto kernel = chan_nhwc_bwd_kernel<Op, T, U, VE>;
-        const int nb = nhwc_bwd_grid(nunits, threads, U);
         double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
-        const size_t smem = sizeof(double) * NR * VE * threads;
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             (int)cudaSharedmemCarveoutMaxShared);
-        if (e == cudaSuccess && smem > 48 * 1024)
-            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(kernel, dim3((unsigned)nb), dim3(threads), smem, a.stream, a.x, a.dy, ca, a.out, nunits, groups,
-                       (int)a.C, partials);
+        unsigned int *err = reinterpret_cast<unsigned int *>(static_cast<char *>(a.workspace) + 4);
+        const bool bulk_ok = ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.dy)) & 15u) == 0;
+        const PipeShape ps = pipe_shape<T>(NR, nunits, threads);
+        int nb;
+        cudaError_t e;
+        if (bulk_ok && ps.stages > 0) {
+            auto kernel = chan_nhwc_bwd_pipe_kernel<Op, T, VE, NhwcCfg<T>::U_PIPE>;
+            nb = ps.grid;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ps.smem);
+            if (e != cudaSuccess) return e;
+            e = launch_pdl(kernel, dim3((unsigned)nb), dim3(threads + 32), ps.smem, a.stream, a.x, a.dy, ca, a.out,
+                           nunits, groups, (int)a.C, ps.stages, partials, err);
+        } else {
+            constexpr int U = NhwcCfg<T>::U_BWD;
+            auto kernel = chan_nhwc_bwd_kernel<Op, T, U, VE>;
+            nb = nhwc_bwd_grid(nunits, threads, U);
+            const size_t smem = sizeof(double) * NR * VE * threads;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e == cudaSuccess && smem > 48 * 1024)
+                e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            e = launch_pdl(kernel, dim3((unsigned)nb), dim3(threads), smem, a.stream, a.x, a.dy, ca, a.out, nunits,
+                           groups, (int)a.C, partials);
+        }
         if (e != cudaSuccess) return e;
         return launch_pdl(chan_colsum_kernel<NR>, dim3((unsigned)(NR * a.C)), dim3(kColsumThreads), 0, a.stream,
                           partials, nb, (int)a.C, out0, out1);

@@ -1,0 +1,38 @@
+// mea_channel_api.h -- host-side interface of the per-channel kernels (fused
+// per-channel affine + activation; Swish with one alpha per channel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace mea {
+
+// Per-channel operations (affine + activation; Swish with per-channel alpha).
+// For the channel Swish, gamma carries alpha and dgamma receives dalpha.
+struct AffineLaunch {
+    int act;                 // mea_act_t (affine + activation)
+    float param;             // activation parameter (affine + activation)
+    int dtype;
+    int layout;              // mea_layout_t
+    int64_t N, C, H, W;
+    const void *x;
+    const void *dy;
+    const float *gamma;
+    const float *beta;
+    void *out;
+    float *dgamma;
+    float *dbeta;
+    void *workspace;
+    cudaStream_t stream;
+};
+
+size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
+cudaError_t launch_affine_fwd(const AffineLaunch &a);
+cudaError_t launch_affine_bwd(const AffineLaunch &a);
+size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
+cudaError_t launch_channel_swish_fwd(const AffineLaunch &a);
+cudaError_t launch_channel_swish_bwd(const AffineLaunch &a);
+
+}  // namespace mea

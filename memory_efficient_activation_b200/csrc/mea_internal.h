@@ -50,32 +50,6 @@ struct ActLaunch {
 cudaError_t launch_act_fwd(const ActLaunch &a);
 cudaError_t launch_act_bwd(const ActLaunch &a);
 
-// Per-channel operations (affine + activation; Swish with per-channel alpha).
-// For the channel Swish, gamma carries alpha and dgamma receives dalpha.
-struct AffineLaunch {
-    int act;                 // mea_act_t (affine + activation)
-    float param;             // activation parameter (affine + activation)
-    int dtype;
-    int layout;              // mea_layout_t
-    int64_t N, C, H, W;
-    const void *x;
-    const void *dy;
-    const float *gamma;
-    const float *beta;
-    void *out;
-    float *dgamma;
-    float *dbeta;
-    void *workspace;
-    cudaStream_t stream;
-};
-
-size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
-cudaError_t launch_affine_fwd(const AffineLaunch &a);
-cudaError_t launch_affine_bwd(const AffineLaunch &a);
-size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
-cudaError_t launch_channel_swish_fwd(const AffineLaunch &a);
-cudaError_t launch_channel_swish_bwd(const AffineLaunch &a);
-
 // Launch with programmatic stream serialisation: the kernel may begin while
 // the previous kernel on the stream drains, and waits (pdl_wait) before it
 // touches memory.  Returns the launch's cudaError_t.

@@ -156,6 +156,30 @@ def test_affine_act_full_workload(act):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("act", ["gelu_erf", "swish", "relu"])
+@pytest.mark.parametrize("shape", [(4, 7, 9, 144), (2, 5, 5, 32), (3, 3, 7, 1152)])
+def test_affine_act_nhwc_unaligned(act, dtype, shape):
+    # tensors that start 8 bytes past a 16-byte boundary: the NHWC backward
+    # then streams with plain loads instead of bulk copies into shared memory
+    # (and for fp32, whose 16-byte units need 16-byte alignment, the forward
+    # and backward take the plane path); same values either way
+    x, dy, g, b, _ = _inputs(shape, "nhwc", dtype, 406)
+    n = x.numel()
+    off = 4 if dtype == "bf16" else 2
+    xb = torch.empty(n + off, dtype=x.dtype, device="cuda")
+    gb = torch.empty(n + off, dtype=x.dtype, device="cuda")
+    xs, gs = xb[off:].view(shape), gb[off:].view(shape)
+    xs.copy_(x.cuda())
+    gs.copy_(dy.cuda())
+    assert xs.data_ptr() % 16 == 8 and gs.data_ptr() % 16 == 8
+    p = _param(act)
+    y = mea.affine_act_fwd(act, xs, g.cuda(), b.cuda(), p, "nhwc")
+    dx, dg, db = mea.affine_act_bwd(act, xs, gs, g.cuda(), b.cuda(), p, "nhwc")
+    torch.cuda.synchronize()
+    _affine_compare(act, dtype, "nhwc", shape, x, dy, g, b, y, dx, dg, db)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("layout,shape", [("nhwc", (3, 7, 7, 144)), ("nchw", (3, 40, 7, 7))])
 def test_affine_act_swish_matches_affine_swish(dtype, layout, shape):
     # affine + Swish is the Swish member of the family with alpha = 1: the
@@ -182,6 +206,7 @@ def test_affine_act_deterministic_and_counter_reset(act, layout, shape):
     outs = [mea.affine_act_bwd(act, x, dy, g, b, 1.0, layout, workspace=ws) for _ in range(4)]
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+    assert int(ws[4:8].view(torch.int32).item()) == 0     # no bounded wait expired
     for o in outs[1:]:
         for a, c in zip(outs[0], o):
             assert torch.equal(a, c)
@@ -265,6 +290,7 @@ def test_swish_channel_deterministic_and_counter_reset(layout, shape):
     outs = [mea.swish_channel_bwd(x, dy, a, layout, workspace=ws) for _ in range(4)]
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+    assert int(ws[4:8].view(torch.int32).item()) == 0
     for o in outs[1:]:
         for p, q in zip(outs[0], o):
             assert torch.equal(p, q)
