@@ -53,6 +53,47 @@ struct AffineOp {
         acc[1] += o;                   // dz
         return h.g * o;                // dx
     }
+
+    // Two channels at once: the affine, the reduction terms and dx as packed
+    // .f32x2 operations (bitwise the scalar results); f' pairwise where the
+    // activation provides it, else per element.
+    struct Ch2 {
+        F2 g, b;
+    };
+    static __device__ __forceinline__ Ch2 pair(const Ch &a, const Ch &c) { return Ch2{pk(a.g, c.g), pk(a.b, c.b)}; }
+    template <bool P>
+    static __device__ __forceinline__ F2 f2(F2 x, const K &k, const Ch2 &h, bool &tail)
+    {
+        float z0, z1, o0, o1;
+        upk(fma2(h.g, x, h.b), z0, z1);
+        if constexpr (HasPairs<A, P>::value) {
+            A::f2(z0, z1, k, tail, o0, o1);
+        } else {
+            o0 = A::template f<P>(z0, k, tail);
+            o1 = A::template f<P>(z1, k, tail);
+        }
+        return pk(o0, o1);
+    }
+    template <bool P>
+    static __device__ __forceinline__ void bwd2(F2 x, F2 dy, const K &k, const Ch2 &h, bool &tail, F2 &o, F2 &)
+    {
+        float z0, z1, d0, d1, o0, o1;
+        upk(fma2(h.g, x, h.b), z0, z1);
+        upk(dy, d0, d1);
+        if constexpr (HasPairs<A, P>::value) {
+            A::df2(z0, z1, d0, d1, k, tail, o0, o1);
+        } else {
+            o0 = A::template df<P>(z0, d0, k, tail);
+            o1 = A::template df<P>(z1, d1, k, tail);
+        }
+        o = pk(o0, o1);
+    }
+    static __device__ __forceinline__ F2 finish2(F2 x, F2 o, F2, const Ch2 &h, F2 (&acc)[NR])
+    {
+        acc[0] = fma2(o, x, acc[0]);
+        acc[1] = add2(acc[1], o);
+        return mul2(h.g, o);
+    }
 };
 
 template <typename T, int MODE>

@@ -11,6 +11,8 @@
 //   bwd<P>(x, dy, ..., o, t)      backward main path -> raw results o, t
 //   bwd_tail<P>(...)              deep-tail recompute of o, t
 //   finish(x, o, t, ch, acc[NR])  dx, and adds the channel's reduction terms
+//   Ch2, pair(ch, ch), bwd2<P>, finish2   the same for two adjacent channels
+//                          in packed .f32x2 registers (pipelined backward)
 //
 // Only x is kept between the passes; the backward recomputes everything from
 // it (the save-input-only idea of "Memory efficient Swish", section "What
@@ -54,6 +56,8 @@ constexpr int kNhwcBwdGridCap = 888;     // 148 x 6
 #define MEA_NHWC_BWD_MAXREGS 72
 #endif
 constexpr int kNhwcBwdMaxRegs = MEA_NHWC_BWD_MAXREGS;
+// Register cap of the NHWC forward: 64 keeps three 288-thread blocks per SM.
+constexpr int kNhwcFwdMaxRegs = 64;
 constexpr int kPlaneThreads = 256;
 constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks
 
@@ -90,6 +94,13 @@ inline int plane_slices(int64_t N, int64_t C)
     if (s > N) s = N;
     if (s < 1) s = 1;
     return (int)s;
+}
+
+__device__ __forceinline__ F2 add2(F2 a, F2 b)
+{
+    F2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
 }
 
 // ------------------------------------------------------------ load units
@@ -162,12 +173,13 @@ struct NhwcCfg<float> {
 // ------------------------------------------------------------ NHWC kernels
 
 // Forward: one tile of blockDim.x * U units per block (as the plain
-// activation kernels).
+// activation kernels); pairs of channels in packed .f32x2 registers.
 template <class Op, typename T, int U, int VE>
-__global__ void __launch_bounds__(kNhwcMaxThreads)
+__global__ void __maxnreg__(kNhwcFwdMaxRegs)
 chan_nhwc_fwd_kernel(const void *__restrict__ x, ChanArgs ca, void *__restrict__ out, int64_t nunits, int groups)
 {
     using L = Unit<T, VE>;
+    using W = typename L::W;
     constexpr bool P = L::P;
     const int tid = threadIdx.x;
     const int g = tid % groups;
@@ -176,28 +188,43 @@ chan_nhwc_fwd_kernel(const void *__restrict__ x, ChanArgs ca, void *__restrict__
     typename Op::Ch ch[VE];
 #pragma unroll
     for (int j = 0; j < VE; ++j) ch[j] = Op::load(ca, g * VE + j);
+    typename Op::Ch2 ch2[VE / 2];
+#pragma unroll
+    for (int p = 0; p < VE / 2; ++p) ch2[p] = Op::pair(ch[2 * p], ch[2 * p + 1]);
     const int64_t base = (int64_t)blockIdx.x * blockDim.x * U + tid;
-    typename L::W xv[U];
+    const bool whole = (int64_t)(blockIdx.x + 1) * blockDim.x * U <= nunits;
+    auto unit = [&](const W &w) -> W {
+        float xf[VE], of[VE];
+        L::unpack(w, xf);
+        bool tail = false;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int64_t i = base + (int64_t)u * blockDim.x;
-        if (i < nunits) xv[u] = L::load(x, i);
-    }
+        for (int p = 0; p < VE / 2; ++p)
+            upk(Op::template f2<P>(pk(xf[2 * p], xf[2 * p + 1]), k, ch2[p], tail), of[2 * p], of[2 * p + 1]);
+        if (tail) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int64_t i = base + (int64_t)u * blockDim.x;
-        if (i < nunits) {
-            float xf[VE], of[VE];
-            L::unpack(xv[u], xf);
-            bool tail = false;
+            for (int j = 0; j < VE; ++j)
+                if (Op::is_tail(xf[j], k, ch[j])) of[j] = Op::template f_tail<P>(xf[j], k, ch[j]);
+        }
+        return L::pack(of);
+    };
+    W xv[U];
+    if (whole) {
+        const W *src = static_cast<const W *>(x) + base;
 #pragma unroll
-            for (int j = 0; j < VE; ++j) of[j] = Op::template f<P>(xf[j], k, ch[j], tail);
-            if (tail) {
+        for (int u = 0; u < U; ++u) xv[u] = L::load(src, u * blockDim.x);
+        W *dst = static_cast<W *>(out) + base;
 #pragma unroll
-                for (int j = 0; j < VE; ++j)
-                    if (Op::is_tail(xf[j], k, ch[j])) of[j] = Op::template f_tail<P>(xf[j], k, ch[j]);
-            }
-            L::store(out, i, L::pack(of));
+        for (int u = 0; u < U; ++u) L::store(dst, u * blockDim.x, unit(xv[u]));
+    } else {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + (int64_t)u * blockDim.x;
+            if (i < nunits) xv[u] = L::load(x, i);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + (int64_t)u * blockDim.x;
+            if (i < nunits) L::store(out, i, unit(xv[u]));
         }
     }
     pdl_trigger();
@@ -325,6 +352,9 @@ constexpr int kPipeMaxStages = 8;
 constexpr int kPipeHeader = 256;
 // 64 registers: three blocks of 288 + 32 threads (C = 144) per SM.
 constexpr int kPipeMaxRegs = 64;
+// Tiles whose fp32 sums a consumer thread carries before adding them to its
+// fp64 sums (kPipeFlushTiles * UT terms per channel in fp32).
+constexpr int kPipeFlushTiles = 4;
 
 template <class Op, typename T, int VE, int UT>
 __global__ void __maxnreg__(kPipeMaxRegs)
@@ -388,43 +418,62 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     typename Op::Ch ch[VE];
 #pragma unroll
     for (int j = 0; j < VE; ++j) ch[j] = Op::load(ca, g * VE + j);
+    typename Op::Ch2 ch2[VE / 2];
+#pragma unroll
+    for (int p = 0; p < VE / 2; ++p) ch2[p] = Op::pair(ch[2 * p], ch[2 * p + 1]);
 #pragma unroll
     for (int r = 0; r < NR; ++r)
 #pragma unroll
         for (int j = 0; j < VE; ++j) acc[(r * VE + j) * consumers + ct] = 0.0;
 
-    auto work = [&](const W (&xv)[UT], const W (&gv)[UT], int64_t base, int64_t limit) {
-        float accf[VE][NR];
+    // fp32 sums of up to kPipeFlushTiles tiles (UT terms per channel each),
+    // then added to the thread's fp64 sums in shared memory.
+    F2 accf[VE / 2][NR];
+    auto clear = [&]() {
 #pragma unroll
-        for (int j = 0; j < VE; ++j)
+        for (int p = 0; p < VE / 2; ++p)
 #pragma unroll
-            for (int r = 0; r < NR; ++r) accf[j][r] = 0.f;
-#pragma unroll
-        for (int u = 0; u < UT; ++u) {
-            const int64_t i = base + (int64_t)u * consumers;
-            if (i < limit) {
-                float xf[VE], gf[VE], o[VE], tt[VE], of[VE];
-                L::unpack(xv[u], xf);
-                L::unpack(gv[u], gf);
-                bool tail = false;
-#pragma unroll
-                for (int j = 0; j < VE; ++j) Op::template bwd<P>(xf[j], gf[j], k, ch[j], tail, o[j], tt[j]);
-                if (tail) {
-#pragma unroll
-                    for (int j = 0; j < VE; ++j)
-                        if (Op::is_tail(xf[j], k, ch[j]))
-                            Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
-                }
-#pragma unroll
-                for (int j = 0; j < VE; ++j) of[j] = Op::finish(xf[j], o[j], tt[j], ch[j], accf[j]);
-                L::store(dx, i, L::pack(of));
-            }
-        }
+            for (int r = 0; r < NR; ++r) accf[p][r] = sp2(0.f);
+    };
+    auto flush = [&]() {
 #pragma unroll
         for (int r = 0; r < NR; ++r)
 #pragma unroll
-            for (int j = 0; j < VE; ++j) acc[(r * VE + j) * consumers + ct] += (double)accf[j][r];
+            for (int p = 0; p < VE / 2; ++p) {
+                float a0, a1;
+                upk(accf[p][r], a0, a1);
+                acc[(r * VE + 2 * p) * consumers + ct] += (double)a0;
+                acc[(r * VE + 2 * p + 1) * consumers + ct] += (double)a1;
+            }
+        clear();
     };
+    // One unit: VE elements of VE consecutive channels.
+    auto unit = [&](const W &xw, const W &gw) -> W {
+        float xf[VE], gf[VE], o[VE], tt[VE], of[VE];
+        L::unpack(xw, xf);
+        L::unpack(gw, gf);
+        bool tail = false;
+#pragma unroll
+        for (int p = 0; p < VE / 2; ++p) {
+            F2 o2, t2 = sp2(0.f);
+            Op::template bwd2<P>(pk(xf[2 * p], xf[2 * p + 1]), pk(gf[2 * p], gf[2 * p + 1]), k, ch2[p], tail, o2,
+                                 t2);
+            upk(o2, o[2 * p], o[2 * p + 1]);
+            upk(t2, tt[2 * p], tt[2 * p + 1]);
+        }
+        if (tail) {
+#pragma unroll
+            for (int j = 0; j < VE; ++j)
+                if (Op::is_tail(xf[j], k, ch[j])) Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
+        }
+#pragma unroll
+        for (int p = 0; p < VE / 2; ++p)
+            upk(Op::finish2(pk(xf[2 * p], xf[2 * p + 1]), pk(o[2 * p], o[2 * p + 1]),
+                            pk(tt[2 * p], tt[2 * p + 1]), ch2[p], accf[p]),
+                of[2 * p], of[2 * p + 1]);
+        return L::pack(of);
+    };
+    clear();
 
     int it = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
@@ -433,31 +482,32 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             atomicExch(err, 1u);
             break;
         }
-        const unsigned char *bx = buf + (size_t)s * 2 * tile_bytes;
+        const W *sx = reinterpret_cast<const W *>(buf + (size_t)s * 2 * tile_bytes) + ct;
+        const W *sg = reinterpret_cast<const W *>(buf + (size_t)s * 2 * tile_bytes + tile_bytes) + ct;
         W xv[UT], gv[UT];
 #pragma unroll
         for (int u = 0; u < UT; ++u) {
-            xv[u] = reinterpret_cast<const W *>(bx)[u * consumers + ct];
-            gv[u] = reinterpret_cast<const W *>(bx + tile_bytes)[u * consumers + ct];
+            xv[u] = sx[u * consumers];
+            gv[u] = sg[u * consumers];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(empty + s));
-        work(xv, gv, t * tile_units + ct, nunits);
+        // a whole tile: every unit is in range
+        W *out = static_cast<W *>(dx) + t * tile_units + ct;
+#pragma unroll
+        for (int u = 0; u < UT; ++u) L::store(out, u * consumers, unit(xv[u], gv[u]));
+        if ((it + 1) % kPipeFlushTiles == 0) flush();
     }
     // The partial tile at the end, if any, belongs to block ntiles % grid.
     if (ntiles * tile_units < nunits && blockIdx.x == ntiles % gridDim.x) {
         const int64_t base = ntiles * tile_units + ct;
-        W xv[UT], gv[UT];
 #pragma unroll
         for (int u = 0; u < UT; ++u) {
             const int64_t i = base + (int64_t)u * consumers;
-            if (i < nunits) {
-                xv[u] = L::load(x, i);
-                gv[u] = L::load(dy, i);
-            }
+            if (i < nunits) L::store(dx, i, unit(L::load(x, i), L::load(dy, i)));
         }
-        work(xv, gv, base, nunits);
     }
+    flush();
     pdl_trigger();
     named_sync(1, consumers);
     const int rows = consumers / groups;

@@ -49,6 +49,35 @@ struct ChannelSwishOp {
         acc[0] += t;
         return o;
     }
+
+    // Two channels at once (each with its own alpha, so f' stays per element).
+    struct Ch2 {
+        Ch a, b;
+    };
+    static __device__ __forceinline__ Ch2 pair(const Ch &a, const Ch &b) { return Ch2{a, b}; }
+    template <bool P>
+    static __device__ __forceinline__ F2 f2(F2 x, const K &, const Ch2 &h, bool &tail)
+    {
+        float x0, x1;
+        upk(x, x0, x1);
+        return pk(Swish::f<P>(x0, h.a, tail), Swish::f<P>(x1, h.b, tail));
+    }
+    template <bool P>
+    static __device__ __forceinline__ void bwd2(F2 x, F2 dy, const K &, const Ch2 &h, bool &tail, F2 &o, F2 &t)
+    {
+        float x0, x1, d0, d1, t0, t1;
+        upk(x, x0, x1);
+        upk(dy, d0, d1);
+        const float o0 = Swish::df_da<P>(x0, d0, h.a, tail, t0);
+        const float o1 = Swish::df_da<P>(x1, d1, h.b, tail, t1);
+        o = pk(o0, o1);
+        t = pk(t0, t1);
+    }
+    static __device__ __forceinline__ F2 finish2(F2, F2 o, F2 t, const Ch2 &, F2 (&acc)[NR])
+    {
+        acc[0] = add2(acc[0], t);
+        return o;
+    }
 };
 
 size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W)

@@ -75,7 +75,10 @@ def _check_sums_against_dx(dx, x, g, dg, db, ch, C):
     """fp32 only: the channel sums agree with the kernel's own dx (dz = dx /
     gamma_c, each dx one fp32 rounding of gamma_c dz), which checks the
     reduction machinery (every element counted once, in its channel) far
-    more tightly than the oracle comparison of the values can."""
+    more tightly than the oracle comparison of the values can.  The kernels
+    add at most 16 terms in fp32 before moving to fp64; a sequential fp32 sum
+    of k terms errs by at most (k - 1) 2^-24 of the sum of |terms|, so with
+    the rounding of each dx the bound is 1.1e-6 of that sum."""
     gg = g.double().numpy()
     dz = to_f64(dx) / gg[ch]
     xd = to_f64(x)
@@ -85,8 +88,8 @@ def _check_sums_against_dx(dx, x, g, dg, db, ch, C):
     tg = np.bincount(ch, np.abs(dz * xd), minlength=C)
     eb = np.abs(db.cpu().double().numpy() - sb)
     eg = np.abs(dg.cpu().double().numpy() - sg)
-    assert np.all(eb <= 3e-7 * tb + 1e-30), eb.max()
-    assert np.all(eg <= 3e-7 * tg + 1e-30), eg.max()
+    assert np.all(eb <= 1.1e-6 * tb + 1e-30), eb.max()
+    assert np.all(eg <= 1.1e-6 * tg + 1e-30), eg.max()
 
 
 def _affine_compare(act, dtype, layout, shape, x, dy, g, b, y, dx, dg, db):
