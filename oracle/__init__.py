@@ -19,7 +19,8 @@ Sources (by page and section):
   efficient version Swish implemented?", "What makes this implementation save
   GPU memory?").
 * "What activations cost, in memory and in arithmetic" (asifuddin.com,
-  problem B07), GIVEN: the activation family.
+  problem B07), GIVEN: the activation family; SOLUTION step 4: the matrix
+  multiply the activation follows (matmul_act_fwd / matmul_act_bwd).
 
 Parity pins for every function here live in ``tests/test_oracle_*.py``.
 """
@@ -97,6 +98,11 @@ def _load():
         lib.oracle_swish_channel_fwd.restype = ctypes.c_int
         lib.oracle_swish_channel_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d]
         lib.oracle_swish_channel_bwd.restype = ctypes.c_int
+        lib.oracle_matmul_act_fwd.argtypes = [ctypes.c_int, i64, i64, i64, d, d, ctypes.c_double, ctypes.c_int,
+                                              d, d, d]
+        lib.oracle_matmul_act_fwd.restype = ctypes.c_int
+        lib.oracle_matmul_act_bwd.argtypes = [ctypes.c_int, i64, i64, i64, d, d, d, ctypes.c_double, d, d, d]
+        lib.oracle_matmul_act_bwd.restype = ctypes.c_int
         lib.oracle_round_bf16.argtypes = [d, ctypes.POINTER(ctypes.c_uint16), i64]
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_f32.argtypes = [d, ctypes.POINTER(ctypes.c_float), i64]
@@ -263,6 +269,45 @@ def swish_channel_bwd(layout: str, shape, x, dy, alpha):
     if rc:
         raise ValueError(f"oracle_swish_channel_bwd failed: {rc}")
     return dx, da, scale
+
+
+def matmul_act_fwd(act: str, X, W, param: float = 1.0, round_z_bf16: bool = True):
+    """Z = X W^T (X [M, K], W [N, K]) and Y = f(Z as stored: rounded to bf16
+    when round_z_bf16).  Returns (Z, Y, absum) in double, absum = sum_k
+    |X[m, k] W[n, k]|."""
+    X, W = np.ascontiguousarray(X, dtype=np.float64), np.ascontiguousarray(W, dtype=np.float64)
+    M, K = X.shape
+    N, K2 = W.shape
+    if K != K2:
+        raise ValueError("X and W disagree in K")
+    Z = np.empty((M, N))
+    Y = np.empty((M, N))
+    S = np.empty((M, N))
+    rc = _load().oracle_matmul_act_fwd(ACTS[act], M, N, K, _ptr(X), _ptr(W), float(param), int(bool(round_z_bf16)),
+                                       _ptr(Z), _ptr(Y), _ptr(S))
+    if rc:
+        raise ValueError(f"oracle_matmul_act_fwd failed: {rc}")
+    return Z, Y, S
+
+
+def matmul_act_bwd(act: str, G, W, Z, param: float = 1.0):
+    """dZ = (G W^T) * f'(Z) (G [M, K], W [N, K], Z [M, N] as stored).
+    Returns (dZ, D, absum): D = G W^T before the derivative, absum = sum_k
+    |G[m, k] W[n, k]|."""
+    G, W = np.ascontiguousarray(G, dtype=np.float64), np.ascontiguousarray(W, dtype=np.float64)
+    Z = np.ascontiguousarray(Z, dtype=np.float64)
+    M, K = G.shape
+    N, K2 = W.shape
+    if K != K2 or Z.shape != (M, N):
+        raise ValueError("shapes disagree")
+    dZ = np.empty((M, N))
+    D = np.empty((M, N))
+    S = np.empty((M, N))
+    rc = _load().oracle_matmul_act_bwd(ACTS[act], M, N, K, _ptr(G), _ptr(W), _ptr(Z), float(param), _ptr(dZ),
+                                       _ptr(D), _ptr(S))
+    if rc:
+        raise ValueError(f"oracle_matmul_act_bwd failed: {rc}")
+    return dZ, D, S
 
 
 def round_bf16(v) -> np.ndarray:

@@ -39,6 +39,12 @@
  *    (Hendrycks and Gimpel, 2016); 1 + tanh(u) is evaluated as 2 Sigmoid(2u).
  *  - Fused affine + Swish: z = gamma_c x + beta_c, y = z Sigmoid(z) (alpha 1),
  *    channel c = i mod C for NHWC and (i / (H W)) mod C for NCHW.
+ *  - Matmul + activation (problem B07, SOLUTION step 4: the activation
+ *    follows a d x d matrix multiply on the same tensor): Z = X W^T with X
+ *    [M x K] and W [N x K] row-major; the activation is evaluated at Z as
+ *    stored (rounded to bf16 when the caller asks), because the backward
+ *    recomputes it from that stored Z.  The backward of the pair is
+ *    dZ = (G W) * f'(Z) for an upstream G [M x K] and W [N x K].
  *
  * Reductions (d alpha, d gamma, d beta) are serial sums in index order in
  * long double.
@@ -433,6 +439,72 @@ int oracle_swish_channel_bwd(int layout, const int64_t shape[4], const double *x
     }
     for (int64_t c = 0; c < C; ++c) dalpha[c] = (double)acc[c];
     free(acc);
+    return 0;
+}
+
+/* ------------------------------------------------- matmul + activation */
+
+static uint16_t bf16_from_double(double v);
+
+static double bf16_value(double v)
+{
+    union {
+        uint32_t u;
+        float f;
+    } b;
+    b.u = (uint32_t)bf16_from_double(v) << 16;
+    return (double)b.f;
+}
+
+/* Z[m][n] = sum_k X[m][k] W[n][k]  (serial over k, long double);
+ * Y[m][n] = f(z) with z = Z[m][n], or z = Z[m][n] rounded to the nearest
+ * bf16 when round_z_bf16 is non-zero (the value a bf16 store of Z holds).
+ * absum (nullable) receives sum_k |X[m][k] W[n][k]|, the scale of the
+ * rounding error of any floating-point evaluation of the sum.  Y may be NULL. */
+int oracle_matmul_act_fwd(int act, int64_t M, int64_t N, int64_t K, const double *X, const double *W,
+                          double param, int round_z_bf16, double *Z, double *Y, double *absum)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || M < 0 || N < 0 || K < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            long double acc = 0.0L, aacc = 0.0L;
+            for (int64_t k = 0; k < K; ++k) {
+                long double t = (long double)X[m * K + k] * (long double)W[n * K + k];
+                acc += t;
+                aacc += fabsl(t);
+            }
+            double z = (double)acc;
+            Z[m * N + n] = z;
+            if (absum) absum[m * N + n] = (double)aacc;
+            if (Y) Y[m * N + n] = act_f(act, round_z_bf16 ? bf16_value(z) : z, param);
+        }
+    }
+    return 0;
+}
+
+/* D[m][n] = sum_k G[m][k] W[n][k] (serial over k, long double) and
+ * dZ[m][n] = D[m][n] f'(Z[m][n]), Z as stored.  D and absum (sum_k
+ * |G[m][k] W[n][k]|) are nullable. */
+int oracle_matmul_act_bwd(int act, int64_t M, int64_t N, int64_t K, const double *G, const double *W,
+                          const double *Z, double param, double *dZ, double *D, double *absum)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || M < 0 || N < 0 || K < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            long double acc = 0.0L, aacc = 0.0L;
+            for (int64_t k = 0; k < K; ++k) {
+                long double t = (long double)G[m * K + k] * (long double)W[n * K + k];
+                acc += t;
+                aacc += fabsl(t);
+            }
+            double d = (double)acc;
+            if (D) D[m * N + n] = d;
+            if (absum) absum[m * N + n] = (double)aacc;
+            dZ[m * N + n] = d * act_df(act, Z[m * N + n], param);
+        }
+    }
     return 0;
 }
 
