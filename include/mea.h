@@ -256,6 +256,43 @@ MEA_API mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layou
                                            const float *alpha, void *dx, float *dalpha,
                                            void *workspace, size_t ws_bytes, mea_stream_t stream);
 
+/* Matrix multiply with the activation fused into its epilogue, forward:
+ *   Z = X W^T  (bf16 inputs, fp32 accumulation on the tensor cores),
+ *   z = Z rounded to bf16 (written when z is non-NULL),
+ *   y = f(Z as stored in bf16) (written when y is non-NULL).
+ *   act, param  activation and its parameter, as in mea_act_fwd.
+ *   M, N, K     X is [M x K], W is [N x K], Z, y are [M x N]; M or N of 0 is
+ *               a no-op; K must be positive.  K and N must be multiples of 8
+ *               (rows of 16-byte multiples), each below 2^31; otherwise
+ *               MEA_ERR_UNSUPPORTED.
+ *   x, w        device, bf16, row-major (K contiguous), read only, 16-byte
+ *               aligned (else MEA_ERR_UNSUPPORTED).
+ *   z, y        device, bf16, row-major [M x N], 16-byte aligned, written;
+ *               at least one non-NULL; neither may overlap x, w or the other.
+ * Only Z needs to be kept for the backward (the save-input-only scheme,
+ * with the matmul output as the saved input); y feeds the next layer.
+ * Source: problem B07 of "What activations cost, in memory and in
+ * arithmetic", SOLUTION step 4 (the activation follows a d x d matrix
+ * multiply on the same tensor; its arithmetic is free beside it, its memory
+ * is not). */
+MEA_API mea_status_t mea_matmul_act_fwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *x,
+                                        const void *w, float param, void *z, void *y, mea_stream_t stream);
+
+/* Matrix multiply with the activation's derivative fused into its epilogue,
+ * backward: dz = (G W^T) * f'(z), f' recomputed from the stored z.
+ *   G           device bf16 [M x K] (the upstream gradient), read only.
+ *   W           device bf16 [N x K]: for a following layer out = y W2^T
+ *               with W2 [K x N], pass W = W2^T (N rows of K).
+ *   z           device bf16 [M x N], the stored pre-activation, read only.
+ *   dz          device bf16 [M x N], written; may be the same pointer as z
+ *               (each element is read before it is written), no partial
+ *               overlap with z, and no overlap with G or W.
+ *   Other arguments and restrictions as in mea_matmul_act_fwd.
+ * The product G W^T never reaches memory. */
+MEA_API mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *g,
+                                        const void *w, const void *z, float param, void *dz,
+                                        mea_stream_t stream);
+
 /* Backward with d alpha that allocates nothing and takes no workspace.
  * No counterpart on the pages: this is a library convenience, not part of
  * the method.  It computes exactly what mea_act_bwd computes (same kernel,

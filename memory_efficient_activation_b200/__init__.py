@@ -11,6 +11,7 @@ stream) into those calls; PyTorch is plumbing here, not the compute path.
 Functions (the C ABI's names without the ``mea_`` prefix):
     act_fwd, act_bwd, affine_swish_fwd, affine_swish_bwd,
     affine_act_fwd, affine_act_bwd, swish_channel_fwd, swish_channel_bwd,
+    matmul_act_fwd, matmul_act_bwd,
     act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes,
     affine_act_bwd_workspace_bytes, swish_channel_bwd_workspace_bytes
 Autograd / modules:
@@ -32,6 +33,7 @@ from ._capi import ACT_IDS, LAYOUT_IDS, MeaError
 __all__ = [
     "act_fwd", "act_bwd", "affine_swish_fwd", "affine_swish_bwd",
     "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
+    "matmul_act_fwd", "matmul_act_bwd",
     "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
     "affine_act_bwd_workspace_bytes", "swish_channel_bwd_workspace_bytes",
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
@@ -293,6 +295,59 @@ def swish_channel_bwd(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, la
                                             ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
     _capi.check("mea_swish_channel_bwd", st)
     return dx, da
+
+
+def _mat2d(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    _need_cuda(t)
+    return t
+
+
+def matmul_act_fwd(act: str, x: torch.Tensor, w: torch.Tensor, param: float = 1.0, want_z: bool = True,
+                   want_y: bool = True, z: torch.Tensor | None = None, y: torch.Tensor | None = None):
+    """Z = x w^T on the tensor cores (x [M, K], w [N, K], bf16), with the
+    activation in the epilogue: returns (z, y), z = Z in bf16 (the tensor to
+    keep for the backward) and y = f(z); either may be skipped (None)."""
+    _mat2d(x, "x")
+    _mat2d(w, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("x and w disagree in K")
+    if want_z and z is None:
+        z = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if want_y and y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    for t in (z, y):
+        if t is not None:
+            _need_cuda(t)
+    st = _capi.lib().mea_matmul_act_fwd(_act_id(act), M, N, K, x.data_ptr(), w.data_ptr(), float(param),
+                                         _ptr(z if want_z else None), _ptr(y if want_y else None), _stream(x))
+    _capi.check("mea_matmul_act_fwd", st)
+    return (z if want_z else None), (y if want_y else None)
+
+
+def matmul_act_bwd(act: str, g: torch.Tensor, w: torch.Tensor, z: torch.Tensor, param: float = 1.0,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """dz = (g w^T) * f'(z) with the product never written: g [M, K] the
+    upstream gradient, w [N, K] (the transpose of the next layer's weight),
+    z [M, N] the stored pre-activation (bf16)."""
+    _mat2d(g, "g")
+    _mat2d(w, "w")
+    _mat2d(z, "z")
+    M, K = g.shape
+    N = w.shape[0]
+    if w.shape[1] != K or z.shape != (M, N):
+        raise ValueError("g, w and z disagree in shape")
+    dz = torch.empty_like(z) if out is None else out
+    _need_cuda(dz)
+    st = _capi.lib().mea_matmul_act_bwd(_act_id(act), M, N, K, g.data_ptr(), w.data_ptr(), z.data_ptr(),
+                                         float(param), dz.data_ptr(), _stream(g))
+    _capi.check("mea_matmul_act_bwd", st)
+    return dz
 
 
 # ---------------------------------------------------------------- autograd

@@ -48,6 +48,8 @@ SIGNATURES = {
     "mea_swish_channel_bwd_workspace_bytes": (_sz, [_i, _i, _shape]),
     "mea_swish_channel_fwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp]),
     "mea_swish_channel_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mea_matmul_act_fwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _f, _vp, _vp, _vp]),
+    "mea_matmul_act_bwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _vp, _f, _vp, _vp]),
     "mea_act_bwd_dparam_noalloc": (_i, [_i, _i, _vp, _vp, _vp, _i64, _f, _vp, _vp, _vp]),
     "mea_status_string": (ctypes.c_char_p, [_i]),
     "mea_last_error": (ctypes.c_char_p, []),

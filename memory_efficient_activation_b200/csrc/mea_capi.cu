@@ -9,6 +9,7 @@
 #include "../../include/mea.h"
 #include "mea_channel_api.h"
 #include "mea_internal.h"
+#include "mea_matmul_api.h"
 
 namespace {
 
@@ -195,7 +196,7 @@ const char *mea_status_string(mea_status_t status)
 
 const char *mea_last_error(void) { return g_err; }
 
-int mea_version(void) { return 1 * 10000 + 1 * 100 + 0; }
+int mea_version(void) { return 1 * 10000 + 2 * 100 + 0; }
 
 mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y, int64_t n, float param,
                          const float *param_dev, mea_stream_t stream)
@@ -325,6 +326,86 @@ mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layout, const
 {
     return chan_bwd(1, "mea_swish_channel_bwd", MEA_SWISH, dtype, layout, shape, x, dy, alpha, nullptr, 1.f, dx,
                     dalpha, nullptr, workspace, ws_bytes, stream);
+}
+
+static mea_status_t check_matmul(const char *name, int act, int64_t M, int64_t N, int64_t K)
+{
+    (void)name;
+    if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", act);
+    if (M < 0 || N < 0 || K < 0) return fail(MEA_ERR_INVALID_ARG, "M, N and K must be non-negative");
+    const int64_t lim = (int64_t)1 << 31;
+    if (M >= lim || N >= lim || K >= lim) return fail(MEA_ERR_UNSUPPORTED, "M, N and K must be below 2^31");
+    return MEA_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mea_status_t mea_matmul_act_fwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *x, const void *w,
+                                float param, void *z, void *y, mea_stream_t stream)
+{
+    clear_error();
+    mea_status_t st = check_matmul("mea_matmul_act_fwd", act, M, N, K);
+    if (st != MEA_OK) return st;
+    if (M == 0 || N == 0) return MEA_OK;
+    if (K == 0) return fail(MEA_ERR_UNSUPPORTED, "K = 0 (an empty product) is not served");
+    if (K % 8 || N % 8) return fail(MEA_ERR_UNSUPPORTED, "K and N must be multiples of 8");
+    if (!x || !w) return fail(MEA_ERR_INVALID_ARG, "x or w is NULL");
+    if (!z && !y) return fail(MEA_ERR_INVALID_ARG, "z and y are both NULL");
+    if (!aligned16(x) || !aligned16(w) || (z && !aligned16(z)) || (y && !aligned16(y)))
+        return fail(MEA_ERR_UNSUPPORTED, "x, w, z and y must be 16-byte aligned");
+    const size_t bx = (size_t)M * K * 2, bw = (size_t)N * K * 2, bo = (size_t)M * N * 2;
+    for (void *o : {z, y}) {
+        if (!o) continue;
+        if (overlaps(o, bo, x, bx) || overlaps(o, bo, w, bw))
+            return fail(MEA_ERR_INVALID_ARG, "an output overlaps x or w");
+    }
+    if (z && y && overlaps(z, bo, y, bo)) return fail(MEA_ERR_INVALID_ARG, "z overlaps y");
+    mea::MatmulLaunch l{};
+    l.act = act;
+    l.mode = 0;
+    l.M = M;
+    l.N = N;
+    l.K = K;
+    l.x = x;
+    l.w = w;
+    l.out0 = z;
+    l.out1 = y;
+    l.param = param;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_matmul_act(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_matmul_act_fwd launch");
+}
+
+mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *g, const void *w,
+                                const void *z, float param, void *dz, mea_stream_t stream)
+{
+    clear_error();
+    mea_status_t st = check_matmul("mea_matmul_act_bwd", act, M, N, K);
+    if (st != MEA_OK) return st;
+    if (M == 0 || N == 0) return MEA_OK;
+    if (K == 0) return fail(MEA_ERR_UNSUPPORTED, "K = 0 (an empty product) is not served");
+    if (K % 8 || N % 8) return fail(MEA_ERR_UNSUPPORTED, "K and N must be multiples of 8");
+    if (!g || !w || !z || !dz) return fail(MEA_ERR_INVALID_ARG, "g, w, z or dz is NULL");
+    if (!aligned16(g) || !aligned16(w) || !aligned16(z) || !aligned16(dz))
+        return fail(MEA_ERR_UNSUPPORTED, "g, w, z and dz must be 16-byte aligned");
+    const size_t bg = (size_t)M * K * 2, bw = (size_t)N * K * 2, bo = (size_t)M * N * 2;
+    if (overlaps(dz, bo, g, bg) || overlaps(dz, bo, w, bw))
+        return fail(MEA_ERR_INVALID_ARG, "dz overlaps g or w");
+    if (partial_overlap(dz, z, bo)) return fail(MEA_ERR_INVALID_ARG, "dz partially overlaps z");
+    mea::MatmulLaunch l{};
+    l.act = act;
+    l.mode = 1;
+    l.M = M;
+    l.N = N;
+    l.K = K;
+    l.x = g;
+    l.w = w;
+    l.zin = z;
+    l.out1 = dz;
+    l.param = param;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_matmul_act(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_matmul_act_bwd launch");
 }
 
 }  // extern "C"

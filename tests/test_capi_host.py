@@ -34,7 +34,7 @@ def _header_enum(name):
 
 def test_every_declared_symbol_is_exported(lib):
     declared = _header_functions()
-    assert len(declared) == 16, declared
+    assert len(declared) == 18, declared
     for fn in declared:
         assert hasattr(lib, fn), fn
         assert fn in _capi.SIGNATURES, fn
@@ -55,7 +55,7 @@ def test_enums_match_header():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.mea_version() == 10100
+    assert lib.mea_version() == 10200
     for st in range(5):
         assert lib.mea_status_string(st)
     assert lib.mea_status_string(99) == b"unknown status"
@@ -176,3 +176,22 @@ def test_affine_act_and_channel_validation(lib):
     assert bc(1, 1, s, X, G, 0x700000, D, 0x720000, 0x800000, cneed - 1, None) == _capi.MEA_ERR_WORKSPACE
     assert bc(1, 1, s, X, G, 0x700000, G + 2, 0x720000, 0x800000, cneed, None) == _capi.MEA_ERR_INVALID_ARG
     assert lib.mea_swish_channel_bwd_workspace_bytes(1, 1, _capi.shape4((1, -2, 1, 1))) == 0
+
+
+def test_matmul_validation(lib):
+    f, b = lib.mea_matmul_act_fwd, lib.mea_matmul_act_bwd
+    A, Wt, Z, Yo = 0x1000000, 0x2000000, 0x3000000, 0x4000000
+    assert f(9, 16, 16, 16, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(0, -1, 16, 16, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(0, 0, 16, 16, None, None, 1.0, None, None, None) == _capi.MEA_OK      # empty: no-op
+    assert f(0, 16, 16, 0, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_UNSUPPORTED  # K = 0
+    assert f(0, 16, 12, 16, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_UNSUPPORTED # N % 8
+    assert f(0, 16, 16, 20, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_UNSUPPORTED # K % 8
+    assert f(0, 16, 16, 16, A + 8, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_UNSUPPORTED
+    assert f(0, 16, 16, 16, A, Wt, 1.0, None, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(0, 16, 16, 16, A, Wt, 1.0, A + 256, None, None) == _capi.MEA_ERR_INVALID_ARG  # z overlaps x
+    assert f(0, 16, 16, 16, A, Wt, 1.0, Z, Z + 256, None) == _capi.MEA_ERR_INVALID_ARG     # z overlaps y
+    assert f(0, 1 << 31, 16, 16, A, Wt, 1.0, Z, Yo, None) == _capi.MEA_ERR_UNSUPPORTED
+    assert b(0, 16, 16, 16, A, Wt, Z, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b(0, 16, 16, 16, A, Wt, Z, 1.0, Z + 16, None) == _capi.MEA_ERR_INVALID_ARG      # partial overlap
+    assert b(0, 16, 16, 16, A, Wt, Z, 1.0, Wt, None) == _capi.MEA_ERR_INVALID_ARG          # dz overlaps w
