@@ -44,6 +44,7 @@ WORKLOAD = "swish_bf16_8x2048x4096"
 SHAPE = (8, 2048, 4096)
 DTYPE = "bf16"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 DOMINANT_KERNEL = "act_kernel<Swish, Bf16, MODE 1> (mea_act_bwd)"
 
 
@@ -74,6 +75,16 @@ def _max_over_ranks(v: float, ws: int) -> float:
         return v
     from memory_efficient_activation_b200 import dist as mdist
     return mdist.max_over_ranks(v, device="cuda")
+
+
+def _bf16_peak():
+    """(TFLOP/s, kind): the measured burst bf16 matmul rate, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured burst"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def _peaks():
@@ -573,6 +584,32 @@ def run_secondary(args):
                         [lambda b=b, d=d, ws=ws, a=a: mea.swish_channel_bwd(b[0], b[1], a, "nchw", out=b[3], dalpha=d,
                                                                             workspace=ws)
                          for b, d, ws in zip(sets, ds, wss)], accounting.channel_swish_bwd_bytes(w.n, "f32", C)))
+    elif wl == "matmul_act_bf16":
+        # the d x d matmul of problem B07 ([8 x 2048, 4096] x [4096, 4096]) with
+        # the activation in its epilogue, and the same work unfused (cuBLAS
+        # through torch.matmul, then the streaming activation kernels)
+        M, N, K = 16384, 4096, 4096
+        flops = 2 * M * N * K
+        tf_peak = _bf16_peak()
+        x = synthetic.normal(M * K, 1.0, 41, synthetic.STREAM_X, "bf16").view(M, K)
+        w = synthetic.normal(N * K, K ** -0.5, 41, synthetic.STREAM_PARAM, "bf16").view(N, K)
+        nbytes = (2 * M * K + N * K + 2 * M * N) * 2
+        k = _sets_for(nbytes)
+        sets = [[x.to(dev), w.to(dev), x.to(dev),
+                 torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                 torch.empty(M, N, dtype=torch.bfloat16, device=dev)] for _ in range(k)]   # x, w, g, z, out
+        for act in ("relu", "swish", "gelu_erf"):
+            ops.append((f"fused_fwd_{act}", [lambda a=act, b=b: mea.matmul_act_fwd(a, b[0], b[1], 1.0, z=b[3], y=b[4])
+                                             for b in sets], flops))
+            ops.append((f"fused_bwd_{act}", [lambda a=act, b=b: mea.matmul_act_bwd(a, b[2], b[1], b[3], 1.0, out=b[4])
+                                             for b in sets], flops))
+        ops.append(("cublas_matmul", [lambda b=b: torch.matmul(b[0], b[1].t(), out=b[3]) for b in sets], flops))
+        ops.append(("act_fwd_gelu_erf_on_z", [lambda b=b: mea.act_fwd("gelu_erf", b[3], out=b[4]) for b in sets],
+                    accounting.fwd_bytes(M * N, "bf16")))
+        ops.append(("act_bwd_gelu_erf_on_z", [lambda b=b: mea.act_bwd("gelu_erf", b[3], b[4], out=b[4]) for b in sets],
+                    accounting.bwd_bytes(M * N, "bf16")))
+        args._flop_ops = {name for name, _, _ in ops if not name.startswith("act_")}
+        args._tf_peak = tf_peak
     elif wl == "memory_study":
         return run_memory_study(args)
     elif wl == "swish_f32_1m":
@@ -589,10 +626,10 @@ def run_secondary(args):
     with torch.cuda.stream(cap), _ClockSampler(0) as clk:
         per, total = _time_ops(ops, args.steps, args.warmup, cap)
     stream.wait_stream(cap)
-    tot_bytes = sum(b for _, _, b in ops)
+    tot_bytes = sum(b for name, _, b in ops if name not in getattr(args, "_flop_ops", ()))
     out = {
         "workload": wl,
-        "value": round(tot_bytes / (total * 1e-3) / 1e9, 2),
+        "value": round(tot_bytes / (total * 1e-3) / 1e9, 2) if not getattr(args, "_flop_ops", None) else None,
         "unit": "GB/s",
         "steps": args.steps,
         "warmup": args.warmup,
@@ -600,8 +637,12 @@ def run_secondary(args):
         "peak_kind": peak_kind,
         "timing": "mean device time per launch from CUDA-graph replays of 24 back-to-back launches rotating over "
                   "buffer sets that together exceed 3x L2",
-        "ops": {name: {"ms": round(per[name], 5), "GB/s": round(b / (per[name] * 1e-3) / 1e9, 1),
-                       "frac": round(b / (per[name] * 1e-3) / 1e9 / peak, 4), "bytes": b, "sets": len(fns)}
+        "ops": {name: ({"ms": round(per[name], 5), "TFLOP/s": round(b / (per[name] * 1e-3) / 1e12, 1),
+                        "frac": round(b / (per[name] * 1e-3) / 1e12 / args._tf_peak[0], 4),
+                        "peak": args._tf_peak, "flops": b, "sets": len(fns)}
+                       if name in getattr(args, "_flop_ops", ()) else
+                       {"ms": round(per[name], 5), "GB/s": round(b / (per[name] * 1e-3) / 1e9, 1),
+                        "frac": round(b / (per[name] * 1e-3) / 1e9 / peak, 4), "bytes": b, "sets": len(fns)})
                 for name, fns, b in ops},
         "clocks": clk.summary(),
     }
@@ -698,7 +739,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="swish_bf16",
                     choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
-                             "affine_family_nhwc_bf16", "swish_channel_f32", "swish_f32_1m", "memory_study"],
+                             "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "swish_f32_1m",
+                             "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:

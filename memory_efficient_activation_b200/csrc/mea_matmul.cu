@@ -14,21 +14,27 @@
 // and in the backward multiplies the product by f'(Z) before it ever
 // reaches memory (no G W^T tensor is written or re-read).
 //
-// Kernel (persistent, one CTA per SM, 192 threads):
-//   warp 0      one thread issues TMA loads of 128 x 64 tiles of X and
-//               256 x 64 tiles of W (128-byte swizzle) into a 4-stage ring
-//   warp 1      allocates 512 tensor-memory columns (two 128 x 256 fp32
-//               accumulators); one thread issues tcgen05.mma (M 128, N 256,
-//               K 16, bf16 in, fp32 accumulate) and commits each stage back
-//               to the producer and each finished accumulator to the
-//               epilogue
-//   warps 2..5  read an accumulator (tcgen05.ld, one row per thread), apply
-//               the epilogue, store, and release the accumulator, while the
-//               MMA warp fills the other one
-// Tiles are assigned round-robin (tile blockIdx.x + i gridDim.x); each
-// tile's sum runs over k in one fixed order, so results do not depend on
-// the grid.  Every barrier wait is bounded: one that expires sets
-// g_matmul_error and the roles stop issuing work.
+// Kernel (persistent, clusters of two CTAs on two SMs, 192 threads each):
+// a CTA pair owns a 256 x 256 output tile and multiplies it with the
+// two-SM form of the tensor-core instruction (tcgen05.mma.cta_group::2):
+// each CTA stages its own 128 rows of X and its own 128 rows of W per K
+// step, and one instruction issued by the pair's first CTA reads A from
+// both CTAs' shared memory (M 256) and B from both (N 256), writing a
+// 128 x 256 fp32 accumulator into each CTA's tensor memory.  Per CTA:
+//   warp 0      one thread issues TMA loads of 128 x 64 tiles of X and W
+//               (128-byte swizzle, no multicast) into a 6-stage ring; the
+//               loads of both CTAs complete on the first CTA's barrier
+//   warp 1      allocates 512 tensor-memory columns (two accumulators) in
+//               both CTAs; in the first CTA one thread issues the MMAs and
+//               commits each stage and each finished accumulator to the
+//               barriers of both CTAs (tcgen05.commit multicast)
+//   warps 2..5  read this CTA's accumulator rows (tcgen05.ld, one row per
+//               thread), apply the epilogue, store, and release the
+//               accumulator to the first CTA, while the other is filled
+// Tiles are assigned round-robin to CTA pairs; each tile's sum runs over k
+// in one fixed order, so results do not depend on the grid.  Every barrier
+// wait is bounded: one that expires sets g_matmul_error and the roles stop
+// issuing work.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -47,12 +53,13 @@ __device__ unsigned int g_matmul_error = 0;
 
 namespace {
 
-constexpr int kBM = kMatmulBM, kBN = kMatmulBN, kBK = kMatmulBK;
+constexpr int kBM = kMatmulBM, kBN = kMatmulBN, kBK = kMatmulBK;   // tile of a CTA pair: 256 x 256
+constexpr int kHalf = 128;                                  // rows of X and of W one CTA stages
 constexpr int kUmmaK = 16;                                  // K of one bf16 MMA
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kThreadsMM = 192;
-constexpr uint32_t kStageA = kBM * kBK * 2;                  // 16 KB
-constexpr uint32_t kStageB = kBN * kBK * 2;                  // 32 KB
+constexpr uint32_t kStageA = kHalf * kBK * 2;                // 16 KB
+constexpr uint32_t kStageB = kHalf * kBK * 2;                // 16 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kAccCols = kBN;                           // fp32 columns per accumulator
 constexpr uint32_t kTmemCols = 2 * kAccCols;                 // 512: all of tensor memory
@@ -60,7 +67,7 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
 
 // Instruction descriptor of tcgen05.mma.kind::f16: fp32 accumulator (bits
 // 4-5 = 1), A and B bf16 (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15,
-// 16 = 0), N / 8 in bits 17-22, M / 16 in bits 24-28.
+// 16 = 0), N / 8 in bits 17-22, M / 16 in bits 24-28 (M 256: the pair).
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
 
@@ -78,30 +85,60 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+// TMA load into this CTA's shared memory that completes on `bar`, a
+// shared::cluster address that may lie in the other CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
 {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(dst),
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate)
+// shared::cluster address of the variable at `saddr` in CTA `rank` of the
+// cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate)
 {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
             tmem_d),
         "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
         : "memory");
 }
 
-// Arrives once on `bar` when every tcgen05.mma this thread issued so far has
-// completed.
-__device__ __forceinline__ void umma_commit(uint32_t bar)
+// Arrives once on the barrier at `bar` in both CTAs of the pair when every
+// tcgen05.mma this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -200,7 +237,7 @@ __device__ __forceinline__ void epilogue32(const uint32_t (&acc)[32], const Coef
 }
 
 template <class A, int MODE>
-__global__ void __launch_bounds__(kThreadsMM, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsMM, 1)
 matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_w, int M,
                   int N, int K, float param, const uint16_t *__restrict__ zin, uint16_t *__restrict__ out0,
                   uint16_t *__restrict__ out1)
@@ -216,39 +253,42 @@ matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();          // 0: issues the MMAs of the pair
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int tiles_m = (M + kBM - 1) / kBM, tiles_n = (N + kBN - 1) / kBN;
     const int ntiles = tiles_m * tiles_n;
     const int kblocks = (K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_addr(full + s), 1);
-            mbar_init(smem_addr(empty + s), 1);
+            mbar_init(smem_addr(full + s), 1);     // the first CTA's producer; bytes of both CTAs
+            mbar_init(smem_addr(empty + s), 1);    // one commit from the first CTA
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_addr(acc_full + b), 1);
-            mbar_init(smem_addr(acc_empty + b), 4);
+            mbar_init(smem_addr(acc_empty + b), 8); // four epilogue warps of each CTA
         }
         mbar_init_fence();
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                      "r"(kTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();                                // barriers of both CTAs initialised
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
-            // TMA producer
+            // TMA producer: this CTA's rows of X and W; completion on the
+            // first CTA's barrier
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int t = pair; t < ntiles && ok; t += npairs) {
                 const int tm = t / tiles_n, tn = t % tiles_n;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int s = it % kStages, round = it / kStages;
@@ -257,23 +297,24 @@ matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_consta
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_addr(full + s);
-                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    const uint32_t fb = cluster_addr(smem_addr(full + s), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(smem_addr(full + s), 2 * kStageBytes);
                     const uint32_t sa = sbase + s * kStageBytes;
-                    tma_load_2d(sa, &tma_x, kb * kBK, tm * kBM, fb);
-                    tma_load_2d(sa + kStageA, &tma_w, kb * kBK, tn * kBN, fb);
+                    tma_load_2d_pair(sa, &tma_x, kb * kBK, tm * kBM + rank * kHalf, fb);
+                    tma_load_2d_pair(sa + kStageA, &tma_w, kb * kBK, tn * kBN + rank * kHalf, fb);
                 }
             }
-            // every load issued has landed before teardown
+            // every load issued has landed before teardown: this CTA's stages
+            // are released (empty) once the MMAs that read them complete
             for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
-                if (!mbar_wait(smem_addr(full + j % kStages), (j / kStages) & 1)) record_error();
+                if (!mbar_wait(smem_addr(empty + j % kStages), (j / kStages) & 1)) record_error();
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // MMA issuer
+        if (lane == 0 && rank == 0) {
+            // MMA issuer of the pair
             int it = 0, lt = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++lt) {
+            for (int t = pair; t < ntiles && ok; t += npairs, ++lt) {
                 const int b = lt & 1, use = lt >> 1;
                 if (use > 0 && !mbar_wait(smem_addr(acc_empty + b), (use & 1) ^ 1)) {
                     record_error();
@@ -292,20 +333,22 @@ matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_consta
                     const uint32_t sa = sbase + s * kStageBytes;
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k)
-                        umma_bf16(d, sdesc_sw128(sa + k * kUmmaK * 2), sdesc_sw128(sa + kStageA + k * kUmmaK * 2),
-                                  (kb | k) != 0);
-                    umma_commit(smem_addr(empty + s));
+                        umma_bf16_pair(d, sdesc_sw128(sa + k * kUmmaK * 2),
+                                       sdesc_sw128(sa + kStageA + k * kUmmaK * 2), (kb | k) != 0);
+                    umma_commit_pair(smem_addr(empty + s));
                 }
-                if (ok) umma_commit(smem_addr(acc_full + b));
+                if (ok) umma_commit_pair(smem_addr(acc_full + b));
             }
         }
         __syncwarp();
     } else {
-        // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31
+        // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 of
+        // this CTA, i.e. rows rank * 128 + 32 (w % 4) + lane of the tile
         const int q = warp & 3;
         const Coef k = A::coef(param);
+        const uint32_t release = cluster_addr(smem_addr(acc_empty), 0);
         int lt = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+        for (int t = pair; t < ntiles; t += npairs, ++lt) {
             const int b = lt & 1, use = lt >> 1;
             if (!mbar_wait(smem_addr(acc_full + b), use & 1)) {
                 record_error();
@@ -313,7 +356,7 @@ matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_consta
             }
             tc_fence_after();
             const int tm = t / tiles_n, tn = t % tiles_n;
-            const int row = tm * kBM + q * 32 + lane;
+            const int row = tm * kBM + (int)rank * kHalf + q * 32 + lane;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t v[32];
@@ -328,15 +371,15 @@ matmul_act_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_consta
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(acc_empty + b));
+            if (lane == 0) mbar_arrive_cluster(release + 8 * b);
         }
     }
     pdl_trigger();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();                                // no CTA leaves while its pair may touch its memory
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -381,9 +424,9 @@ cudaError_t launch_one(const MatmulLaunch &a, const CUtensorMap &mx, const CUten
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t tiles = ((a.M + kBM - 1) / kBM) * ((a.N + kBN - 1) / kBN);
-    const int sms = sm_count();
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kThreadsMM), kSmemBytes, a.stream, mx, mw, (int)a.M,
+    const int pairs_max = sm_count() / 2;
+    const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
+    return launch_pdl(kernel, dim3((unsigned)(2 * pairs)), dim3(kThreadsMM), kSmemBytes, a.stream, mx, mw, (int)a.M,
                       (int)a.N, (int)a.K, a.param, static_cast<const uint16_t *>(a.zin),
                       static_cast<uint16_t *>(a.out0), static_cast<uint16_t *>(a.out1));
 }
@@ -408,7 +451,7 @@ cudaError_t by_act(const MatmulLaunch &a, const CUtensorMap &mx, const CUtensorM
 cudaError_t launch_matmul_act(const MatmulLaunch &a)
 {
     CUtensorMap mx, mw;
-    if (!make_map(&mx, a.x, a.M, a.K, kBM) || !make_map(&mw, a.w, a.N, a.K, kBN)) return cudaErrorInvalidValue;
+    if (!make_map(&mx, a.x, a.M, a.K, kHalf) || !make_map(&mw, a.w, a.N, a.K, kHalf)) return cudaErrorInvalidValue;
     return a.mode == 0 ? by_act<0>(a, mx, mw) : by_act<1>(a, mx, mw);
 }
 

@@ -29,7 +29,7 @@ struct MatmulLaunch {
 cudaError_t launch_matmul_act(const MatmulLaunch &a);
 
 // Tile shape of the kernel (rows of X, rows of W, K per pipeline stage).
-constexpr int kMatmulBM = 128;
+constexpr int kMatmulBM = 256;
 constexpr int kMatmulBN = 256;
 constexpr int kMatmulBK = 64;
 
