@@ -610,6 +610,8 @@ def run_secondary(args):
                     accounting.bwd_bytes(M * N, "bf16")))
         args._flop_ops = {name for name, _, _ in ops if not name.startswith("act_")}
         args._tf_peak = tf_peak
+    elif wl == "mlp_bf16":
+        return run_mlp(args)
     elif wl == "memory_study":
         return run_memory_study(args)
     elif wl == "swish_f32_1m":
@@ -649,6 +651,60 @@ def run_secondary(args):
     if wl == "swish_f32_1m":
         out["note"] = "21 MB of traffic per step fits in the 126 MB L2: an L2-resident figure, not HBM bandwidth"
     return out
+
+
+def run_mlp(args, M: int = 16384, d: int = 4096, h: int = 4096, act: str = "gelu_tanh"):
+    """One MLP block (Linear d -> h, activation, Linear h -> d; bf16, no bias)
+    at the d x d size of problem B07, forward + backward: the memory-efficient
+    block (fused matmul epilogues, keeps x and z) against the same block in
+    plain PyTorch autograd (F.linear, F.gelu, F.linear).  Reports time per
+    step, matmul throughput (6 matmuls of 2 M d h FLOPs), the activation
+    memory held between forward and backward, and the peak during a step."""
+    import torch.nn.functional as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    m = mea.MemoryEfficientMLP(d, h, act).to(dev)
+    x = synthetic.normal(M * d, 1.0, 43, synthetic.STREAM_X, "bf16").view(M, d).to(dev).requires_grad_(True)
+    dout = synthetic.normal(M * d, 1.0, 43, synthetic.STREAM_DY, "bf16").view(M, d).to(dev)
+
+    def ours():
+        return m(x)
+
+    def plain():
+        return F.linear(F.gelu(F.linear(x, m.w1), approximate="tanh"), m.w2)
+
+    flops = 6 * 2 * M * d * h
+    res = {}
+    with _ClockSampler(0) as clk:
+        for name, fwd in (("memory_efficient", ours), ("plain_pytorch", plain)):
+            for _ in range(max(3, args.warmup)):
+                fwd().backward(dout)
+            x.grad = None
+            m.w1.grad = None
+            m.w2.grad = None
+            torch.cuda.synchronize()
+            base = torch.cuda.memory_allocated()
+            out = fwd()
+            torch.cuda.synchronize()
+            held = torch.cuda.memory_allocated() - base - out.numel() * out.element_size()
+            torch.cuda.reset_peak_memory_stats()
+            out.backward(dout)
+            torch.cuda.synchronize()
+            peak = torch.cuda.max_memory_allocated() - base
+            del out
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            for _ in range(args.steps):
+                fwd().backward(dout)
+            e.record()
+            torch.cuda.synchronize()
+            ms = s.elapsed_time(e) / args.steps
+            res[name] = {"ms_per_step": round(ms, 4), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1),
+                         "activation_bytes_held": int(held), "backward_peak_bytes": int(peak)}
+    return {"workload": "mlp_bf16", "shape": {"tokens": M, "d_model": d, "d_hidden": h}, "act": act,
+            "steps": args.steps, "warmup": args.warmup, "bf16_peak": _bf16_peak(), "results": res,
+            "speedup": round(res["plain_pytorch"]["ms_per_step"] / res["memory_efficient"]["ms_per_step"], 4),
+            "clocks": clk.summary()}
 
 
 class _PlainSwish(torch.nn.Module):
@@ -739,8 +795,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="swish_bf16",
                     choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
-                             "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "swish_f32_1m",
-                             "memory_study"],
+                             "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "mlp_bf16",
+                             "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:

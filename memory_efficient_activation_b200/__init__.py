@@ -18,7 +18,8 @@ Autograd / modules:
     ActivationFunction, MemoryEfficientActivation, MemoryEfficientSwish,
     AffineSwishFunction, MemoryEfficientAffineSwish,
     AffineActFunction, MemoryEfficientAffineActivation,
-    SwishChannelFunction, MemoryEfficientChannelSwish
+    SwishChannelFunction, MemoryEfficientChannelSwish,
+    MLPFunction, MemoryEfficientMLP
 """
 from __future__ import annotations
 
@@ -39,7 +40,8 @@ __all__ = [
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
     "AffineSwishFunction", "MemoryEfficientAffineSwish",
     "AffineActFunction", "MemoryEfficientAffineActivation",
-    "SwishChannelFunction", "MemoryEfficientChannelSwish", "MeaError", "ACTIVATIONS",
+    "SwishChannelFunction", "MemoryEfficientChannelSwish", "MLPFunction", "MemoryEfficientMLP",
+    "MeaError", "ACTIVATIONS",
 ]
 
 ACTIVATIONS = tuple(ACT_IDS)
@@ -501,3 +503,57 @@ class MemoryEfficientChannelSwish(torch.nn.Module):
 
     def forward(self, x):
         return SwishChannelFunction.apply(x, self.alpha, self.layout)
+
+
+class MLPFunction(torch.autograd.Function):
+    """out = f(x W1^T) W2^T that keeps x and z = x W1^T (bf16) for the
+    backward, not f(z): the first matmul writes z and f(z) from one epilogue,
+    and the backward multiplies dout W2 by f'(z) inside the matmul that forms
+    it (matmul_act_bwd), recomputing f(z) only for W2's gradient.  The two
+    other products (f(z) W2^T forward; dW2, dW1, dx backward) are plain
+    matmuls (torch.matmul)."""
+
+    @staticmethod
+    def forward(ctx, x, w1, w2, act: str, param: float):
+        z, y = matmul_act_fwd(act, x, w1, param)
+        out = torch.matmul(y, w2.t())
+        ctx.act, ctx.param = act, param
+        ctx.save_for_backward(x, w1, w2, z)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        x, w1, w2, z = ctx.saved_tensors
+        dout = dout.contiguous()
+        y = act_fwd(ctx.act, z, ctx.param)
+        dw2 = torch.matmul(dout.t(), y)
+        del y                                  # freed before dz exists: one hidden-sized buffer at a time
+        dz = matmul_act_bwd(ctx.act, dout, w2.t().contiguous(), z, ctx.param)
+        dw1 = torch.matmul(dz.t(), x)
+        dx = torch.matmul(dz, w1)
+        return dx, dw1, dw2, None, None
+
+
+class MemoryEfficientMLP(torch.nn.Module):
+    """Linear(d_model -> d_hidden, no bias) -> activation -> Linear(d_hidden
+    -> d_model, no bias) in bf16, keeping only the input and the hidden
+    pre-activation for the backward.  d_model and d_hidden must be multiples
+    of 8; inputs are [..., d_model] bf16 CUDA tensors."""
+
+    def __init__(self, d_model: int, d_hidden: int, act: str = "gelu_tanh", param: float | None = None):
+        super().__init__()
+        _act_id(act)
+        if d_model % 8 or d_hidden % 8:
+            raise ValueError("d_model and d_hidden must be multiples of 8")
+        self.act = act
+        self.param = (0.01 if act == "leaky_relu" else 1.0) if param is None else float(param)
+        self.w1 = torch.nn.Parameter(torch.empty(d_hidden, d_model, dtype=torch.bfloat16))
+        self.w2 = torch.nn.Parameter(torch.empty(d_model, d_hidden, dtype=torch.bfloat16))
+        with torch.no_grad():
+            self.w1.normal_(0.0, d_model ** -0.5)
+            self.w2.normal_(0.0, d_hidden ** -0.5)
+
+    def forward(self, x):
+        shape = x.shape
+        out = MLPFunction.apply(x.reshape(-1, shape[-1]).contiguous(), self.w1, self.w2, self.act, self.param)
+        return out.view(*shape[:-1], out.shape[-1])

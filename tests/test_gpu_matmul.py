@@ -194,3 +194,59 @@ def test_matmul_act_matches_unfused_path():
         # dz2 saw the product rounded to bf16 first; the fused path did not
         dist = np.abs(_ordered(bf16_bits(dz)) - _ordered(bf16_bits(dz2)))
         assert dist.max() <= 1, (act, dist.max())
+
+
+def _mlp_ref(act, p, x, w1, w2):
+    """float64 torch autograd of the same MLP (a library check of the
+    module's plumbing, not of the kernels' rounding)."""
+    import torch.nn.functional as F
+    fn = {
+        "relu": lambda t: torch.relu(t),
+        "leaky_relu": lambda t: F.leaky_relu(t, negative_slope=p),
+        "sigmoid": torch.sigmoid,
+        "tanh": torch.tanh,
+        "gelu_erf": lambda t: F.gelu(t, approximate="none"),
+        "gelu_tanh": lambda t: F.gelu(t, approximate="tanh"),
+        "swish": lambda t: t * torch.sigmoid(p * t),
+    }[act]
+    xd = x.double().requires_grad_(True)
+    w1d = w1.double().requires_grad_(True)
+    w2d = w2.double().requires_grad_(True)
+    out = fn(xd @ w1d.t()) @ w2d.t()
+    return out, xd, w1d, w2d
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "swish", "relu"])
+def test_memory_efficient_mlp_module(act):
+    # normwise agreement with float64 autograd: every bf16 store (z, f(z),
+    # dz, and the outputs) rounds by at most 2^-9 relative, and the two
+    # matmul stages compound a few of them: 1e-2 normwise bounds it
+    torch.manual_seed(0)
+    M, d, h = 512, 256, 1024
+    m = mea.MemoryEfficientMLP(d, h, act).cuda()
+    x = _bf16(M * d, 1.0, 37, synthetic.STREAM_X).view(4, M // 4, d).cuda().requires_grad_(True)
+    dout = _bf16(M * d, 1.0, 37, synthetic.STREAM_DY).view(4, M // 4, d).cuda()
+    saved = []
+
+    def pack(t):
+        saved.append(t)
+        return t
+
+    with torch.autograd.graph.saved_tensors_hooks(pack, lambda t: t):
+        out = m(x)
+    out.backward(dout)
+    torch.cuda.synchronize()
+    p = m.param
+    ref, xd, w1d, w2d = _mlp_ref(act, p, x.detach().cpu().view(M, d), m.w1.detach().cpu(), m.w2.detach().cpu())
+    ref.backward(dout.cpu().view(M, d).double())
+
+    def rel(a, b):
+        return float((a.double().cpu() - b).norm() / b.norm())
+
+    assert rel(out.view(M, d), ref.detach()) < 1e-2
+    assert rel(x.grad.view(M, d), xd.grad) < 1e-2
+    assert rel(m.w1.grad, w1d.grad) < 1e-2
+    assert rel(m.w2.grad, w2d.grad) < 1e-2
+    # saved for the backward: x, w1, w2 and z = x w1^T, not f(z)
+    hidden = [t for t in saved if t.dim() == 2 and t.shape == (M, h)]
+    assert len(hidden) == 1
