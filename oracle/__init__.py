@@ -21,6 +21,9 @@ Sources (by page and section):
 * "What activations cost, in memory and in arithmetic" (asifuddin.com,
   problem B07), GIVEN: the activation family; SOLUTION step 4: the matrix
   multiply the activation follows (matmul_act_fwd / matmul_act_bwd).
+* "A memory-efficient implementation of DenseNets", "Motivation": the
+  concatenation and batch normalization whose outputs are re-populated in
+  the backward (concat_bn_relu_fwd / concat_bn_relu_bwd).
 
 Parity pins for every function here live in ``tests/test_oracle_*.py``.
 """
@@ -103,6 +106,10 @@ def _load():
         lib.oracle_matmul_act_fwd.restype = ctypes.c_int
         lib.oracle_matmul_act_bwd.argtypes = [ctypes.c_int, i64, i64, i64, d, d, d, ctypes.c_double, d, d, d]
         lib.oracle_matmul_act_bwd.restype = ctypes.c_int
+        lib.oracle_bn_relu_fwd.argtypes = [i64, i64, i64, d, d, d, ctypes.c_double, d, d, d, d]
+        lib.oracle_bn_relu_fwd.restype = ctypes.c_int
+        lib.oracle_bn_relu_bwd.argtypes = [i64, i64, i64, d, d, d, d, d, d, ctypes.c_double, d, d, d, d]
+        lib.oracle_bn_relu_bwd.restype = ctypes.c_int
         lib.oracle_round_bf16.argtypes = [d, ctypes.POINTER(ctypes.c_uint16), i64]
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_f32.argtypes = [d, ctypes.POINTER(ctypes.c_float), i64]
@@ -308,6 +315,47 @@ def matmul_act_bwd(act: str, G, W, Z, param: float = 1.0):
     if rc:
         raise ValueError(f"oracle_matmul_act_bwd failed: {rc}")
     return dZ, D, S
+
+
+def concat_bn_relu_fwd(pieces, gamma, beta, eps: float = 1e-5):
+    """y = max(BN(concat(pieces, channel axis)), 0) with batch statistics.
+    pieces: NCHW arrays [N, k_i, H, W].  Returns (y [N, C, H, W], mean [C],
+    biased var [C], y_scale)."""
+    x = np.ascontiguousarray(np.concatenate([np.asarray(p, dtype=np.float64) for p in pieces], axis=1))
+    N, C = x.shape[0], x.shape[1]
+    HW = int(np.prod(x.shape[2:]))
+    gamma, beta = _f64(gamma), _f64(beta)
+    y = np.empty_like(x)
+    ys = np.empty_like(x)
+    mean = np.empty(C)
+    var = np.empty(C)
+    rc = _load().oracle_bn_relu_fwd(N, C, HW, _ptr(x), _ptr(gamma), _ptr(beta), float(eps), _ptr(y), _ptr(mean),
+                                    _ptr(var), _ptr(ys))
+    if rc:
+        raise ValueError(f"oracle_bn_relu_fwd failed: {rc}")
+    return y, mean, var, ys
+
+
+def concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, var, eps: float = 1e-5):
+    """Backward of concat_bn_relu_fwd from the pieces, dy [N, C, H, W] and the
+    batch statistics.  Returns (list of d piece, dgamma, dbeta, dx_scale as a
+    list split like the pieces)."""
+    pieces = [np.asarray(p, dtype=np.float64) for p in pieces]
+    x = np.ascontiguousarray(np.concatenate(pieces, axis=1))
+    dy = np.ascontiguousarray(np.asarray(dy, dtype=np.float64)).reshape(x.shape)
+    N, C = x.shape[0], x.shape[1]
+    HW = int(np.prod(x.shape[2:]))
+    gamma, beta, mean, var = _f64(gamma), _f64(beta), _f64(mean), _f64(var)
+    dx = np.empty_like(x)
+    sc = np.empty_like(x)
+    dg = np.empty(C)
+    db = np.empty(C)
+    rc = _load().oracle_bn_relu_bwd(N, C, HW, _ptr(x), _ptr(dy), _ptr(gamma), _ptr(beta), _ptr(mean), _ptr(var),
+                                    float(eps), _ptr(dx), _ptr(dg), _ptr(db), _ptr(sc))
+    if rc:
+        raise ValueError(f"oracle_bn_relu_bwd failed: {rc}")
+    cuts = np.cumsum([p.shape[1] for p in pieces])[:-1]
+    return np.split(dx, cuts, axis=1), dg, db, np.split(sc, cuts, axis=1)
 
 
 def round_bf16(v) -> np.ndarray:

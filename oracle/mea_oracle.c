@@ -39,6 +39,15 @@
  *    (Hendrycks and Gimpel, 2016); 1 + tanh(u) is evaluated as 2 Sigmoid(2u).
  *  - Fused affine + Swish: z = gamma_c x + beta_c, y = z Sigmoid(z) (alpha 1),
  *    channel c = i mod C for NHWC and (i / (H W)) mod C for NCHW.
+ *  - Concatenation + batch normalization + ReLU ("A memory-efficient
+ *    implementation of DenseNets", section "Motivation": the outputs of every
+ *    concatenation and batch normalization live in shared allocations and
+ *    are re-populated in the backward).  The page names the operations only;
+ *    batch normalization here is the standard training-mode definition:
+ *    per-channel mean and biased variance over N, H, W, xhat = (x - mean) /
+ *    sqrt(var + eps), y = max(gamma xhat + beta, 0); running statistics move
+ *    by momentum towards the batch mean and the unbiased variance.  The
+ *    caller concatenates the pieces (along channels) before calling.
  *  - Matmul + activation (problem B07, SOLUTION step 4: the activation
  *    follows a d x d matrix multiply on the same tensor): Z = X W^T with X
  *    [M x K] and W [N x K] row-major; the activation is evaluated at Z as
@@ -504,6 +513,90 @@ int oracle_matmul_act_bwd(int act, int64_t M, int64_t N, int64_t K, const double
             if (absum) absum[m * N + n] = (double)aacc;
             dZ[m * N + n] = d * act_df(act, Z[m * N + n], param);
         }
+    }
+    return 0;
+}
+
+/* ---------------------------------------- batch normalization + ReLU */
+
+/* x: NCHW [N, C, HW] (channel c of sample n is the plane x[(n C + c) HW ..]).
+ * Outputs: y = max(gamma xhat + beta, 0); mean[c], var[c] (biased); y_scale
+ * (nullable) = |gamma| r |x| + |gamma| r |mean| + |beta|, r = 1 / sqrt(var +
+ * eps): the magnitude of the terms any evaluation of gamma xhat + beta adds.
+ * Sums are serial in index order, long double, two passes (mean first). */
+int oracle_bn_relu_fwd(int64_t N, int64_t C, int64_t HW, const double *x, const double *gamma,
+                       const double *beta, double eps, double *y, double *mean, double *var, double *y_scale)
+{
+    if (N < 0 || C < 0 || HW < 0) return -1;
+    const int64_t n = N * HW;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        long double s = 0.0L;
+        for (int64_t b = 0; b < N; ++b)
+            for (int64_t i = 0; i < HW; ++i) s += (long double)x[(b * C + c) * HW + i];
+        const long double mu = n > 0 ? s / (long double)n : 0.0L;
+        long double v = 0.0L;
+        for (int64_t b = 0; b < N; ++b)
+            for (int64_t i = 0; i < HW; ++i) {
+                const long double d = (long double)x[(b * C + c) * HW + i] - mu;
+                v += d * d;
+            }
+        const long double var_c = n > 0 ? v / (long double)n : 0.0L;
+        mean[c] = (double)mu;
+        var[c] = (double)var_c;
+        const double r = 1.0 / sqrt((double)var_c + eps);
+        for (int64_t b = 0; b < N; ++b)
+            for (int64_t i = 0; i < HW; ++i) {
+                const int64_t j = (b * C + c) * HW + i;
+                const double xh = (x[j] - (double)mu) * r;
+                const double z = gamma[c] * xh + beta[c];
+                y[j] = z > 0.0 ? z : 0.0;
+                if (y_scale) y_scale[j] = fabs(gamma[c]) * r * (fabs(x[j]) + fabs((double)mu)) + fabs(beta[c]);
+            }
+    }
+    return 0;
+}
+
+/* Backward of y = max(gamma xhat + beta, 0) with batch statistics, from x,
+ * dy and the batch mean / biased variance (nothing else saved):
+ *   dz = dy [gamma xhat + beta > 0];  dbeta = sum dz;  dgamma = sum dz xhat;
+ *   dx = gamma r (dz - dbeta / n - xhat dgamma / n).
+ * dx_scale (nullable) = |gamma| r (|dz| + sum|dz| / n + |xhat| sum|dz xhat| / n),
+ * the magnitude of the terms that dx adds up. */
+int oracle_bn_relu_bwd(int64_t N, int64_t C, int64_t HW, const double *x, const double *dy, const double *gamma,
+                       const double *beta, const double *mean, const double *var, double eps, double *dx,
+                       double *dgamma, double *dbeta, double *dx_scale)
+{
+    if (N < 0 || C < 0 || HW < 0) return -1;
+    const int64_t n = N * HW;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        const double r = 1.0 / sqrt(var[c] + eps);
+        long double sdz = 0.0L, sdzx = 0.0L, adz = 0.0L, adzx = 0.0L;
+        for (int64_t b = 0; b < N; ++b)
+            for (int64_t i = 0; i < HW; ++i) {
+                const int64_t j = (b * C + c) * HW + i;
+                const double xh = (x[j] - mean[c]) * r;
+                const double dz = gamma[c] * xh + beta[c] > 0.0 ? dy[j] : 0.0;
+                sdz += (long double)dz;
+                sdzx += (long double)dz * (long double)xh;
+                adz += fabsl((long double)dz);
+                adzx += fabsl((long double)dz * (long double)xh);
+            }
+        dbeta[c] = (double)sdz;
+        dgamma[c] = (double)sdzx;
+        const double k = gamma[c] * r;
+        for (int64_t b = 0; b < N; ++b)
+            for (int64_t i = 0; i < HW; ++i) {
+                const int64_t j = (b * C + c) * HW + i;
+                const double xh = (x[j] - mean[c]) * r;
+                const double dz = gamma[c] * xh + beta[c] > 0.0 ? dy[j] : 0.0;
+                dx[j] = n > 0 ? k * (dz - (double)sdz / (double)n - xh * (double)sdzx / (double)n) : 0.0;
+                if (dx_scale)
+                    dx_scale[j] = n > 0 ? fabs(k) * (fabs(dz) + (double)adz / (double)n +
+                                                     fabs(xh) * (double)adzx / (double)n)
+                                        : 0.0;
+            }
     }
     return 0;
 }
