@@ -612,6 +612,8 @@ def run_secondary(args):
         args._tf_peak = tf_peak
     elif wl == "mlp_bf16":
         return run_mlp(args)
+    elif wl == "densenet_bn_bf16":
+        return run_densenet_bn(args)
     elif wl == "memory_study":
         return run_memory_study(args)
     elif wl == "swish_f32_1m":
@@ -707,6 +709,79 @@ def run_mlp(args, M: int = 16384, d: int = 4096, h: int = 4096, act: str = "gelu
             "clocks": clk.summary()}
 
 
+def run_densenet_bn(args, N: int = 64, ks=(64, 32, 32, 32, 32, 32), spatial=(56, 56)):
+    """Concatenation + batch normalization + ReLU of one DenseNet-121 layer
+    (first dense block, sixth layer: 224 channels at 56 x 56, batch 64, bf16)
+    over one training step (forward, the backward's re-population of the
+    output, backward): the kernels that never form the concatenation and keep
+    only the statistics, against torch.cat + F.batch_norm + relu under
+    autograd.  Reports time per step, the bytes each path moves per step
+    (algorithmic: the tensors each kernel must read and write), and the
+    activation memory held between forward and backward."""
+    import torch.nn.functional as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    HW = spatial[0] * spatial[1]
+    C = sum(ks)
+    pieces = [synthetic.normal(N * k * HW, 1.5, 70 + i, synthetic.STREAM_X, "bf16").view((N, k) + spatial).to(dev)
+              for i, k in enumerate(ks)]
+    g = torch.from_numpy(synthetic.uniform_f64(C, 0.5, 1.5, 71, synthetic.STREAM_GAMMA)).float().to(dev)
+    b = torch.from_numpy(synthetic.normal_f64(C, 0.3, 71, synthetic.STREAM_BETA)).float().to(dev)
+    dy = synthetic.normal(N * C * HW, 1.0, 72, synthetic.STREAM_DY, "bf16").view((N, C) + spatial).to(dev)
+    y = torch.empty((N, C) + spatial, dtype=torch.bfloat16, device=dev)
+    dps = [torch.empty_like(p) for p in pieces]
+    rmean = torch.zeros(C, device=dev)
+    rvar = torch.ones(C, device=dev)
+    ws = torch.zeros(int(mea._capi.lib().mea_concat_bn_relu_workspace_bytes(N, C)), dtype=torch.uint8, device=dev)
+    T = N * C * HW * 2
+    ours_bytes = 10 * T       # fwd: stats read x, apply read x + write y; re-populate: read x + write y;
+    #                           bwd: reduce read x + dy, dx read x + dy + write dx
+
+    def ours():
+        _, mean, invstd = mea.concat_bn_relu_fwd(pieces, g, b, 1e-5, 0.1, rmean, rvar, out=y, workspace=ws)
+        mea.concat_bn_relu_apply(pieces, g, b, mean, invstd, out=y)
+        mea.concat_bn_relu_bwd(pieces, dy, g, b, mean, invstd, dpieces=dps, workspace=ws)
+
+    pr = [p.detach().clone().requires_grad_(True) for p in pieces]
+    gr = g.clone().requires_grad_(True)
+    br = b.clone().requires_grad_(True)
+
+    def plain_fwd():
+        return torch.relu(F.batch_norm(torch.cat(pr, 1), rmean, rvar, gr, br, training=True, momentum=0.1, eps=1e-5))
+
+    def plain():
+        plain_fwd().backward(dy)
+
+    res = {}
+    with _ClockSampler(0) as clk:
+        for name, fn in (("memory_efficient", ours), ("plain_pytorch", plain)):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            for _ in range(args.steps):
+                fn()
+            e.record()
+            torch.cuda.synchronize()
+            res[name] = {"ms_per_step": round(s.elapsed_time(e) / args.steps, 4)}
+    # activation memory held between forward and backward
+    base = torch.cuda.memory_allocated()
+    out = plain_fwd()
+    torch.cuda.synchronize()
+    res["plain_pytorch"]["activation_bytes_held"] = int(torch.cuda.memory_allocated() - base
+                                                        - out.numel() * out.element_size())
+    del out
+    res["memory_efficient"]["activation_bytes_held"] = 2 * C * 4      # mean and invstd
+    res["memory_efficient"]["GB/s"] = round(ours_bytes / (res["memory_efficient"]["ms_per_step"] * 1e-3) / 1e9, 1)
+    res["memory_efficient"]["frac"] = round(res["memory_efficient"]["GB/s"] / _peaks()[0], 4)
+    return {"workload": "densenet_bn_bf16", "shape": {"N": N, "pieces": list(ks), "H": spatial[0], "W": spatial[1]},
+            "steps": args.steps, "warmup": args.warmup, "algorithmic_bytes_per_step": ours_bytes,
+            "peak_hbm_gbs": _peaks(), "results": res,
+            "speedup": round(res["plain_pytorch"]["ms_per_step"] / res["memory_efficient"]["ms_per_step"], 4),
+            "clocks": clk.summary()}
+
+
 class _PlainSwish(torch.nn.Module):
     """The plain autograd Swish of the pages' first listing: x * sigmoid(alpha x)
     built from PyTorch ops, which keeps every intermediate for the backward.
@@ -796,7 +871,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="swish_bf16",
                     choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
                              "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "mlp_bf16",
-                             "swish_f32_1m", "memory_study"],
+                             "densenet_bn_bf16", "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:

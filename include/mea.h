@@ -293,6 +293,70 @@ MEA_API mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int
                                         const void *w, const void *z, float param, void *dz,
                                         mea_stream_t stream);
 
+/* Concatenation + batch normalization + ReLU without the concatenated
+ * tensor (DenseNet's memory-efficient layer): the input is the channel
+ * concatenation of `npieces` NCHW pieces, never formed in memory.
+ *   pieces        HOST array of npieces DEVICE pointers; piece i is a dense
+ *                 [N, channels[i], HW] tensor of `dtype`, 16-byte aligned for
+ *                 the vector path (any alignment is served).
+ *   channels      HOST array of npieces channel counts (each >= 1); C = their
+ *                 sum (below 2^31); 1 <= npieces <= 128.
+ *   N, HW         batch and plane size (H W); N HW >= 1.
+ *   gamma, beta   device fp32 [C].
+ *   mean, invstd  device fp32 [C], written: the batch mean and
+ *                 1 / sqrt(var + eps), var the biased batch variance.  These
+ *                 2 C floats are all the backward needs besides the pieces.
+ *   running_mean,
+ *   running_var   device fp32 [C] or both NULL: moved by `momentum` towards
+ *                 the batch mean and the unbiased batch variance.
+ *   y             device [N, C, HW] of `dtype`, written: max(gamma xhat +
+ *                 beta, 0).  Meant to be a buffer shared by every layer: the
+ *                 backward re-populates it (mea_concat_bn_relu_apply).  Must
+ *                 not overlap a piece.
+ *   workspace     device scratch of mea_concat_bn_relu_workspace_bytes(N, C)
+ *                 bytes, 16-byte aligned (no counter; no zero-fill needed).
+ * Source: "A memory-efficient implementation of DenseNets", section
+ * "Motivation" (shared allocations for every concatenation and batch
+ * normalization output, re-populated in the backward); batch normalization
+ * in its standard training-mode definition. */
+MEA_API size_t mea_concat_bn_relu_workspace_bytes(int64_t N, int64_t C);
+
+MEA_API mea_status_t mea_concat_bn_relu_fwd(mea_dtype_t dtype, int npieces, const void *const *pieces,
+                                            const int64_t *channels, int64_t N, int64_t HW,
+                                            const float *gamma, const float *beta, float eps,
+                                            float momentum, float *running_mean, float *running_var,
+                                            float *mean, float *invstd, void *y, void *workspace,
+                                            size_t ws_bytes, mea_stream_t stream);
+
+/* Re-populates y = max(gamma (x - mean) invstd + beta, 0) from the pieces
+ * and saved statistics (no reduction): the backward's recompute of the
+ * forward output, bitwise equal to what mea_concat_bn_relu_fwd wrote.
+ * Arguments as in mea_concat_bn_relu_fwd. */
+MEA_API mea_status_t mea_concat_bn_relu_apply(mea_dtype_t dtype, int npieces, const void *const *pieces,
+                                              const int64_t *channels, int64_t N, int64_t HW,
+                                              const float *gamma, const float *beta,
+                                              const float *mean, const float *invstd, void *y,
+                                              mea_stream_t stream);
+
+/* Backward from the pieces, dy and the saved statistics (the ReLU mask and
+ * xhat are recomputed):
+ *   dz = dy [gamma' x + beta' > 0] (the forward's own test);
+ *   dbeta = sum dz, dgamma = sum dz xhat (fp64 sums in a fixed order,
+ *   OVERWRITTEN, fp32); dx = gamma invstd (dz - dbeta / n - xhat dgamma / n).
+ *   dy            device [N, C, HW] of `dtype`, read only.
+ *   dpieces       HOST array of npieces DEVICE pointers, the gradients of the
+ *                 pieces (same shapes); overwritten, or added to when
+ *                 `accumulate` is non-zero (a piece feeds several layers).
+ *                 dpieces[i] may be pieces[i] itself (no partial overlap).
+ *   workspace     as in mea_concat_bn_relu_fwd. */
+MEA_API mea_status_t mea_concat_bn_relu_bwd(mea_dtype_t dtype, int npieces, const void *const *pieces,
+                                            const int64_t *channels, int64_t N, int64_t HW,
+                                            const void *dy, const float *gamma, const float *beta,
+                                            const float *mean, const float *invstd,
+                                            void *const *dpieces, int accumulate, float *dgamma,
+                                            float *dbeta, void *workspace, size_t ws_bytes,
+                                            mea_stream_t stream);
+
 /* Backward with d alpha that allocates nothing and takes no workspace.
  * No counterpart on the pages: this is a library convenience, not part of
  * the method.  It computes exactly what mea_act_bwd computes (same kernel,

@@ -12,6 +12,7 @@ Functions (the C ABI's names without the ``mea_`` prefix):
     act_fwd, act_bwd, affine_swish_fwd, affine_swish_bwd,
     affine_act_fwd, affine_act_bwd, swish_channel_fwd, swish_channel_bwd,
     matmul_act_fwd, matmul_act_bwd,
+    concat_bn_relu_fwd, concat_bn_relu_apply, concat_bn_relu_bwd,
     act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes,
     affine_act_bwd_workspace_bytes, swish_channel_bwd_workspace_bytes
 Autograd / modules:
@@ -19,7 +20,8 @@ Autograd / modules:
     AffineSwishFunction, MemoryEfficientAffineSwish,
     AffineActFunction, MemoryEfficientAffineActivation,
     SwishChannelFunction, MemoryEfficientChannelSwish,
-    MLPFunction, MemoryEfficientMLP
+    MLPFunction, MemoryEfficientMLP,
+    SharedBuffer, ConcatBNReLUConvFunction, MemoryEfficientDenseBottleneck
 """
 from __future__ import annotations
 
@@ -35,12 +37,14 @@ __all__ = [
     "act_fwd", "act_bwd", "affine_swish_fwd", "affine_swish_bwd",
     "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
     "matmul_act_fwd", "matmul_act_bwd",
+    "concat_bn_relu_fwd", "concat_bn_relu_apply", "concat_bn_relu_bwd",
     "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
     "affine_act_bwd_workspace_bytes", "swish_channel_bwd_workspace_bytes",
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
     "AffineSwishFunction", "MemoryEfficientAffineSwish",
     "AffineActFunction", "MemoryEfficientAffineActivation",
     "SwishChannelFunction", "MemoryEfficientChannelSwish", "MLPFunction", "MemoryEfficientMLP",
+    "SharedBuffer", "ConcatBNReLUConvFunction", "MemoryEfficientDenseBottleneck",
     "MeaError", "ACTIVATIONS",
 ]
 
@@ -352,6 +356,84 @@ def matmul_act_bwd(act: str, g: torch.Tensor, w: torch.Tensor, z: torch.Tensor, 
     return dz
 
 
+def _bn_pieces(pieces):
+    if not pieces:
+        raise ValueError("at least one piece")
+    N, HW = pieces[0].shape[0], int(pieces[0][0, 0].numel())
+    dtype = pieces[0].dtype
+    for p in pieces:
+        _need_cuda(p)
+        if p.dim() < 2 or p.shape[0] != N or int(p[0, 0].numel()) != HW or p.dtype != dtype:
+            raise ValueError("pieces must share N, the spatial size and the dtype")
+    chans = [int(p.shape[1]) for p in pieces]
+    return N, HW, chans, _capi.ptr_array([p.data_ptr() for p in pieces]), _capi.int64_array(chans)
+
+
+def concat_bn_relu_fwd(pieces, gamma, beta, eps: float = 1e-5, momentum: float = 0.1, running_mean=None,
+                       running_var=None, out=None, workspace=None):
+    """y = max(BN(cat(pieces, dim=1)), 0) with batch statistics, without
+    forming the concatenation.  Returns (y, mean, invstd)."""
+    N, HW, chans, parr, carr = _bn_pieces(pieces)
+    C = sum(chans)
+    _chan_params(C, gamma, beta)
+    dev = pieces[0].device
+    shape = (N, C) + tuple(pieces[0].shape[2:])
+    y = torch.empty(shape, dtype=pieces[0].dtype, device=dev) if out is None else out
+    _need_cuda(y)
+    mean = torch.empty(C, dtype=torch.float32, device=dev)
+    invstd = torch.empty(C, dtype=torch.float32, device=dev)
+    need = int(_capi.lib().mea_concat_bn_relu_workspace_bytes(N, C))
+    ws = workspace if workspace is not None else _pool.get(dev, _stream(y), need)
+    st = _capi.lib().mea_concat_bn_relu_fwd(_dtype_id(y), len(pieces), parr, carr, N, HW, gamma.data_ptr(),
+                                             beta.data_ptr(), float(eps), float(momentum), _ptr(running_mean),
+                                             _ptr(running_var), mean.data_ptr(), invstd.data_ptr(), y.data_ptr(),
+                                             ws.data_ptr(), ws.numel() * ws.element_size(), _stream(y))
+    _capi.check("mea_concat_bn_relu_fwd", st)
+    return y, mean, invstd
+
+
+def concat_bn_relu_apply(pieces, gamma, beta, mean, invstd, out=None):
+    """Re-populates y from the pieces and saved statistics (the forward's
+    output, bitwise)."""
+    N, HW, chans, parr, carr = _bn_pieces(pieces)
+    C = sum(chans)
+    _chan_params(C, gamma, beta, mean, invstd)
+    shape = (N, C) + tuple(pieces[0].shape[2:])
+    y = torch.empty(shape, dtype=pieces[0].dtype, device=pieces[0].device) if out is None else out
+    _need_cuda(y)
+    st = _capi.lib().mea_concat_bn_relu_apply(_dtype_id(y), len(pieces), parr, carr, N, HW, gamma.data_ptr(),
+                                               beta.data_ptr(), mean.data_ptr(), invstd.data_ptr(), y.data_ptr(),
+                                               _stream(y))
+    _capi.check("mea_concat_bn_relu_apply", st)
+    return y
+
+
+def concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, invstd, dpieces=None, accumulate: bool = False,
+                       workspace=None):
+    """Returns (list of piece gradients, dgamma, dbeta); the ReLU mask and
+    xhat are recomputed from the pieces."""
+    N, HW, chans, parr, carr = _bn_pieces(pieces)
+    C = sum(chans)
+    _need_cuda(dy)
+    _chan_params(C, gamma, beta, mean, invstd)
+    dev = pieces[0].device
+    if dpieces is None:
+        dpieces = [torch.zeros_like(p) if accumulate else torch.empty_like(p) for p in pieces]
+    for d in dpieces:
+        _need_cuda(d)
+    dg = torch.empty(C, dtype=torch.float32, device=dev)
+    db = torch.empty(C, dtype=torch.float32, device=dev)
+    need = int(_capi.lib().mea_concat_bn_relu_workspace_bytes(N, C))
+    ws = workspace if workspace is not None else _pool.get(dev, _stream(dy), need)
+    st = _capi.lib().mea_concat_bn_relu_bwd(_dtype_id(dy), len(pieces), parr, carr, N, HW, dy.data_ptr(),
+                                             gamma.data_ptr(), beta.data_ptr(), mean.data_ptr(), invstd.data_ptr(),
+                                             _capi.ptr_array([d.data_ptr() for d in dpieces]), int(bool(accumulate)),
+                                             dg.data_ptr(), db.data_ptr(), ws.data_ptr(),
+                                             ws.numel() * ws.element_size(), _stream(dy))
+    _capi.check("mea_concat_bn_relu_bwd", st)
+    return dpieces, dg, db
+
+
 # ---------------------------------------------------------------- autograd
 
 class ActivationFunction(torch.autograd.Function):
@@ -557,3 +639,81 @@ class MemoryEfficientMLP(torch.nn.Module):
         shape = x.shape
         out = MLPFunction.apply(x.reshape(-1, shape[-1]).contiguous(), self.w1, self.w2, self.act, self.param)
         return out.view(*shape[:-1], out.shape[-1])
+
+
+class SharedBuffer:
+    """One device buffer reused by every layer for its batch-normalization
+    output (grown on demand).  A layer's output lives there only until the
+    next layer overwrites it; the backward re-populates it."""
+
+    def __init__(self):
+        self._buf = None
+
+    def get(self, shape, dtype, device) -> torch.Tensor:
+        n = 1
+        for d in shape:
+            n *= int(d)
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        if self._buf is None or self._buf.numel() < nbytes or self._buf.device != torch.device(device):
+            self._buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return self._buf[:nbytes].view(dtype).view(shape)
+
+
+class ConcatBNReLUConvFunction(torch.autograd.Function):
+    """conv1x1(relu(BN(cat(pieces)))) with batch statistics, keeping only the
+    pieces (which the network keeps anyway), the weights and 2 C floats of
+    statistics: the normalized tensor lives in a shared buffer and the
+    backward re-populates it before the weight gradient needs it.  The 1x1
+    convolution is a batched matmul (torch.matmul)."""
+
+    @staticmethod
+    def forward(ctx, shared, weight, gamma, beta, running_mean, running_var, eps, momentum, *pieces):
+        N = pieces[0].shape[0]
+        C = sum(int(p.shape[1]) for p in pieces)
+        spatial = tuple(pieces[0].shape[2:])
+        y = shared.get((N, C) + spatial, pieces[0].dtype, pieces[0].device)
+        y, mean, invstd = concat_bn_relu_fwd(list(pieces), gamma, beta, eps, momentum, running_mean, running_var,
+                                             out=y)
+        out = torch.matmul(weight.view(weight.shape[0], C), y.view(N, C, -1))
+        ctx.shared, ctx.spatial = shared, spatial
+        ctx.save_for_backward(weight, gamma, beta, mean, invstd, *pieces)
+        return out.view((N, weight.shape[0]) + spatial)
+
+    @staticmethod
+    def backward(ctx, dout):
+        weight, gamma, beta, mean, invstd, *pieces = ctx.saved_tensors
+        N = pieces[0].shape[0]
+        C = sum(int(p.shape[1]) for p in pieces)
+        w2 = weight.view(weight.shape[0], C)
+        y = ctx.shared.get((N, C) + ctx.spatial, pieces[0].dtype, pieces[0].device)
+        concat_bn_relu_apply(pieces, gamma, beta, mean, invstd, out=y)
+        do = dout.contiguous().view(N, w2.shape[0], -1)
+        dw = torch.matmul(do, y.view(N, C, -1).transpose(1, 2)).sum(dim=0)
+        dy = torch.matmul(w2.t(), do).view_as(y)
+        dpieces, dg, db = concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, invstd)
+        return (None, dw.view_as(weight), dg, db, None, None, None, None, *dpieces)
+
+
+class MemoryEfficientDenseBottleneck(torch.nn.Module):
+    """The bottleneck of a DenseNet layer: concatenation of the previous
+    feature maps, batch normalization, ReLU and a 1x1 convolution to
+    `out_channels`, with the concatenated and normalized tensors kept only in
+    `shared` (one buffer for every layer).  NCHW bf16 or fp32."""
+
+    def __init__(self, in_channels: int, out_channels: int, shared: SharedBuffer | None = None,
+                 eps: float = 1e-5, momentum: float = 0.1, dtype=torch.bfloat16):
+        super().__init__()
+        self.shared = shared if shared is not None else SharedBuffer()
+        self.eps, self.momentum = eps, momentum
+        self.weight = torch.nn.Parameter(torch.empty(out_channels, in_channels, 1, 1, dtype=dtype))
+        with torch.no_grad():
+            self.weight.normal_(0.0, in_channels ** -0.5)
+        self.gamma = torch.nn.Parameter(torch.ones(in_channels, dtype=torch.float32))
+        self.beta = torch.nn.Parameter(torch.zeros(in_channels, dtype=torch.float32))
+        self.register_buffer("running_mean", torch.zeros(in_channels, dtype=torch.float32))
+        self.register_buffer("running_var", torch.ones(in_channels, dtype=torch.float32))
+
+    def forward(self, *pieces):
+        return ConcatBNReLUConvFunction.apply(self.shared, self.weight, self.gamma, self.beta, self.running_mean,
+                                              self.running_var, self.eps, self.momentum,
+                                              *[p.contiguous() for p in pieces])

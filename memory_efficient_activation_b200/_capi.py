@@ -35,6 +35,7 @@ _f = ctypes.c_float
 _i = ctypes.c_int
 _sz = ctypes.c_size_t
 _shape = ctypes.POINTER(ctypes.c_int64)
+_ptrs = ctypes.POINTER(ctypes.c_void_p)
 SIGNATURES = {
     "mea_act_fwd": (_i, [_i, _i, _vp, _vp, _i64, _f, _vp, _vp]),
     "mea_act_bwd_workspace_bytes": (_sz, [_i, _i64, _i]),
@@ -50,6 +51,12 @@ SIGNATURES = {
     "mea_swish_channel_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mea_matmul_act_fwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _f, _vp, _vp, _vp]),
     "mea_matmul_act_bwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _vp, _f, _vp, _vp]),
+    "mea_concat_bn_relu_workspace_bytes": (_sz, [_i64, _i64]),
+    "mea_concat_bn_relu_fwd": (_i, [_i, _i, _ptrs, _shape, _i64, _i64, _vp, _vp, _f, _f, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _sz, _vp]),
+    "mea_concat_bn_relu_apply": (_i, [_i, _i, _ptrs, _shape, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mea_concat_bn_relu_bwd": (_i, [_i, _i, _ptrs, _shape, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ptrs, _i, _vp,
+                                    _vp, _vp, _sz, _vp]),
     "mea_act_bwd_dparam_noalloc": (_i, [_i, _i, _vp, _vp, _vp, _i64, _f, _vp, _vp, _vp]),
     "mea_status_string": (ctypes.c_char_p, [_i]),
     "mea_last_error": (ctypes.c_char_p, []),
@@ -95,3 +102,12 @@ def shape4(shape) -> ctypes.Array:
     if len(vals) != 4:
         raise ValueError("shape must have four entries (N, C, H, W)")
     return (ctypes.c_int64 * 4)(*vals)
+
+
+def ptr_array(ptrs) -> ctypes.Array:
+    """Host array of device pointers (void *const *)."""
+    return (ctypes.c_void_p * len(ptrs))(*[int(p) for p in ptrs])
+
+
+def int64_array(vals) -> ctypes.Array:
+    return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])

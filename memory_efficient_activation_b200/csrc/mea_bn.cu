@@ -1,0 +1,433 @@
+// mea_bn.cu -- channel concatenation + batch normalization (batch
+// statistics) + ReLU without the concatenated tensor, and with its output
+// only in a caller-owned buffer that the backward re-populates.
+//
+// "A memory-efficient implementation of DenseNets", section "Motivation":
+// every concatenation and batch-normalization output of a DenseNet goes into
+// shared allocations reused by all layers, and the backward re-populates
+// them from the layer inputs, which turns the feature-map memory from
+// quadratic to linear in depth.  Here the concatenation is never formed:
+// the kernels read the pieces in place through a table of (pointer, channel
+// offset), so the only per-layer state kept for the backward is the batch
+// mean and inverse standard deviation (2 C floats).
+//
+//   forward   bn_stats_kernel      per (channel, batch slice): fp64 sums of
+//                                  x and x^2 -> partials
+//             bn_finalize_kernel   per channel, slices in order: mean,
+//                                  invstd = 1 / sqrt(var + eps), running
+//                                  statistics (momentum; unbiased variance)
+//             bn_apply_kernel      y = max(gamma' x + beta', 0), gamma' =
+//                                  gamma invstd, beta' = beta - mean gamma'
+//   backward  bn_bwd_reduce_kernel per (channel, slice): recompute the ReLU
+//                                  mask from x; fp64 sums of dz and dz xhat
+//             bn_bwd_finalize      dbeta, dgamma and the coefficients of dx
+//             bn_dx_kernel         dx = gamma invstd (dz - dbeta / n -
+//                                  xhat dgamma / n), written or added into
+//                                  the pieces' gradients
+// Blocks own (channel c, slice s of the batch) and stream the contiguous
+// H W planes of that channel (16-byte vectors when a plane is a multiple of
+// 16 bytes and the pieces are aligned).  All sums are per block in a fixed
+// order and combined per channel in slice order: bitwise reproducible.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "mea_bn_api.h"
+#include "mea_device.cuh"
+#include "mea_internal.h"
+
+namespace mea {
+namespace {
+
+constexpr int kBnThreads = 256;
+constexpr int kBnBlocksTarget = 1184;     // C * S is sized to about this many blocks (148 x 8)
+constexpr int kBnFinThreads = 128;
+
+int bn_slices(int64_t N, int64_t C)
+{
+    int64_t s = (kBnBlocksTarget + C - 1) / C;
+    if (s > N) s = N;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+// Piece holding global channel c (one thread searches, the block shares it).
+__device__ __forceinline__ int piece_of(const BnPieces &t, int c)
+{
+    int lo = 0, hi = t.npieces - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t.off[mid] <= c) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct PlaneJob {
+    int64_t c, n0, n1;
+    int piece, j, k;     // piece index, channel within the piece, channels of the piece
+};
+
+__device__ __forceinline__ PlaneJob plane_job(const BnPieces &t, int64_t N, int slices)
+{
+    __shared__ int sp;
+    PlaneJob p;
+    p.c = blockIdx.x / slices;
+    const int s = blockIdx.x % slices;
+    p.n0 = (int64_t)s * N / slices;
+    p.n1 = (int64_t)(s + 1) * N / slices;
+    if (threadIdx.x == 0) sp = piece_of(t, (int)p.c);
+    __syncthreads();
+    p.piece = sp;
+    p.j = (int)p.c - t.off[p.piece];
+    p.k = t.off[p.piece + 1] - t.off[p.piece];
+    return p;
+}
+
+// Calls f(value_index_in_piece, index_in_concatenation, V floats or 1 float)
+// over the block's planes.  vec: the 16-byte vector path applies.
+template <typename T, class F>
+__device__ __forceinline__ void for_planes(const PlaneJob &p, int64_t C, int64_t HW, bool vec, F &&f)
+{
+    using S = Store<T>;
+    constexpr int V = S::V;
+    if (vec) {
+        const int64_t hwv = HW / V;
+        const int64_t total = (p.n1 - p.n0) * hwv;
+        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
+            const int64_t n = p.n0 + q / hwv, v = q % hwv;
+            f.template vec<V>(((n * p.k + p.j) * HW) / V + v, ((n * C + p.c) * HW) / V + v);
+        }
+    } else {
+        const int64_t total = (p.n1 - p.n0) * HW;
+        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
+            const int64_t n = p.n0 + q / HW, i = q % HW;
+            f.one((n * p.k + p.j) * HW + i, (n * C + p.c) * HW + i);
+        }
+    }
+}
+
+// ------------------------------------------------------------ forward
+
+template <typename T>
+struct StatsF {
+    const void *x;
+    double s1 = 0.0, s2 = 0.0;
+    template <int V>
+    __device__ __forceinline__ void vec(int64_t vi, int64_t)
+    {
+        float xf[V];
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const double d = xf[j];
+            s1 += d;
+            s2 = fma(d, d, s2);
+        }
+    }
+    __device__ __forceinline__ void one(int64_t i, int64_t)
+    {
+        const double d = Store<T>::load1(x, i);
+        s1 += d;
+        s2 = fma(d, d, s2);
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads)
+bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, double *__restrict__ partials)
+{
+    pdl_wait();
+    const PlaneJob p = plane_job(t, N, slices);
+    StatsF<T> f{t.ptr[p.piece]};
+    for_planes<T>(p, C, HW, vec, f);
+    pdl_trigger();
+    __shared__ double red[32];
+    const double a = block_sum(f.s1, red);
+    const double b = block_sum(f.s2, red);
+    if (threadIdx.x == 0) {
+        partials[2 * blockIdx.x] = a;
+        partials[2 * blockIdx.x + 1] = b;
+    }
+}
+
+__global__ void __launch_bounds__(kBnFinThreads)
+bn_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n, float eps, float momentum,
+                   float *__restrict__ mean, float *__restrict__ invstd, float *__restrict__ running_mean,
+                   float *__restrict__ running_var)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < slices; ++s) {
+        s1 += partials[2 * (c * slices + s)];
+        s2 += partials[2 * (c * slices + s) + 1];
+    }
+    const double mu = s1 / n;
+    double var = s2 / n - mu * mu;
+    if (var < 0.0) var = 0.0;
+    mean[c] = (float)mu;
+    invstd[c] = (float)(1.0 / sqrt(var + (double)eps));
+    if (running_mean) {
+        const double unbiased = n > 1.0 ? var * n / (n - 1.0) : var;
+        running_mean[c] = (float)((1.0 - momentum) * running_mean[c] + momentum * mu);
+        running_var[c] = (float)((1.0 - momentum) * running_var[c] + momentum * unbiased);
+    }
+}
+
+template <typename T>
+struct ApplyF {
+    const void *x;
+    void *y;
+    float g, b;
+    template <int V>
+    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
+    {
+        float xf[V], of[V];
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) of[j] = fmaxf(fmaf(g, xf[j], b), 0.f);
+        st_v4(static_cast<uint4 *>(y) + vo, Store<T>::pack(of));
+    }
+    __device__ __forceinline__ void one(int64_t i, int64_t o)
+    {
+        Store<T>::store1(y, o, fmaxf(fmaf(g, Store<T>::load1(x, i), b), 0.f));
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads)
+bn_apply_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, const float *__restrict__ gamma,
+                const float *__restrict__ beta, const float *__restrict__ mean, const float *__restrict__ invstd,
+                void *__restrict__ y)
+{
+    pdl_wait();
+    const PlaneJob p = plane_job(t, N, slices);
+    const float gp = gamma[p.c] * invstd[p.c];
+    ApplyF<T> f{t.ptr[p.piece], y, gp, fmaf(-mean[p.c], gp, beta[p.c])};
+    for_planes<T>(p, C, HW, vec, f);
+    pdl_trigger();
+}
+
+// ------------------------------------------------------------ backward
+
+// dz and xhat of one element, recomputed from x: z = gamma' x + beta' (the
+// forward's arithmetic, so the ReLU mask is the forward's).
+struct BwdCoef {
+    float gp, bp, mu, r;
+};
+
+template <typename T>
+struct ReduceF {
+    const void *x;
+    const void *dy;
+    BwdCoef k;
+    double s1 = 0.0, s2 = 0.0;
+    __device__ __forceinline__ void elem(float xv, float g)
+    {
+        const float dz = fmaf(k.gp, xv, k.bp) > 0.f ? g : 0.f;
+        const float xh = (xv - k.mu) * k.r;
+        s1 += (double)dz;
+        s2 = fma((double)dz, (double)xh, s2);
+    }
+    template <int V>
+    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
+    {
+        float xf[V], gf[V];
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vo), gf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) elem(xf[j], gf[j]);
+    }
+    __device__ __forceinline__ void one(int64_t i, int64_t o) { elem(Store<T>::load1(x, i), Store<T>::load1(dy, o)); }
+};
+
+__device__ __forceinline__ BwdCoef bwd_coef(const float *gamma, const float *beta, const float *mean,
+                                            const float *invstd, int64_t c)
+{
+    BwdCoef k;
+    k.mu = mean[c];
+    k.r = invstd[c];
+    k.gp = gamma[c] * k.r;
+    k.bp = fmaf(-k.mu, k.gp, beta[c]);
+    return k;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads)
+bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices, int vec,
+                     const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
+                     const float *__restrict__ invstd, double *__restrict__ partials)
+{
+    pdl_wait();
+    const PlaneJob p = plane_job(t, N, slices);
+    ReduceF<T> f{t.ptr[p.piece], dy, bwd_coef(gamma, beta, mean, invstd, p.c)};
+    for_planes<T>(p, C, HW, vec, f);
+    pdl_trigger();
+    __shared__ double red[32];
+    const double a = block_sum(f.s1, red);
+    const double b = block_sum(f.s2, red);
+    if (threadIdx.x == 0) {
+        partials[2 * blockIdx.x] = a;
+        partials[2 * blockIdx.x + 1] = b;
+    }
+}
+
+// dbeta, dgamma, and dx = a dz + b + c xhat with a = gamma r, b = -a dbeta / n,
+// c = -a dgamma / n (coef[3 ch + 0..2]).
+__global__ void __launch_bounds__(kBnFinThreads)
+bn_bwd_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n,
+                       const float *__restrict__ gamma, const float *__restrict__ invstd, float *__restrict__ dgamma,
+                       float *__restrict__ dbeta, float *__restrict__ coef)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < slices; ++s) {
+        s1 += partials[2 * (c * slices + s)];
+        s2 += partials[2 * (c * slices + s) + 1];
+    }
+    dbeta[c] = (float)s1;
+    dgamma[c] = (float)s2;
+    const double a = (double)gamma[c] * (double)invstd[c];
+    coef[3 * c] = (float)a;
+    coef[3 * c + 1] = (float)(-a * s1 / n);
+    coef[3 * c + 2] = (float)(-a * s2 / n);
+}
+
+template <typename T>
+struct DxF {
+    const void *x;
+    const void *dy;
+    void *dx;
+    BwdCoef k;
+    float a, b, cc;
+    bool acc;
+    __device__ __forceinline__ float elem(float xv, float g, float prev)
+    {
+        const float dz = fmaf(k.gp, xv, k.bp) > 0.f ? g : 0.f;
+        const float xh = (xv - k.mu) * k.r;
+        const float d = fmaf(a, dz, fmaf(cc, xh, b));
+        return acc ? prev + d : d;
+    }
+    template <int V>
+    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
+    {
+        float xf[V], gf[V], pf[V], of[V];
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vo), gf);
+        if (acc) Store<T>::unpack(*(static_cast<const uint4 *>(dx) + vi), pf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) of[j] = elem(xf[j], gf[j], acc ? pf[j] : 0.f);
+        st_v4(static_cast<uint4 *>(dx) + vi, Store<T>::pack(of));
+    }
+    __device__ __forceinline__ void one(int64_t i, int64_t o)
+    {
+        const float prev = acc ? Store<T>::load1(dx, i) : 0.f;
+        Store<T>::store1(dx, i, elem(Store<T>::load1(x, i), Store<T>::load1(dy, o), prev));
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads)
+bn_dx_kernel(BnPieces t, BnOutPieces d, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices,
+             int vec, const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
+             const float *__restrict__ invstd, const float *__restrict__ coef, int accumulate)
+{
+    pdl_wait();
+    const PlaneJob p = plane_job(t, N, slices);
+    DxF<T> f{t.ptr[p.piece], dy, d.ptr[p.piece], bwd_coef(gamma, beta, mean, invstd, p.c), coef[3 * p.c],
+             coef[3 * p.c + 1], coef[3 * p.c + 2], accumulate != 0};
+    for_planes<T>(p, C, HW, vec, f);
+    pdl_trigger();
+}
+
+// ------------------------------------------------------------ launchers
+
+bool vec_ok(const BnLaunch &a, int bytes, bool with_d)
+{
+    if ((a.HW * bytes) % 16) return false;
+    uintptr_t al = 0;
+    for (int i = 0; i < a.in.npieces; ++i) {
+        al |= reinterpret_cast<uintptr_t>(a.in.ptr[i]);
+        if (with_d) al |= reinterpret_cast<uintptr_t>(a.din.ptr[i]);
+    }
+    al |= reinterpret_cast<uintptr_t>(a.y) | reinterpret_cast<uintptr_t>(a.dy);
+    return (al & 15u) == 0;
+}
+
+template <typename T>
+cudaError_t fwd_t(const BnLaunch &a, bool stats)
+{
+    const int slices = bn_slices(a.N, a.C);
+    const int64_t grid = a.C * slices;
+    if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    const int vec = vec_ok(a, Store<T>::kBytes, false);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+    cudaError_t e = cudaSuccess;
+    if (stats) {
+        e = launch_pdl(bn_stats_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
+                       slices, vec, partials);
+        if (e != cudaSuccess) return e;
+        const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
+        e = launch_pdl(bn_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
+                       static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.eps, a.momentum,
+                       a.mean, a.invstd, a.running_mean, a.running_var);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(bn_apply_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
+                      slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
+                      static_cast<const float *>(a.invstd), a.y);
+}
+
+template <typename T>
+cudaError_t bwd_t(const BnLaunch &a)
+{
+    const int slices = bn_slices(a.N, a.C);
+    const int64_t grid = a.C * slices;
+    if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    const int vec = vec_ok(a, Store<T>::kBytes, true);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+    float *coef = reinterpret_cast<float *>(partials + 2 * grid);
+    cudaError_t e = launch_pdl(bn_bwd_reduce_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in,
+                               a.dy, a.N, a.C, a.HW, slices, vec, a.gamma, a.beta,
+                               static_cast<const float *>(a.mean), static_cast<const float *>(a.invstd), partials);
+    if (e != cudaSuccess) return e;
+    const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
+    e = launch_pdl(bn_bwd_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
+                   static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.gamma,
+                   static_cast<const float *>(a.invstd), a.dgamma, a.dbeta, coef);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(bn_dx_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.din, a.dy, a.N,
+                      a.C, a.HW, slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
+                      static_cast<const float *>(a.invstd), static_cast<const float *>(coef), a.accumulate);
+}
+
+}  // namespace
+
+size_t bn_workspace_bytes(int64_t N, int64_t C)
+{
+    const size_t grid = (size_t)C * (size_t)bn_slices(N, C);
+    return kWsHeader + sizeof(double) * 2 * grid + sizeof(float) * 3 * (size_t)C + 16;
+}
+
+cudaError_t launch_bn_fwd(const BnLaunch &a)
+{
+    return a.dtype == kBF16 ? fwd_t<Bf16>(a, true) : fwd_t<float>(a, true);
+}
+
+cudaError_t launch_bn_apply(const BnLaunch &a)
+{
+    return a.dtype == kBF16 ? fwd_t<Bf16>(a, false) : fwd_t<float>(a, false);
+}
+
+cudaError_t launch_bn_bwd(const BnLaunch &a)
+{
+    return a.dtype == kBF16 ? bwd_t<Bf16>(a) : bwd_t<float>(a);
+}
+
+}  // namespace mea

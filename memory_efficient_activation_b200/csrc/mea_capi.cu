@@ -7,6 +7,7 @@
 #include <cstdio>
 
 #include "../../include/mea.h"
+#include "mea_bn_api.h"
 #include "mea_channel_api.h"
 #include "mea_internal.h"
 #include "mea_matmul_api.h"
@@ -196,7 +197,7 @@ const char *mea_status_string(mea_status_t status)
 
 const char *mea_last_error(void) { return g_err; }
 
-int mea_version(void) { return 1 * 10000 + 2 * 100 + 0; }
+int mea_version(void) { return 1 * 10000 + 3 * 100 + 0; }
 
 mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y, int64_t n, float param,
                          const float *param_dev, mea_stream_t stream)
@@ -406,6 +407,145 @@ mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int64_t K, 
     l.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = mea::launch_matmul_act(l);
     return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_matmul_act_bwd launch");
+}
+
+static mea_status_t bn_common(const char *name, int dtype, int npieces, const void *const *pieces,
+                              const int64_t *channels, int64_t N, int64_t HW, mea::BnLaunch *l, size_t *plane_bytes)
+{
+    (void)name;
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", dtype);
+    if (npieces < 1 || npieces > mea::kBnMaxPieces)
+        return fail(MEA_ERR_UNSUPPORTED, "npieces = %d is outside 1..%d", npieces, mea::kBnMaxPieces);
+    if (!pieces || !channels) return fail(MEA_ERR_INVALID_ARG, "pieces or channels is NULL");
+    if (N < 0 || HW < 0) return fail(MEA_ERR_INVALID_ARG, "N and HW must be non-negative");
+    if (N == 0 || HW == 0) return fail(MEA_ERR_INVALID_ARG, "batch statistics need N HW >= 1");
+    int64_t C = 0;
+    l->in.npieces = npieces;
+    for (int i = 0; i < npieces; ++i) {
+        if (channels[i] < 1) return fail(MEA_ERR_INVALID_ARG, "channels[%d] = %lld", i, (long long)channels[i]);
+        if (!pieces[i]) return fail(MEA_ERR_INVALID_ARG, "pieces[%d] is NULL", i);
+        l->in.ptr[i] = pieces[i];
+        l->in.off[i] = (int)C;
+        C += channels[i];
+        if (C >= ((int64_t)1 << 31)) return fail(MEA_ERR_UNSUPPORTED, "more than 2^31 channels");
+    }
+    l->in.off[npieces] = (int)C;
+    if (N > kMaxElems / HW || N * HW > kMaxElems / C) return fail(MEA_ERR_INVALID_ARG, "tensor too large");
+    l->dtype = dtype;
+    l->N = N;
+    l->C = C;
+    l->HW = HW;
+    *plane_bytes = (size_t)N * HW * dtype_bytes(dtype);
+    return MEA_OK;
+}
+
+size_t mea_concat_bn_relu_workspace_bytes(int64_t N, int64_t C)
+{
+    if (N < 1 || C < 1) return 0;
+    return mea::bn_workspace_bytes(N, C);
+}
+
+mea_status_t mea_concat_bn_relu_fwd(mea_dtype_t dtype, int npieces, const void *const *pieces, const int64_t *channels,
+                                    int64_t N, int64_t HW, const float *gamma, const float *beta, float eps,
+                                    float momentum, float *running_mean, float *running_var, float *mean,
+                                    float *invstd, void *y, void *workspace, size_t ws_bytes, mea_stream_t stream)
+{
+    clear_error();
+    mea::BnLaunch l{};
+    size_t pb = 0;
+    mea_status_t st = bn_common("mea_concat_bn_relu_fwd", dtype, npieces, pieces, channels, N, HW, &l, &pb);
+    if (st != MEA_OK) return st;
+    if (!gamma || !beta || !mean || !invstd || !y) return fail(MEA_ERR_INVALID_ARG, "gamma, beta, mean, invstd or y is NULL");
+    if (!running_mean != !running_var) return fail(MEA_ERR_INVALID_ARG, "running_mean and running_var go together");
+    if (!(eps >= 0.f)) return fail(MEA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = mea::bn_workspace_bytes(N, l.C);
+    if (!workspace || ws_bytes < need)
+        return fail(MEA_ERR_WORKSPACE, "needs %zu bytes of workspace, got %zu%s", need, ws_bytes, workspace ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    for (int i = 0; i < npieces; ++i)
+        if (overlaps(y, pb * l.C, pieces[i], pb * channels[i])) return fail(MEA_ERR_INVALID_ARG, "y overlaps piece %d", i);
+    l.gamma = gamma;
+    l.beta = beta;
+    l.eps = eps;
+    l.momentum = momentum;
+    l.running_mean = running_mean;
+    l.running_var = running_var;
+    l.mean = mean;
+    l.invstd = invstd;
+    l.y = y;
+    l.workspace = workspace;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_bn_fwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_concat_bn_relu_fwd launch");
+}
+
+mea_status_t mea_concat_bn_relu_apply(mea_dtype_t dtype, int npieces, const void *const *pieces,
+                                      const int64_t *channels, int64_t N, int64_t HW, const float *gamma,
+                                      const float *beta, const float *mean, const float *invstd, void *y,
+                                      mea_stream_t stream)
+{
+    clear_error();
+    mea::BnLaunch l{};
+    size_t pb = 0;
+    mea_status_t st = bn_common("mea_concat_bn_relu_apply", dtype, npieces, pieces, channels, N, HW, &l, &pb);
+    if (st != MEA_OK) return st;
+    if (!gamma || !beta || !mean || !invstd || !y) return fail(MEA_ERR_INVALID_ARG, "gamma, beta, mean, invstd or y is NULL");
+    for (int i = 0; i < npieces; ++i)
+        if (overlaps(y, pb * l.C, pieces[i], pb * channels[i])) return fail(MEA_ERR_INVALID_ARG, "y overlaps piece %d", i);
+    l.gamma = gamma;
+    l.beta = beta;
+    l.mean = const_cast<float *>(mean);
+    l.invstd = const_cast<float *>(invstd);
+    l.y = y;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_bn_apply(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_concat_bn_relu_apply launch");
+}
+
+mea_status_t mea_concat_bn_relu_bwd(mea_dtype_t dtype, int npieces, const void *const *pieces, const int64_t *channels,
+                                    int64_t N, int64_t HW, const void *dy, const float *gamma, const float *beta,
+                                    const float *mean, const float *invstd, void *const *dpieces, int accumulate,
+                                    float *dgamma, float *dbeta, void *workspace, size_t ws_bytes,
+                                    mea_stream_t stream)
+{
+    clear_error();
+    mea::BnLaunch l{};
+    size_t pb = 0;
+    mea_status_t st = bn_common("mea_concat_bn_relu_bwd", dtype, npieces, pieces, channels, N, HW, &l, &pb);
+    if (st != MEA_OK) return st;
+    if (!dy || !gamma || !beta || !mean || !invstd || !dgamma || !dbeta || !dpieces)
+        return fail(MEA_ERR_INVALID_ARG, "dy, gamma, beta, mean, invstd, dgamma, dbeta or dpieces is NULL");
+    const size_t need = mea::bn_workspace_bytes(N, l.C);
+    if (!workspace || ws_bytes < need)
+        return fail(MEA_ERR_WORKSPACE, "needs %zu bytes of workspace, got %zu%s", need, ws_bytes, workspace ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return fail(MEA_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+    const size_t cb = (size_t)l.C * sizeof(float);
+    if (overlaps(dgamma, cb, dbeta, cb)) return fail(MEA_ERR_INVALID_ARG, "dgamma overlaps dbeta");
+    for (int i = 0; i < npieces; ++i) {
+        if (!dpieces[i]) return fail(MEA_ERR_INVALID_ARG, "dpieces[%d] is NULL", i);
+        const size_t bi = pb * channels[i];
+        if (overlaps(dpieces[i], bi, dy, pb * l.C)) return fail(MEA_ERR_INVALID_ARG, "dpieces[%d] overlaps dy", i);
+        for (int j = 0; j < npieces; ++j) {
+            const size_t bj = pb * channels[j];
+            if (j == i ? partial_overlap(dpieces[i], pieces[j], bi) : overlaps(dpieces[i], bi, pieces[j], bj))
+                return fail(MEA_ERR_INVALID_ARG, "dpieces[%d] overlaps piece %d", i, j);
+            if (j != i && overlaps(dpieces[i], bi, dpieces[j], bj))
+                return fail(MEA_ERR_INVALID_ARG, "dpieces[%d] overlaps dpieces[%d]", i, j);
+        }
+        l.din.ptr[i] = dpieces[i];
+    }
+    l.dy = dy;
+    l.gamma = gamma;
+    l.beta = beta;
+    l.mean = const_cast<float *>(mean);
+    l.invstd = const_cast<float *>(invstd);
+    l.accumulate = accumulate;
+    l.dgamma = dgamma;
+    l.dbeta = dbeta;
+    l.workspace = workspace;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_bn_bwd(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_concat_bn_relu_bwd launch");
 }
 
 }  // extern "C"

@@ -34,7 +34,7 @@ def _header_enum(name):
 
 def test_every_declared_symbol_is_exported(lib):
     declared = _header_functions()
-    assert len(declared) == 18, declared
+    assert len(declared) == 22, declared
     for fn in declared:
         assert hasattr(lib, fn), fn
         assert fn in _capi.SIGNATURES, fn
@@ -55,7 +55,7 @@ def test_enums_match_header():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.mea_version() == 10200
+    assert lib.mea_version() == 10300
     for st in range(5):
         assert lib.mea_status_string(st)
     assert lib.mea_status_string(99) == b"unknown status"
@@ -195,3 +195,30 @@ def test_matmul_validation(lib):
     assert b(0, 16, 16, 16, A, Wt, Z, 1.0, None, None) == _capi.MEA_ERR_INVALID_ARG
     assert b(0, 16, 16, 16, A, Wt, Z, 1.0, Z + 16, None) == _capi.MEA_ERR_INVALID_ARG      # partial overlap
     assert b(0, 16, 16, 16, A, Wt, Z, 1.0, Wt, None) == _capi.MEA_ERR_INVALID_ARG          # dz overlaps w
+
+
+def test_concat_bn_validation(lib):
+    P = _capi.ptr_array([0x1000000, 0x2000000])
+    ch = _capi.int64_array([3, 5])
+    f = lib.mea_concat_bn_relu_fwd
+    ws = lib.mea_concat_bn_relu_workspace_bytes(4, 8)
+    assert ws >= 256 + 16 * 8
+    assert lib.mea_concat_bn_relu_workspace_bytes(0, 8) == 0
+    G, B, Mu, Is, Yb, Wk = 0x3000000, 0x3100000, 0x3200000, 0x3300000, 0x4000000, 0x5000000
+    assert f(1, 0, P, ch, 4, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, Yb, Wk, ws, None) == _capi.MEA_ERR_UNSUPPORTED
+    assert f(1, 129, P, ch, 4, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, Yb, Wk, ws, None) == _capi.MEA_ERR_UNSUPPORTED
+    assert f(1, 2, P, ch, 0, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, Yb, Wk, ws, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(1, 2, P, _capi.int64_array([3, 0]), 4, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, Yb, Wk, ws, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    assert f(1, 2, P, ch, 4, 9, G, B, 1e-5, 0.1, 0x6000000, None, Mu, Is, Yb, Wk, ws, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(1, 2, P, ch, 4, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, Yb, Wk, ws - 1, None) == _capi.MEA_ERR_WORKSPACE
+    # y overlapping a piece
+    assert f(1, 2, P, ch, 4, 9, G, B, 1e-5, 0.1, None, None, Mu, Is, 0x2000010, Wk, ws, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    b = lib.mea_concat_bn_relu_bwd
+    D = _capi.ptr_array([0x7000000, 0x7000040])      # dpieces overlapping each other
+    assert b(1, 2, P, ch, 4, 9, Yb, G, B, Mu, Is, D, 0, 0x3400000, 0x3500000, Wk, ws, None) \
+        == _capi.MEA_ERR_INVALID_ARG
+    D = _capi.ptr_array([0x1000000 + 2, 0x8000000])  # partial overlap with its own piece
+    assert b(1, 2, P, ch, 4, 9, Yb, G, B, Mu, Is, D, 0, 0x3400000, 0x3500000, Wk, ws, None) \
+        == _capi.MEA_ERR_INVALID_ARG
