@@ -11,26 +11,31 @@
 // offset), so the only per-layer state kept for the backward is the batch
 // mean and inverse standard deviation (2 C floats).
 //
-//   forward   bn_stats_kernel      per (channel, batch slice): fp64 sums of
-//                                  x and x^2 -> partials
+//   forward   bn_stats_kernel      per (channel, batch slice): sums of d =
+//                                  x - shift and d^2 (shift: one element of
+//                                  the channel), fp32 within a 16-byte
+//                                  vector, fp64 across -> partials
 //             bn_finalize_kernel   per channel, slices in order: mean,
 //                                  invstd = 1 / sqrt(var + eps), running
 //                                  statistics (momentum; unbiased variance)
 //             bn_apply_kernel      y = max(gamma' x + beta', 0), gamma' =
 //                                  gamma invstd, beta' = beta - mean gamma'
 //   backward  bn_bwd_reduce_kernel per (channel, slice): recompute the ReLU
-//                                  mask from x; fp64 sums of dz and dz xhat
+//                                  mask from x; sums of dz and dz xhat
+//                                  (fp32 within a vector, fp64 across)
 //             bn_bwd_finalize      dbeta, dgamma and the coefficients of dx
 //             bn_dx_kernel         dx = gamma invstd (dz - dbeta / n -
 //                                  xhat dgamma / n), written or added into
 //                                  the pieces' gradients
 // Blocks own (channel c, slice s of the batch) and stream the contiguous
 // H W planes of that channel (16-byte vectors when a plane is a multiple of
-// 16 bytes and the pieces are aligned).  All sums are per block in a fixed
+// 16 bytes and the pieces are aligned), four items in flight per thread,
+// (sample, position) from the item index by a multiply-shift division.  All sums are per block in a fixed
 // order and combined per channel in slice order: bitwise reproducible.
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "mea_bn_api.h"
 #include "mea_device.cuh"
@@ -84,70 +89,184 @@ __device__ __forceinline__ PlaneJob plane_job(const BnPieces &t, int64_t N, int 
     return p;
 }
 
-// Calls f(value_index_in_piece, index_in_concatenation, V floats or 1 float)
-// over the block's planes.  vec: the 16-byte vector path applies.
-template <typename T, class F>
-__device__ __forceinline__ void for_planes(const PlaneJob &p, int64_t C, int64_t HW, bool vec, F &&f)
-{
-    using S = Store<T>;
-    constexpr int V = S::V;
-    if (vec) {
-        const int64_t hwv = HW / V;
-        const int64_t total = (p.n1 - p.n0) * hwv;
-        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
-            const int64_t n = p.n0 + q / hwv, v = q % hwv;
-            f.template vec<V>(((n * p.k + p.j) * HW) / V + v, ((n * C + p.c) * HW) / V + v);
-        }
-    } else {
-        const int64_t total = (p.n1 - p.n0) * HW;
-        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
-            const int64_t n = p.n0 + q / HW, i = q % HW;
-            f.one((n * p.k + p.j) * HW + i, (n * C + p.c) * HW + i);
-        }
-    }
-}
-
-// ------------------------------------------------------------ forward
-
-template <typename T>
-struct StatsF {
-    const void *x;
-    double s1 = 0.0, s2 = 0.0;
-    template <int V>
-    __device__ __forceinline__ void vec(int64_t vi, int64_t)
+// Unsigned division by a fixed d >= 1 for dividends below 2^31: q = (hi(n m)
+// + n) >> s with s = ceil(log2 d), m = floor(2^32 (2^s - d) / d) + 1 (the
+// round-up method of Granlund and Montgomery, "Division by invariant integers
+// using multiplication", 1994).
+struct DivU32 {
+    uint32_t d, m, s;
+    __device__ __forceinline__ explicit DivU32(uint32_t dd) : d(dd)
     {
-        float xf[V];
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const double d = xf[j];
-            s1 += d;
-            s2 = fma(d, d, s2);
-        }
+        s = 0;
+        while ((1u << s) < d && s < 31) ++s;
+        m = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << s) - d)) / d + 1);
     }
-    __device__ __forceinline__ void one(int64_t i, int64_t)
+    __device__ __forceinline__ void divmod(uint32_t n, uint32_t &q, uint32_t &r) const
     {
-        const double d = Store<T>::load1(x, i);
-        s1 += d;
-        s2 = fma(d, d, s2);
+        q = (__umulhi(n, m) + n) >> s;
+        r = n - q * d;
     }
 };
 
+constexpr int kBnUnroll = 4;     // items in flight per thread
+
+// Runs f over the block's planes in items of VL elements (one 16-byte vector,
+// or one element), kBnUnroll items per thread per step: f.template step<U>
+// gets each item's index in the piece (ii) and in the concatenation (io), in
+// item units, and whether it exists (ok).
+template <int VL, class F>
+__device__ __forceinline__ void stream_items(const PlaneJob &p, int64_t C, int64_t HW, F &f)
+{
+    const uint32_t per = (uint32_t)(HW / VL);
+    const uint32_t total = (uint32_t)(p.n1 - p.n0) * per;
+    const DivU32 div(per);
+    const uint32_t bd = blockDim.x;
+    for (uint32_t q0 = threadIdx.x; q0 < total; q0 += kBnUnroll * bd) {
+        int64_t ii[kBnUnroll], io[kBnUnroll];
+        bool ok[kBnUnroll];
+#pragma unroll
+        for (int u = 0; u < kBnUnroll; ++u) {
+            const uint32_t q = q0 + u * bd;
+            ok[u] = q < total;
+            uint32_t nr, v;
+            div.divmod(ok[u] ? q : 0u, nr, v);
+            const int64_t n = p.n0 + nr;
+            ii[u] = (n * p.k + p.j) * per + v;
+            io[u] = (n * C + p.c) * per + v;
+        }
+        f.step(ii, io, ok);
+    }
+}
+
+template <typename T, class F>
+__device__ __forceinline__ void for_planes(const PlaneJob &p, int64_t C, int64_t HW, bool vec, F &f)
+{
+    if (vec) {
+        auto fv = f.template items<Store<T>::V>();
+        stream_items<Store<T>::V>(p, C, HW, fv);
+        f.absorb(fv);
+    } else {
+        auto fs = f.template items<1>();
+        stream_items<1>(p, C, HW, fs);
+        f.absorb(fs);
+    }
+}
+
+// Item access: VL = V loads a 16-byte vector, VL = 1 one element.  Loads
+// keep the raw bits (unpacked when used) so four items in flight cost few
+// registers.
+template <typename T, int VL>
+struct Item {
+    using Raw = typename std::conditional<VL == 1, float, uint4>::type;
+    static __device__ __forceinline__ Raw load(const void *p, int64_t i)
+    {
+        if constexpr (VL == 1) {
+            return Store<T>::load1(p, i);
+        } else {
+            return ld_nc_v4(static_cast<const uint4 *>(p) + i);
+        }
+    }
+    static __device__ __forceinline__ Raw load_rw(const void *p, int64_t i)
+    {
+        if constexpr (VL == 1) {
+            return Store<T>::load1(p, i);
+        } else {
+            return *(static_cast<const uint4 *>(p) + i);
+        }
+    }
+    static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[VL])
+    {
+        if constexpr (VL == 1) {
+            f[0] = r;
+        } else {
+            Store<T>::unpack(r, f);
+        }
+    }
+    static __device__ __forceinline__ void store(void *p, int64_t i, const float (&f)[VL])
+    {
+        if constexpr (VL == 1) {
+            Store<T>::store1(p, i, f[0]);
+        } else {
+            st_v4(static_cast<uint4 *>(p) + i, Store<T>::pack(f));
+        }
+    }
+};
+
+// ------------------------------------------------------------ forward
+
+// Sums of d = x - shift and d^2: fp32 within an item, fp64 across items.
+// shift is one element of the channel (the same for every block of the
+// channel), which keeps E[d^2] near the variance however large the mean.
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads)
+struct StatsF {
+    const void *x;
+    float shift;
+    double s1 = 0.0, s2 = 0.0;
+    template <int VL>
+    struct It {
+        const void *x;
+        float shift;
+        double s1 = 0.0, s2 = 0.0;
+        __device__ __forceinline__ void step(const int64_t (&ii)[kBnUnroll], const int64_t (&)[kBnUnroll],
+                                             const bool (&ok)[kBnUnroll])
+        {
+            typename Item<T, VL>::Raw xr[kBnUnroll];
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u)
+                if (ok[u]) xr[u] = Item<T, VL>::load(x, ii[u]);
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u) {
+                if (!ok[u]) continue;
+                float xf[VL];
+                Item<T, VL>::unpack(xr[u], xf);
+                float a = 0.f, b = 0.f;
+#pragma unroll
+                for (int j = 0; j < VL; ++j) {
+                    const float d = xf[j] - shift;
+                    a += d;
+                    b = fmaf(d, d, b);
+                }
+                s1 += (double)a;
+                s2 += (double)b;
+            }
+        }
+    };
+    template <int VL>
+    __device__ __forceinline__ It<VL> items() const
+    {
+        return It<VL>{x, shift};
+    }
+    template <class I>
+    __device__ __forceinline__ void absorb(const I &i)
+    {
+        s1 = i.s1;
+        s2 = i.s2;
+    }
+};
+
+__device__ __forceinline__ int64_t first_of_channel(const BnPieces &t, const PlaneJob &p, int64_t HW)
+{
+    (void)t;
+    return (int64_t)p.j * HW;       // sample 0, channel j of the piece, element 0
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads, 3)
 bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, double *__restrict__ partials)
 {
     pdl_wait();
     const PlaneJob p = plane_job(t, N, slices);
-    StatsF<T> f{t.ptr[p.piece]};
+    const void *x = t.ptr[p.piece];
+    StatsF<T> f{x, Store<T>::load1(x, first_of_channel(t, p, HW))};
     for_planes<T>(p, C, HW, vec, f);
     pdl_trigger();
     __shared__ double red[32];
     const double a = block_sum(f.s1, red);
     const double b = block_sum(f.s2, red);
     if (threadIdx.x == 0) {
-        partials[2 * blockIdx.x] = a;
-        partials[2 * blockIdx.x + 1] = b;
+        partials[3 * blockIdx.x] = a;
+        partials[3 * blockIdx.x + 1] = b;
+        partials[3 * blockIdx.x + 2] = (double)f.shift;
     }
 }
 
@@ -162,12 +281,14 @@ bn_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, d
     if (c >= C) return;
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < slices; ++s) {
-        s1 += partials[2 * (c * slices + s)];
-        s2 += partials[2 * (c * slices + s) + 1];
+        s1 += partials[3 * (c * slices + s)];
+        s2 += partials[3 * (c * slices + s) + 1];
     }
-    const double mu = s1 / n;
-    double var = s2 / n - mu * mu;
+    const double shift = partials[3 * c * slices + 2];
+    const double md = s1 / n;                 // mean of d = x - shift
+    double var = s2 / n - md * md;
     if (var < 0.0) var = 0.0;
+    const double mu = shift + md;
     mean[c] = (float)mu;
     invstd[c] = (float)(1.0 / sqrt(var + (double)eps));
     if (running_mean) {
@@ -182,23 +303,42 @@ struct ApplyF {
     const void *x;
     void *y;
     float g, b;
-    template <int V>
-    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
-    {
-        float xf[V], of[V];
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
+    template <int VL>
+    struct It {
+        const void *x;
+        void *y;
+        float g, b;
+        __device__ __forceinline__ void step(const int64_t (&ii)[kBnUnroll], const int64_t (&io)[kBnUnroll],
+                                             const bool (&ok)[kBnUnroll])
+        {
+            typename Item<T, VL>::Raw xr[kBnUnroll];
 #pragma unroll
-        for (int j = 0; j < V; ++j) of[j] = fmaxf(fmaf(g, xf[j], b), 0.f);
-        st_v4(static_cast<uint4 *>(y) + vo, Store<T>::pack(of));
-    }
-    __device__ __forceinline__ void one(int64_t i, int64_t o)
+            for (int u = 0; u < kBnUnroll; ++u)
+                if (ok[u]) xr[u] = Item<T, VL>::load(x, ii[u]);
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u) {
+                if (!ok[u]) continue;
+                float xf[VL], of[VL];
+                Item<T, VL>::unpack(xr[u], xf);
+#pragma unroll
+                for (int j = 0; j < VL; ++j) of[j] = fmaxf(fmaf(g, xf[j], b), 0.f);
+                Item<T, VL>::store(y, io[u], of);
+            }
+        }
+    };
+    template <int VL>
+    __device__ __forceinline__ It<VL> items() const
     {
-        Store<T>::store1(y, o, fmaxf(fmaf(g, Store<T>::load1(x, i), b), 0.f));
+        return It<VL>{x, y, g, b};
+    }
+    template <class I>
+    __device__ __forceinline__ void absorb(const I &)
+    {
     }
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads)
+__global__ void __launch_bounds__(kBnThreads, 3)
 bn_apply_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, const float *__restrict__ gamma,
                 const float *__restrict__ beta, const float *__restrict__ mean, const float *__restrict__ invstd,
                 void *__restrict__ y)
@@ -219,31 +359,6 @@ struct BwdCoef {
     float gp, bp, mu, r;
 };
 
-template <typename T>
-struct ReduceF {
-    const void *x;
-    const void *dy;
-    BwdCoef k;
-    double s1 = 0.0, s2 = 0.0;
-    __device__ __forceinline__ void elem(float xv, float g)
-    {
-        const float dz = fmaf(k.gp, xv, k.bp) > 0.f ? g : 0.f;
-        const float xh = (xv - k.mu) * k.r;
-        s1 += (double)dz;
-        s2 = fma((double)dz, (double)xh, s2);
-    }
-    template <int V>
-    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
-    {
-        float xf[V], gf[V];
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vo), gf);
-#pragma unroll
-        for (int j = 0; j < V; ++j) elem(xf[j], gf[j]);
-    }
-    __device__ __forceinline__ void one(int64_t i, int64_t o) { elem(Store<T>::load1(x, i), Store<T>::load1(dy, o)); }
-};
-
 __device__ __forceinline__ BwdCoef bwd_coef(const float *gamma, const float *beta, const float *mean,
                                             const float *invstd, int64_t c)
 {
@@ -256,7 +371,60 @@ __device__ __forceinline__ BwdCoef bwd_coef(const float *gamma, const float *bet
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads)
+struct ReduceF {
+    const void *x;
+    const void *dy;
+    BwdCoef k;
+    double s1 = 0.0, s2 = 0.0;
+    template <int VL>
+    struct It {
+        const void *x;
+        const void *dy;
+        BwdCoef k;
+        double s1 = 0.0, s2 = 0.0;
+        __device__ __forceinline__ void step(const int64_t (&ii)[kBnUnroll], const int64_t (&io)[kBnUnroll],
+                                             const bool (&ok)[kBnUnroll])
+        {
+            typename Item<T, VL>::Raw xr[kBnUnroll], gr[kBnUnroll];
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u)
+                if (ok[u]) {
+                    xr[u] = Item<T, VL>::load(x, ii[u]);
+                    gr[u] = Item<T, VL>::load(dy, io[u]);
+                }
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u) {
+                if (!ok[u]) continue;
+                float xf[VL], gf[VL];
+                Item<T, VL>::unpack(xr[u], xf);
+                Item<T, VL>::unpack(gr[u], gf);
+                float a = 0.f, b = 0.f;
+#pragma unroll
+                for (int j = 0; j < VL; ++j) {
+                    const float dz = fmaf(k.gp, xf[j], k.bp) > 0.f ? gf[j] : 0.f;
+                    a += dz;
+                    b = fmaf(dz, (xf[j] - k.mu) * k.r, b);
+                }
+                s1 += (double)a;
+                s2 += (double)b;
+            }
+        }
+    };
+    template <int VL>
+    __device__ __forceinline__ It<VL> items() const
+    {
+        return It<VL>{x, dy, k};
+    }
+    template <class I>
+    __device__ __forceinline__ void absorb(const I &i)
+    {
+        s1 = i.s1;
+        s2 = i.s2;
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kBnThreads, 3)
 bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices, int vec,
                      const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
                      const float *__restrict__ invstd, double *__restrict__ partials)
@@ -270,8 +438,8 @@ bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t
     const double a = block_sum(f.s1, red);
     const double b = block_sum(f.s2, red);
     if (threadIdx.x == 0) {
-        partials[2 * blockIdx.x] = a;
-        partials[2 * blockIdx.x + 1] = b;
+        partials[3 * blockIdx.x] = a;
+        partials[3 * blockIdx.x + 1] = b;
     }
 }
 
@@ -288,8 +456,8 @@ bn_bwd_finalize_kernel(const double *__restrict__ partials, int64_t C, int slice
     if (c >= C) return;
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < slices; ++s) {
-        s1 += partials[2 * (c * slices + s)];
-        s2 += partials[2 * (c * slices + s) + 1];
+        s1 += partials[3 * (c * slices + s)];
+        s2 += partials[3 * (c * slices + s) + 1];
     }
     dbeta[c] = (float)s1;
     dgamma[c] = (float)s2;
@@ -307,33 +475,54 @@ struct DxF {
     BwdCoef k;
     float a, b, cc;
     bool acc;
-    __device__ __forceinline__ float elem(float xv, float g, float prev)
-    {
-        const float dz = fmaf(k.gp, xv, k.bp) > 0.f ? g : 0.f;
-        const float xh = (xv - k.mu) * k.r;
-        const float d = fmaf(a, dz, fmaf(cc, xh, b));
-        return acc ? prev + d : d;
-    }
-    template <int V>
-    __device__ __forceinline__ void vec(int64_t vi, int64_t vo)
-    {
-        float xf[V], gf[V], pf[V], of[V];
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
-        Store<T>::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vo), gf);
-        if (acc) Store<T>::unpack(*(static_cast<const uint4 *>(dx) + vi), pf);
+    template <int VL>
+    struct It {
+        const void *x;
+        const void *dy;
+        void *dx;
+        BwdCoef k;
+        float a, b, cc;
+        bool acc;
+        __device__ __forceinline__ void step(const int64_t (&ii)[kBnUnroll], const int64_t (&io)[kBnUnroll],
+                                             const bool (&ok)[kBnUnroll])
+        {
+            typename Item<T, VL>::Raw xr[kBnUnroll], gr[kBnUnroll];
 #pragma unroll
-        for (int j = 0; j < V; ++j) of[j] = elem(xf[j], gf[j], acc ? pf[j] : 0.f);
-        st_v4(static_cast<uint4 *>(dx) + vi, Store<T>::pack(of));
-    }
-    __device__ __forceinline__ void one(int64_t i, int64_t o)
+            for (int u = 0; u < kBnUnroll; ++u)
+                if (ok[u]) {
+                    xr[u] = Item<T, VL>::load(x, ii[u]);
+                    gr[u] = Item<T, VL>::load(dy, io[u]);
+                }
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u) {
+                if (!ok[u]) continue;
+                float xf[VL], gf[VL], pf[VL], of[VL];
+                Item<T, VL>::unpack(xr[u], xf);
+                Item<T, VL>::unpack(gr[u], gf);
+                if (acc) Item<T, VL>::unpack(Item<T, VL>::load_rw(dx, ii[u]), pf);
+#pragma unroll
+                for (int j = 0; j < VL; ++j) {
+                    const float dz = fmaf(k.gp, xf[j], k.bp) > 0.f ? gf[j] : 0.f;
+                    const float d = fmaf(a, dz, fmaf(cc, (xf[j] - k.mu) * k.r, b));
+                    of[j] = acc ? pf[j] + d : d;
+                }
+                Item<T, VL>::store(dx, ii[u], of);
+            }
+        }
+    };
+    template <int VL>
+    __device__ __forceinline__ It<VL> items() const
     {
-        const float prev = acc ? Store<T>::load1(dx, i) : 0.f;
-        Store<T>::store1(dx, i, elem(Store<T>::load1(x, i), Store<T>::load1(dy, o), prev));
+        return It<VL>{x, dy, dx, k, a, b, cc, acc};
+    }
+    template <class I>
+    __device__ __forceinline__ void absorb(const I &)
+    {
     }
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads)
+__global__ void __launch_bounds__(kBnThreads, 3)
 bn_dx_kernel(BnPieces t, BnOutPieces d, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices,
              int vec, const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
              const float *__restrict__ invstd, const float *__restrict__ coef, int accumulate)
@@ -392,7 +581,7 @@ cudaError_t bwd_t(const BnLaunch &a)
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const int vec = vec_ok(a, Store<T>::kBytes, true);
     double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
-    float *coef = reinterpret_cast<float *>(partials + 2 * grid);
+    float *coef = reinterpret_cast<float *>(partials + 3 * grid);
     cudaError_t e = launch_pdl(bn_bwd_reduce_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in,
                                a.dy, a.N, a.C, a.HW, slices, vec, a.gamma, a.beta,
                                static_cast<const float *>(a.mean), static_cast<const float *>(a.invstd), partials);
@@ -412,7 +601,7 @@ cudaError_t bwd_t(const BnLaunch &a)
 size_t bn_workspace_bytes(int64_t N, int64_t C)
 {
     const size_t grid = (size_t)C * (size_t)bn_slices(N, C);
-    return kWsHeader + sizeof(double) * 2 * grid + sizeof(float) * 3 * (size_t)C + 16;
+    return kWsHeader + sizeof(double) * 3 * grid + sizeof(float) * 3 * (size_t)C + 16;
 }
 
 cudaError_t launch_bn_fwd(const BnLaunch &a)

@@ -431,6 +431,7 @@ static mea_status_t bn_common(const char *name, int dtype, int npieces, const vo
     }
     l->in.off[npieces] = (int)C;
     if (N > kMaxElems / HW || N * HW > kMaxElems / C) return fail(MEA_ERR_INVALID_ARG, "tensor too large");
+    if (N * HW >= ((int64_t)1 << 31)) return fail(MEA_ERR_UNSUPPORTED, "N HW must be below 2^31");
     l->dtype = dtype;
     l->N = N;
     l->C = C;

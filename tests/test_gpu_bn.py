@@ -5,9 +5,8 @@ ABI, and the memory-efficient DenseNet bottleneck built on them.
 Rules (tests/_compare.py): y is held to one bf16 ulp or, in fp32, 1e-5 of
 its condition scale (|gamma| r (|x| + |mean|) + |beta|, the terms any
 evaluation of gamma xhat + beta adds); with bf16 storage a y that misses the
-ulp rule may meet the fp32 rule against that scale.  The statistics are
-fp32 roundings of fp64 sums: mean within 1e-6 relative (plus 1e-12 of the
-mean |x|), invstd within 2e-6 relative.  dx is held to the same rules with
+ulp rule may meet the fp32 rule against that scale.  The statistics: see
+_check_stats (fp32 sums of at most 8 shifted values, then fp64).  dx is held to the same rules with
 the oracle's scale |gamma| r (|dz| + sum|dz| / n + |xhat| sum|dz xhat| / n).
 An element whose exact gamma xhat + beta lies within 1e-5 of its scale of
 zero may take either side of the ReLU: its dz may differ by dy, which adds
@@ -49,11 +48,18 @@ def _np(ps):
 
 
 def _check_stats(mean, invstd, rm, rv, pieces):
+    # The kernels sum d = x - shift (shift: an element of the channel) in
+    # fp32 over at most 8 values, then in fp64: the sum of d errs by at most
+    # 8 2^-24 of sum |d|, and sum |d| / n <= mean|x| + max|x|; the fp32
+    # results add one rounding.  E[d^2] errs likewise, relative to E[d^2] =
+    # var + (mean - shift)^2 <= var + (|mean| + max|x|)^2.
     x = np.concatenate(_np(pieces), axis=1)
     am = np.abs(x).mean(axis=(0, 2))
-    assert np.all(np.abs(mean.cpu().double().numpy() - rm) <= 1e-6 * np.abs(rm) + 1e-12 * am + 1e-30)
+    mx = np.abs(x).max(axis=(0, 2))
+    assert np.all(np.abs(mean.cpu().double().numpy() - rm) <= 1e-6 * np.abs(rm) + 5e-7 * (am + mx))
     ri = 1.0 / np.sqrt(rv + EPS)
-    assert np.all(np.abs(invstd.cpu().double().numpy() - ri) <= 2e-6 * ri)
+    tol = 2e-6 + 5e-7 * (np.abs(rm) + mx) ** 2 / (rv + EPS)
+    assert np.all(np.abs(invstd.cpu().double().numpy() - ri) <= tol * ri)
 
 
 def _ambiguous(pieces, g, b, rm, rv, ys):
