@@ -42,6 +42,7 @@
 #include "mea_internal.h"
 #include "mea_math.cuh"
 #include "mea_pipe.cuh"
+#include "mea_stream.cuh"
 
 namespace mea {
 
@@ -543,15 +544,15 @@ chan_colsum_kernel(const double *__restrict__ partials, int nb, int C, float *__
 
 // ------------------------------------------------------------ plane path
 
+constexpr int kPlaneUnroll = 4;   // items in flight per thread
+
 template <class Op, typename T, int MODE, bool NHWC>
-__global__ void __launch_bounds__(kPlaneThreads)
+__global__ void __launch_bounds__(kPlaneThreads, 3)
 chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca, void *__restrict__ out,
                   int64_t N, int64_t C, int64_t HW, int slices, int vec_ok, float *__restrict__ out0,
                   float *__restrict__ out1, void *__restrict__ ws)
 {
-    using S = Store<T>;
-    constexpr int V = S::V;
-    constexpr bool P = S::P;
+    constexpr bool P = Store<T>::P;
     constexpr int NR = Op::NR;
     const int64_t c = blockIdx.x / slices;
     const int s = blockIdx.x % slices;
@@ -563,50 +564,69 @@ chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanA
 #pragma unroll
     for (int r = 0; r < NR; ++r) acc[r] = 0.0;
 
-    auto one = [&](float xi, float gi, float &res) {
-        bool tail = false;
-        if constexpr (MODE == 0) {
-            res = Op::template f<P>(xi, k, ch, tail);
-            if (tail) res = Op::template f_tail<P>(xi, k, ch);
-        } else {
-            float o, t;
-            Op::template bwd<P>(xi, gi, k, ch, tail, o, t);
-            if (tail) Op::template bwd_tail<P>(xi, gi, k, ch, o, t);
-            float tmp[NR];
+    // The block's planes in items of VL elements (a 16-byte vector, or one
+    // element), kPlaneUnroll items per thread per step, loads first; the
+    // reduction terms of an item are added in fp32, then in fp64.
+    auto run = [&](auto vl) {
+        constexpr int VL = decltype(vl)::value;
+        using I = Item<T, VL>;
+        const uint32_t per = (uint32_t)(HW / VL);
+        const uint32_t total = (uint32_t)(n1 - n0) * per;
+        const DivU32 div(per);
+        const uint32_t bd = blockDim.x;
+        for (uint32_t q0 = threadIdx.x; q0 < total; q0 += kPlaneUnroll * bd) {
+            int64_t idx[kPlaneUnroll];
+            typename I::Raw xr[kPlaneUnroll], gr[kPlaneUnroll];
 #pragma unroll
-            for (int r = 0; r < NR; ++r) tmp[r] = 0.f;
-            res = Op::finish(xi, o, t, ch, tmp);
+            for (int u = 0; u < kPlaneUnroll; ++u) {
+                const uint32_t q = q0 + u * bd;
+                uint32_t nr, v;
+                div.divmod(q < total ? q : 0u, nr, v);
+                const int64_t n = n0 + nr;
+                idx[u] = NHWC ? (n * HW + v) * C + c : (n * C + c) * per + v;
+                if (q < total) {
+                    xr[u] = I::load(x, idx[u]);
+                    if constexpr (MODE == 1) gr[u] = I::load(dy, idx[u]);
+                }
+            }
 #pragma unroll
-            for (int r = 0; r < NR; ++r) acc[r] += (double)tmp[r];
+            for (int u = 0; u < kPlaneUnroll; ++u) {
+                if (q0 + u * bd >= total) continue;
+                float xf[VL], gf[VL], of[VL];
+                I::unpack(xr[u], xf);
+                if constexpr (MODE == 1) I::unpack(gr[u], gf);
+                bool tail = false;
+                if constexpr (MODE == 0) {
+#pragma unroll
+                    for (int j = 0; j < VL; ++j) of[j] = Op::template f<P>(xf[j], k, ch, tail);
+                    if (tail) {
+#pragma unroll
+                        for (int j = 0; j < VL; ++j)
+                            if (Op::is_tail(xf[j], k, ch)) of[j] = Op::template f_tail<P>(xf[j], k, ch);
+                    }
+                } else {
+                    float o[VL], t[VL];
+#pragma unroll
+                    for (int j = 0; j < VL; ++j) Op::template bwd<P>(xf[j], gf[j], k, ch, tail, o[j], t[j]);
+                    if (tail) {
+#pragma unroll
+                        for (int j = 0; j < VL; ++j)
+                            if (Op::is_tail(xf[j], k, ch)) Op::template bwd_tail<P>(xf[j], gf[j], k, ch, o[j], t[j]);
+                    }
+                    float tmp[NR];
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) tmp[r] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < VL; ++j) of[j] = Op::finish(xf[j], o[j], t[j], ch, tmp);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) acc[r] += (double)tmp[r];
+                }
+                I::store(out, idx[u], of);
+            }
         }
     };
-
-    if (!NHWC && vec_ok) {
-        // NCHW planes are contiguous and each starts on a 16-byte boundary.
-        const int64_t hwv = HW / V;
-        const int64_t total = (n1 - n0) * hwv;
-        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
-            const int64_t n = n0 + q / hwv;
-            const int64_t vi = (n * C + c) * hwv + q % hwv;
-            float xf[V], gf[V], of[V];
-            S::unpack(ld_nc_v4(static_cast<const uint4 *>(x) + vi), xf);
-            if constexpr (MODE == 1) S::unpack(ld_nc_v4(static_cast<const uint4 *>(dy) + vi), gf);
-#pragma unroll
-            for (int j = 0; j < V; ++j) one(xf[j], MODE == 1 ? gf[j] : 0.f, of[j]);
-            st_v4(static_cast<uint4 *>(out) + vi, S::pack(of));
-        }
-    } else {
-        const int64_t total = (n1 - n0) * HW;
-        for (int64_t p = threadIdx.x; p < total; p += blockDim.x) {
-            const int64_t n = n0 + p / HW, hw = p % HW;
-            const int64_t i = NHWC ? (n * HW + hw) * C + c : (n * C + c) * HW + hw;
-            const float xi = S::load1(x, i);
-            const float gi = MODE == 1 ? S::load1(dy, i) : 0.f;
-            float o;
-            one(xi, gi, o);
-            S::store1(out, i, o);
-        }
-    }
+    if (!NHWC && vec_ok) run(std::integral_constant<int, Store<T>::V>{});
+    else run(std::integral_constant<int, 1>{});
     pdl_trigger();
     if constexpr (MODE == 0) {
         return;
