@@ -22,7 +22,7 @@
 // both CTAs' shared memory (M 256) and B from both (N 256), writing a
 // 128 x 256 fp32 accumulator into each CTA's tensor memory.  Per CTA:
 //   warp 0      one thread issues TMA loads of 128 x 64 tiles of X and W
-//               (128-byte swizzle, no multicast) into a 6-stage ring; the
+//               (128-byte swizzle, no multicast) into a 7-stage ring; the
 //               loads of both CTAs complete on the first CTA's barrier
 //   warp 1      allocates 512 tensor-memory columns (two accumulators) in
 //               both CTAs; in the first CTA one thread issues the MMAs and
@@ -56,7 +56,7 @@ namespace {
 constexpr int kBM = kMatmulBM, kBN = kMatmulBN, kBK = kMatmulBK;   // tile of a CTA pair: 256 x 256
 constexpr int kHalf = 128;                                  // rows of X and of W one CTA stages
 constexpr int kUmmaK = 16;                                  // K of one bf16 MMA
-constexpr int kStages = 6;
+constexpr int kStages = 7;
 constexpr int kThreadsMM = 192;
 constexpr uint32_t kStageA = kHalf * kBK * 2;                // 16 KB
 constexpr uint32_t kStageB = kHalf * kBK * 2;                // 16 KB
