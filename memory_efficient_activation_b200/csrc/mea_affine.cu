@@ -9,9 +9,36 @@
 // movement and the deterministic reductions are the per-channel kernels of
 // mea_channel.cuh; this file supplies the arithmetic (AffineOp) and the
 // dispatch over activation and storage dtype.
+#include <type_traits>
+
 #include "mea_channel.cuh"
 
 namespace mea {
+
+// Swish'(z) dy for two elements of bf16 storage: the operations of
+// Swish::df<false> in the same order, the multiplies and adds as packed
+// .f32x2 pairs (each result rounded as the scalar instruction rounds it), so
+// the values are bitwise those of two scalar calls.
+__device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, float d1, const Coef &k, bool &tail,
+                                               float &o0, float &o1)
+{
+    const F2 z = pk(z0, z1);
+    float t0, t1;
+    upk(mul2(z, sp2(k.c_hi)), t0, t1);
+    const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
+    tail |= (t0 > kTailT) | (t1 > kTailT);
+    const F2 E = pk(e0, e1);
+    float a0, a1;
+    upk(add2(sp2(1.f), E), a0, a1);
+    const F2 s = pk(rcp_ftz(a0), rcp_ftz(a1));
+    float p0, p1, es0, es1, om0, om1;
+    upk(mul2(sp2(k.p), z), p0, p1);
+    upk(mul2(E, s), es0, es1);
+    upk(fma2(s, sp2(-1.f), sp2(1.f)), om0, om1);    // 1 - s, rounded once
+    const float sm0 = p0 > 0.f ? es0 : om0, sm1 = p1 > 0.f ? es1 : om1;
+    const F2 zs = mul2(pk(fminf(p0, kBig), fminf(p1, kBig)), s);
+    upk(mul2(pk(d0, d1), fma2(zs, pk(sm0, sm1), s)), o0, o1);
+}
 
 template <class A>
 struct AffineOp {
@@ -82,6 +109,8 @@ struct AffineOp {
         upk(dy, d0, d1);
         if constexpr (HasPairs<A, P>::value) {
             A::df2(z0, z1, d0, d1, k, tail, o0, o1);
+        } else if constexpr (std::is_same<A, Swish>::value && !P) {
+            swish_df2_bf16(z0, z1, d0, d1, k, tail, o0, o1);
         } else {
             o0 = A::template df<P>(z0, d0, k, tail);
             o1 = A::template df<P>(z1, d1, k, tail);

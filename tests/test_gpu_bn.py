@@ -201,3 +201,18 @@ def test_dense_bottleneck_module():
     assert rel(m.gamma.grad, gd.grad) < 1e-2
     assert rel(m.beta.grad, bd.grad) < 1e-2
     assert rel(m.weight.grad, wd.grad) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_concat_bn_relu_one_value_per_channel(dtype):
+    # N H W = 1: the batch variance is 0 and xhat = 0, so y = max(beta, 0) up
+    # to the rounding of the folded gamma' x + beta' (held to the oracle's
+    # rules), invstd = eps^-1/2, and dgamma = 0 exactly (x equals its mean)
+    _run(1, [5, 3], (1, 1), dtype, 69)
+    pieces = [p.cuda() for p in _pieces(1, [5, 3], (1, 1), dtype, 69)]
+    g, b = [t.cuda() for t in _params(8, 70)]
+    y, mean, invstd = mea.concat_bn_relu_fwd(pieces, g, b, EPS)
+    dps, dg, db = mea.concat_bn_relu_bwd(pieces, torch.ones_like(y), g, b, mean, invstd)
+    torch.cuda.synchronize()
+    assert torch.allclose(invstd.cpu(), torch.full((8,), EPS ** -0.5), rtol=1e-6)
+    assert torch.all(dg == 0)

@@ -250,3 +250,10 @@ def test_memory_efficient_mlp_module(act):
     # saved for the backward: x, w1, w2 and z = x w1^T, not f(z)
     hidden = [t for t in saved if t.dim() == 2 and t.shape == (M, h)]
     assert len(hidden) == 1
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (7, 16, 24), (100, 8, 64), (129, 264, 8)])
+def test_matmul_act_tiny_and_ragged(M, N, K):
+    # single rows, the narrowest N and K the C ABI takes, M that leaves the
+    # second CTA of the pair (or most of the first) without rows
+    _run("swish", M, N, K, 38)
