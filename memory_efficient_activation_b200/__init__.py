@@ -13,6 +13,7 @@ Functions (the C ABI's names without the ``mea_`` prefix):
     affine_act_fwd, affine_act_bwd, swish_channel_fwd, swish_channel_bwd,
     matmul_act_fwd, matmul_act_bwd,
     concat_bn_relu_fwd, concat_bn_relu_apply, concat_bn_relu_bwd,
+    act_fwd_bwd_host,
     act_bwd_workspace_bytes, affine_swish_bwd_workspace_bytes,
     affine_act_bwd_workspace_bytes, swish_channel_bwd_workspace_bytes
 Autograd / modules:
@@ -38,6 +39,7 @@ __all__ = [
     "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
     "matmul_act_fwd", "matmul_act_bwd",
     "concat_bn_relu_fwd", "concat_bn_relu_apply", "concat_bn_relu_bwd",
+    "act_fwd_bwd_host",
     "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
     "affine_act_bwd_workspace_bytes", "swish_channel_bwd_workspace_bytes",
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
@@ -432,6 +434,65 @@ def concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, invstd, dpieces=None, accu
                                              ws.numel() * ws.element_size(), _stream(dy))
     _capi.check("mea_concat_bn_relu_bwd", st)
     return dpieces, dg, db
+
+
+class _HostPipe:
+    """Device buffers and streams reused by act_fwd_bwd_host (per device)."""
+
+    def __init__(self, device, numel, dtype):
+        self.key = (device, numel, dtype)
+        self.bufs = [torch.empty(numel, dtype=dtype, device=device) for _ in range(4)]   # x, dy, y, dx
+        self.streams = [torch.cuda.Stream(device) for _ in range(3)]                     # copy in, compute, copy out
+
+
+_host_pipes: dict = {}
+
+
+def act_fwd_bwd_host(act: str, hx: torch.Tensor, hdy: torch.Tensor, param: float = 1.0,
+                     hy: torch.Tensor | None = None, hdx: torch.Tensor | None = None, chunks: int = 8,
+                     device=None):
+    """Forward and backward of an activation on data in pinned host memory:
+    y = f(x) and dx = dy f'(x) copied back to host.  The tensor is split into
+    `chunks` pieces that flow through three streams (host to device, the two
+    kernels, device to host), so the copy of one piece overlaps the kernels of
+    the previous one and the copy back of the one before (PCIe carries both
+    directions at once).  Returns (hy, hdx); the work is queued behind the
+    current stream and the current stream waits for its end."""
+    if hx.is_cuda or hdy.is_cuda:
+        raise ValueError("hx and hdy must be host tensors")
+    if hx.shape != hdy.shape or hx.dtype != hdy.dtype:
+        raise ValueError("hx and hdy must match")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    n = hx.numel()
+    hy = torch.empty_like(hx).pin_memory() if hy is None else hy
+    hdx = torch.empty_like(hx).pin_memory() if hdx is None else hdx
+    key = (dev, n, hx.dtype)
+    pipe = _host_pipes.get(dev)
+    if pipe is None or pipe.key != key:
+        pipe = _HostPipe(dev, n, hx.dtype)
+        _host_pipes[dev] = pipe
+    x, dy, y, dx = pipe.bufs
+    s_in, s_run, s_out = pipe.streams
+    cur = torch.cuda.current_stream(dev)
+    fx, fdy, fy, fdx = hx.reshape(-1), hdy.reshape(-1), hy.reshape(-1), hdx.reshape(-1)
+    step = -(-n // max(1, chunks))
+    step = -(-step // 256) * 256                 # pieces start 16-byte aligned
+    s_in.wait_stream(cur)
+    for lo in range(0, n, step):
+        hi = min(n, lo + step)
+        with torch.cuda.stream(s_in):
+            x[lo:hi].copy_(fx[lo:hi], non_blocking=True)
+            dy[lo:hi].copy_(fdy[lo:hi], non_blocking=True)
+        s_run.wait_stream(s_in)
+        with torch.cuda.stream(s_run):
+            act_fwd(act, x[lo:hi], param, out=y[lo:hi])
+            act_bwd(act, x[lo:hi], dy[lo:hi], param, out=dx[lo:hi])
+        s_out.wait_stream(s_run)
+        with torch.cuda.stream(s_out):
+            fy[lo:hi].copy_(y[lo:hi], non_blocking=True)
+            fdx[lo:hi].copy_(dx[lo:hi], non_blocking=True)
+    cur.wait_stream(s_out)
+    return hy, hdx
 
 
 # ---------------------------------------------------------------- autograd
