@@ -45,6 +45,7 @@ SHAPE = (8, 2048, 4096)
 DTYPE = "bf16"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0        # the B200's nominal HBM3e bandwidth (8 TB/s per GPU, DGX figure)
 DOMINANT_KERNEL = "act_kernel<Swish, Bf16, MODE 1> (mea_act_bwd)"
 
 
@@ -276,6 +277,7 @@ def run_ours(args, rank, ws, local):
         "timing": f"CUDA events around each kernel on every {every}th step of the timed region",
         "fwd_frac": round(accounting.fwd_bytes(n, DTYPE) / (fwd_ms * 1e-3) / 1e9 / peak, 4),
         "step_frac": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "step_frac_of_nominal_8tbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
     }
 
     out = {
