@@ -6,7 +6,18 @@
  * backward recomputes what it needs from the saved input x in the same pass
  * and writes dx = dy * f'(x) (plus d alpha for a learnable Swish alpha,
  * scalar or one per channel, or d gamma / d beta for the fused per-channel
- * affine + activation).
+ * affine + activation).  The same recompute principle is applied beside two
+ * neighbouring operations: a matrix multiply with the activation in its
+ * epilogue (mea_matmul_act_*: only the product Z is kept, f'(Z) is applied
+ * inside the backward matmul) and DenseNet's concatenation + batch
+ * normalization + ReLU (mea_concat_bn_relu_*: the concatenation is never
+ * formed, only the batch statistics are kept, the output is re-populated).
+ *
+ * Entry points: mea_act_fwd / mea_act_bwd (+ _workspace_bytes,
+ * mea_act_bwd_dparam_noalloc); mea_affine_swish_* and mea_affine_act_*;
+ * mea_swish_channel_*; mea_matmul_act_fwd / _bwd; mea_concat_bn_relu_fwd /
+ * _apply / _bwd (+ _workspace_bytes); mea_status_string, mea_last_error,
+ * mea_version.
  *
  * Sources, by page and section:
  *  - "Memory efficient Swish" (adeeplearner blog, 2021-05-17):
@@ -43,9 +54,11 @@
  *    path): reductions run on a grid fixed by the shape and sum in a fixed
  *    order, independent of the stream, the run and the GPU's SM count.
  *  - Workspaces: the first 4 bytes are a completion counter (see
- *    mea_act_bwd); bytes 4..7 are an error word that a kernel sets non-zero
- *    if one of its bounded waits on shared-memory barriers expires (which
- *    does not happen in correct operation); results are then undefined.
+ *    mea_act_bwd); bytes 4..7 are an error word that the per-channel
+ *    backward sets non-zero if one of its bounded waits on shared-memory
+ *    barriers expires (which does not happen in correct operation); results
+ *    are then undefined.  The matmul kernels, which take no workspace, record
+ *    the same condition in a device word of the library.
  */
 #ifndef MEA_H
 #define MEA_H
