@@ -398,6 +398,13 @@ MEA_API mea_status_t mea_act_bwd_dparam_noalloc(mea_act_t act, mea_dtype_t dtype
                                                 const float *param_dev, float *dparam_dev,
                                                 mea_stream_t stream);
 
+/* Reads (and with clear non-zero, resets) the matmul kernels' device error
+ * word on the current device: non-zero if a bounded barrier wait in a
+ * mea_matmul_act_* kernel expired since the last clear (which does not
+ * happen in correct operation).  Synchronises the current device.  Returns
+ * -1 if the word cannot be read (a CUDA error; see mea_last_error). */
+MEA_API int mea_matmul_error_word(int clear);
+
 /* Static description of a status code. */
 MEA_API const char *mea_status_string(mea_status_t status);
 

@@ -51,6 +51,7 @@ SIGNATURES = {
     "mea_swish_channel_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mea_matmul_act_fwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _f, _vp, _vp, _vp]),
     "mea_matmul_act_bwd": (_i, [_i, _i64, _i64, _i64, _vp, _vp, _vp, _f, _vp, _vp]),
+    "mea_matmul_error_word": (_i, [_i]),
     "mea_concat_bn_relu_workspace_bytes": (_sz, [_i64, _i64]),
     "mea_concat_bn_relu_fwd": (_i, [_i, _i, _ptrs, _shape, _i64, _i64, _vp, _vp, _f, _f, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),

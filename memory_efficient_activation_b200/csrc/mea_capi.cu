@@ -409,6 +409,18 @@ mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int64_t K, 
     return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_matmul_act_bwd launch");
 }
 
+int mea_matmul_error_word(int clear)
+{
+    clear_error();
+    unsigned int w = 0;
+    cudaError_t e = mea::matmul_error_word(clear, &w);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "mea_matmul_error_word");
+        return -1;
+    }
+    return (int)w;
+}
+
 static mea_status_t bn_common(const char *name, int dtype, int npieces, const void *const *pieces,
                               const int64_t *channels, int64_t N, int64_t HW, mea::BnLaunch *l, size_t *plane_bytes)
 {

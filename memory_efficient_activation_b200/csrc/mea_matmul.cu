@@ -448,6 +448,16 @@ cudaError_t by_act(const MatmulLaunch &a, const CUtensorMap &mx, const CUtensorM
 
 }  // namespace
 
+cudaError_t matmul_error_word(int clear, unsigned int *word)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(word, g_matmul_error, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_matmul_error, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
 cudaError_t launch_matmul_act(const MatmulLaunch &a)
 {
     CUtensorMap mx, mw;

@@ -27,6 +27,7 @@ struct MatmulLaunch {
 };
 
 cudaError_t launch_matmul_act(const MatmulLaunch &a);
+cudaError_t matmul_error_word(int clear, unsigned int *word);   // synchronous
 
 // Tile shape of the kernel (rows of X, rows of W, K per pipeline stage).
 constexpr int kMatmulBM = 256;

@@ -257,3 +257,9 @@ def test_matmul_act_tiny_and_ragged(M, N, K):
     # single rows, the narrowest N and K the C ABI takes, M that leaves the
     # second CTA of the pair (or most of the first) without rows
     _run("swish", M, N, K, 38)
+
+
+def test_matmul_error_word_clear():
+    # no bounded wait expired in any matmul launched by this test session
+    assert mea._capi.lib().mea_matmul_error_word(1) == 0
+    assert mea._capi.lib().mea_matmul_error_word(0) == 0
