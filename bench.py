@@ -611,6 +611,8 @@ def run_secondary(args):
         return run_mlp(args)
     elif wl == "densenet_bn_bf16":
         return run_densenet_bn(args)
+    elif wl == "densenet_bc100":
+        return run_densenet_bc100(args)
     elif wl == "memory_study":
         return run_memory_study(args)
     elif wl == "swish_f32_1m":
@@ -779,6 +781,121 @@ def run_densenet_bn(args, N: int = 64, ks=(64, 32, 32, 32, 32, 32), spatial=(56,
             "clocks": clk.summary()}
 
 
+def _densenet_bc(efficient: bool, growth: int = 12, depth: int = 100, classes: int = 10, dtype=torch.float32):
+    """DenseNet-BC (bottleneck + compression 0.5) for 32 x 32 inputs, random
+    weights: three dense blocks of (depth - 4) / 6 layers; a layer is
+    BN-ReLU-conv1x1 (4 growth channels) then BN-ReLU-conv3x3 (growth
+    channels) on the concatenation of every earlier feature map of its block.
+    efficient: the first BN-ReLU-conv1x1 of each layer is the memory-efficient
+    bottleneck (concatenation never formed, normalized tensor in one buffer
+    shared by all layers, re-populated in the backward); otherwise torch.cat
+    + BatchNorm2d + ReLU + Conv2d."""
+    import torch.nn as nn
+    layers_per_block = (depth - 4) // 6
+    shared = mea.SharedBuffer()
+
+    class Layer(nn.Module):
+        def __init__(self, cin):
+            super().__init__()
+            if efficient:
+                self.b1 = mea.MemoryEfficientDenseBottleneck(cin, 4 * growth, shared, dtype=dtype)
+            else:
+                self.n1 = nn.BatchNorm2d(cin)
+                self.c1 = nn.Conv2d(cin, 4 * growth, 1, bias=False)
+            self.n2 = nn.BatchNorm2d(4 * growth)
+            self.c2 = nn.Conv2d(4 * growth, growth, 3, padding=1, bias=False)
+
+        def forward(self, feats):
+            if efficient:
+                h = self.b1(*feats)
+            else:
+                h = self.c1(torch.relu(self.n1(torch.cat(feats, 1))))
+            return self.c2(torch.relu(self.n2(h)))
+
+    class Net(nn.Module):
+        def __init__(self):
+            super().__init__()
+            c = 2 * growth
+            self.stem = nn.Conv2d(3, c, 3, padding=1, bias=False)
+            self.blocks = nn.ModuleList()
+            self.trans = nn.ModuleList()
+            for bi in range(3):
+                blk = nn.ModuleList()
+                for _ in range(layers_per_block):
+                    blk.append(Layer(c))
+                    c += growth
+                self.blocks.append(blk)
+                if bi < 2:
+                    self.trans.append(nn.Sequential(nn.BatchNorm2d(c), nn.ReLU(), nn.Conv2d(c, c // 2, 1, bias=False),
+                                                    nn.AvgPool2d(2)))
+                    c //= 2
+            self.final = nn.BatchNorm2d(c)
+            self.fc = nn.Linear(c, classes)
+
+        def forward(self, x):
+            h = self.stem(x)
+            for bi, blk in enumerate(self.blocks):
+                feats = [h]
+                for layer in blk:
+                    feats.append(layer(feats))
+                h = torch.cat(feats, 1)
+                if bi < 2:
+                    h = self.trans[bi](h)
+            h = torch.relu(self.final(h)).mean(dim=(2, 3))
+            return self.fc(h)
+
+    return Net().to(dtype)
+
+
+def run_densenet_bc100(args, batch: int = 64):
+    """One training step (forward, backward) of DenseNet-BC-100 (growth 12)
+    on a synthetic batch of 64 32 x 32 images, fp32, random weights: the page's
+    "Performance" comparison (naive against memory-efficient implementation,
+    memory per GPU and time per minibatch) re-measured on one B200 with the
+    memory-efficient bottleneck kernels.  No dataset: inputs and the loss
+    weights are synthetic."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    torch.backends.cudnn.benchmark = True     # both networks: cuDNN picks its fastest convolution algorithms
+    x = torch.from_numpy(synthetic.normal_f64(batch * 3 * 32 * 32, 1.0, 80, synthetic.STREAM_X)).float()
+    x = x.view(batch, 3, 32, 32).to(dev)
+    wloss = torch.from_numpy(synthetic.normal_f64(batch * 10, 1.0, 80, synthetic.STREAM_DY)).float().view(batch, 10).to(dev)
+    res = {}
+    for name, eff in (("naive", False), ("memory_efficient", True)):
+        torch.manual_seed(0)
+        net = _densenet_bc(eff).to(dev)
+        net.train()
+
+        def step():
+            net.zero_grad(set_to_none=True)
+            (net(x) * wloss).sum().backward()
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+        step()
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            step()
+        e.record()
+        torch.cuda.synchronize()
+        res[name] = {"peak_memory_bytes": int(peak), "peak_above_weights_bytes": int(peak - base),
+                     "ms_per_minibatch": round(s.elapsed_time(e) / args.steps, 3),
+                     "parameters": int(sum(p.numel() for p in net.parameters()))}
+        del net
+        torch.cuda.empty_cache()
+    return {"workload": "densenet_bc100", "batch": batch, "image": [3, 32, 32], "dtype": "fp32",
+            "data": "synthetic (no dataset, random weights)", "steps": args.steps, "warmup": args.warmup,
+            "results": res,
+            "memory_ratio": round(res["memory_efficient"]["peak_memory_bytes"] / res["naive"]["peak_memory_bytes"], 4),
+            "time_ratio": round(res["memory_efficient"]["ms_per_minibatch"] / res["naive"]["ms_per_minibatch"], 4)}
+
+
 class _PlainSwish(torch.nn.Module):
     """The plain autograd Swish of the pages' first listing: x * sigmoid(alpha x)
     built from PyTorch ops, which keeps every intermediate for the backward.
@@ -868,7 +985,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="swish_bf16",
                     choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
                              "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "mlp_bf16",
-                             "densenet_bn_bf16", "swish_f32_1m", "memory_study"],
+                             "densenet_bn_bf16", "densenet_bc100", "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -725,7 +725,8 @@ class ConcatBNReLUConvFunction(torch.autograd.Function):
     pieces (which the network keeps anyway), the weights and 2 C floats of
     statistics: the normalized tensor lives in a shared buffer and the
     backward re-populates it before the weight gradient needs it.  The 1x1
-    convolution is a batched matmul (torch.matmul)."""
+    convolution and its gradients are the library's (cuDNN through
+    torch.nn.functional.conv2d and torch.nn.grad), as in a plain layer."""
 
     @staticmethod
     def forward(ctx, shared, weight, gamma, beta, running_mean, running_var, eps, momentum, *pieces):
@@ -735,31 +736,32 @@ class ConcatBNReLUConvFunction(torch.autograd.Function):
         y = shared.get((N, C) + spatial, pieces[0].dtype, pieces[0].device)
         y, mean, invstd = concat_bn_relu_fwd(list(pieces), gamma, beta, eps, momentum, running_mean, running_var,
                                              out=y)
-        out = torch.matmul(weight.view(weight.shape[0], C), y.view(N, C, -1))
+        out = torch.nn.functional.conv2d(y, weight)
         ctx.shared, ctx.spatial = shared, spatial
         ctx.save_for_backward(weight, gamma, beta, mean, invstd, *pieces)
-        return out.view((N, weight.shape[0]) + spatial)
+        return out
 
     @staticmethod
     def backward(ctx, dout):
         weight, gamma, beta, mean, invstd, *pieces = ctx.saved_tensors
         N = pieces[0].shape[0]
         C = sum(int(p.shape[1]) for p in pieces)
-        w2 = weight.view(weight.shape[0], C)
         y = ctx.shared.get((N, C) + ctx.spatial, pieces[0].dtype, pieces[0].device)
         concat_bn_relu_apply(pieces, gamma, beta, mean, invstd, out=y)
-        do = dout.contiguous().view(N, w2.shape[0], -1)
-        dw = torch.matmul(do, y.view(N, C, -1).transpose(1, 2)).sum(dim=0)
-        dy = torch.matmul(w2.t(), do).view_as(y)
+        dout = dout.contiguous()
+        dw = torch.nn.grad.conv2d_weight(y, weight.shape, dout)
+        dy = torch.nn.grad.conv2d_input(y.shape, weight, dout)
         dpieces, dg, db = concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, invstd)
-        return (None, dw.view_as(weight), dg, db, None, None, None, None, *dpieces)
+        return (None, dw, dg, db, None, None, None, None, *dpieces)
 
 
 class MemoryEfficientDenseBottleneck(torch.nn.Module):
     """The bottleneck of a DenseNet layer: concatenation of the previous
     feature maps, batch normalization, ReLU and a 1x1 convolution to
     `out_channels`, with the concatenated and normalized tensors kept only in
-    `shared` (one buffer for every layer).  NCHW bf16 or fp32."""
+    `shared` (one buffer for every layer).  NCHW bf16 or fp32; the gradient
+    of the normalized tensor (the 1x1 convolution's input gradient) is a
+    transient of the backward."""
 
     def __init__(self, in_channels: int, out_channels: int, shared: SharedBuffer | None = None,
                  eps: float = 1e-5, momentum: float = 0.1, dtype=torch.bfloat16):

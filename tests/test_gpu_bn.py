@@ -14,6 +14,8 @@ zero may take either side of the ReLU: its dz may differ by dy, which adds
 dbeta (dgamma) allowance.  dgamma and dbeta: 1e-5 relative plus 1e-5 of
 the sum of their terms' magnitudes.
 """
+import copy
+
 import numpy as np
 import pytest
 import torch
@@ -216,3 +218,60 @@ def test_concat_bn_relu_one_value_per_channel(dtype):
     torch.cuda.synchronize()
     assert torch.allclose(invstd.cpu(), torch.full((8,), EPS ** -0.5), rtol=1e-6)
     assert torch.all(dg == 0)
+
+
+def test_densenet_bc_efficient_matches_naive():
+    # the same DenseNet-BC (depth 16: two layers per block), same weights,
+    # fp32: the memory-efficient bottleneck gives the naive network's logits
+    # and gradients up to summation order (batch statistics in fp64 here,
+    # cuDNN's own in the naive layers)
+    import bench
+    tf32 = (torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32)
+    torch.backends.cudnn.allow_tf32 = False      # both networks in plain fp32 convolutions
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        _densenet_compare(bench)
+    finally:
+        torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32 = tf32
+
+
+def _densenet_compare(bench):
+    # Both fp32 networks against the naive one evaluated in float64: a wiring
+    # fault (a stale shared buffer, a piece gradient lost or counted twice)
+    # moves the logits and gradients by O(1).  The library convolutions both
+    # networks call (cuDNN's algorithm choices) put the naive network's own
+    # fp32 gradients up to ~1e-3 from float64 here, so the bound is 1e-2.
+    torch.manual_seed(0)
+    naive = bench._densenet_bc(False, depth=16).cuda()
+    eff = bench._densenet_bc(True, depth=16).cuda()
+    with torch.no_grad():
+        for bn, be in zip(naive.blocks, eff.blocks):
+            for ln, le in zip(bn, be):
+                le.b1.weight.copy_(ln.c1.weight)
+                le.b1.gamma.copy_(ln.n1.weight)
+                le.b1.beta.copy_(ln.n1.bias)
+                le.n2.load_state_dict(ln.n2.state_dict())
+                le.c2.load_state_dict(ln.c2.state_dict())
+        for name in ("stem", "trans", "final", "fc"):
+            getattr(eff, name).load_state_dict(getattr(naive, name).state_dict())
+    ref = copy.deepcopy(naive).double()
+    x = torch.from_numpy(synthetic.normal_f64(8 * 3 * 32 * 32, 1.0, 81, synthetic.STREAM_X)).view(8, 3, 32, 32)
+    outs = []
+    for net, xx in ((naive, x.float().cuda()), (eff, x.float().cuda()), (ref, x.cuda())):
+        net.train()
+        out = net(xx)
+        out.square().sum().backward()
+        outs.append(out.detach().double())
+    torch.cuda.synchronize()
+
+    def rel(a, b):
+        return float((a.detach().double() - b.detach()).norm() / b.detach().norm())
+
+    assert rel(outs[1], outs[2]) < 1e-3
+    for bn, be, br in zip(naive.blocks, eff.blocks, ref.blocks):
+        for ln, le, lr in zip(bn, be, br):
+            assert rel(le.b1.weight.grad, lr.c1.weight.grad) < 1e-2
+            assert rel(le.b1.gamma.grad, lr.n1.weight.grad) < 1e-2
+            assert rel(le.b1.beta.grad, lr.n1.bias.grad) < 1e-2
+            assert rel(le.c2.weight.grad, lr.c2.weight.grad) < 1e-2
+    assert rel(eff.stem.weight.grad, ref.stem.weight.grad) < 1e-2
