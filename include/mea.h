@@ -327,9 +327,8 @@ MEA_API mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int
  *                 backward re-populates it (mea_concat_bn_relu_apply).  Must
  *                 not overlap a piece.
  *   workspace     device scratch of mea_concat_bn_relu_workspace_bytes(N, C)
- *                 bytes, 16-byte aligned, with the completion-counter rule of
- *                 mea_act_bwd (zero-fill once; each call leaves the counter at
- *                 zero; no concurrent sharing).
+ *                 bytes, 16-byte aligned (no counter: no zero-fill needed;
+ *                 calls that share it must not run concurrently).
  * Source: "A memory-efficient implementation of DenseNets", section
  * "Motivation" (shared allocations for every concatenation and batch
  * normalization output, re-populated in the backward); batch normalization

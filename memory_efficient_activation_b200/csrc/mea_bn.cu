@@ -15,18 +15,15 @@
 //                                  x - shift and d^2 (shift: one element of
 //                                  the channel), fp32 within a 16-byte
 //                                  vector, fp64 across -> partials
-//                                  and, in the last block to finish
-//                                  (atomic ticket), per channel in slice
-//                                  order: mean, invstd = 1 / sqrt(var +
-//                                  eps), running statistics (momentum;
-//                                  unbiased variance)
+//             bn_finalize_kernel   per channel, slices in order: mean,
+//                                  invstd = 1 / sqrt(var + eps), running
+//                                  statistics (momentum; unbiased variance)
 //             bn_apply_kernel      y = max(gamma' x + beta', 0), gamma' =
 //                                  gamma invstd, beta' = beta - mean gamma'
 //   backward  bn_bwd_reduce_kernel per (channel, slice): recompute the ReLU
 //                                  mask from x; sums of dz and dz xhat
 //                                  (fp32 within a vector, fp64 across)
-//                                  and, in the last block, dbeta, dgamma and
-//                                  the coefficients of dx
+//             bn_bwd_finalize      dbeta, dgamma and the coefficients of dx
 //             bn_dx_kernel         dx = gamma invstd (dz - dbeta / n -
 //                                  xhat dgamma / n), written or added into
 //                                  the pieces' gradients
@@ -49,6 +46,7 @@ namespace {
 
 constexpr int kBnThreads = 256;
 constexpr int kBnBlocksTarget = 1184;     // C * S is sized to about this many blocks (148 x 8)
+constexpr int kBnFinThreads = 128;
 
 int bn_slices(int64_t N, int64_t C)
 {
@@ -193,40 +191,11 @@ __device__ __forceinline__ int64_t first_of_channel(const BnPieces &t, const Pla
     return (int64_t)p.j * HW;       // sample 0, channel j of the piece, element 0
 }
 
-// Per channel, slices in order: mean, invstd, running statistics.
-__device__ __forceinline__ void bn_finalize_channel(const double *partials, int64_t c, int slices, double n,
-                                                    float eps, float momentum, float *mean, float *invstd,
-                                                    float *running_mean, float *running_var)
-{
-    double s1 = 0.0, s2 = 0.0;
-    for (int s = 0; s < slices; ++s) {
-        s1 += __ldcg(partials + 3 * (c * slices + s));
-        s2 += __ldcg(partials + 3 * (c * slices + s) + 1);
-    }
-    const double shift = __ldcg(partials + 3 * c * slices + 2);
-    const double md = s1 / n;                 // mean of d = x - shift
-    double var = s2 / n - md * md;
-    if (var < 0.0) var = 0.0;
-    const double mu = shift + md;
-    mean[c] = (float)mu;
-    invstd[c] = (float)(1.0 / sqrt(var + (double)eps));
-    if (running_mean) {
-        const double unbiased = n > 1.0 ? var * n / (n - 1.0) : var;
-        running_mean[c] = (float)((1.0 - momentum) * running_mean[c] + momentum * mu);
-        running_var[c] = (float)((1.0 - momentum) * running_var[c] + momentum * unbiased);
-    }
-}
-
-// Statistics pass; the last block to finish (atomic ticket in the
-// workspace header, returned to zero) finalizes every channel.
 template <typename T>
 __global__ void __launch_bounds__(kBnThreads, 3)
-bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, void *__restrict__ ws,
-                float eps, float momentum, float *__restrict__ mean, float *__restrict__ invstd,
-                float *__restrict__ running_mean, float *__restrict__ running_var)
+bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, double *__restrict__ partials)
 {
     pdl_wait();
-    double *partials = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
     const PlaneJob p = plane_job(t, N, slices);
     const void *x = t.ptr[p.piece];
     StatsF<T> f{x, Store<T>::load1(x, first_of_channel(t, p, HW))};
@@ -240,10 +209,34 @@ bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int ve
         partials[3 * blockIdx.x + 1] = b;
         partials[3 * blockIdx.x + 2] = (double)f.shift;
     }
-    if (!last_block_done(static_cast<unsigned int *>(ws))) return;
-    const double n = (double)(N * HW);
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
-        bn_finalize_channel(partials, c, slices, n, eps, momentum, mean, invstd, running_mean, running_var);
+}
+
+__global__ void __launch_bounds__(kBnFinThreads)
+bn_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n, float eps, float momentum,
+                   float *__restrict__ mean, float *__restrict__ invstd, float *__restrict__ running_mean,
+                   float *__restrict__ running_var)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < slices; ++s) {
+        s1 += partials[3 * (c * slices + s)];
+        s2 += partials[3 * (c * slices + s) + 1];
+    }
+    const double shift = partials[3 * c * slices + 2];
+    const double md = s1 / n;                 // mean of d = x - shift
+    double var = s2 / n - md * md;
+    if (var < 0.0) var = 0.0;
+    const double mu = shift + md;
+    mean[c] = (float)mu;
+    invstd[c] = (float)(1.0 / sqrt(var + (double)eps));
+    if (running_mean) {
+        const double unbiased = n > 1.0 ? var * n / (n - 1.0) : var;
+        running_mean[c] = (float)((1.0 - momentum) * running_mean[c] + momentum * mu);
+        running_var[c] = (float)((1.0 - momentum) * running_var[c] + momentum * unbiased);
+    }
 }
 
 template <typename T>
@@ -371,35 +364,13 @@ struct ReduceF {
     }
 };
 
-// dbeta, dgamma, and dx = a dz + b + c xhat with a = gamma r, b = -a dbeta / n,
-// c = -a dgamma / n (coef[3 ch + 0..2]); slices in order.
-__device__ __forceinline__ void bn_bwd_finalize_channel(const double *partials, int64_t c, int slices, double n,
-                                                        const float *gamma, const float *invstd, float *dgamma,
-                                                        float *dbeta, float *coef)
-{
-    double s1 = 0.0, s2 = 0.0;
-    for (int s = 0; s < slices; ++s) {
-        s1 += __ldcg(partials + 3 * (c * slices + s));
-        s2 += __ldcg(partials + 3 * (c * slices + s) + 1);
-    }
-    dbeta[c] = (float)s1;
-    dgamma[c] = (float)s2;
-    const double a = (double)gamma[c] * (double)invstd[c];
-    coef[3 * c] = (float)a;
-    coef[3 * c + 1] = (float)(-a * s1 / n);
-    coef[3 * c + 2] = (float)(-a * s2 / n);
-}
-
-// Reduction pass of the backward; the last block (ticket) finalizes.
 template <typename T>
 __global__ void __launch_bounds__(kBnThreads, 3)
 bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices, int vec,
                      const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
-                     const float *__restrict__ invstd, void *__restrict__ ws, float *__restrict__ dgamma,
-                     float *__restrict__ dbeta, float *__restrict__ coef)
+                     const float *__restrict__ invstd, double *__restrict__ partials)
 {
     pdl_wait();
-    double *partials = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
     const PlaneJob p = plane_job(t, N, slices);
     ReduceF<T> f{t.ptr[p.piece], dy, bwd_coef(gamma, beta, mean, invstd, p.c)};
     for_planes<T>(p, C, HW, vec, f);
@@ -411,10 +382,30 @@ bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t
         partials[3 * blockIdx.x] = a;
         partials[3 * blockIdx.x + 1] = b;
     }
-    if (!last_block_done(static_cast<unsigned int *>(ws))) return;
-    const double n = (double)(N * HW);
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
-        bn_bwd_finalize_channel(partials, c, slices, n, gamma, invstd, dgamma, dbeta, coef);
+}
+
+// dbeta, dgamma, and dx = a dz + b + c xhat with a = gamma r, b = -a dbeta / n,
+// c = -a dgamma / n (coef[3 ch + 0..2]).
+__global__ void __launch_bounds__(kBnFinThreads)
+bn_bwd_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n,
+                       const float *__restrict__ gamma, const float *__restrict__ invstd, float *__restrict__ dgamma,
+                       float *__restrict__ dbeta, float *__restrict__ coef)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < slices; ++s) {
+        s1 += partials[3 * (c * slices + s)];
+        s2 += partials[3 * (c * slices + s) + 1];
+    }
+    dbeta[c] = (float)s1;
+    dgamma[c] = (float)s2;
+    const double a = (double)gamma[c] * (double)invstd[c];
+    coef[3 * c] = (float)a;
+    coef[3 * c + 1] = (float)(-a * s1 / n);
+    coef[3 * c + 2] = (float)(-a * s2 / n);
 }
 
 template <typename T>
@@ -506,10 +497,16 @@ cudaError_t fwd_t(const BnLaunch &a, bool stats)
     const int64_t grid = a.C * slices;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const int vec = vec_ok(a, Store<T>::kBytes, false);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+    cudaError_t e = cudaSuccess;
     if (stats) {
-        cudaError_t e = launch_pdl(bn_stats_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N,
-                                   a.C, a.HW, slices, vec, a.workspace, a.eps, a.momentum, a.mean, a.invstd,
-                                   a.running_mean, a.running_var);
+        e = launch_pdl(bn_stats_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
+                       slices, vec, partials);
+        if (e != cudaSuccess) return e;
+        const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
+        e = launch_pdl(bn_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
+                       static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.eps, a.momentum,
+                       a.mean, a.invstd, a.running_mean, a.running_var);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(bn_apply_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
@@ -528,8 +525,12 @@ cudaError_t bwd_t(const BnLaunch &a)
     float *coef = reinterpret_cast<float *>(partials + 3 * grid);
     cudaError_t e = launch_pdl(bn_bwd_reduce_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in,
                                a.dy, a.N, a.C, a.HW, slices, vec, a.gamma, a.beta,
-                               static_cast<const float *>(a.mean), static_cast<const float *>(a.invstd), a.workspace,
-                               a.dgamma, a.dbeta, coef);
+                               static_cast<const float *>(a.mean), static_cast<const float *>(a.invstd), partials);
+    if (e != cudaSuccess) return e;
+    const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
+    e = launch_pdl(bn_bwd_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
+                   static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.gamma,
+                   static_cast<const float *>(a.invstd), a.dgamma, a.dbeta, coef);
     if (e != cudaSuccess) return e;
     return launch_pdl(bn_dx_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.din, a.dy, a.N,
                       a.C, a.HW, slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
