@@ -299,6 +299,11 @@ struct Tanh {
 // be subnormal (-w^2 + P(t) < -124 ln 2, i.e. x below about -13.1) but
 // x Phi(x) is still normal, the element is recomputed with the exponentials
 // scaled by 2^64.
+//
+// The bf16 forward uses the same form with a degree-5 polynomial fitted
+// here (csrc/fit_erfc_bf16.py: near-minimax over |w| <= 9.6, error of
+// log erfc below 7.7e-6, far inside the bf16 rounding of the result); the
+// backward, whose value cancels near x = -0.75, keeps the degree-9 one.
 struct GeluErf {
     static constexpr float kNegRsqrt2Hi = -0.707106769084930419921875f;
     static constexpr float kNegRsqrt2Lo = -1.2101617104478969362e-08f;
@@ -322,6 +327,18 @@ struct GeluErf {
         p = fmaf(p, t, 0.37409196f);
         p = fmaf(p, t, 1.00002368f);
         p = fmaf(p, t, -1.26551223f);
+        return fmaf(-a, a, p) * kLog2ef;
+    }
+    // Degree-5 form of nr_parts for the bf16 forward.
+    static __device__ __forceinline__ float nr5_parts(float a, float &t)
+    {
+        t = rcp_ftz(fmaf(0.5f, a, 1.0f));
+        float p = 0.228795588f;
+        p = fmaf(p, t, -0.709205508f);
+        p = fmaf(p, t, 0.474508315f);
+        p = fmaf(p, t, 0.254436046f);
+        p = fmaf(p, t, 1.01801503f);
+        p = fmaf(p, t, -1.26654184f);
         return fmaf(-a, a, p) * kLog2ef;
     }
     static __device__ __forceinline__ bool is_tail(float x, const Coef &)
@@ -367,6 +384,22 @@ struct GeluErf {
         p = fma2(p, t, sp2(-1.26551223f));
         u = mul2(fma2(pk(-fabsf(w0), -fabsf(w1)), a, p), sp2(kLog2ef));
     }
+    static __device__ __forceinline__ void nr5_parts2(F2 x, float &w0, float &w1, F2 &t, F2 &u)
+    {
+        const F2 w = mul2(x, sp2(kNegRsqrt2Hi));
+        upk(w, w0, w1);
+        const F2 a = pk(fabsf(w0), fabsf(w1));
+        float d0, d1;
+        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
+        t = pk(rcp_ftz(d0), rcp_ftz(d1));
+        F2 p = sp2(0.228795588f);
+        p = fma2(p, t, sp2(-0.709205508f));
+        p = fma2(p, t, sp2(0.474508315f));
+        p = fma2(p, t, sp2(0.254436046f));
+        p = fma2(p, t, sp2(1.01801503f));
+        p = fma2(p, t, sp2(-1.26654184f));
+        u = mul2(fma2(pk(-fabsf(w0), -fabsf(w1)), a, p), sp2(kLog2ef));
+    }
     static __device__ __forceinline__ F2 erfc2(float w0, float w1, F2 t, float u0, float u1)
     {
         float a0, a1;
@@ -378,7 +411,7 @@ struct GeluErf {
         const F2 x = pk(x0, x1);
         float w0, w1, u0, u1;
         F2 t, u;
-        nr_parts2(x, w0, w1, t, u);
+        nr5_parts2(x, w0, w1, t, u);
         upk(u, u0, u1);
         tail |= ((u0 < -kTailT) && (x0 < 0.f)) || ((u1 < -kTailT) && (x1 < 0.f));
         upk(mul2(mul2(sp2(0.5f), x), erfc2(w0, w1, t, u0, u1)), o0, o1);
@@ -411,7 +444,7 @@ struct GeluErf {
         } else {
             const float w = x * kNegRsqrt2Hi;
             float t;
-            const float u = nr_parts(fabsf(w), t);
+            const float u = nr5_parts(fabsf(w), t);
             tail |= (u < -kTailT) && (x < 0.f);
             const float ans = t * ex2_ftz(u);
             const float ec = w >= 0.f ? ans : 2.f - ans;
