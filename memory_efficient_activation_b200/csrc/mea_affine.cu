@@ -15,10 +15,17 @@
 
 namespace mea {
 
-// Swish'(z) dy for two elements of bf16 storage: the operations of
-// Swish::df<false> in the same order, the multiplies and adds as packed
-// .f32x2 pairs (each result rounded as the scalar instruction rounds it), so
-// the values are bitwise those of two scalar calls.
+// Swish'(z) dy for two elements of bf16 storage, in the fewest packed
+// .f32x2 operations: with E = 2^t = e^(-alpha z) and s = 1 / (1 + E),
+// Sigmoid(-alpha z) = E s (a product, no cancellation on either side), and
+//   dz = dy (s (1 + alpha z E s))
+// (s times the bracket first: s may be as small as 2^-124, and dy s could
+// fall below the normal range where the final result does not).
+// Every finite product stays finite while |t| <= kTailT; the tail flag is
+// raised for |t| > kTailT (deep negative z, and z beyond +86 or +inf, where
+// alpha z E s could be inf * 0), and the caller recomputes such elements
+// with the scalar form.  Rounding differs from the scalar form by a few fp32
+// ulps, far inside a bf16 ulp.
 __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, float d1, const Coef &k, bool &tail,
                                                float &o0, float &o1)
 {
@@ -26,18 +33,13 @@ __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, flo
     float t0, t1;
     upk(mul2(z, sp2(k.c_hi)), t0, t1);
     const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
-    tail |= (t0 > kTailT) | (t1 > kTailT);
+    tail |= (fabsf(t0) > kTailT) | (fabsf(t1) > kTailT);
     const F2 E = pk(e0, e1);
     float a0, a1;
     upk(add2(sp2(1.f), E), a0, a1);
     const F2 s = pk(rcp_ftz(a0), rcp_ftz(a1));
-    float p0, p1, es0, es1, om0, om1;
-    upk(mul2(sp2(k.p), z), p0, p1);
-    upk(mul2(E, s), es0, es1);
-    upk(fma2(s, sp2(-1.f), sp2(1.f)), om0, om1);    // 1 - s, rounded once
-    const float sm0 = p0 > 0.f ? es0 : om0, sm1 = p1 > 0.f ? es1 : om1;
-    const F2 zs = mul2(pk(fminf(p0, kBig), fminf(p1, kBig)), s);
-    upk(mul2(pk(d0, d1), fma2(zs, pk(sm0, sm1), s)), o0, o1);
+    const F2 r = fma2(mul2(sp2(k.p), z), mul2(E, s), sp2(1.f));
+    upk(mul2(pk(d0, d1), mul2(s, r)), o0, o1);
 }
 
 template <class A>

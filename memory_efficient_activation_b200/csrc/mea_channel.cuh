@@ -392,10 +392,12 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
 
     if (warp == 0) {
         if (lane == 0) {
-            int it = 0;
+            // stage s of pass `phase` (it = phase * stages + s), stepped
+            // without a division
+            int it = 0, s = 0;
+            uint32_t phase = 0;
             for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-                const int s = it % stages;
-                if (it >= stages && !mbar_wait(smem_addr(empty + s), ((it / stages) & 1) ^ 1)) {
+                if (it >= stages && !mbar_wait(smem_addr(empty + s), (phase & 1) ^ 1)) {
                     atomicExch(err, 1u);
                     break;
                 }
@@ -405,6 +407,10 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
                 bulk_load(smem_addr(bx), static_cast<const unsigned char *>(x) + t * tile_bytes, tile_bytes, fb);
                 bulk_load(smem_addr(bx + tile_bytes), static_cast<const unsigned char *>(dy) + t * tile_bytes,
                           tile_bytes, fb);
+                if (++s == stages) {
+                    s = 0;
+                    ++phase;
+                }
             }
             // Every issued copy lands before the block may exit.
             for (int j = it > stages ? it - stages : 0; j < it; ++j)
@@ -463,9 +469,17 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             upk(t2, tt[2 * p], tt[2 * p + 1]);
         }
         if (tail) {
+            // the pairwise form may flag elements that are not deep-tail
+            // (it tests |t|): those are recomputed by the scalar form
 #pragma unroll
-            for (int j = 0; j < VE; ++j)
-                if (Op::is_tail(xf[j], k, ch[j])) Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
+            for (int j = 0; j < VE; ++j) {
+                if (Op::is_tail(xf[j], k, ch[j])) {
+                    Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
+                } else {
+                    bool unused = false;
+                    Op::template bwd<P>(xf[j], gf[j], k, ch[j], unused, o[j], tt[j]);
+                }
+            }
         }
 #pragma unroll
         for (int p = 0; p < VE / 2; ++p)
@@ -476,10 +490,10 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     };
     clear();
 
-    int it = 0;
+    int it = 0, s = 0;
+    uint32_t phase = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-        const int s = it % stages;
-        if (!mbar_wait(smem_addr(full + s), (it / stages) & 1)) {
+        if (!mbar_wait(smem_addr(full + s), phase & 1)) {
             atomicExch(err, 1u);
             break;
         }
@@ -498,6 +512,10 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
 #pragma unroll
         for (int u = 0; u < UT; ++u) L::store(out, u * consumers, unit(xv[u], gv[u]));
         if ((it + 1) % kPipeFlushTiles == 0) flush();
+        if (++s == stages) {
+            s = 0;
+            ++phase;
+        }
     }
     // The partial tile at the end, if any, belongs to block ntiles % grid.
     if (ntiles * tile_units < nunits && blockIdx.x == ntiles % gridDim.x) {
