@@ -42,6 +42,45 @@ __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, flo
     upk(mul2(pk(d0, d1), mul2(s, r)), o0, o1);
 }
 
+// GELU-tanh for two elements of bf16 storage: t = z (c1 + c3 z^2) as in
+// GeluTanh, E = 2^t, s = 1 / (1 + E) = Sigmoid(v), Sigmoid(-v) = E s, and
+//   y = z s,   dz = dy (s (1 + z v' E s)),  v' = k1 + 3 k3 z^2,
+// The forward flags t > kTailT (deep negative z) for the tail form; the
+// backward uses swish_df2_bf16's rule (|t| > kTailT flags the element for
+// the scalar form; inside, z v' E s is finite).
+template <bool kBothSides>
+__device__ __forceinline__ F2 gelu_tanh_parts2(F2 z, F2 &z2, bool &tail, F2 &E)
+{
+    z2 = mul2(z, z);
+    float t0, t1;
+    upk(mul2(z, fma2(sp2(GeluTanh::kC3f), z2, sp2(GeluTanh::kC1f))), t0, t1);
+    const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
+    if constexpr (kBothSides)
+        tail |= (fabsf(t0) > kTailT) | (fabsf(t1) > kTailT);
+    else
+        tail |= (t0 > kTailT) | (t1 > kTailT);
+    E = pk(e0, e1);
+    float a0, a1;
+    upk(add2(sp2(1.f), E), a0, a1);
+    return pk(rcp_ftz(a0), rcp_ftz(a1));
+}
+__device__ __forceinline__ void gelu_tanh_f2_bf16(float z0, float z1, bool &tail, float &o0, float &o1)
+{
+    const F2 z = pk(z0, z1);
+    F2 z2, E;
+    upk(mul2(z, gelu_tanh_parts2<false>(z, z2, tail, E)), o0, o1);
+}
+__device__ __forceinline__ void gelu_tanh_df2_bf16(float z0, float z1, float d0, float d1, bool &tail, float &o0,
+                                                   float &o1)
+{
+    const F2 z = pk(z0, z1);
+    F2 z2, E;
+    const F2 s = gelu_tanh_parts2<true>(z, z2, tail, E);
+    const F2 q = mul2(z, fma2(sp2(GeluTanh::kK3x3f), z2, sp2(GeluTanh::kK1f)));
+    const F2 r = fma2(q, mul2(E, s), sp2(1.f));
+    upk(mul2(pk(d0, d1), mul2(s, r)), o0, o1);
+}
+
 template <class A>
 struct AffineOp {
     static constexpr int NR = 2;   // dgamma, dbeta
@@ -97,6 +136,8 @@ struct AffineOp {
         upk(fma2(h.g, x, h.b), z0, z1);
         if constexpr (HasPairs<A, P>::value) {
             A::f2(z0, z1, k, tail, o0, o1);
+        } else if constexpr (std::is_same<A, GeluTanh>::value && !P) {
+            gelu_tanh_f2_bf16(z0, z1, tail, o0, o1);
         } else {
             o0 = A::template f<P>(z0, k, tail);
             o1 = A::template f<P>(z1, k, tail);
@@ -113,6 +154,8 @@ struct AffineOp {
             A::df2(z0, z1, d0, d1, k, tail, o0, o1);
         } else if constexpr (std::is_same<A, Swish>::value && !P) {
             swish_df2_bf16(z0, z1, d0, d1, k, tail, o0, o1);
+        } else if constexpr (std::is_same<A, GeluTanh>::value && !P) {
+            gelu_tanh_df2_bf16(z0, z1, d0, d1, tail, o0, o1);
         } else {
             o0 = A::template df<P>(z0, d0, k, tail);
             o1 = A::template df<P>(z1, d1, k, tail);

@@ -49,6 +49,15 @@ __device__ __forceinline__ float ex2_ftz(float t)
     return r;
 }
 
+// The MUFU hyperbolic tangent (tanh.approx.f32, sm_75 and later; the PTX ISA
+// states a maximum relative error of about 2^-11, a quarter of a bf16 ulp or
+// less).  Used for bf16 storage only.
+__device__ __forceinline__ float tanh_mufu(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ float rcp_ftz(float v)
 {
     float r;
@@ -236,7 +245,7 @@ struct Sigmoid {
 };
 
 // ----------------------------------------------------------------- Tanh
-// Forward: CUDA's tanhf.  Backward: 1 - tanh^2 x = 4 Sigmoid(2|x|)
+// Forward: CUDA's tanhf for fp32 storage, the MUFU tanh for bf16.  Backward: 1 - tanh^2 x = 4 Sigmoid(2|x|)
 // Sigmoid(-2|x|) = 4 E s^2 with E = 2^t, t = -2|x| log2 e (t <= 0),
 // s = 1/(1+E) = Sigmoid(2|x|) and Sigmoid(-2|x|) = E s.
 struct Tanh {
@@ -254,10 +263,17 @@ struct Tanh {
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &, bool &)
     {
-        return tanhf(x);
+        if constexpr (P)
+            return tanhf(x);
+        else
+            return tanh_mufu(x);
     }
     template <bool P>
-    static __device__ __forceinline__ float f_tail(float x, const Coef &) { return tanhf(x); }
+    static __device__ __forceinline__ float f_tail(float x, const Coef &k)
+    {
+        bool unused = false;
+        return f<P>(x, k, unused);
+    }
     template <bool P>
     static __device__ __forceinline__ float df(float x, float dy, const Coef &k, bool &tail)
     {
