@@ -162,9 +162,12 @@ struct NhwcCfg;
 #define MEA_NHWC_BWD_U 2
 #endif
 // U_PIPE: units per consumer thread per tile of the pipelined backward.
+#ifndef MEA_PIPE_UT_BF16
+#define MEA_PIPE_UT_BF16 4
+#endif
 template <>
 struct NhwcCfg<Bf16> {
-    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U, U_PIPE = 4;
+    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U, U_PIPE = MEA_PIPE_UT_BF16;
 };
 template <>
 struct NhwcCfg<float> {
@@ -351,8 +354,15 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
 // then `stages` x {x tile, dy tile}.
 constexpr int kPipeMaxStages = 8;
 constexpr int kPipeHeader = 256;
-// 64 registers: three blocks of 288 + 32 threads (C = 144) per SM.
-constexpr int kPipeMaxRegs = 64;
+// 96 registers: two blocks of 288 + 32 threads (C = 144) per SM.  Against
+// three blocks of 64 registers (3 stages each), two blocks of 96 with 5
+// stages each keep more bytes in flight and more independent elements per
+// thread: measured on [128, 56, 56, 144] bf16, Swish 0.83 -> 0.87 of copy
+// bandwidth, GELU-tanh 0.79 -> 0.84, ReLU unchanged.
+#ifndef MEA_PIPE_MAXREGS
+#define MEA_PIPE_MAXREGS 96
+#endif
+constexpr int kPipeMaxRegs = MEA_PIPE_MAXREGS;
 // Tiles whose fp32 sums a consumer thread carries before adding them to its
 // fp64 sums (kPipeFlushTiles * UT terms per channel in fp32).
 constexpr int kPipeFlushTiles = 4;
@@ -695,11 +705,17 @@ inline bool nhwc_fast(const AffineLaunch &a)
 }
 
 // Pipelined backward: shared memory per block is held to kPipeSmemBudget so
-// that three blocks fit an SM (228 KB, 1 KB of it reserved per block), and
-// the grid is at most kPipeGrid blocks (one wave of three per SM on a B200;
+// that two blocks fit an SM (228 KB, 1 KB of it reserved per block), and
+// the grid is at most kPipeGrid blocks (one wave of two per SM on a B200;
 // a constant, so the summation order does not depend on the device).
-constexpr int kPipeSmemBudget = 75 * 1024;
-constexpr int kPipeGrid = 444;
+#ifndef MEA_PIPE_SMEM_KB
+#define MEA_PIPE_SMEM_KB 110
+#endif
+#ifndef MEA_PIPE_GRID
+#define MEA_PIPE_GRID 296
+#endif
+constexpr int kPipeSmemBudget = MEA_PIPE_SMEM_KB * 1024;
+constexpr int kPipeGrid = MEA_PIPE_GRID;
 
 struct PipeShape {
     int stages;          // 0: the pipelined kernel is not used
