@@ -42,6 +42,20 @@ __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, flo
     upk(mul2(pk(d0, d1), mul2(s, r)), o0, o1);
 }
 
+// Swish (y = z Sigmoid(alpha z)) and the sigmoid for two elements of bf16
+// storage: the operations of Swish::f<false> / Sigmoid::f<false> with the
+// multiplies and adds as packed .f32x2 pairs, bitwise the scalar results.
+__device__ __forceinline__ F2 sigmoid_parts2(F2 z, const Coef &k, bool &tail)
+{
+    float t0, t1;
+    upk(mul2(z, sp2(k.c_hi)), t0, t1);
+    const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
+    tail |= (t0 > kTailT) | (t1 > kTailT);
+    float a0, a1;
+    upk(add2(sp2(1.f), pk(e0, e1)), a0, a1);
+    return pk(rcp_ftz(a0), rcp_ftz(a1));
+}
+
 // GELU-tanh for two elements of bf16 storage: t = z (c1 + c3 z^2) as in
 // GeluTanh, E = 2^t, s = 1 / (1 + E) = Sigmoid(v), Sigmoid(-v) = E s, and
 //   y = z s,   dz = dy (s (1 + z v' E s)),  v' = k1 + 3 k3 z^2,
@@ -138,6 +152,11 @@ struct AffineOp {
             A::f2(z0, z1, k, tail, o0, o1);
         } else if constexpr (std::is_same<A, GeluTanh>::value && !P) {
             gelu_tanh_f2_bf16(z0, z1, tail, o0, o1);
+        } else if constexpr (std::is_same<A, Swish>::value && !P) {
+            const F2 z = pk(z0, z1);
+            upk(mul2(z, sigmoid_parts2(z, k, tail)), o0, o1);
+        } else if constexpr (std::is_same<A, Sigmoid>::value && !P) {
+            upk(sigmoid_parts2(pk(z0, z1), k, tail), o0, o1);
         } else {
             o0 = A::template f<P>(z0, k, tail);
             o1 = A::template f<P>(z1, k, tail);

@@ -58,7 +58,10 @@ constexpr int kNhwcBwdGridCap = 888;     // 148 x 6
 #endif
 constexpr int kNhwcBwdMaxRegs = MEA_NHWC_BWD_MAXREGS;
 // Register cap of the NHWC forward: 64 keeps three 288-thread blocks per SM.
-constexpr int kNhwcFwdMaxRegs = 64;
+#ifndef MEA_NHWC_FWD_MAXREGS
+#define MEA_NHWC_FWD_MAXREGS 64
+#endif
+constexpr int kNhwcFwdMaxRegs = MEA_NHWC_FWD_MAXREGS;
 constexpr int kPlaneThreads = 256;
 constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks
 
@@ -165,9 +168,12 @@ struct NhwcCfg;
 #ifndef MEA_PIPE_UT_BF16
 #define MEA_PIPE_UT_BF16 4
 #endif
+#ifndef MEA_NHWC_FWD_U_BF16
+#define MEA_NHWC_FWD_U_BF16 16
+#endif
 template <>
 struct NhwcCfg<Bf16> {
-    static constexpr int VE = 4, U_FWD = 16, U_BWD = MEA_NHWC_BWD_U, U_PIPE = MEA_PIPE_UT_BF16;
+    static constexpr int VE = 4, U_FWD = MEA_NHWC_FWD_U_BF16, U_BWD = MEA_NHWC_BWD_U, U_PIPE = MEA_PIPE_UT_BF16;
 };
 template <>
 struct NhwcCfg<float> {
