@@ -1,0 +1,68 @@
+"""Host-side checks of the polynomial constants the bf16 GELU-erf kernels use
+(mea_math.cuh, GeluErf::nr_parts and GeluErf::nr5_parts), read from the
+source text and evaluated in float64 against scipy's scaled complementary
+error function.  Both approximate log(erfc(a) / t) + a^2 by a polynomial in
+t = 1 / (1 + a / 2) (Press et al., "Numerical Recipes in C", 2nd ed.,
+section 6.2); the claims checked are the fractional error bounds that the
+kernel comments and the design notes state: 1.2e-7 for the degree-9 form
+(the published bound) and 7.7e-6 for the degree-5 refit, over the range
+each is used on (a up to 9.6, where the kernels' tail branch takes over).
+"""
+import os
+import re
+
+import numpy as np
+from scipy.special import erfcx
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "memory_efficient_activation_b200", "csrc", "mea_math.cuh")
+
+
+def _horner_coefficients(func: str) -> list[float]:
+    """The Horner chain of `func` in GeluErf, highest degree first."""
+    text = open(SRC).read()
+    start = text.index("struct GeluErf")
+    body = text[text.index(f"float {func}(float a, float &t)", start):]
+    body = body[:body.index("return")]
+    first = float(re.search(r"float p = ([-0-9.eE]+)f;", body).group(1))
+    rest = [float(v) for v in re.findall(r"p = fmaf\(p, t, ([-0-9.eE]+)f\);", body)]
+    return [first] + rest
+
+
+def _max_fractional_error(coef_high_first, a_max=9.6, points=200001):
+    a = np.linspace(0.0, a_max, points)
+    t = 1.0 / (1.0 + a / 2.0)
+    coef32 = np.array(coef_high_first, dtype=np.float32).astype(np.float64)
+    p = np.polyval(coef32, t)
+    # erfc(a) = t exp(-a^2 + P(t)) and erfcx(a) = exp(a^2) erfc(a)
+    approx_over_exact = t * np.exp(p) / erfcx(a)
+    return float(np.max(np.abs(approx_over_exact - 1.0)))
+
+
+def test_degree9_matches_published_bound():
+    c = _horner_coefficients("nr_parts")
+    assert len(c) == 10
+    assert _max_fractional_error(c) < 1.2e-7
+
+
+def test_degree5_refit_bound():
+    c = _horner_coefficients("nr5_parts")
+    assert len(c) == 6
+    err = _max_fractional_error(c)
+    assert err < 7.7e-6
+    # far inside half a bf16 ulp (2^-9 relative), the forward's output precision
+    assert err < 2.0 ** -9 / 100
+
+
+def test_degree5_is_the_fit_script_result():
+    import importlib.util
+    path = os.path.join(os.path.dirname(SRC), "fit_erfc_bf16.py")
+    spec = importlib.util.spec_from_file_location("fit_erfc_bf16", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    coef, err = mod.fit(points=100001, iterations=120)
+    kernel = np.array(_horner_coefficients("nr5_parts")[::-1], dtype=np.float32)
+    # the refit with fewer points lands on the same fp32 constants to within
+    # a few ulps of each (the Lawson iteration converges to the same minimax)
+    assert np.allclose(coef, kernel, rtol=1e-4, atol=1e-5), (coef, kernel)
+    assert err < 7.7e-6
