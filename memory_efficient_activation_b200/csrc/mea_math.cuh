@@ -318,14 +318,48 @@ struct Tanh {
 //
 // The bf16 forward uses the same form with a degree-5 polynomial fitted
 // here (csrc/fit_erfc_bf16.py: near-minimax over |w| <= 9.6, error of
-// log erfc below 7.7e-6, far inside the bf16 rounding of the result); the
-// backward, whose value cancels near x = -0.75, keeps the degree-9 one.
+// log erfc below 7.7e-6, far inside the bf16 rounding of the result).  The
+// backward, whose value cancels near x = -0.75, needs the full accuracy; it
+// writes erfc(|w|) = t e^(-w^2) Q(t) with Q(t) = erfcx(|w|) / t fitted as a
+// degree-8 polynomial (same script; fractional error 5e-8 in exact
+// arithmetic, about 2e-7 evaluated in fp32, as the degree-9 form), so that
+// the Gaussian e^(-w^2) of f' is the only exponential.  Its tail test is on
+// that exponential's argument (-w^2 log2 e < -124); the deep-tail recompute
+// is the scaled form above.
 struct GeluErf {
     static constexpr float kNegRsqrt2Hi = -0.707106769084930419921875f;
     static constexpr float kNegRsqrt2Lo = -1.2101617104478969362e-08f;
     static constexpr float kTwoRsqrtPi = 1.12837916709551257f;     // 2 / sqrt(pi)
     static constexpr float kRsqrt2Pi = 0.398942280401432678f;      // 1 / sqrt(2 pi)
     static constexpr float kLog2ef = 1.44269504088896340736f;
+    // Backward: erfc(a) = t e^(-a^2) Q(t), t = 1 / (1 + a / 2), with
+    // Q(t) = erfcx(a) / t fitted directly (degree 8, coefficients of t^0 ..
+    // t^8; csrc/fit_erfc_bf16.py), so that the one exponential e^(-a^2)
+    // serves both erfc and the Gaussian of f' (q8, q8_2).
+    static __device__ __forceinline__ float q8(float t)
+    {
+        float q = -0.058932472f;
+        q = fmaf(q, t, 0.283905655f);
+        q = fmaf(q, t, -0.485806316f);
+        q = fmaf(q, t, 0.276463121f);
+        q = fmaf(q, t, -0.0255132243f);
+        q = fmaf(q, t, 0.202212647f);
+        q = fmaf(q, t, 0.243224636f);
+        q = fmaf(q, t, 0.282358527f);
+        return fmaf(q, t, 0.282087386f);
+    }
+    static __device__ __forceinline__ F2 q8_2(F2 t)
+    {
+        F2 q = sp2(-0.058932472f);
+        q = fma2(q, t, sp2(0.283905655f));
+        q = fma2(q, t, sp2(-0.485806316f));
+        q = fma2(q, t, sp2(0.276463121f));
+        q = fma2(q, t, sp2(-0.0255132243f));
+        q = fma2(q, t, sp2(0.202212647f));
+        q = fma2(q, t, sp2(0.243224636f));
+        q = fma2(q, t, sp2(0.282358527f));
+        return fma2(q, t, sp2(0.282087386f));
+    }
 
     static __device__ __forceinline__ Coef coef(float) { return Coef{1.f, 0.f, 0.f}; }
 
@@ -436,16 +470,21 @@ struct GeluErf {
                                                float &o0, float &o1)
     {
         const F2 x = pk(x0, x1);
-        float w0, w1, u0, u1;
-        F2 t, u;
-        nr_parts2(x, w0, w1, t, u);
-        upk(u, u0, u1);
-        tail |= ((u0 < -kTailT) && (x0 < 0.f)) || ((u1 < -kTailT) && (x1 < 0.f));
-        const F2 ec = erfc2(w0, w1, t, u0, u1);
-        const F2 w = pk(w0, w1);
+        const F2 w = mul2(x, sp2(kNegRsqrt2Hi));
+        float w0, w1;
+        upk(w, w0, w1);
+        const F2 a = pk(fabsf(w0), fabsf(w1));
+        float d0, d1;
+        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
+        const F2 t = pk(rcp_ftz(d0), rcp_ftz(d1));
+        const F2 q = q8_2(t);
         float v0, v1;
         upk(mul2(mul2(w, w), sp2(-kLog2ef)), v0, v1);
+        tail |= ((v0 < -kTailT) && (x0 < 0.f)) || ((v1 < -kTailT) && (x1 < 0.f));
         const F2 g = pk(ex2_ftz(v0), ex2_ftz(v1));
+        float a0, a1;
+        upk(mul2(mul2(t, q), g), a0, a1);
+        const F2 ec = pk(w0 >= 0.f ? a0 : 2.f - a0, w1 >= 0.f ? a1 : 2.f - a1);
         const F2 d = fma2(mul2(x, sp2(kRsqrt2Pi)), g, mul2(sp2(0.5f), ec));
         upk(mul2(pk(dy0, dy1), d), o0, o1);
     }
@@ -490,12 +529,13 @@ struct GeluErf {
             return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
         } else {
             const float w = x * kNegRsqrt2Hi;
-            float t;
-            const float u = nr_parts(fabsf(w), t);
-            tail |= (u < -kTailT) && (x < 0.f);
-            const float ans = t * ex2_ftz(u);
+            const float t = rcp_ftz(fmaf(0.5f, fabsf(w), 1.0f));
+            const float q = q8(t);
+            const float v = (w * w) * -kLog2ef;
+            tail |= (v < -kTailT) && (x < 0.f);
+            const float g = ex2_ftz(v);
+            const float ans = (t * q) * g;
             const float ec = w >= 0.f ? ans : 2.f - ans;
-            const float g = ex2_ftz(-(w * w) * kLog2ef);
             return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
         }
     }

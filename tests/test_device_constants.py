@@ -1,12 +1,15 @@
 """Host-side checks of the polynomial constants the bf16 GELU-erf kernels use
-(mea_math.cuh, GeluErf::nr_parts and GeluErf::nr5_parts), read from the
-source text and evaluated in float64 against scipy's scaled complementary
-error function.  Both approximate log(erfc(a) / t) + a^2 by a polynomial in
-t = 1 / (1 + a / 2) (Press et al., "Numerical Recipes in C", 2nd ed.,
-section 6.2); the claims checked are the fractional error bounds that the
-kernel comments and the design notes state: 1.2e-7 for the degree-9 form
-(the published bound) and 7.7e-6 for the degree-5 refit, over the range
-each is used on (a up to 9.6, where the kernels' tail branch takes over).
+(mea_math.cuh, GeluErf::nr_parts, nr5_parts and q8), read from the source
+text and evaluated in float64 against scipy's scaled complementary error
+function.  All are polynomials in t = 1 / (1 + a / 2) (Press et al.,
+"Numerical Recipes in C", 2nd ed., section 6.2).  nr_parts and nr5_parts
+approximate log(erfc(a) / t) + a^2; q8 approximates erfcx(a) / t.  The
+claims checked are the fractional error bounds that the kernel comments and
+the design notes state, over the range each is used on (a up to 9.6, where
+the kernels' tail branch takes over):
+  - 1.2e-7 for the degree-9 form (the published bound);
+  - 7.7e-6 for the degree-5 refit;
+  - 5e-8 for the degree-8 Q.
 """
 import os
 import re
@@ -26,6 +29,17 @@ def _horner_coefficients(func: str) -> list[float]:
     body = body[:body.index("return")]
     first = float(re.search(r"float p = ([-0-9.eE]+)f;", body).group(1))
     rest = [float(v) for v in re.findall(r"p = fmaf\(p, t, ([-0-9.eE]+)f\);", body)]
+    return [first] + rest
+
+
+def _q8_coefficients() -> list[float]:
+    """q8's Horner chain, highest degree first."""
+    text = open(SRC).read()
+    start = text.index("struct GeluErf")
+    body = text[text.index("float q8(float t)", start):]
+    body = body[:body.index("}")]
+    first = float(re.search(r"float q = ([-0-9.eE]+)f;", body).group(1))
+    rest = [float(v) for v in re.findall(r"fmaf\(q, t, ([-0-9.eE]+)f\)", body)]
     return [first] + rest
 
 
@@ -66,3 +80,23 @@ def test_degree5_is_the_fit_script_result():
     # a few ulps of each (the Lawson iteration converges to the same minimax)
     assert np.allclose(coef, kernel, rtol=1e-4, atol=1e-5), (coef, kernel)
     assert err < 7.7e-6
+
+
+def test_q8_bound_and_fit():
+    c = _q8_coefficients()
+    assert len(c) == 9
+    a = np.linspace(0.0, 9.6, 200001)
+    t = 1.0 / (1.0 + a / 2.0)
+    q = np.polyval(np.array(c, dtype=np.float32).astype(np.float64), t)
+    # erfc(a) = t e^(-a^2) Q(t)  <=>  Q(t) = erfcx(a) / t
+    err = float(np.max(np.abs(q * t / erfcx(a) - 1.0)))
+    assert err < 5e-8
+    assert abs(q[0] - 1.0) < 1e-7          # a = 0: erfc(0) = 1 = t Q(t) with t = 1
+    import importlib.util
+    path = os.path.join(os.path.dirname(SRC), "fit_erfc_bf16.py")
+    spec = importlib.util.spec_from_file_location("fit_erfc_bf16", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    coef, ferr = mod.fit_q(points=100001, iterations=100)
+    assert np.allclose(coef, np.array(c[::-1], dtype=np.float32), rtol=1e-4, atol=1e-6), (coef, c)
+    assert ferr < 1e-7                      # a shorter refit, less converged
