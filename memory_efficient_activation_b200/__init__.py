@@ -462,6 +462,12 @@ def act_fwd_bwd_host(act: str, hx: torch.Tensor, hdy: torch.Tensor, param: float
         raise ValueError("hx and hdy must be host tensors")
     if hx.shape != hdy.shape or hx.dtype != hdy.dtype:
         raise ValueError("hx and hdy must match")
+    for name, out in (("hy", hy), ("hdx", hdx)):
+        # results are copied into the flat view of the output, so it must be
+        # that tensor's own storage: contiguous, on the host, same size and dtype
+        if out is not None and (out.is_cuda or not out.is_contiguous() or out.numel() != hx.numel()
+                                or out.dtype != hx.dtype):
+            raise ValueError(f"{name} must be a contiguous host tensor with hx's size and dtype")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     n = hx.numel()
     hy = torch.empty_like(hx).pin_memory() if hy is None else hy

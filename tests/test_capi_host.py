@@ -222,3 +222,23 @@ def test_concat_bn_validation(lib):
     D = _capi.ptr_array([0x1000000 + 2, 0x8000000])  # partial overlap with its own piece
     assert b(1, 2, P, ch, 4, 9, Yb, G, B, Mu, Is, D, 0, 0x3400000, 0x3500000, Wk, ws, None) \
         == _capi.MEA_ERR_INVALID_ARG
+
+
+def test_host_pipeline_validates_outputs():
+    import torch
+    import memory_efficient_activation_b200 as mea
+    # results are copied into the flat view of hy / hdx: a tensor whose
+    # reshape would be a copy (non-contiguous), or of another size or dtype,
+    # is refused before any device work
+    x = torch.zeros(64, dtype=torch.bfloat16)
+    dy = torch.zeros(64, dtype=torch.bfloat16)
+    bad = [torch.zeros(128, dtype=torch.bfloat16)[::2],          # non-contiguous
+           torch.zeros(63, dtype=torch.bfloat16),
+           torch.zeros(64, dtype=torch.float32)]
+    for b in bad:
+        with pytest.raises(ValueError):
+            mea.act_fwd_bwd_host("swish", x, dy, hy=b)
+        with pytest.raises(ValueError):
+            mea.act_fwd_bwd_host("swish", x, dy, hdx=b)
+    with pytest.raises(ValueError):
+        mea.act_fwd_bwd_host("swish", x, dy[:32])
