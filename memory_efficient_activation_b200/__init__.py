@@ -69,6 +69,29 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+def _like(ref: torch.Tensor, t: torch.Tensor, name: str) -> torch.Tensor:
+    """A tensor the kernels read or write with ref's layout: contiguous, on
+    ref's device, with ref's dtype and element count (anything else would
+    make the kernel run off its end or onto another device)."""
+    _need_cuda(t)
+    if t.device != ref.device or t.dtype != ref.dtype or t.numel() != ref.numel():
+        raise ValueError(f"{name} must be a contiguous tensor on {ref.device} with x's dtype and size")
+    return t
+
+
+def _on_device(ref: torch.Tensor, t: torch.Tensor, name: str, dtype=None, numel=None) -> torch.Tensor:
+    """A companion tensor (parameter, gradient, workspace) on ref's device,
+    contiguous, optionally of a given dtype and at least `numel` elements."""
+    _need_cuda(t)
+    if t.device != ref.device:
+        raise ValueError(f"{name} must be on {ref.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} needs at least {numel} elements")
+    return t
+
+
 def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
@@ -134,10 +157,9 @@ def act_fwd(act: str, x: torch.Tensor, param: float = 1.0, param_dev: torch.Tens
     """y = f(x).  param: alpha (Swish) or slope (LeakyReLU); param_dev: an
     optional one-element fp32 CUDA tensor read on the device instead."""
     _need_cuda(x)
-    y = torch.empty_like(x) if out is None else out
-    _need_cuda(y)
+    y = torch.empty_like(x) if out is None else _like(x, out, "out")
     if param_dev is not None:
-        _need_cuda(param_dev)
+        _on_device(x, param_dev, "param_dev", torch.float32, 1)
     st = _capi.lib().mea_act_fwd(_act_id(act), _dtype_id(x), x.data_ptr(), y.data_ptr(), x.numel(),
                                   float(param), _ptr(param_dev), _stream(x))
     _capi.check("mea_act_fwd", st)
@@ -152,16 +174,17 @@ def act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, param: float = 1.0,
     _need_cuda(x, dy)
     if dy.dtype != x.dtype or dy.shape != x.shape:
         raise ValueError("dy must match x in dtype and shape")
-    dx = torch.empty_like(x) if out is None else out
-    _need_cuda(dx)
+    _like(x, dy, "dy")
+    dx = torch.empty_like(x) if out is None else _like(x, out, "out")
     ws_ptr, ws_bytes = None, 0
     if dparam is not None:
-        _need_cuda(dparam)
+        _on_device(x, dparam, "dparam", torch.float32, 1)
         ws_bytes = act_bwd_workspace_bytes(act, x.numel(), True)
-        ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), ws_bytes)
+        ws = _on_device(x, workspace, "workspace") if workspace is not None else \
+            _pool.get(x.device, _stream(x), ws_bytes)
         ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
     if param_dev is not None:
-        _need_cuda(param_dev)
+        _on_device(x, param_dev, "param_dev", torch.float32, 1)
     st = _capi.lib().mea_act_bwd(_act_id(act), _dtype_id(x), x.data_ptr(), dy.data_ptr(), dx.data_ptr(),
                                   x.numel(), float(param), _ptr(param_dev), _ptr(dparam), ws_ptr, ws_bytes,
                                   _stream(x))
@@ -181,11 +204,13 @@ def _affine_shape(x: torch.Tensor, layout: str):
     return (N, C, H, W)
 
 
-def _chan_params(C: int, *ps):
+def _chan_params(C: int, *ps, device=None):
     for p in ps:
         _need_cuda(p)
         if p.dtype != torch.float32 or p.numel() != C:
             raise ValueError(f"per-channel parameters must be fp32 with {C} elements")
+        if device is not None and p.device != device:
+            raise ValueError(f"per-channel parameters must be on {device}")
 
 
 def affine_swish_fwd(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, layout: str = "nhwc",
@@ -194,9 +219,8 @@ def affine_swish_fwd(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, l
     'nhwc' or (N, C, H, W) for 'nchw'; gamma and beta are fp32 [C]."""
     _need_cuda(x)
     shape = _affine_shape(x, layout)
-    _chan_params(shape[1], gamma, beta)
-    y = torch.empty_like(x) if out is None else out
-    _need_cuda(y)
+    _chan_params(shape[1], gamma, beta, device=x.device)
+    y = torch.empty_like(x) if out is None else _like(x, out, "out")
     st = _capi.lib().mea_affine_swish_fwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
                                            gamma.data_ptr(), beta.data_ptr(), y.data_ptr(), _stream(x))
     _capi.check("mea_affine_swish_fwd", st)
@@ -213,13 +237,14 @@ def affine_swish_bwd(x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, bet
         raise ValueError("dy must match x in dtype and shape")
     shape = _affine_shape(x, layout)
     C = shape[1]
-    _chan_params(C, gamma, beta)
-    dx = torch.empty_like(x) if out is None else out
+    _chan_params(C, gamma, beta, device=x.device)
+    _like(x, dy, "dy")
+    dx = torch.empty_like(x) if out is None else _like(x, out, "out")
     dg = torch.empty(C, dtype=torch.float32, device=x.device) if dgamma is None else dgamma
     db = torch.empty(C, dtype=torch.float32, device=x.device) if dbeta is None else dbeta
-    _need_cuda(dx, dg, db)
+    _chan_params(C, dg, db, device=x.device)
     need = affine_swish_bwd_workspace_bytes(x.dtype, layout, shape)
-    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    ws = _on_device(x, workspace, "workspace") if workspace is not None else _pool.get(x.device, _stream(x), need)
     st = _capi.lib().mea_affine_swish_bwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
                                            dy.data_ptr(), gamma.data_ptr(), beta.data_ptr(), dx.data_ptr(),
                                            dg.data_ptr(), db.data_ptr(), ws.data_ptr(),
@@ -234,9 +259,8 @@ def affine_act_fwd(act: str, x: torch.Tensor, gamma: torch.Tensor, beta: torch.T
     (param: LeakyReLU slope or Swish alpha)."""
     _need_cuda(x)
     shape = _affine_shape(x, layout)
-    _chan_params(shape[1], gamma, beta)
-    y = torch.empty_like(x) if out is None else out
-    _need_cuda(y)
+    _chan_params(shape[1], gamma, beta, device=x.device)
+    y = torch.empty_like(x) if out is None else _like(x, out, "out")
     st = _capi.lib().mea_affine_act_fwd(_act_id(act), _dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape),
                                          x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), float(param),
                                          y.data_ptr(), _stream(x))
@@ -254,13 +278,14 @@ def affine_act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, gamma: torch.Ten
         raise ValueError("dy must match x in dtype and shape")
     shape = _affine_shape(x, layout)
     C = shape[1]
-    _chan_params(C, gamma, beta)
-    dx = torch.empty_like(x) if out is None else out
+    _chan_params(C, gamma, beta, device=x.device)
+    _like(x, dy, "dy")
+    dx = torch.empty_like(x) if out is None else _like(x, out, "out")
     dg = torch.empty(C, dtype=torch.float32, device=x.device) if dgamma is None else dgamma
     db = torch.empty(C, dtype=torch.float32, device=x.device) if dbeta is None else dbeta
-    _need_cuda(dx, dg, db)
+    _chan_params(C, dg, db, device=x.device)
     need = affine_act_bwd_workspace_bytes(x.dtype, layout, shape)
-    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    ws = _on_device(x, workspace, "workspace") if workspace is not None else _pool.get(x.device, _stream(x), need)
     st = _capi.lib().mea_affine_act_bwd(_act_id(act), _dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape),
                                          x.data_ptr(), dy.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
                                          float(param), dx.data_ptr(), dg.data_ptr(), db.data_ptr(), ws.data_ptr(),
@@ -274,9 +299,8 @@ def swish_channel_fwd(x: torch.Tensor, alpha: torch.Tensor, layout: str = "nchw"
     """y = x Sigmoid(alpha_c x), alpha fp32 [C]."""
     _need_cuda(x)
     shape = _affine_shape(x, layout)
-    _chan_params(shape[1], alpha)
-    y = torch.empty_like(x) if out is None else out
-    _need_cuda(y)
+    _chan_params(shape[1], alpha, device=x.device)
+    y = torch.empty_like(x) if out is None else _like(x, out, "out")
     st = _capi.lib().mea_swish_channel_fwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
                                             alpha.data_ptr(), y.data_ptr(), _stream(x))
     _capi.check("mea_swish_channel_fwd", st)
@@ -292,12 +316,13 @@ def swish_channel_bwd(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, la
         raise ValueError("dy must match x in dtype and shape")
     shape = _affine_shape(x, layout)
     C = shape[1]
-    _chan_params(C, alpha)
-    dx = torch.empty_like(x) if out is None else out
+    _chan_params(C, alpha, device=x.device)
+    _like(x, dy, "dy")
+    dx = torch.empty_like(x) if out is None else _like(x, out, "out")
     da = torch.empty(C, dtype=torch.float32, device=x.device) if dalpha is None else dalpha
-    _need_cuda(dx, da)
+    _chan_params(C, da, device=x.device)
     need = swish_channel_bwd_workspace_bytes(x.dtype, layout, shape)
-    ws = workspace if workspace is not None else _pool.get(x.device, _stream(x), need)
+    ws = _on_device(x, workspace, "workspace") if workspace is not None else _pool.get(x.device, _stream(x), need)
     st = _capi.lib().mea_swish_channel_bwd(_dtype_id(x), LAYOUT_IDS[layout], _capi.shape4(shape), x.data_ptr(),
                                             dy.data_ptr(), alpha.data_ptr(), dx.data_ptr(), da.data_ptr(),
                                             ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))

@@ -242,3 +242,85 @@ def test_host_pipeline_validates_outputs():
             mea.act_fwd_bwd_host("swish", x, dy, hdx=b)
     with pytest.raises(ValueError):
         mea.act_fwd_bwd_host("swish", x, dy[:32])
+
+
+def test_binding_companion_tensor_checks(monkeypatch):
+    # the device-independent part of the checks on outputs and companion
+    # tensors (device placement itself needs a GPU): dtype, size, contiguity
+    import torch
+    import memory_efficient_activation_b200 as mea
+    monkeypatch.setattr(mea, "_need_cuda", lambda *ts: None)
+    ref = torch.zeros(10, dtype=torch.bfloat16)
+    assert mea._like(ref, torch.zeros(10, dtype=torch.bfloat16), "out") is not None
+    for bad in (torch.zeros(10, dtype=torch.float32), torch.zeros(11, dtype=torch.bfloat16)):
+        with pytest.raises(ValueError):
+            mea._like(ref, bad, "out")
+    mea._on_device(ref, torch.zeros(1), "dparam", torch.float32, 1)
+    with pytest.raises(ValueError):
+        mea._on_device(ref, torch.zeros(1, dtype=torch.bfloat16), "dparam", torch.float32, 1)
+    with pytest.raises(ValueError):
+        mea._on_device(ref, torch.zeros(0), "dparam", torch.float32, 1)
+    mea._chan_params(4, torch.zeros(4), torch.zeros(4), device=torch.device("cpu"))
+    with pytest.raises(ValueError):
+        mea._chan_params(4, torch.zeros(5))
+    with pytest.raises(ValueError):
+        mea._chan_params(4, torch.zeros(4, dtype=torch.float64))
+
+
+class _FakeLib:
+    """Stands in for libmea.so: every entry point returns MEA_OK (0) and
+    records its name, so the binding's marshalling runs on the CPU."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append(name)
+            return 0
+        return fn
+
+
+def test_binding_call_patterns_with_stand_in_library(monkeypatch):
+    # the calling patterns of the modules, tests and benchmark pass the
+    # binding's checks and reach the C ABI; mismatched companions do not
+    import torch
+    import memory_efficient_activation_b200 as mea
+    from memory_efficient_activation_b200 import _capi
+    fake = _FakeLib()
+    monkeypatch.setattr(_capi, "lib", lambda: fake)
+    monkeypatch.setattr(mea, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(mea, "_stream", lambda t: 0)
+    bf = torch.bfloat16
+    x = torch.zeros(2, 4, 4, 16, dtype=bf)
+    dy = torch.zeros_like(x)
+    g, b = torch.ones(16), torch.zeros(16)
+    a1 = torch.tensor([1.5])
+    mea.act_fwd("swish", x, 1.0, out=torch.empty_like(x))
+    mea.act_fwd("swish", x, 0.0, param_dev=a1)
+    mea.act_bwd("swish", x, dy, 1.0, out=dy)                      # dx over dy
+    mea.act_bwd("swish", x, dy, 0.0, param_dev=a1, dparam=torch.empty(1),
+                workspace=torch.zeros(4096, dtype=torch.uint8))
+    mea.affine_swish_fwd(x, g, b, "nhwc", out=torch.empty_like(x))
+    mea.affine_swish_bwd(x, dy, g, b, "nhwc", out=torch.empty_like(x), dgamma=torch.empty(16),
+                         dbeta=torch.empty(16), workspace=torch.zeros(1 << 16, dtype=torch.uint8))
+    mea.affine_act_fwd("gelu_tanh", x, g, b, 1.0, "nhwc")
+    mea.affine_act_bwd("gelu_tanh", x, dy, g, b, 1.0, "nhwc")
+    xc = torch.zeros(2, 16, 4, 4)
+    mea.swish_channel_fwd(xc, g, "nchw", out=torch.empty_like(xc))
+    mea.swish_channel_bwd(xc, torch.zeros_like(xc), g, "nchw", dalpha=torch.empty(16))
+    assert fake.calls.count("mea_act_fwd") == 2 and fake.calls.count("mea_act_bwd") == 2
+    assert "mea_affine_swish_bwd" in fake.calls and "mea_swish_channel_bwd" in fake.calls
+    n = len(fake.calls)
+    for call in (
+        lambda: mea.act_fwd("swish", x, 1.0, out=torch.empty(2, 4, 4, 16)),            # fp32 out for bf16 x
+        lambda: mea.act_bwd("swish", x, dy, 1.0, out=torch.empty(10, dtype=bf)),        # wrong size
+        lambda: mea.act_bwd("swish", x, dy, 0.0, dparam=torch.empty(1, dtype=bf)),      # bf16 d alpha
+        lambda: mea.act_fwd("swish", x, 0.0, param_dev=torch.empty(0)),                # empty alpha
+        lambda: mea.affine_swish_bwd(x, dy, g, b, "nhwc", dgamma=torch.empty(15)),      # dgamma size
+        lambda: mea.swish_channel_bwd(xc, torch.zeros_like(xc), g, "nchw",
+                                      dalpha=torch.empty(16, dtype=torch.float64)),
+    ):
+        with pytest.raises(ValueError):
+            call()
+    assert len(fake.calls) == n                     # nothing reached the library
