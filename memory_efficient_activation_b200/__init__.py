@@ -92,6 +92,14 @@ def _on_device(ref: torch.Tensor, t: torch.Tensor, name: str, dtype=None, numel=
     return t
 
 
+def _shaped(t: torch.Tensor, shape, dtype, device, name: str) -> torch.Tensor:
+    """An output of a given shape, dtype and device (contiguous)."""
+    _need_cuda(t)
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device:
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}")
+    return t
+
+
 def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
@@ -350,13 +358,14 @@ def matmul_act_fwd(act: str, x: torch.Tensor, w: torch.Tensor, param: float = 1.
     N = w.shape[0]
     if w.shape[1] != K:
         raise ValueError("x and w disagree in K")
-    if want_z and z is None:
-        z = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    if want_y and y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    for t in (z, y):
-        if t is not None:
-            _need_cuda(t)
+    if w.device != x.device:
+        raise ValueError("x and w must be on the same device")
+    if want_z:
+        z = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if z is None else \
+            _shaped(z, (M, N), torch.bfloat16, x.device, "z")
+    if want_y:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else \
+            _shaped(y, (M, N), torch.bfloat16, x.device, "y")
     st = _capi.lib().mea_matmul_act_fwd(_act_id(act), M, N, K, x.data_ptr(), w.data_ptr(), float(param),
                                          _ptr(z if want_z else None), _ptr(y if want_y else None), _stream(x))
     _capi.check("mea_matmul_act_fwd", st)
@@ -375,8 +384,9 @@ def matmul_act_bwd(act: str, g: torch.Tensor, w: torch.Tensor, z: torch.Tensor, 
     N = w.shape[0]
     if w.shape[1] != K or z.shape != (M, N):
         raise ValueError("g, w and z disagree in shape")
-    dz = torch.empty_like(z) if out is None else out
-    _need_cuda(dz)
+    if w.device != g.device or z.device != g.device:
+        raise ValueError("g, w and z must be on the same device")
+    dz = torch.empty_like(z) if out is None else _shaped(out, (M, N), torch.bfloat16, g.device, "out")
     st = _capi.lib().mea_matmul_act_bwd(_act_id(act), M, N, K, g.data_ptr(), w.data_ptr(), z.data_ptr(),
                                          float(param), dz.data_ptr(), _stream(g))
     _capi.check("mea_matmul_act_bwd", st)
@@ -392,6 +402,8 @@ def _bn_pieces(pieces):
         _need_cuda(p)
         if p.dim() < 2 or p.shape[0] != N or int(p[0, 0].numel()) != HW or p.dtype != dtype:
             raise ValueError("pieces must share N, the spatial size and the dtype")
+        if p.device != pieces[0].device:
+            raise ValueError("pieces must be on one device")
     chans = [int(p.shape[1]) for p in pieces]
     return N, HW, chans, _capi.ptr_array([p.data_ptr() for p in pieces]), _capi.int64_array(chans)
 
@@ -402,15 +414,18 @@ def concat_bn_relu_fwd(pieces, gamma, beta, eps: float = 1e-5, momentum: float =
     forming the concatenation.  Returns (y, mean, invstd)."""
     N, HW, chans, parr, carr = _bn_pieces(pieces)
     C = sum(chans)
-    _chan_params(C, gamma, beta)
     dev = pieces[0].device
+    _chan_params(C, gamma, beta, device=dev)
+    for r in (running_mean, running_var):
+        if r is not None:
+            _chan_params(C, r, device=dev)
     shape = (N, C) + tuple(pieces[0].shape[2:])
-    y = torch.empty(shape, dtype=pieces[0].dtype, device=dev) if out is None else out
-    _need_cuda(y)
+    y = torch.empty(shape, dtype=pieces[0].dtype, device=dev) if out is None else \
+        _shaped(out, shape, pieces[0].dtype, dev, "out")
     mean = torch.empty(C, dtype=torch.float32, device=dev)
     invstd = torch.empty(C, dtype=torch.float32, device=dev)
     need = int(_capi.lib().mea_concat_bn_relu_workspace_bytes(N, C))
-    ws = workspace if workspace is not None else _pool.get(dev, _stream(y), need)
+    ws = _on_device(y, workspace, "workspace") if workspace is not None else _pool.get(dev, _stream(y), need)
     st = _capi.lib().mea_concat_bn_relu_fwd(_dtype_id(y), len(pieces), parr, carr, N, HW, gamma.data_ptr(),
                                              beta.data_ptr(), float(eps), float(momentum), _ptr(running_mean),
                                              _ptr(running_var), mean.data_ptr(), invstd.data_ptr(), y.data_ptr(),
@@ -424,10 +439,11 @@ def concat_bn_relu_apply(pieces, gamma, beta, mean, invstd, out=None):
     output, bitwise)."""
     N, HW, chans, parr, carr = _bn_pieces(pieces)
     C = sum(chans)
-    _chan_params(C, gamma, beta, mean, invstd)
+    dev = pieces[0].device
+    _chan_params(C, gamma, beta, mean, invstd, device=dev)
     shape = (N, C) + tuple(pieces[0].shape[2:])
-    y = torch.empty(shape, dtype=pieces[0].dtype, device=pieces[0].device) if out is None else out
-    _need_cuda(y)
+    y = torch.empty(shape, dtype=pieces[0].dtype, device=dev) if out is None else \
+        _shaped(out, shape, pieces[0].dtype, dev, "out")
     st = _capi.lib().mea_concat_bn_relu_apply(_dtype_id(y), len(pieces), parr, carr, N, HW, gamma.data_ptr(),
                                                beta.data_ptr(), mean.data_ptr(), invstd.data_ptr(), y.data_ptr(),
                                                _stream(y))
@@ -441,17 +457,19 @@ def concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, invstd, dpieces=None, accu
     xhat are recomputed from the pieces."""
     N, HW, chans, parr, carr = _bn_pieces(pieces)
     C = sum(chans)
-    _need_cuda(dy)
-    _chan_params(C, gamma, beta, mean, invstd)
     dev = pieces[0].device
+    _shaped(dy, (N, C) + tuple(pieces[0].shape[2:]), pieces[0].dtype, dev, "dy")
+    _chan_params(C, gamma, beta, mean, invstd, device=dev)
     if dpieces is None:
         dpieces = [torch.zeros_like(p) if accumulate else torch.empty_like(p) for p in pieces]
-    for d in dpieces:
-        _need_cuda(d)
+    if len(dpieces) != len(pieces):
+        raise ValueError("one gradient tensor per piece")
+    for p, d in zip(pieces, dpieces):
+        _shaped(d, p.shape, p.dtype, dev, "dpieces[i]")
     dg = torch.empty(C, dtype=torch.float32, device=dev)
     db = torch.empty(C, dtype=torch.float32, device=dev)
     need = int(_capi.lib().mea_concat_bn_relu_workspace_bytes(N, C))
-    ws = workspace if workspace is not None else _pool.get(dev, _stream(dy), need)
+    ws = _on_device(dy, workspace, "workspace") if workspace is not None else _pool.get(dev, _stream(dy), need)
     st = _capi.lib().mea_concat_bn_relu_bwd(_dtype_id(dy), len(pieces), parr, carr, N, HW, dy.data_ptr(),
                                              gamma.data_ptr(), beta.data_ptr(), mean.data_ptr(), invstd.data_ptr(),
                                              _capi.ptr_array([d.data_ptr() for d in dpieces]), int(bool(accumulate)),

@@ -324,3 +324,40 @@ def test_binding_call_patterns_with_stand_in_library(monkeypatch):
         with pytest.raises(ValueError):
             call()
     assert len(fake.calls) == n                     # nothing reached the library
+
+
+def test_binding_matmul_and_bn_patterns_with_stand_in_library(monkeypatch):
+    import torch
+    import memory_efficient_activation_b200 as mea
+    from memory_efficient_activation_b200 import _capi
+    fake = _FakeLib()
+    monkeypatch.setattr(_capi, "lib", lambda: fake)
+    monkeypatch.setattr(mea, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(mea, "_stream", lambda t: 0)
+    bf = torch.bfloat16
+    x, w = torch.zeros(16, 8, dtype=bf), torch.zeros(24, 8, dtype=bf)
+    z, y = mea.matmul_act_fwd("swish", x, w)
+    assert z.shape == (16, 24) and y.shape == (16, 24)
+    mea.matmul_act_fwd("swish", x, w, z=torch.empty(16, 24, dtype=bf), want_y=False)
+    g = torch.zeros(16, 8, dtype=bf)
+    mea.matmul_act_bwd("swish", g, w, z, out=z)                     # dz written over z
+    pieces = [torch.zeros(2, 3, 4, 4), torch.zeros(2, 5, 4, 4)]
+    gam, bet = torch.ones(8), torch.zeros(8)
+    yb, mean, invstd = mea.concat_bn_relu_fwd(pieces, gam, bet, 1e-5, 0.1, torch.zeros(8), torch.ones(8),
+                                              out=torch.empty(2, 8, 4, 4))
+    mea.concat_bn_relu_apply(pieces, gam, bet, mean, invstd, out=yb)
+    mea.concat_bn_relu_bwd(pieces, torch.zeros(2, 8, 4, 4), gam, bet, mean, invstd,
+                           dpieces=[torch.zeros_like(p) for p in pieces], accumulate=True)
+    n = len(fake.calls)
+    for call in (
+        lambda: mea.matmul_act_fwd("swish", x, w, z=torch.empty(16, 23, dtype=bf)),
+        lambda: mea.matmul_act_bwd("swish", g, w, z, out=torch.empty(16, 24)),           # fp32 out
+        lambda: mea.concat_bn_relu_fwd(pieces, gam, bet, out=torch.empty(2, 7, 4, 4)),
+        lambda: mea.concat_bn_relu_fwd(pieces, gam, bet, 1e-5, 0.1, torch.zeros(7), torch.ones(8)),
+        lambda: mea.concat_bn_relu_bwd(pieces, torch.zeros(2, 8, 4, 4, dtype=bf), gam, bet, mean, invstd),
+        lambda: mea.concat_bn_relu_bwd(pieces, torch.zeros(2, 8, 4, 4), gam, bet, mean, invstd,
+                                       dpieces=[torch.zeros_like(pieces[0])]),
+    ):
+        with pytest.raises(ValueError):
+            call()
+    assert len(fake.calls) == n
