@@ -489,6 +489,9 @@ class _HostPipe:
 
 
 _host_pipes: dict = {}
+# One pipeline submission at a time: calls from several threads share a
+# device's buffers and streams.
+_host_pipe_lock = threading.Lock()
 
 
 def act_fwd_bwd_host(act: str, hx: torch.Tensor, hdy: torch.Tensor, param: float = 1.0,
@@ -516,10 +519,19 @@ def act_fwd_bwd_host(act: str, hx: torch.Tensor, hdy: torch.Tensor, param: float
     hy = torch.empty_like(hx).pin_memory() if hy is None else hy
     hdx = torch.empty_like(hx).pin_memory() if hdx is None else hdx
     key = (dev, n, hx.dtype)
-    pipe = _host_pipes.get(dev)
-    if pipe is None or pipe.key != key:
-        pipe = _HostPipe(dev, n, hx.dtype)
-        _host_pipes[dev] = pipe
+    with _host_pipe_lock:
+        pipe = _host_pipes.get(dev)
+        if pipe is None or pipe.key != key:
+            if pipe is not None:
+                # the old buffers may still be in use by queued work
+                torch.cuda.current_stream(dev).wait_stream(pipe.streams[2])
+            pipe = _HostPipe(dev, n, hx.dtype)
+            _host_pipes[dev] = pipe
+        return _host_pipe_run(pipe, dev, act, hx, hdy, hy, hdx, param, chunks)
+
+
+def _host_pipe_run(pipe, dev, act, hx, hdy, hy, hdx, param, chunks):
+    n = hx.numel()
     x, dy, y, dx = pipe.bufs
     s_in, s_run, s_out = pipe.streams
     cur = torch.cuda.current_stream(dev)
@@ -527,6 +539,7 @@ def act_fwd_bwd_host(act: str, hx: torch.Tensor, hdy: torch.Tensor, param: float
     step = -(-n // max(1, chunks))
     step = -(-step // 256) * 256                 # pieces start 16-byte aligned
     s_in.wait_stream(cur)
+    s_in.wait_stream(s_out)                      # a previous call's pieces are out of the buffers
     for lo in range(0, n, step):
         hi = min(n, lo + step)
         with torch.cuda.stream(s_in):
