@@ -1,0 +1,78 @@
+/* A plain C99 consumer of include/mea.h: compiled with gcc -std=c99
+ * -pedantic -Werror and linked against libmea.so by test_capi_c.py.  It
+ * makes only calls that the library refuses (or serves as no-ops) during
+ * argument validation, so it runs without a GPU.  Pointer arguments are fake
+ * addresses that no call dereferences.  Prints "ok" and exits 0 when every
+ * check holds; otherwise prints the first failed check and exits 1. */
+#include <stdio.h>
+#include <string.h>
+
+#include "mea.h"
+
+#define CHECK(cond)                                                          \
+    do {                                                                     \
+        if (!(cond)) {                                                       \
+            printf("failed: %s (line %d): %s\n", #cond, __LINE__,            \
+                   mea_last_error());                                        \
+            return 1;                                                        \
+        }                                                                    \
+    } while (0)
+
+int main(void)
+{
+    void *x = (void *)0x100000, *y = (void *)0x200000, *dy = (void *)0x300000, *dx = (void *)0x400000;
+    float *dparam = (float *)0x500000;
+    void *ws = (void *)0x600000;
+    const int64_t shape[4] = {2, 144, 3, 3};
+    const int64_t bad_shape[4] = {2, -1, 3, 3};
+    size_t need;
+
+    CHECK(mea_version() > 0);
+    CHECK(strcmp(mea_status_string(MEA_OK), "") != 0);
+    CHECK(strcmp(mea_status_string(MEA_ERR_CUDA), "") != 0);
+
+    /* n = 0 is a no-op, NULL pointers included, and clears the last error */
+    CHECK(mea_act_fwd(MEA_SWISH, MEA_BF16, NULL, NULL, 0, 1.0f, NULL, NULL) == MEA_OK);
+    CHECK(mea_last_error()[0] == '\0');
+
+    /* bad enums, negative sizes, NULL pointers, overlapping outputs */
+    CHECK(mea_act_fwd((mea_act_t)7, MEA_BF16, x, y, 10, 1.0f, NULL, NULL) == MEA_ERR_INVALID_ARG);
+    CHECK(mea_last_error()[0] != '\0');
+    CHECK(mea_act_fwd(MEA_SWISH, (mea_dtype_t)2, x, y, 10, 1.0f, NULL, NULL) == MEA_ERR_INVALID_ARG);
+    CHECK(mea_act_fwd(MEA_SWISH, MEA_BF16, x, y, -1, 1.0f, NULL, NULL) == MEA_ERR_INVALID_ARG);
+    CHECK(mea_act_fwd(MEA_SWISH, MEA_BF16, NULL, y, 10, 1.0f, NULL, NULL) == MEA_ERR_INVALID_ARG);
+    CHECK(mea_act_fwd(MEA_SWISH, MEA_BF16, x, (char *)x + 2, 10, 1.0f, NULL, NULL) == MEA_ERR_INVALID_ARG);
+
+    /* the d alpha backward needs a workspace of the advertised size */
+    need = mea_act_bwd_workspace_bytes(MEA_SWISH, 1000, 1);
+    CHECK(need >= 8);
+    CHECK(mea_act_bwd(MEA_SWISH, MEA_BF16, x, dy, dx, 1000, 1.0f, NULL, dparam, NULL, need, NULL) ==
+          MEA_ERR_WORKSPACE);
+    CHECK(mea_act_bwd(MEA_SWISH, MEA_BF16, x, dy, dx, 1000, 1.0f, NULL, dparam, ws, need - 1, NULL) ==
+          MEA_ERR_WORKSPACE);
+    CHECK(mea_act_bwd(MEA_RELU, MEA_BF16, x, dy, dx, 1000, 1.0f, NULL, dparam, ws, need, NULL) ==
+          MEA_ERR_UNSUPPORTED);
+
+    /* per-channel entry points */
+    need = mea_affine_swish_bwd_workspace_bytes(MEA_BF16, MEA_NHWC, shape);
+    CHECK(need > 0);
+    CHECK(mea_affine_swish_bwd_workspace_bytes(MEA_BF16, MEA_NHWC, bad_shape) == 0);
+    CHECK(mea_affine_swish_fwd(MEA_BF16, MEA_NHWC, bad_shape, x, (float *)dy, (float *)dx, y, NULL) ==
+          MEA_ERR_INVALID_ARG);
+    CHECK(mea_affine_act_fwd((mea_act_t)9, MEA_BF16, MEA_NHWC, shape, x, (float *)dy, (float *)dx, 1.0f, y,
+                             NULL) == MEA_ERR_INVALID_ARG);
+    CHECK(mea_swish_channel_fwd(MEA_F32, (mea_layout_t)3, shape, x, (float *)dy, y, NULL) ==
+          MEA_ERR_INVALID_ARG);
+
+    /* matmul: K = 0 is not served, N must be a multiple of 8 */
+    CHECK(mea_matmul_act_fwd(MEA_SWISH, 256, 256, 0, x, y, 1.0f, dy, dx, NULL) == MEA_ERR_UNSUPPORTED);
+    CHECK(mea_matmul_act_fwd(MEA_SWISH, 256, 250, 64, x, y, 1.0f, dy, dx, NULL) == MEA_ERR_UNSUPPORTED);
+
+    /* batch normalization: 1..128 pieces are served */
+    CHECK(mea_concat_bn_relu_workspace_bytes(64, 224) > 0);
+    CHECK(mea_concat_bn_relu_apply(MEA_BF16, 0, NULL, NULL, 64, 3136, (float *)dy, (float *)dx, (float *)dy,
+                                   (float *)dx, y, NULL) == MEA_ERR_UNSUPPORTED);
+
+    printf("ok\n");
+    return 0;
+}
