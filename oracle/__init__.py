@@ -26,6 +26,31 @@ Sources (by page and section):
   the backward (concat_bn_relu_fwd / concat_bn_relu_bwd).
 
 Parity pins for every function here live in ``tests/test_oracle_*.py``.
+Each function is checked against something other than itself:
+
+* act_fwd, act_bwd, act_deriv: test_oracle_swish.py and test_oracle_family.py.
+  Checks: closed forms (Swish(0), f'(0) = 1/2, f''(0) = alpha/2, the
+  Lambert-W minimum); odd-part identities; limits; central finite
+  differences; torch float64 autograd; scipy expit / ndtr and the textbook
+  Phi(1).
+* act_bwd_scale: test_oracle_swish.py.  The scale is at least |dx| and equal
+  to it away from the zeros of f'.
+* swish_dalpha: test_oracle_swish.py (finite differences in alpha, brute-force
+  sums) and test_oracle_channel.py (per-channel sums).
+* affine_swish_*, affine_act_*, swish_channel_*: test_oracle_affine.py and
+  test_oracle_channel.py.  Checks: torch autograd; brute force on tiny
+  inputs; finite differences of the parameter gradients; reduction to the
+  plain activation at gamma = 1, beta = 0, and to a scalar alpha when all
+  alphas are equal.
+* matmul_act_*: test_oracle_matmul.py.  Checks: a hand-worked example;
+  numpy matmul; a permutation that catches a transposed operand; rank-one
+  products; torch autograd for the backward.
+* concat_bn_relu_*: test_oracle_bn.py.  Checks: torch.cat + F.batch_norm +
+  relu autograd in float64; a hand-worked example; the batch-normalization
+  invariants.
+* round_bf16, round_f32: test_oracle_rounding.py.  Checks: torch's and
+  numpy's round-to-nearest-even casts; ties to even and range boundaries;
+  identity on every finite bf16 value.
 """
 from __future__ import annotations
 
