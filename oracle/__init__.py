@@ -45,9 +45,16 @@ Each function is checked against something other than itself:
 * matmul_act_*: test_oracle_matmul.py.  Checks: a hand-worked example;
   numpy matmul; a permutation that catches a transposed operand; rank-one
   products; torch autograd for the backward.
+* affine_act_zround: test_oracle_channel.py.  Checks: exact first-order
+  values for ReLU; u |z f'(z)| against the pinned derivative and u |z f''(z)|
+  against Swish's closed-form second derivative and torch float64 double
+  backward for GELU-tanh.
 * concat_bn_relu_*: test_oracle_bn.py.  Checks: torch.cat + F.batch_norm +
   relu autograd in float64; a hand-worked example; the batch-normalization
   invariants.
+* bn_running_update: test_oracle_bn.py.  Checks: torch F.batch_norm's
+  running_mean / running_var update (training, momentum 0.1) in float64; a
+  hand-worked example.
 * round_bf16, round_f32: test_oracle_rounding.py.  Checks: torch's and
   numpy's round-to-nearest-even casts; ties to even and range boundaries;
   identity on every finite bf16 value.
@@ -122,6 +129,11 @@ def _load():
         lib.oracle_affine_act_bwd.argtypes = [ctypes.c_int, ctypes.c_int, shp, d, d, d, d, ctypes.c_double,
                                               d, d, d, d]
         lib.oracle_affine_act_bwd.restype = ctypes.c_int
+        lib.oracle_affine_act_zround.argtypes = [ctypes.c_int, ctypes.c_int, shp, d, d, d, d, ctypes.c_double,
+                                                 d, d]
+        lib.oracle_affine_act_zround.restype = ctypes.c_int
+        lib.oracle_bn_running_update.argtypes = [i64, i64, d, d, ctypes.c_double, d, d]
+        lib.oracle_bn_running_update.restype = ctypes.c_int
         lib.oracle_swish_channel_fwd.argtypes = [ctypes.c_int, shp, d, d, d]
         lib.oracle_swish_channel_fwd.restype = ctypes.c_int
         lib.oracle_swish_channel_bwd.argtypes = [ctypes.c_int, shp, d, d, d, d, d, d]
@@ -139,6 +151,8 @@ def _load():
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_f32.argtypes = [d, ctypes.POINTER(ctypes.c_float), i64]
         lib.oracle_round_f32.restype = None
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -156,6 +170,11 @@ def _ptr(a: np.ndarray, ctype=ctypes.c_double):
 def num_threads() -> int:
     """OpenMP threads the elementwise loops use."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Set the OpenMP threads of the elementwise loops (n >= 1)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def act_fwd(act: str, x, param: float = 1.0) -> np.ndarray:
@@ -278,6 +297,22 @@ def affine_act_bwd(act: str, layout: str, shape, x, dy, gamma, beta, param: floa
     return dx, dg, db, scale
 
 
+def affine_act_zround(act: str, layout: str, shape, x, dy, gamma, beta, param: float = 1.0):
+    """Returns (ey, edx): per element, the largest change of y = f(z) and of
+    dx = gamma_c dy f'(z) when z = gamma_c x + beta_c moves by one binary32
+    rounding (to z (1 -+ 2^-24)).  The part of an fp32 evaluation's error that
+    comes from forming z in fp32."""
+    s = _shape4(shape)
+    x, dy, gamma, beta = _f64(x), _f64(dy), _f64(gamma), _f64(beta)
+    ey = np.empty_like(x)
+    edx = np.empty_like(x)
+    rc = _load().oracle_affine_act_zround(ACTS[act], LAYOUTS[layout], _ptr(s, ctypes.c_int64), _ptr(x), _ptr(dy),
+                                          _ptr(gamma), _ptr(beta), float(param), _ptr(ey), _ptr(edx))
+    if rc:
+        raise ValueError(f"oracle_affine_act_zround failed: {rc}")
+    return ey, edx
+
+
 def swish_channel_fwd(layout: str, shape, x, alpha) -> np.ndarray:
     """y = x Sigmoid(alpha_c x); shape is (N, C, H, W)."""
     s = _shape4(shape)
@@ -381,6 +416,18 @@ def concat_bn_relu_bwd(pieces, dy, gamma, beta, mean, var, eps: float = 1e-5):
         raise ValueError(f"oracle_bn_relu_bwd failed: {rc}")
     cuts = np.cumsum([p.shape[1] for p in pieces])[:-1]
     return np.split(dx, cuts, axis=1), dg, db, np.split(sc, cuts, axis=1)
+
+
+def bn_running_update(running_mean, running_var, mean, var, n: int, momentum: float = 0.1):
+    """Running statistics after one training step: returns new (running_mean,
+    running_var) from the batch mean and biased variance over n values per
+    channel (the unbiased variance var n / (n - 1) enters running_var)."""
+    rm, rv = _f64(running_mean).copy(), _f64(running_var).copy()
+    mean, var = _f64(mean), _f64(var)
+    rc = _load().oracle_bn_running_update(rm.size, int(n), _ptr(mean), _ptr(var), float(momentum), _ptr(rm), _ptr(rv))
+    if rc:
+        raise ValueError(f"oracle_bn_running_update failed: {rc}")
+    return rm, rv
 
 
 def round_bf16(v) -> np.ndarray:

@@ -46,8 +46,9 @@
  *    batch normalization here is the standard training-mode definition:
  *    per-channel mean and biased variance over N, H, W, xhat = (x - mean) /
  *    sqrt(var + eps), y = max(gamma xhat + beta, 0); running statistics move
- *    by momentum towards the batch mean and the unbiased variance.  The
- *    caller concatenates the pieces (along channels) before calling.
+ *    by momentum towards the batch mean and the unbiased variance
+ *    (oracle_bn_running_update).  The caller concatenates the pieces (along
+ *    channels) before calling.
  *  - Matmul + activation (problem B07, SOLUTION step 4: the activation
  *    follows a d x d matrix multiply on the same tensor): Z = X W^T with X
  *    [M x K] and W [N x K] row-major; the activation is evaluated at Z as
@@ -419,6 +420,36 @@ int oracle_affine_act_bwd(int act, int layout, const int64_t shape[4], const dou
     return 0;
 }
 
+/* How much the affine outputs move when z = gamma_c x + beta_c is rounded
+ * once to binary32.  Any fp32 evaluation (the configurations compute in fp32)
+ * forms z in binary32, which moves it by at most u |z|, u = 2^-24 (round to
+ * nearest); no arithmetic after that rounding can recover the exact z.  For
+ * each element: ey = the largest change of y = f(z), and edx = the largest
+ * change of dx = gamma_c dy f'(z), when z moves to z (1 - u) or z (1 + u),
+ * evaluated in double as differences of the definitions at those points.
+ * Near-linear f gives ey = u |z f'(z)| and edx = u |z gamma_c dy f''(z)| to
+ * first order.  The tests add these to the fp32 tolerance of the affine
+ * outputs. */
+int oracle_affine_act_zround(int act, int layout, const int64_t shape[4], const double *x, const double *dy,
+                             const double *gamma, const double *beta, double param, double *ey, double *edx)
+{
+    if (act < 0 || act >= OR_NUM_ACTS || (layout != OR_NCHW && layout != OR_NHWC)) return -1;
+    const double u = ldexp(1.0, -24);
+    int64_t n = shape[0] * shape[1] * shape[2] * shape[3];
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = channel_of(layout, shape, i);
+        double z = gamma[c] * x[i] + beta[c];
+        double lo = z * (1.0 - u), hi = z * (1.0 + u);
+        double f0 = act_f(act, z, param), d0 = act_df(act, z, param);
+        double fy = fmax(fabs(act_f(act, lo, param) - f0), fabs(act_f(act, hi, param) - f0));
+        double fd = fmax(fabs(act_df(act, lo, param) - d0), fabs(act_df(act, hi, param) - d0));
+        ey[i] = fy;
+        edx[i] = fabs(gamma[c] * dy[i]) * fd;
+    }
+    return 0;
+}
+
 /* Swish with one alpha per channel: y = x Sigmoid(alpha_c x). */
 int oracle_swish_channel_fwd(int layout, const int64_t shape[4], const double *x,
                              const double *alpha, double *y)
@@ -601,6 +632,24 @@ int oracle_bn_relu_bwd(int64_t N, int64_t C, int64_t HW, const double *x, const 
     return 0;
 }
 
+/* Running statistics after one training step of batch normalization, per
+ * channel: running_mean <- (1 - momentum) running_mean + momentum mean and
+ * running_var <- (1 - momentum) running_var + momentum var n / (n - 1), the
+ * unbiased batch variance over n = N H W values (standard training-mode
+ * definition).  For n = 1 the unbiased variance is undefined; the biased one
+ * (zero) is used.  running_mean and running_var are updated in place. */
+int oracle_bn_running_update(int64_t C, int64_t n, const double *mean, const double *var, double momentum,
+                             double *running_mean, double *running_var)
+{
+    if (C < 0 || n < 1) return -1;
+    for (int64_t c = 0; c < C; ++c) {
+        double unbiased = n > 1 ? var[c] * (double)n / (double)(n - 1) : var[c];
+        running_mean[c] = (1.0 - momentum) * running_mean[c] + momentum * mean[c];
+        running_var[c] = (1.0 - momentum) * running_var[c] + momentum * unbiased;
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------ storage rounding */
 
 /* Round a double to the nearest bfloat16 (1 sign bit, 8 exponent bits with
@@ -652,6 +701,17 @@ void oracle_round_f32(const double *v, float *out, int64_t n)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) out[i] = (float)v[i];
+}
+
+/* Threads the OpenMP loops use from now on (the baseline's single-core
+ * figure); n < 1 is ignored. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
 }
 
 int oracle_num_threads(void)

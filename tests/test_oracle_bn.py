@@ -91,3 +91,28 @@ def test_invariants_above_threshold():
     r = 1.0 / np.sqrt(var + eps)
     assert np.allclose((dx * xh).sum(axis=(0, 2)), g * r * dg * eps / (var + eps), rtol=1e-9, atol=1e-13)
     assert np.allclose(db, dy.sum(axis=(0, 2)), rtol=1e-12)
+
+
+@pytest.mark.parametrize("N,C,HW", [(4, 6, 7), (2, 3, 1), (8, 5, 25)])
+def test_running_update_matches_torch(N, C, HW):
+    # torch's training-mode F.batch_norm updates running_mean / running_var in
+    # place with momentum and the unbiased batch variance
+    x = synthetic.normal_f64(N * C * HW, 1.3, 54, 0, mean=0.4).reshape(N, C, HW)
+    rm0 = synthetic.normal_f64(C, 0.5, 55, 3)
+    rv0 = synthetic.uniform_f64(C, 0.5, 2.0, 55, 4)
+    g, b = _params(C, 56)
+    _, mean, var, _ = oracle.concat_bn_relu_fwd([x], g, b, 1e-5)
+    rm, rv = oracle.bn_running_update(rm0, rv0, mean, var, N * HW, 0.1)
+    trm, trv = torch.from_numpy(rm0.copy()), torch.from_numpy(rv0.copy())
+    F.batch_norm(torch.from_numpy(x.copy()), trm, trv, torch.from_numpy(g), torch.from_numpy(b), training=True,
+                 momentum=0.1, eps=1e-5)
+    assert np.allclose(rm, trm.numpy(), rtol=1e-13, atol=1e-15)
+    assert np.allclose(rv, trv.numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_running_update_hand_worked():
+    # one channel, values {1, 3}: mean 2, biased variance 1, unbiased 2;
+    # momentum 0.25 from (0, 1): mean 0.75 * 0 + 0.25 * 2 = 0.5,
+    # var 0.75 * 1 + 0.25 * 2 = 1.25
+    rm, rv = oracle.bn_running_update([0.0], [1.0], [2.0], [1.0], 2, 0.25)
+    assert rm[0] == 0.5 and rv[0] == 1.25
