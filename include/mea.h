@@ -14,7 +14,9 @@
  * formed, only the batch statistics are kept, the output is re-populated).
  *
  * Entry points: mea_act_fwd / mea_act_bwd (+ _workspace_bytes,
- * mea_act_bwd_dparam_noalloc); mea_affine_swish_* and mea_affine_act_*;
+ * mea_act_bwd_dparam_noalloc); mea_act_fwd_grouped / mea_act_bwd_grouped
+ * (+ _workspace_bytes: many independent tensors in one launch);
+ * mea_affine_swish_* and mea_affine_act_*;
  * mea_swish_channel_*; mea_matmul_act_fwd / _bwd; mea_concat_bn_relu_fwd /
  * _apply / _bwd (+ _workspace_bytes); mea_status_string, mea_last_error,
  * mea_version.
@@ -165,6 +167,59 @@ MEA_API mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x
                          void *dx, int64_t n, float param, const float *param_dev,
                          float *dparam_dev, void *workspace, size_t ws_bytes,
                          mea_stream_t stream);
+
+/* One tensor of a grouped call (mea_act_fwd_grouped / mea_act_bwd_grouped). */
+typedef struct {
+    const void *x;            /* device, n elements, read only (the saved tensor) */
+    const void *dy;           /* backward: device, n elements; ignored by the forward */
+    void *out;                /* device, n elements: y (forward) or dx (backward) */
+    int64_t n;                /* element count, >= 0 */
+    float param;              /* as in mea_act_fwd */
+    const float *param_dev;   /* as in mea_act_fwd (nullable) */
+    float *dparam_dev;        /* backward, MEA_SWISH: as in mea_act_bwd; set in every
+                                 segment or in none; ignored by the forward */
+} mea_act_segment_t;
+
+/* Forward over several independent tensors in one launch: for every segment
+ * s, out_s = f(x_s), with one activation and dtype for all.  Each segment's
+ * result is bitwise the result of mea_act_fwd on that segment alone.  One
+ * grid instead of nseg launches removes each small tensor's ramp-up, drain
+ * and launch gap (the small feature maps of a network's branches or of
+ * several micro-batches).
+ *   segs         host array of nseg (>= 0) segments; read during the call only.
+ *                Segments are launched up to 32 per kernel.
+ *   Every segment is validated as mea_act_fwd validates its tensors, and no
+ *   segment's output may overlap any other segment's input or output
+ *   (MEA_ERR_INVALID_ARG, nothing launched).
+ * Source: as mea_act_fwd; one launch for many tensors is this library's
+ * (the pages call the activation once per layer). */
+MEA_API mea_status_t mea_act_fwd_grouped(mea_act_t act, mea_dtype_t dtype, int nseg,
+                                         const mea_act_segment_t *segs, mea_stream_t stream);
+
+/* Bytes of device workspace mea_act_bwd_grouped needs for these segments:
+ * 0 unless their dparam_dev are set; else the sum over segments of
+ * mea_act_bwd_workspace_bytes rounded up to 256 bytes.  Pure host
+ * arithmetic. */
+MEA_API size_t mea_act_bwd_grouped_workspace_bytes(mea_act_t act, int nseg, const mea_act_segment_t *segs);
+
+/* Backward over several independent tensors in one launch: for every
+ * segment, dx_s = dy_s * f'(x_s), and with dparam_dev set (MEA_SWISH, every
+ * segment) d alpha_s, each bitwise what mea_act_bwd gives for that segment
+ * alone (same reduction grid and summation order).
+ *   segs         as in mea_act_fwd_grouped; dx may alias that segment's dy
+ *                or x exactly, no other overlap with any segment.
+ *   workspace,
+ *   ws_bytes     when d alpha is asked for: device scratch of at least
+ *                mea_act_bwd_grouped_workspace_bytes(), 256-byte aligned,
+ *                any contents (every call writes the partial sums it reads:
+ *                no counter, no zero-fill).  The d alpha sums are formed by
+ *                a second, small kernel (one block per segment) queued on
+ *                the same stream.  Calls sharing a workspace must not run
+ *                concurrently on the GPU.
+ * Source: as mea_act_bwd. */
+MEA_API mea_status_t mea_act_bwd_grouped(mea_act_t act, mea_dtype_t dtype, int nseg,
+                                         const mea_act_segment_t *segs, void *workspace, size_t ws_bytes,
+                                         mea_stream_t stream);
 
 /* Bytes of device workspace mea_affine_swish_bwd needs for this dtype,
  * layout and logical shape {N, C, H, W} (host pointer).  Pure host
@@ -386,11 +441,13 @@ MEA_API mea_status_t mea_concat_bn_relu_bwd(mea_dtype_t dtype, int npieces, cons
  *   Every element count is served (the reduction grid is capped so that its
  *   scratch fits the array); a request needing more scratch than the array
  *   holds would be refused with MEA_ERR_WORKSPACE.
- *   The first call on a device (with that device current) looks up the
- *   array's device address with cudaGetSymbolAddress; make that first call
- *   before any stream capture.  Every call clears the array's completion
- *   counter with cudaMemsetAsync on `stream` and then launches the kernel;
- *   it calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Every call looks up the array's device address on the current device
+ *   with cudaGetSymbolAddress (so the address stays right after a device
+ *   reset); the first call on a device may load the library's device code,
+ *   so make it before any stream capture.  Every call clears the array's
+ *   completion counter with cudaMemsetAsync on `stream` and then launches
+ *   the kernel; it calls no cudaMalloc, cudaFree or other allocating
+ *   routine.
  *   All calls on a device share the one array: calls whose kernels may run
  *   at the same time on the GPU (unordered streams) race and must not be
  *   issued; calls ordered on one stream are safe. */
@@ -398,6 +455,24 @@ MEA_API mea_status_t mea_act_bwd_dparam_noalloc(mea_act_t act, mea_dtype_t dtype
                                                 const void *dy, void *dx, int64_t n, float param,
                                                 const float *param_dev, float *dparam_dev,
                                                 mea_stream_t stream);
+
+/* Self-test of the bounded waits (failure detection without a GPU fault).
+ * No counterpart on the pages.  Runs the pipelined NHWC backward of the
+ * fused affine + Swish on the caller's tensors (arguments as for
+ * mea_affine_swish_bwd with layout MEA_NHWC; dx, dgamma, dbeta are not
+ * written) with the shared-memory copies of its producer withheld, so that
+ * no stage barrier ever completes.  Every wait then gives up after a few
+ * milliseconds, records the workspace's error word and lets its warp
+ * finish, exactly the path a wait takes if a copy never lands.  The call
+ * synchronises `stream`, stores the error word in *expired (1: the waits
+ * expired and the kernel returned; the context stays usable) and clears the
+ * word.  MEA_ERR_UNSUPPORTED when the shape or alignment does not take the
+ * pipelined path (C a multiple of 4, x and dy 16-byte aligned, enough
+ * tiles). */
+MEA_API mea_status_t mea_affine_bwd_wait_selftest(mea_dtype_t dtype, const int64_t shape[4], const void *x,
+                                                  const void *dy, const float *gamma, const float *beta, void *dx,
+                                                  void *workspace, size_t ws_bytes, int *expired,
+                                                  mea_stream_t stream);
 
 /* Reads (and with clear non-zero, resets) the matmul kernels' device error
  * word on the current device: non-zero if a bounded barrier wait in a

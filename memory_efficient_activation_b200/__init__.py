@@ -35,19 +35,19 @@ from . import _capi
 from ._capi import ACT_IDS, LAYOUT_IDS, MeaError
 
 __all__ = [
-    "act_fwd", "act_bwd", "affine_swish_fwd", "affine_swish_bwd",
+    "act_fwd", "act_bwd", "act_fwd_grouped", "act_bwd_grouped", "affine_swish_fwd", "affine_swish_bwd",
     "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
     "matmul_act_fwd", "matmul_act_bwd",
     "concat_bn_relu_fwd", "concat_bn_relu_apply", "concat_bn_relu_bwd",
     "act_fwd_bwd_host",
-    "act_bwd_workspace_bytes", "affine_swish_bwd_workspace_bytes",
+    "act_bwd_workspace_bytes", "act_bwd_grouped_workspace_bytes", "affine_swish_bwd_workspace_bytes",
     "affine_act_bwd_workspace_bytes", "swish_channel_bwd_workspace_bytes",
     "ActivationFunction", "MemoryEfficientActivation", "MemoryEfficientSwish",
     "AffineSwishFunction", "MemoryEfficientAffineSwish",
     "AffineActFunction", "MemoryEfficientAffineActivation",
     "SwishChannelFunction", "MemoryEfficientChannelSwish", "MLPFunction", "MemoryEfficientMLP",
     "SharedBuffer", "ConcatBNReLUConvFunction", "MemoryEfficientDenseBottleneck",
-    "MeaError", "ACTIVATIONS",
+    "affine_bwd_wait_selftest", "MeaError", "ACTIVATIONS",
 ]
 
 ACTIVATIONS = tuple(ACT_IDS)
@@ -198,6 +198,89 @@ def act_bwd(act: str, x: torch.Tensor, dy: torch.Tensor, param: float = 1.0,
                                   _stream(x))
     _capi.check("mea_act_bwd", st)
     return dx
+
+
+def _group_args(xs, name, params, param_devs, dys=None, dparams=None, outs=None):
+    """Checks a grouped call's tensor lists (same device and dtype, shapes
+    matching x) and builds its mea_act_segment_t array; returns (segments,
+    outputs)."""
+    xs = list(xs)
+    k = len(xs)
+    if k == 0:
+        return (_capi.ActSegment * 0)(), []
+    _need_cuda(*xs)
+    ref = xs[0]
+    for x in xs:
+        if x.device != ref.device or x.dtype != ref.dtype:
+            raise ValueError(f"{name}: every tensor must share the first one's device and dtype")
+    params = [1.0] * k if params is None else ([float(params)] * k if isinstance(params, (int, float))
+                                               else [float(p) for p in params])
+    param_devs = [None] * k if param_devs is None else list(param_devs)
+    dparams = [None] * k if dparams is None else list(dparams)
+    if len(params) != k or len(param_devs) != k or len(dparams) != k or (dys is not None and len(dys) != k):
+        raise ValueError(f"{name}: every list must have one entry per tensor")
+    if outs is None:
+        outs = [torch.empty_like(x) for x in xs]
+    else:
+        outs = [_like(x, o, "out") for x, o in zip(xs, outs)]
+    segs = (_capi.ActSegment * k)()
+    for i, x in enumerate(xs):
+        if param_devs[i] is not None:
+            _on_device(x, param_devs[i], "param_dev", torch.float32, 1)
+        if dparams[i] is not None:
+            _on_device(x, dparams[i], "dparam", torch.float32, 1)
+        dy = None
+        if dys is not None:
+            dy = _like(x, dys[i], "dy")
+        segs[i] = _capi.ActSegment(x.data_ptr(), dy.data_ptr() if dy is not None else None, outs[i].data_ptr(),
+                                   x.numel(), params[i], _ptr(param_devs[i]), _ptr(dparams[i]))
+    return segs, outs
+
+
+def act_bwd_grouped_workspace_bytes(act: str, sizes, want_dparam: bool) -> int:
+    """Workspace bytes of a grouped backward over tensors of these element
+    counts (0 without d alpha)."""
+    sizes = [int(n) for n in sizes]
+    if not want_dparam or not sizes:
+        return 0
+    segs = (_capi.ActSegment * len(sizes))()
+    for i, n in enumerate(sizes):
+        # the size query reads only n and whether d alpha is asked for
+        segs[i] = _capi.ActSegment(None, None, None, n, 1.0, None, 1)
+    return int(_capi.lib().mea_act_bwd_grouped_workspace_bytes(_act_id(act), len(sizes), segs))
+
+
+def act_fwd_grouped(act: str, xs, params=None, param_devs=None, outs=None) -> list:
+    """y_i = f(x_i) for every tensor of xs in one launch (many small,
+    independent tensors: one grid instead of one launch each).  params: one
+    float for all or one per tensor; param_devs: optional one-element fp32
+    CUDA tensors.  Each y_i is bitwise what act_fwd gives for x_i."""
+    segs, outs = _group_args(xs, "act_fwd_grouped", params, param_devs, outs=outs)
+    if len(outs) == 0:
+        return []
+    st = _capi.lib().mea_act_fwd_grouped(_act_id(act), _dtype_id(xs[0]), len(outs), segs, _stream(xs[0]))
+    _capi.check("mea_act_fwd_grouped", st)
+    return outs
+
+
+def act_bwd_grouped(act: str, xs, dys, params=None, param_devs=None, dparams=None, outs=None,
+                    workspace: torch.Tensor | None = None) -> list:
+    """dx_i = dy_i * f'(x_i) for every pair in one launch; with dparams (one
+    one-element fp32 CUDA tensor per tensor, Swish) each is overwritten with
+    that tensor's d alpha.  Each result is bitwise what act_bwd gives."""
+    segs, outs = _group_args(xs, "act_bwd_grouped", params, param_devs, dys=dys, dparams=dparams, outs=outs)
+    if len(outs) == 0:
+        return []
+    ws_ptr, ws_bytes = None, 0
+    if dparams is not None:
+        need = int(_capi.lib().mea_act_bwd_grouped_workspace_bytes(_act_id(act), len(outs), segs))
+        ws = _on_device(xs[0], workspace, "workspace") if workspace is not None else \
+            _pool.get(xs[0].device, _stream(xs[0]), need)
+        ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+    st = _capi.lib().mea_act_bwd_grouped(_act_id(act), _dtype_id(xs[0]), len(outs), segs, ws_ptr, ws_bytes,
+                                         _stream(xs[0]))
+    _capi.check("mea_act_bwd_grouped", st)
+    return outs
 
 
 def _affine_shape(x: torch.Tensor, layout: str):
@@ -842,3 +925,26 @@ class MemoryEfficientDenseBottleneck(torch.nn.Module):
         return ConcatBNReLUConvFunction.apply(self.shared, self.weight, self.gamma, self.beta, self.running_mean,
                                               self.running_var, self.eps, self.momentum,
                                               *[p.contiguous() for p in pieces])
+
+
+def affine_bwd_wait_selftest(x: torch.Tensor, dy: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+                             workspace: torch.Tensor | None = None) -> int:
+    """Self-test of the bounded waits: runs the pipelined NHWC backward of the
+    fused affine + Swish on these tensors (x, dy: (N, H, W, C)) with its
+    shared-memory copies withheld, so that every stage wait expires; returns
+    the error word the kernel recorded (1 when the waits expired and the
+    kernel returned, as designed).  Synchronises the current stream."""
+    _need_cuda(x, dy)
+    _like(x, dy, "dy")
+    shape = _affine_shape(x, "nhwc")
+    _chan_params(shape[1], gamma, beta, device=x.device)
+    need = affine_swish_bwd_workspace_bytes(x.dtype, "nhwc", shape)
+    ws = torch.zeros(need, dtype=torch.uint8, device=x.device) if workspace is None else \
+        _on_device(x, workspace, "workspace")
+    dx = torch.empty_like(x)
+    expired = ctypes.c_int(0)
+    st = _capi.lib().mea_affine_bwd_wait_selftest(_dtype_id(x), _capi.shape4(shape), x.data_ptr(), dy.data_ptr(),
+                                                  gamma.data_ptr(), beta.data_ptr(), dx.data_ptr(), ws.data_ptr(),
+                                                  ws.numel(), ctypes.byref(expired), _stream(x))
+    _capi.check("mea_affine_bwd_wait_selftest", st)
+    return int(expired.value)

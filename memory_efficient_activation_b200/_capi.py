@@ -36,10 +36,22 @@ _i = ctypes.c_int
 _sz = ctypes.c_size_t
 _shape = ctypes.POINTER(ctypes.c_int64)
 _ptrs = ctypes.POINTER(ctypes.c_void_p)
+
+
+class ActSegment(ctypes.Structure):
+    """mea_act_segment_t: one tensor of a grouped call."""
+    _fields_ = [("x", _vp), ("dy", _vp), ("out", _vp), ("n", _i64), ("param", _f), ("param_dev", _vp),
+                ("dparam_dev", _vp)]
+
+
+_segs = ctypes.POINTER(ActSegment)
 SIGNATURES = {
     "mea_act_fwd": (_i, [_i, _i, _vp, _vp, _i64, _f, _vp, _vp]),
     "mea_act_bwd_workspace_bytes": (_sz, [_i, _i64, _i]),
     "mea_act_bwd": (_i, [_i, _i, _vp, _vp, _vp, _i64, _f, _vp, _vp, _vp, _sz, _vp]),
+    "mea_act_fwd_grouped": (_i, [_i, _i, _i, _segs, _vp]),
+    "mea_act_bwd_grouped_workspace_bytes": (_sz, [_i, _i, _segs]),
+    "mea_act_bwd_grouped": (_i, [_i, _i, _i, _segs, _vp, _sz, _vp]),
     "mea_affine_swish_bwd_workspace_bytes": (_sz, [_i, _i, _shape]),
     "mea_affine_swish_fwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp]),
     "mea_affine_swish_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -59,6 +71,8 @@ SIGNATURES = {
     "mea_concat_bn_relu_bwd": (_i, [_i, _i, _ptrs, _shape, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ptrs, _i, _vp,
                                     _vp, _vp, _sz, _vp]),
     "mea_act_bwd_dparam_noalloc": (_i, [_i, _i, _vp, _vp, _vp, _i64, _f, _vp, _vp, _vp]),
+    "mea_affine_bwd_wait_selftest": (_i, [_i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                          ctypes.POINTER(ctypes.c_int), _vp]),
     "mea_status_string": (ctypes.c_char_p, [_i]),
     "mea_last_error": (ctypes.c_char_p, []),
     "mea_version": (_i, []),

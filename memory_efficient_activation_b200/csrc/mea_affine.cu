@@ -21,11 +21,12 @@ namespace mea {
 //   dz = dy (s (1 + alpha z E s))
 // (s times the bracket first: s may be as small as 2^-124, and dy s could
 // fall below the normal range where the final result does not).
-// Every finite product stays finite while |t| <= kTailT; the tail flag is
-// raised for |t| > kTailT (deep negative z, and z beyond +86 or +inf, where
-// alpha z E s could be inf * 0), and the caller recomputes such elements
-// with the scalar form.  Rounding differs from the scalar form by a few fp32
-// ulps, far inside a bf16 ulp.
+// Every finite product stays finite while |t| <= kTailT.  One u = t -
+// Swish::kRootT gives both flags: |u| > Swish::kTailU (which contains |t| >
+// kTailT: deep negative z, and z beyond +86 or +inf, where alpha z E s could
+// be inf * 0) and |u| < Swish::kRootWinT (alpha z near the zero of Swish');
+// the caller recomputes the flagged elements.  Rounding differs from the
+// scalar form by a few fp32 ulps, far inside a bf16 ulp.
 __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, float d1, const Coef &k, bool &tail,
                                                float &o0, float &o1)
 {
@@ -33,7 +34,10 @@ __device__ __forceinline__ void swish_df2_bf16(float z0, float z1, float d0, flo
     float t0, t1;
     upk(mul2(z, sp2(k.c_hi)), t0, t1);
     const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
-    tail |= (fabsf(t0) > kTailT) | (fabsf(t1) > kTailT);
+    float u0, u1;
+    upk(add2(pk(t0, t1), sp2(-Swish::kRootT)), u0, u1);
+    tail |= (fabsf(u0) < Swish::kRootWinT) | (fabsf(u1) < Swish::kRootWinT) | (fabsf(u0) > Swish::kTailU) |
+            (fabsf(u1) > Swish::kTailU);
     const F2 E = pk(e0, e1);
     float a0, a1;
     upk(add2(sp2(1.f), E), a0, a1);
@@ -60,8 +64,8 @@ __device__ __forceinline__ F2 sigmoid_parts2(F2 z, const Coef &k, bool &tail)
 // GeluTanh, E = 2^t, s = 1 / (1 + E) = Sigmoid(v), Sigmoid(-v) = E s, and
 //   y = z s,   dz = dy (s (1 + z v' E s)),  v' = k1 + 3 k3 z^2,
 // The forward flags t > kTailT (deep negative z) for the tail form; the
-// backward uses swish_df2_bf16's rule (|t| > kTailT flags the element for
-// the scalar form; inside, z v' E s is finite).
+// backward uses swish_df2_bf16's two guards on u = t - GeluTanh::kRootT
+// (inside them z v' E s is finite and z is away from the zero of f').
 template <bool kBothSides>
 __device__ __forceinline__ F2 gelu_tanh_parts2(F2 z, F2 &z2, bool &tail, F2 &E)
 {
@@ -69,10 +73,15 @@ __device__ __forceinline__ F2 gelu_tanh_parts2(F2 z, F2 &z2, bool &tail, F2 &E)
     float t0, t1;
     upk(mul2(z, fma2(sp2(GeluTanh::kC3f), z2, sp2(GeluTanh::kC1f))), t0, t1);
     const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
-    if constexpr (kBothSides)
-        tail |= (fabsf(t0) > kTailT) | (fabsf(t1) > kTailT);
-    else
+    if constexpr (kBothSides) {
+        // backward: the guards of swish_df2_bf16, on GeluTanh's constants
+        float u0, u1;
+        upk(add2(pk(t0, t1), sp2(-GeluTanh::kRootT)), u0, u1);
+        tail |= (fabsf(u0) < GeluTanh::kRootWinT) | (fabsf(u1) < GeluTanh::kRootWinT) |
+                (fabsf(u0) > GeluTanh::kTailU) | (fabsf(u1) > GeluTanh::kTailU);
+    } else {
         tail |= (t0 > kTailT) | (t1 > kTailT);
+    }
     E = pk(e0, e1);
     float a0, a1;
     upk(add2(sp2(1.f), E), a0, a1);
@@ -117,17 +126,45 @@ struct AffineOp {
         return A::template f_tail<P>(z(x, h), k);
     }
     static __device__ __forceinline__ bool is_tail(float x, const K &k, const Ch &h) { return A::is_tail(z(x, h), k); }
+    // Every element the backward main paths (scalar or packed) may flag: the
+    // deep tails, the packed forms' overflow guards and, with bf16 storage,
+    // the neighbourhood of the zero of f'.  Only these are recomputed.
+    template <bool P>
+    static __device__ __forceinline__ bool flag_bwd(float x, const K &k, const Ch &h)
+    {
+        const float zz = z(x, h);
+        if constexpr (!P && A::kHasRoot) return A::template bwd_flagged<P>(zz, k) || A::near_root(zz, k);
+        return A::template bwd_flagged<P>(zz, k);
+    }
     // o = dz
     template <bool P>
     static __device__ __forceinline__ void bwd(float x, float dy, const K &k, const Ch &h, bool &tail, float &o,
                                                float &)
     {
-        o = A::template df<P>(z(x, h), dy, k, tail);
+        const float zz = z(x, h);
+        o = A::template df<P>(zz, dy, k, tail);
+        if constexpr (!P && A::kHasRoot) tail |= A::near_root(zz, k);
     }
+    // A flagged element: near the zero of f' (bf16 storage), d = v - v0 from
+    // z = gamma x + beta formed in fp64 and f' from its Taylor polynomial
+    // there; in the deep tail the scaled tail form; else (a packed form's
+    // overflow guard) the scalar main form.
     template <bool P>
     static __device__ __forceinline__ void bwd_tail(float x, float dy, const K &k, const Ch &h, float &o, float &)
     {
-        o = A::template df_tail<P>(z(x, h), dy, k);
+        const float zz = z(x, h);
+        if constexpr (!P && A::kHasRoot) {
+            if (A::near_root(zz, k)) {
+                o = root_df<A>(root_d(h.g, x, h.b, A::root_scale(k), A::kRootD), dy);
+                return;
+            }
+        }
+        if (A::is_tail(zz, k)) {
+            o = A::template df_tail<P>(zz, dy, k);
+            return;
+        }
+        bool unused = false;
+        o = A::template df<P>(zz, dy, k, unused);
     }
     static __device__ __forceinline__ float finish(float x, float o, float, const Ch &h, float (&acc)[NR])
     {
@@ -167,8 +204,16 @@ struct AffineOp {
     static __device__ __forceinline__ void bwd2(F2 x, F2 dy, const K &k, const Ch2 &h, bool &tail, F2 &o, F2 &)
     {
         float z0, z1, d0, d1, o0, o1;
-        upk(fma2(h.g, x, h.b), z0, z1);
+        const F2 zp = fma2(h.g, x, h.b);
+        upk(zp, z0, z1);
         upk(dy, d0, d1);
+        if constexpr (!P && std::is_same<A, GeluErf>::value) {
+            // the same test as A::near_root, on both elements (the packed
+            // Swish and GELU-tanh forms test their own exponent instead)
+            float e0, e1;
+            upk(add2(zp, sp2(-A::kRootHi)), e0, e1);
+            tail |= (fabsf(e0) < kRootWin) | (fabsf(e1) < kRootWin);
+        }
         if constexpr (HasPairs<A, P>::value) {
             A::df2(z0, z1, d0, d1, k, tail, o0, o1);
         } else if constexpr (std::is_same<A, Swish>::value && !P) {
@@ -218,6 +263,13 @@ cudaError_t launch_affine_fwd(const AffineLaunch &a)
 cudaError_t launch_affine_bwd(const AffineLaunch &a)
 {
     return a.dtype == kBF16 ? by_act<Bf16, 1>(a) : by_act<float, 1>(a);
+}
+
+cudaError_t launch_affine_bwd_wait_selftest(const AffineLaunch &a)
+{
+    const ChanArgs ca{a.gamma, a.beta, 1.f};
+    return a.dtype == kBF16 ? launch_channel_wait_selftest<AffineOp<Swish>, Bf16>(a, ca)
+                            : launch_channel_wait_selftest<AffineOp<Swish>, float>(a, ca);
 }
 
 }  // namespace mea

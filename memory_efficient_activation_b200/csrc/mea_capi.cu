@@ -1,10 +1,12 @@
 // mea_capi.cu -- the C ABI of include/mea.h: argument validation, error
 // reporting and dispatch to the kernel launchers.  Host code only.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <vector>
 
 #include "../../include/mea.h"
 #include "mea_bn_api.h"
@@ -15,6 +17,16 @@
 namespace {
 
 thread_local char g_err[512];
+
+// One NVTX range per C-ABI call, named for the entry point, so that a
+// profiler's timeline shows which call issued which kernels.  With no tool
+// attached the NVTX calls return at once.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 
 void clear_error() { g_err[0] = '\0'; }
 
@@ -202,6 +214,7 @@ int mea_version(void) { return 1 * 10000 + 3 * 100 + 0; }
 mea_status_t mea_act_fwd(mea_act_t act, mea_dtype_t dtype, const void *x, void *y, int64_t n, float param,
                          const float *param_dev, mea_stream_t stream)
 {
+    Range range_("mea_act_fwd");
     clear_error();
     if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
     if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
@@ -235,6 +248,7 @@ mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const 
                          float param, const float *param_dev, float *dparam_dev, void *workspace,
                          size_t ws_bytes, mea_stream_t stream)
 {
+    Range range_("mea_act_bwd");
     clear_error();
     if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
     if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
@@ -270,6 +284,167 @@ mea_status_t mea_act_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const 
     return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_act_bwd launch");
 }
 
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Validates the segments of a grouped call (each as the single-tensor call
+// validates its tensors; no output overlapping another segment's tensors)
+// and fills the launch table.  bwd: dy is read and dx may alias dy or x.
+static mea_status_t grouped_segments(const char *name, int nseg, const mea_act_segment_t *segs, int dtype,
+                                     bool bwd, std::vector<mea::ActSeg> &out)
+{
+    if (nseg < 0) return fail(MEA_ERR_INVALID_ARG, "%s: nseg = %d", name, nseg);
+    if (nseg > 0 && !segs) return fail(MEA_ERR_INVALID_ARG, "%s: segs is NULL", name);
+    const size_t es = dtype_bytes(dtype);
+    for (int i = 0; i < nseg; ++i) {
+        const mea_act_segment_t &g = segs[i];
+        if (g.n < 0 || g.n > kMaxElems)
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: n = %lld out of range", name, i, (long long)g.n);
+        if (g.n == 0) continue;
+        if (!g.x || !g.out || (bwd && !g.dy))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: a tensor pointer is NULL", name, i);
+        const size_t b = (size_t)g.n * es;
+        if (!bwd && overlaps(g.x, b, g.out, b))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: y overlaps x", name, i);
+        if (bwd && (partial_overlap(g.out, g.dy, b) || partial_overlap(g.out, g.x, b)))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: dx partially overlaps x or dy", name, i);
+    }
+    for (int i = 0; i < nseg; ++i) {
+        if (segs[i].n == 0) continue;
+        const size_t bi = (size_t)segs[i].n * es;
+        for (int j = 0; j < nseg; ++j) {
+            if (j == i || segs[j].n == 0) continue;
+            const size_t bj = (size_t)segs[j].n * es;
+            if (overlaps(segs[i].out, bi, segs[j].x, bj) || overlaps(segs[i].out, bi, segs[j].out, bj) ||
+                (bwd && overlaps(segs[i].out, bi, segs[j].dy, bj)))
+                return fail(MEA_ERR_INVALID_ARG, "%s: the output of segment %d overlaps a tensor of segment %d",
+                            name, i, j);
+        }
+    }
+    out.resize((size_t)nseg);
+    for (int i = 0; i < nseg; ++i) {
+        mea::ActSeg a{};
+        a.x = segs[i].x;
+        a.dy = bwd ? segs[i].dy : nullptr;
+        a.out = segs[i].out;
+        a.n = segs[i].n;
+        a.param = segs[i].param;
+        a.param_dev = segs[i].param_dev;
+        a.dparam = bwd ? segs[i].dparam_dev : nullptr;
+        out[(size_t)i] = a;
+    }
+    return MEA_OK;
+}
+
+mea_status_t mea_act_fwd_grouped(mea_act_t act, mea_dtype_t dtype, int nseg, const mea_act_segment_t *segs,
+                                 mea_stream_t stream)
+{
+    Range range_("mea_act_fwd_grouped");
+    clear_error();
+    if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    std::vector<mea::ActSeg> tab;
+    mea_status_t st = grouped_segments("mea_act_fwd_grouped", nseg, segs, dtype, false, tab);
+    if (st != MEA_OK) return st;
+    if (nseg == 0) return MEA_OK;
+    mea::ActGroupLaunch l{act, dtype, nseg, tab.data(), reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = mea::launch_act_fwd_grouped(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_act_fwd_grouped launch");
+}
+
+size_t mea_act_bwd_grouped_workspace_bytes(mea_act_t act, int nseg, const mea_act_segment_t *segs)
+{
+    if (nseg <= 0 || !segs || !segs[0].dparam_dev) return 0;
+    size_t total = 0;
+    for (int i = 0; i < nseg; ++i) total += round256(mea_act_bwd_workspace_bytes(act, segs[i].n, 1));
+    return total;
+}
+
+mea_status_t mea_act_bwd_grouped(mea_act_t act, mea_dtype_t dtype, int nseg, const mea_act_segment_t *segs,
+                                 void *workspace, size_t ws_bytes, mea_stream_t stream)
+{
+    Range range_("mea_act_bwd_grouped");
+    clear_error();
+    if (!valid_act(act)) return fail(MEA_ERR_INVALID_ARG, "act = %d is not a mea_act_t", (int)act);
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    std::vector<mea::ActSeg> tab;
+    mea_status_t st = grouped_segments("mea_act_bwd_grouped", nseg, segs, dtype, true, tab);
+    if (st != MEA_OK) return st;
+    if (nseg == 0) return MEA_OK;
+    const bool da = segs[0].dparam_dev != nullptr;
+    for (int i = 1; i < nseg; ++i)
+        if ((segs[i].dparam_dev != nullptr) != da)
+            return fail(MEA_ERR_INVALID_ARG, "mea_act_bwd_grouped: dparam_dev must be set in every segment or "
+                                             "in none (segment %d differs)", i);
+    if (da) {
+        if (act != MEA_SWISH)
+            return fail(MEA_ERR_UNSUPPORTED, "a parameter gradient exists only for MEA_SWISH (d alpha)");
+        const size_t need = mea_act_bwd_grouped_workspace_bytes(act, nseg, segs);
+        if (!workspace || ws_bytes < need)
+            return fail(MEA_ERR_WORKSPACE, "grouped d alpha needs %zu bytes of workspace, got %zu%s", need, ws_bytes,
+                        workspace ? "" : " (NULL)");
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return fail(MEA_ERR_WORKSPACE, "grouped workspace must be 256-byte aligned");
+        size_t off = 0;
+        for (int i = 0; i < nseg; ++i) {
+            tab[(size_t)i].ws = static_cast<char *>(workspace) + off;
+            off += round256(mea_act_bwd_workspace_bytes(act, segs[i].n, 1));
+        }
+    } else {
+        bool any = false;
+        for (int i = 0; i < nseg; ++i) any |= segs[i].n > 0;
+        if (!any) return MEA_OK;
+    }
+    mea::ActGroupLaunch l{act, dtype, nseg, tab.data(), reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = mea::launch_act_bwd_grouped(l);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_act_bwd_grouped launch");
+}
+
+mea_status_t mea_affine_bwd_wait_selftest(mea_dtype_t dtype, const int64_t shape[4], const void *x, const void *dy,
+                                          const float *gamma, const float *beta, void *dx, void *workspace,
+                                          size_t ws_bytes, int *expired, mea_stream_t stream)
+{
+    Range range_("mea_affine_bwd_wait_selftest");
+    clear_error();
+    if (!expired) return fail(MEA_ERR_INVALID_ARG, "expired is NULL");
+    *expired = 0;
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", (int)dtype);
+    int64_t n = 0;
+    mea_status_t st = check_shape(shape, &n);
+    if (st != MEA_OK) return st;
+    if (n == 0 || !x || !dy || !dx || !gamma || !beta)
+        return fail(MEA_ERR_INVALID_ARG, "the self-test needs a non-empty NHWC problem and every tensor pointer");
+    const size_t need = chan_ws_bytes(0, dtype, MEA_NHWC, shape);
+    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u))
+        return fail(MEA_ERR_WORKSPACE, "the self-test needs %zu bytes of 16-byte aligned workspace", need);
+    mea::AffineLaunch l{};
+    l.act = MEA_SWISH;
+    l.param = 1.f;
+    l.dtype = dtype;
+    l.layout = MEA_NHWC;
+    l.N = shape[0];
+    l.C = shape[1];
+    l.H = shape[2];
+    l.W = shape[3];
+    l.x = x;
+    l.dy = dy;
+    l.gamma = gamma;
+    l.beta = beta;
+    l.out = dx;
+    l.workspace = workspace;
+    l.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mea::launch_affine_bwd_wait_selftest(l);
+    if (e == cudaErrorNotSupported)
+        return fail(MEA_ERR_UNSUPPORTED, "this shape or alignment does not take the pipelined NHWC backward");
+    if (e == cudaSuccess) e = cudaStreamSynchronize(l.stream);
+    unsigned int word = 0;
+    unsigned int *err = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + 4);
+    if (e == cudaSuccess) e = cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "mea_affine_bwd_wait_selftest");
+    *expired = (int)word;
+    return MEA_OK;
+}
+
 size_t mea_affine_swish_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4])
 {
     return chan_ws_bytes(0, dtype, layout, shape);
@@ -278,6 +453,7 @@ size_t mea_affine_swish_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t layo
 mea_status_t mea_affine_swish_fwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
                                   const float *gamma, const float *beta, void *y, mea_stream_t stream)
 {
+    Range range_("mea_affine_swish_fwd");
     return chan_fwd(0, "mea_affine_swish_fwd", MEA_SWISH, dtype, layout, shape, x, gamma, beta, 1.f, y, stream);
 }
 
@@ -285,6 +461,7 @@ mea_status_t mea_affine_swish_bwd(mea_dtype_t dtype, mea_layout_t layout, const 
                                   const void *dy, const float *gamma, const float *beta, void *dx, float *dgamma,
                                   float *dbeta, void *workspace, size_t ws_bytes, mea_stream_t stream)
 {
+    Range range_("mea_affine_swish_bwd");
     return chan_bwd(0, "mea_affine_swish_bwd", MEA_SWISH, dtype, layout, shape, x, dy, gamma, beta, 1.f, dx, dgamma,
                     dbeta, workspace, ws_bytes, stream);
 }
@@ -298,6 +475,7 @@ mea_status_t mea_affine_act_fwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t l
                                 const void *x, const float *gamma, const float *beta, float param, void *y,
                                 mea_stream_t stream)
 {
+    Range range_("mea_affine_act_fwd");
     return chan_fwd(0, "mea_affine_act_fwd", act, dtype, layout, shape, x, gamma, beta, param, y, stream);
 }
 
@@ -306,6 +484,7 @@ mea_status_t mea_affine_act_bwd(mea_act_t act, mea_dtype_t dtype, mea_layout_t l
                                 void *dx, float *dgamma, float *dbeta, void *workspace, size_t ws_bytes,
                                 mea_stream_t stream)
 {
+    Range range_("mea_affine_act_bwd");
     return chan_bwd(0, "mea_affine_act_bwd", act, dtype, layout, shape, x, dy, gamma, beta, param, dx, dgamma, dbeta,
                     workspace, ws_bytes, stream);
 }
@@ -318,6 +497,7 @@ size_t mea_swish_channel_bwd_workspace_bytes(mea_dtype_t dtype, mea_layout_t lay
 mea_status_t mea_swish_channel_fwd(mea_dtype_t dtype, mea_layout_t layout, const int64_t shape[4], const void *x,
                                    const float *alpha, void *y, mea_stream_t stream)
 {
+    Range range_("mea_swish_channel_fwd");
     return chan_fwd(1, "mea_swish_channel_fwd", MEA_SWISH, dtype, layout, shape, x, alpha, nullptr, 1.f, y, stream);
 }
 
@@ -325,6 +505,7 @@ mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layout, const
                                    const void *dy, const float *alpha, void *dx, float *dalpha, void *workspace,
                                    size_t ws_bytes, mea_stream_t stream)
 {
+    Range range_("mea_swish_channel_bwd");
     return chan_bwd(1, "mea_swish_channel_bwd", MEA_SWISH, dtype, layout, shape, x, dy, alpha, nullptr, 1.f, dx,
                     dalpha, nullptr, workspace, ws_bytes, stream);
 }
@@ -344,6 +525,7 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 mea_status_t mea_matmul_act_fwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *x, const void *w,
                                 float param, void *z, void *y, mea_stream_t stream)
 {
+    Range range_("mea_matmul_act_fwd");
     clear_error();
     mea_status_t st = check_matmul("mea_matmul_act_fwd", act, M, N, K);
     if (st != MEA_OK) return st;
@@ -380,6 +562,7 @@ mea_status_t mea_matmul_act_fwd(mea_act_t act, int64_t M, int64_t N, int64_t K, 
 mea_status_t mea_matmul_act_bwd(mea_act_t act, int64_t M, int64_t N, int64_t K, const void *g, const void *w,
                                 const void *z, float param, void *dz, mea_stream_t stream)
 {
+    Range range_("mea_matmul_act_bwd");
     clear_error();
     mea_status_t st = check_matmul("mea_matmul_act_bwd", act, M, N, K);
     if (st != MEA_OK) return st;
@@ -463,6 +646,7 @@ mea_status_t mea_concat_bn_relu_fwd(mea_dtype_t dtype, int npieces, const void *
                                     float momentum, float *running_mean, float *running_var, float *mean,
                                     float *invstd, void *y, void *workspace, size_t ws_bytes, mea_stream_t stream)
 {
+    Range range_("mea_concat_bn_relu_fwd");
     clear_error();
     mea::BnLaunch l{};
     size_t pb = 0;
@@ -497,6 +681,7 @@ mea_status_t mea_concat_bn_relu_apply(mea_dtype_t dtype, int npieces, const void
                                       const float *beta, const float *mean, const float *invstd, void *y,
                                       mea_stream_t stream)
 {
+    Range range_("mea_concat_bn_relu_apply");
     clear_error();
     mea::BnLaunch l{};
     size_t pb = 0;
@@ -521,6 +706,7 @@ mea_status_t mea_concat_bn_relu_bwd(mea_dtype_t dtype, int npieces, const void *
                                     float *dgamma, float *dbeta, void *workspace, size_t ws_bytes,
                                     mea_stream_t stream)
 {
+    Range range_("mea_concat_bn_relu_bwd");
     clear_error();
     mea::BnLaunch l{};
     size_t pb = 0;

@@ -9,7 +9,11 @@
 //   Ch load(ChanArgs, c)   constants of channel c
 //   f<P>, f_tail<P>, is_tail      forward value, deep-tail recompute, test
 //   bwd<P>(x, dy, ..., o, t)      backward main path -> raw results o, t
-//   bwd_tail<P>(...)              deep-tail recompute of o, t
+//   flag_bwd<P>, bwd_tail<P>      per-element test for, and recompute of,
+//                                 every element a backward main path may flag
+//                                 (deep tails, packed-form overflow guards;
+//                                 with bf16 storage the neighbourhood of the
+//                                 zero of f')
 //   finish(x, o, t, ch, acc[NR])  dx, and adds the channel's reduction terms
 //   Ch2, pair(ch, ch), bwd2<P>, finish2   the same for two adjacent channels
 //                          in packed .f32x2 registers (pipelined backward)
@@ -311,7 +315,8 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
                 if (tail) {
 #pragma unroll
                     for (int j = 0; j < VE; ++j)
-                        if (Op::is_tail(xf[j], k, ch[j])) Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], t[j]);
+                        if (Op::template flag_bwd<P>(xf[j], k, ch[j]))
+                            Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], t[j]);
                 }
 #pragma unroll
                 for (int j = 0; j < VE; ++j) of[j] = Op::finish(xf[j], o[j], t[j], ch[j], accf[j]);
@@ -373,7 +378,12 @@ constexpr int kPipeMaxRegs = MEA_PIPE_MAXREGS;
 // fp64 sums (kPipeFlushTiles * UT terms per channel in fp32).
 constexpr int kPipeFlushTiles = 4;
 
-template <class Op, typename T, int VE, int UT>
+// kWaitOut: the bounded-wait self-test.  The producer announces each stage's
+// bytes but issues no copy, so no stage barrier ever completes (a flag that
+// nothing sets); every wait gives up after kMbarSpinsSelfTest polls, records
+// the error word and lets its role finish.  No copy is in flight when the
+// block exits, and dx is not written.
+template <class Op, typename T, int VE, int UT, bool kWaitOut = false>
 __global__ void __maxnreg__(kPipeMaxRegs)
 chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca,
                           void *__restrict__ dx, int64_t nunits, int groups, int C, int stages,
@@ -395,6 +405,7 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     const uint32_t tile_bytes = (uint32_t)(tile_units * UB);
     const int64_t ntiles = nunits / tile_units;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t spins = kWaitOut ? kMbarSpinsSelfTest : kMbarSpins;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -413,16 +424,18 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             int it = 0, s = 0;
             uint32_t phase = 0;
             for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-                if (it >= stages && !mbar_wait(smem_addr(empty + s), (phase & 1) ^ 1)) {
+                if (it >= stages && !mbar_wait(smem_addr(empty + s), (phase & 1) ^ 1, spins)) {
                     atomicExch(err, 1u);
                     break;
                 }
                 const uint32_t fb = smem_addr(full + s);
                 mbar_arrive_expect_tx(fb, 2 * tile_bytes);
-                unsigned char *bx = buf + (size_t)s * 2 * tile_bytes;
-                bulk_load(smem_addr(bx), static_cast<const unsigned char *>(x) + t * tile_bytes, tile_bytes, fb);
-                bulk_load(smem_addr(bx + tile_bytes), static_cast<const unsigned char *>(dy) + t * tile_bytes,
-                          tile_bytes, fb);
+                if constexpr (!kWaitOut) {
+                    unsigned char *bx = buf + (size_t)s * 2 * tile_bytes;
+                    bulk_load(smem_addr(bx), static_cast<const unsigned char *>(x) + t * tile_bytes, tile_bytes, fb);
+                    bulk_load(smem_addr(bx + tile_bytes), static_cast<const unsigned char *>(dy) + t * tile_bytes,
+                              tile_bytes, fb);
+                }
                 if (++s == stages) {
                     s = 0;
                     ++phase;
@@ -430,7 +443,7 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             }
             // Every issued copy lands before the block may exit.
             for (int j = it > stages ? it - stages : 0; j < it; ++j)
-                if (!mbar_wait(smem_addr(full + j % stages), (j / stages) & 1)) atomicExch(err, 1u);
+                if (!mbar_wait(smem_addr(full + j % stages), (j / stages) & 1, spins)) atomicExch(err, 1u);
         }
         return;
     }
@@ -485,17 +498,13 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             upk(t2, tt[2 * p], tt[2 * p + 1]);
         }
         if (tail) {
-            // the pairwise form may flag elements that are not deep-tail
-            // (it tests |t|): those are recomputed by the scalar form
+            // only the flagged elements: bwd_tail picks the near-zero,
+            // deep-tail or scalar form (the packed forms also flag elements
+            // whose products could overflow)
 #pragma unroll
-            for (int j = 0; j < VE; ++j) {
-                if (Op::is_tail(xf[j], k, ch[j])) {
+            for (int j = 0; j < VE; ++j)
+                if (Op::template flag_bwd<P>(xf[j], k, ch[j]))
                     Op::template bwd_tail<P>(xf[j], gf[j], k, ch[j], o[j], tt[j]);
-                } else {
-                    bool unused = false;
-                    Op::template bwd<P>(xf[j], gf[j], k, ch[j], unused, o[j], tt[j]);
-                }
-            }
         }
 #pragma unroll
         for (int p = 0; p < VE / 2; ++p)
@@ -509,7 +518,7 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     int it = 0, s = 0;
     uint32_t phase = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-        if (!mbar_wait(smem_addr(full + s), phase & 1)) {
+        if (!mbar_wait(smem_addr(full + s), phase & 1, spins)) {
             atomicExch(err, 1u);
             break;
         }
@@ -645,7 +654,8 @@ chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanA
                     if (tail) {
 #pragma unroll
                         for (int j = 0; j < VL; ++j)
-                            if (Op::is_tail(xf[j], k, ch)) Op::template bwd_tail<P>(xf[j], gf[j], k, ch, o[j], t[j]);
+                            if (Op::template flag_bwd<P>(xf[j], k, ch))
+                                Op::template bwd_tail<P>(xf[j], gf[j], k, ch, o[j], t[j]);
                     }
                     float tmp[NR];
 #pragma unroll
@@ -673,7 +683,7 @@ chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanA
             const double b = block_sum(acc[r], red);
             if (threadIdx.x == 0) partials[(r * C + c) * slices + s] = b;
         }
-        if (!last_block_done(ticket)) return;
+        if (!last_block_done(ticket, gridDim.x)) return;
         for (int64_t o = threadIdx.x; o < NR * C; o += blockDim.x) {
             double t = 0.0;
             for (int q = 0; q < slices; ++q) t += __ldcg(partials + o * slices + q);
@@ -829,6 +839,31 @@ cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out
                           a.stream, a.x, a.dy, ca, a.out, a.N, a.C, HW, slices, vec_ok, out0, out1, a.workspace);
     return launch_pdl(chan_plane_kernel<Op, T, MODE, false>, dim3((unsigned)grid), dim3(kPlaneThreads), 0, a.stream,
                       a.x, a.dy, ca, a.out, a.N, a.C, HW, slices, vec_ok, out0, out1, a.workspace);
+}
+
+// The bounded-wait self-test: the pipelined NHWC backward of Op with its
+// copies withheld (see kWaitOut).  cudaErrorNotSupported when the shape or
+// the alignment does not take the pipelined path.
+template <class Op, typename T>
+cudaError_t launch_channel_wait_selftest(const AffineLaunch &a, const ChanArgs &ca)
+{
+    if (!nhwc_fast<T>(a)) return cudaErrorNotSupported;
+    constexpr int VE = NhwcCfg<T>::VE;
+    const int groups = (int)(a.C / VE);
+    const int threads = nhwc_threads(groups);
+    const int64_t nunits = a.N * a.C * a.H * a.W / VE;
+    const bool bulk_ok = ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.dy)) & 15u) == 0;
+    const PipeShape ps = pipe_shape<T>(Op::NR, nunits, threads);
+    if (!bulk_ok || ps.stages <= 0) return cudaErrorNotSupported;
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+    unsigned int *err = reinterpret_cast<unsigned int *>(static_cast<char *>(a.workspace) + 4);
+    auto kernel = chan_nhwc_bwd_pipe_kernel<Op, T, VE, NhwcCfg<T>::U_PIPE, true>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ps.smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, dim3((unsigned)ps.grid), dim3(threads + 32), ps.smem, a.stream, a.x, a.dy, ca, a.out,
+                      nunits, groups, (int)a.C, ps.stages, partials, err);
 }
 
 }  // namespace mea

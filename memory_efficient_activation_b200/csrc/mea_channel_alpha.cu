@@ -32,6 +32,13 @@ struct ChannelSwishOp {
         return Swish::f_tail<P>(x, h);
     }
     static __device__ __forceinline__ bool is_tail(float x, const K &, const Ch &h) { return Swish::is_tail(x, h); }
+    // Every element the backward main path may flag (deep tail; with bf16
+    // storage the neighbourhood of the zero of f').
+    template <bool P>
+    static __device__ __forceinline__ bool flag_bwd(float x, const K &, const Ch &h)
+    {
+        return Swish::bwd_flagged<P>(x, h);
+    }
     // o = dx, t = d alpha term
     template <bool P>
     static __device__ __forceinline__ void bwd(float x, float dy, const K &, const Ch &h, bool &tail, float &o,
@@ -39,10 +46,17 @@ struct ChannelSwishOp {
     {
         o = Swish::df_da<P>(x, dy, h, tail, t);
     }
+    // A flagged element: the near-zero or deep-tail recompute, else the main
+    // form.
     template <bool P>
     static __device__ __forceinline__ void bwd_tail(float x, float dy, const K &, const Ch &h, float &o, float &t)
     {
-        o = Swish::df_da_tail<P>(x, dy, h, t);
+        if (Swish::is_tail_bwd<P>(x, h)) {
+            o = Swish::df_da_tail<P>(x, dy, h, t);
+            return;
+        }
+        bool unused = false;
+        o = Swish::df_da<P>(x, dy, h, unused, t);
     }
     static __device__ __forceinline__ float finish(float, float o, float t, const Ch &, float (&acc)[NR])
     {

@@ -31,6 +31,9 @@ struct AffineLaunch {
 size_t affine_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
 cudaError_t launch_affine_fwd(const AffineLaunch &a);
 cudaError_t launch_affine_bwd(const AffineLaunch &a);
+// The bounded-wait self-test (affine + Swish, NHWC pipelined backward with its
+// copies withheld); cudaErrorNotSupported off the pipelined path.
+cudaError_t launch_affine_bwd_wait_selftest(const AffineLaunch &a);
 size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64_t C, int64_t H, int64_t W);
 cudaError_t launch_channel_swish_fwd(const AffineLaunch &a);
 cudaError_t launch_channel_swish_bwd(const AffineLaunch &a);

@@ -167,14 +167,14 @@ __device__ __forceinline__ double block_sum(double v, double *red)
 // that finishes last (after all other blocks have published their partials
 // with a fence).  The counter wraps back to zero, leaving the workspace as
 // it was found.  Nothing waits.
-__device__ __forceinline__ bool last_block_done(unsigned int *ticket)
+__device__ __forceinline__ bool last_block_done(unsigned int *ticket, unsigned int nblk)
 {
     __shared__ int is_last;
     __threadfence();          // every thread's partial stores are visible device-wide
     __syncthreads();
     if (threadIdx.x == 0) {
-        unsigned int t = atomicInc(ticket, gridDim.x - 1);
-        is_last = (t == gridDim.x - 1);
+        unsigned int t = atomicInc(ticket, nblk - 1);
+        is_last = (t == nblk - 1);
     }
     __syncthreads();
     const bool last = is_last != 0;

@@ -50,6 +50,34 @@ struct ActLaunch {
 cudaError_t launch_act_fwd(const ActLaunch &a);
 cudaError_t launch_act_bwd(const ActLaunch &a);
 
+// One tensor of a grouped launch (act_group_kernel).
+struct ActSeg {
+    const void *x;
+    const void *dy;          // backward only
+    void *out;               // y or dx
+    int64_t n;
+    const float *param_dev;  // nullable
+    float *dparam;           // nullable (Swish d alpha: every segment or none)
+    void *ws;                // this segment's ticket + fp64 partials (d alpha)
+    float param;
+    int vec_ok;              // set by the launcher
+};
+constexpr int kMaxSegs = 32;  // segments per launch (the table is passed as a kernel parameter)
+struct ActSegTable {
+    ActSeg seg[kMaxSegs];
+    int start[kMaxSegs + 1];  // first block of each segment; start[nseg] is the grid
+    int nseg;
+};
+struct ActGroupLaunch {
+    int act;
+    int dtype;
+    int nseg;                 // any count: launched kMaxSegs at a time
+    const ActSeg *segs;
+    cudaStream_t stream;
+};
+cudaError_t launch_act_fwd_grouped(const ActGroupLaunch &a);
+cudaError_t launch_act_bwd_grouped(const ActGroupLaunch &a);
+
 // Launch with programmatic stream serialisation: the kernel may begin while
 // the previous kernel on the stream drains, and waits (pdl_wait) before it
 // touches memory.  Returns the launch's cudaError_t.

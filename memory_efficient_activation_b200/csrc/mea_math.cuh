@@ -130,8 +130,50 @@ __device__ __forceinline__ void scaled_log2e(float m, float &hi, float &lo)
     lo = fmaf(m, kLog2eLo, fmaf(m, kLog2eHi, -hi));
 }
 
+// ------------------------------------------------- near the zero of f'
+// Swish' (as a function of v = alpha x), GELU-erf' and GELU-tanh' each vanish
+// at one point v0 < 0, where the terms of f' cancel.  The main paths form
+// the argument with one fp32 rounding (alpha x, or gamma x + beta in the
+// per-channel kernels) and evaluate f' in fp32: an absolute error of about
+// 1.5e-7 (times |dy|), which within about 1e-4 of v0 is a large part of f'
+// itself.  With bf16 storage every output must stay within one bf16 ulp of
+// the exact result, so there the elements with |v - v0| < kRootWin are
+// recomputed from d = v - v0 formed in fp64 (root_d), as the Taylor
+// polynomial
+//   f'(v0 + d) = d (f''(v0) + d f'''(v0) / 2),
+// whose next term is below 1e-7 of f' over the window.  Outside the window
+// |f'| > 2.1e-4, so the main path's error stays below 1e-3 of f', inside half
+// a bf16 ulp.  The constants (v0 in fp64 and its fp32 rounding for the
+// window test, f''(v0), f'''(v0) / 2) come from csrc/near_root_constants.py.
+// fp32 storage keeps the main path: its rule is relative to the condition
+// scale of f', which that error meets.
+constexpr float kRootWin = 0.0009765625f;   // 2^-10
+
+// d = m (g x + b) - v0 in fp64: g x is exact there, each FMA rounds once
+// (2^-53 relative) and v0 is held to 2^-53, so d carries an absolute error
+// below 5e-16 and the recomputed f' is within a bf16 half-ulp of the exact
+// value wherever |d| > 2e-13.  Taken only for the few elements inside the
+// window.
+__device__ __forceinline__ float root_d(float g, float x, float b, float m, double v0)
+{
+    const double z = fma((double)g, (double)x, (double)b);
+    return (float)fma((double)m, z, -v0);
+}
+
+// dy f'(v0 + d) from the Taylor polynomial of activation A at its zero.
+template <class A>
+__device__ __forceinline__ float root_df(float d, float dy)
+{
+    return dy * (d * fmaf(A::kRootF3h, d, A::kRootF2));
+}
+
 // ------------------------------------------------------------------ ReLU
 struct ReLU {
+    static constexpr bool kHasRoot = false;
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float, const Coef &) { return false; }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
     static __device__ __forceinline__ Coef coef(float) { return Coef{0.f, 0.f, 0.f}; }
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &, bool &)
@@ -152,6 +194,11 @@ struct ReLU {
 
 // ------------------------------------------------------------- LeakyReLU
 struct LeakyReLU {
+    static constexpr bool kHasRoot = false;
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float, const Coef &) { return false; }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
     static __device__ __forceinline__ Coef coef(float slope) { return Coef{slope, 0.f, 0.f}; }
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &k, bool &)
@@ -173,6 +220,12 @@ struct LeakyReLU {
 // -------------------------------------------------------------- Sigmoid
 // t = -x log2 e; s = 1 / (1 + 2^t).
 struct Sigmoid {
+    static constexpr bool kHasRoot = false;
+    // Every element a backward main path flags (df: |t| > kTailT).
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float x, const Coef &k) { return fabsf(x * k.c_hi) > kTailT; }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
     static __device__ __forceinline__ Coef coef(float)
     {
         Coef k;
@@ -249,6 +302,12 @@ struct Sigmoid {
 // Sigmoid(-2|x|) = 4 E s^2 with E = 2^t, t = -2|x| log2 e (t <= 0),
 // s = 1/(1+E) = Sigmoid(2|x|) and Sigmoid(-2|x|) = E s.
 struct Tanh {
+    static constexpr bool kHasRoot = false;
+    // Every element a backward main path flags (df: t < -120).
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float x, const Coef &k) { return fabsf(x) * k.c_hi < -120.f; }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
     static __device__ __forceinline__ Coef coef(float)
     {
         Coef k;
@@ -327,6 +386,19 @@ struct Tanh {
 // that exponential's argument (-w^2 log2 e < -124); the deep-tail recompute
 // is the scaled form above.
 struct GeluErf {
+    // Zero of f' (Phi(x) + x phi(x) = 0) for the compensated recompute of the
+    // per-channel kernels; the plain kernels see x exactly, and the bf16 x
+    // nearest the zero keep |f'| >= 7e-4, so they need none.
+    static constexpr bool kHasRoot = true;
+    static constexpr double kRootD = -0.75179152469356445746;
+    static constexpr float kRootHi = -0.7517915368080139f;      // fp32(kRootD)
+    static constexpr float kRootF2 = 0.43149399757385254f;
+    static constexpr float kRootF3h = 0.38828498125076294f;
+    static __device__ __forceinline__ float root_scale(const Coef &) { return 1.f; }
+    static __device__ __forceinline__ bool near_root(float z, const Coef &)
+    {
+        return fabsf(__fsub_rn(z, kRootHi)) < kRootWin;
+    }
     static constexpr float kNegRsqrt2Hi = -0.707106769084930419921875f;
     static constexpr float kNegRsqrt2Lo = -1.2101617104478969362e-08f;
     static constexpr float kTwoRsqrtPi = 1.12837916709551257f;     // 2 / sqrt(pi)
@@ -391,12 +463,22 @@ struct GeluErf {
         p = fmaf(p, t, -1.26654184f);
         return fmaf(-a, a, p) * kLog2ef;
     }
-    static __device__ __forceinline__ bool is_tail(float x, const Coef &)
+    // The bf16 main paths serve x >= kTailX, where every exponential they take
+    // (down to 2^-113 for the Gaussian, about 2^-115 for erfc) stays normal
+    // and a = |x| / sqrt 2 stays inside the range the fitted polynomials were
+    // fitted on (a <= 9.6, x >= -13.6); the elements below are recomputed with
+    // the exponentials scaled by 2^64.  One comparison, so that the per-element
+    // test of the recompute loops costs next to nothing.
+    static constexpr float kTailX = -12.5f;
+    static __device__ __forceinline__ bool is_tail(float x, const Coef &) { return x < kTailX; }
+    // Every element a backward main path flags (bf16 only: x < kTailX).
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float x, const Coef &k)
     {
-        if (!(x < 0.f)) return false;
-        float t;
-        return nr_parts(x * kNegRsqrt2Hi, t) < -kTailT;
+        return !P && is_tail(x, k);
     }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
 
     // returns erfc(-x / sqrt 2) and sets g = e^(-x^2 / 2) (accurate path)
     static __device__ __forceinline__ float erfc_and_gauss_precise(float x, float &g)
@@ -463,7 +545,7 @@ struct GeluErf {
         F2 t, u;
         nr5_parts2(x, w0, w1, t, u);
         upk(u, u0, u1);
-        tail |= ((u0 < -kTailT) && (x0 < 0.f)) || ((u1 < -kTailT) && (x1 < 0.f));
+        tail |= (x0 < kTailX) | (x1 < kTailX);
         upk(mul2(mul2(sp2(0.5f), x), erfc2(w0, w1, t, u0, u1)), o0, o1);
     }
     static __device__ __forceinline__ void df2(float x0, float x1, float dy0, float dy1, const Coef &, bool &tail,
@@ -480,7 +562,7 @@ struct GeluErf {
         const F2 q = q8_2(t);
         float v0, v1;
         upk(mul2(mul2(w, w), sp2(-kLog2ef)), v0, v1);
-        tail |= ((v0 < -kTailT) && (x0 < 0.f)) || ((v1 < -kTailT) && (x1 < 0.f));
+        tail |= (x0 < kTailX) | (x1 < kTailX);
         const F2 g = pk(ex2_ftz(v0), ex2_ftz(v1));
         float a0, a1;
         upk(mul2(mul2(t, q), g), a0, a1);
@@ -500,7 +582,7 @@ struct GeluErf {
             const float w = x * kNegRsqrt2Hi;
             float t;
             const float u = nr5_parts(fabsf(w), t);
-            tail |= (u < -kTailT) && (x < 0.f);
+            tail |= x < kTailX;
             const float ans = t * ex2_ftz(u);
             const float ec = w >= 0.f ? ans : 2.f - ans;
             return (0.5f * x) * ec;
@@ -532,7 +614,7 @@ struct GeluErf {
             const float t = rcp_ftz(fmaf(0.5f, fabsf(w), 1.0f));
             const float q = q8(t);
             const float v = (w * w) * -kLog2ef;
-            tail |= (v < -kTailT) && (x < 0.f);
+            tail |= x < kTailX;
             const float g = ex2_ftz(v);
             const float ans = (t * q) * g;
             const float ec = w >= 0.f ? ans : 2.f - ans;
@@ -567,6 +649,24 @@ struct HasPairs<GeluErf, false> {
 // t = -v log2 e = x (c1 + c3 x^2).  Backward:
 // Sigmoid(v) + x v' Sigmoid(v) Sigmoid(-v), v' = k1 + 3 k3 x^2.
 struct GeluTanh {
+    // Zero of f' (as for GeluErf: used by the per-channel kernels only).
+    static constexpr bool kHasRoot = true;
+    static constexpr double kRootD = -0.75246142207101625849;
+    static constexpr float kRootHi = -0.7524614334106445f;      // fp32(kRootD)
+    static constexpr float kRootF2 = 0.4304001033306122f;
+    static constexpr float kRootF3h = 0.38751843571662903f;
+    static __device__ __forceinline__ float root_scale(const Coef &) { return 1.f; }
+    // Tested on the exponent t = z (c1 + c3 z^2) as the bf16 forms compute it
+    // (see SwishT): v0 maps to kRootT, 2^-10 in z to kRootWinT, and the packed
+    // backward's u = t - kRootT serves both of its guards.
+    static constexpr float kRootT = 1.7761809825897217f;
+    static constexpr float kRootWinT = 0.0024190107360482216f;
+    static constexpr float kTailU = 122.0f;
+    static __device__ __forceinline__ bool near_root(float z, const Coef &)
+    {
+        float tl;
+        return fabsf(__fsub_rn(expo_arg<false>(z, tl), kRootT)) < kRootWinT;
+    }
     static constexpr double kK1 = 1.5957691216057307;            // 2 sqrt(2/pi)
     static constexpr double kK3 = 1.5957691216057307 * 0.044715;
     static constexpr float kK1f = (float)kK1;
@@ -595,6 +695,20 @@ struct GeluTanh {
     {
         float tl;
         return expo_arg<false>(x, tl) > kTailT;
+    }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
+    // Every element a backward main path flags: t > kTailT (scalar form);
+    // for bf16, |u| < kRootWinT or |u| > kTailU, u = t - kRootT (the packed
+    // form of the per-channel kernels, which contains the scalar one's).
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float x, const Coef &)
+    {
+        float tl;
+        const float t = expo_arg<P>(x, tl);
+        if constexpr (P) return t > kTailT;
+        const float u = __fsub_rn(t, kRootT);
+        return fabsf(u) < kRootWinT || fabsf(u) > kTailU;
     }
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &, bool &tail)
@@ -651,7 +765,39 @@ struct GeluTanh {
 // ---------------------------------------------------------------- Swish
 // y = x Sigmoid(z), z = alpha x; t = x c, c = -alpha log2 e (float-float).
 // dx = dy (s + z s Sigmoid(-z)); d alpha term = dy x^2 s Sigmoid(-z).
-struct Swish {
+// RC: whether the bf16 backward recomputes the neighbourhood of the zero of
+// f' (see "near the zero of f'").  Swish (RC = true) is the general form.
+// With alpha a power of two (or zero) and bf16 x, alpha x is exact and lies
+// on the bf16 grid scaled by 2^k, which is the bf16 grid again, so the
+// inputs nearest v0 keep |f'| >= 6e-4 and the main path is within one ulp:
+// the streaming kernels then use SwishT<false>, without the test.
+template <bool RC>
+struct SwishT {
+    // Zero of Swish_1'(v) = Sigmoid(v) + v Sigmoid(v) Sigmoid(-v), at
+    // v0 = -(1 + W(1/e)); x Sigmoid(alpha x) has x-derivative Swish_1'(alpha x),
+    // so an element is near it when alpha x is.  With alpha = 1 and bf16 x the
+    // nearest inputs keep |f'| >= 6e-4; any other alpha can put alpha x
+    // anywhere, hence the compensated recompute (bf16 storage).
+    static constexpr bool kHasRoot = RC;
+    static constexpr double kRootD = -1.2784645427610737951;
+    static constexpr float kRootHi = -1.2784645557403564f;      // fp32(kRootD)
+    static constexpr float kRootF2 = 0.2178117036819458f;
+    static constexpr float kRootF3h = 0.14664879441261292f;
+    // The window is tested on the sigmoid's exponent variable t = x c_hi =
+    // -alpha x log2(e) (rounded once, as every main path forms it): v0 maps to
+    // kRootT and 2^-10 in v to kRootWinT.  The packed backward then takes one
+    // u = t - kRootT for both of its guards: |u| < kRootWinT (near v0) and
+    // |u| > kTailU, which contains |t| > kTailT.
+    static constexpr float kRootT = 1.8444344997406006f;      // -v0 log2(e)
+    static constexpr float kRootWinT = 0.001408881857059896f; // 2^-10 log2(e)
+    static constexpr float kTailU = 122.0f;
+    static __device__ __forceinline__ float root_scale(const Coef &k) { return k.p; }
+    static __device__ __forceinline__ bool near_root(float z, const Coef &k)
+    {
+        return fabsf(__fsub_rn(__fmul_rn(z, k.c_hi), kRootT)) < kRootWinT;
+    }
+    // d = alpha x - v0
+    static __device__ __forceinline__ float root_dx(float x, const Coef &k) { return root_d(1.f, x, 0.f, k.p, kRootD); }
     static __device__ __forceinline__ Coef coef(float alpha)
     {
         Coef k;
@@ -676,6 +822,25 @@ struct Swish {
         return s64;
     }
     static __device__ __forceinline__ bool is_tail(float x, const Coef &k) { return x * k.c_hi > kTailT; }
+    template <bool P>
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k)
+    {
+        if constexpr (!P && RC) return is_tail(x, k) || near_root(x, k);
+        return is_tail(x, k);
+    }
+    // Every element a backward main path flags: t > kTailT (scalar form),
+    // |t| > kTailT (the packed bf16 form of the per-channel kernels), and with
+    // bf16 storage the neighbourhood of the zero of f'.
+    template <bool P>
+    static __device__ __forceinline__ bool bwd_flagged(float x, const Coef &k)
+    {
+        if constexpr (!P && RC) {
+            const float u = __fsub_rn(__fmul_rn(x, k.c_hi), kRootT);
+            return fabsf(u) < kRootWinT || fabsf(u) > kTailU;
+        }
+        if constexpr (!P) return fabsf(x * k.c_hi) > kTailT;
+        return x * k.c_hi > kTailT;
+    }
 
     template <bool P>
     static __device__ __forceinline__ float f(float x, const Coef &k, bool &tail)
@@ -697,14 +862,20 @@ struct Swish {
         float E = expo<P>(x, k, t);
         tail |= t > kTailT;
         float s = rcp_ftz(1.f + E);
-        float z = k.p * x;
+        float z = __fmul_rn(k.p, x);
+        if constexpr (!P && RC) tail |= fabsf(__fsub_rn(t, kRootT)) < kRootWinT;
         float sm = z > 0.f ? E * s : 1.f - s;
         z = fminf(z, kBig);
         return dy * fmaf(z * s, sm, s);
     }
+    // Elements flagged by df: near the zero of f' (bf16 storage), or the deep
+    // negative tail.
     template <bool P>
     static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
     {
+        if constexpr (!P && RC) {
+            if (near_root(x, k)) return root_df<SwishT>(root_dx(x, k), dy);
+        }
         float z = fmaxf(k.p * x, -kBig);
         return ((dy * tail_s64<P>(x, k)) * (1.f + z)) * kTwoM64;
     }
@@ -717,20 +888,31 @@ struct Swish {
         float E = expo<P>(x, k, t);
         tail |= t > kTailT;
         float s = rcp_ftz(1.f + E);
-        float z = k.p * x;
+        float z = __fmul_rn(k.p, x);
+        if constexpr (!P && RC) tail |= fabsf(__fsub_rn(t, kRootT)) < kRootWinT;
         float sm = z > 0.f ? E * s : 1.f - s;
         term = (((x * s) * sm) * x) * dy;
         z = fminf(z, kBig);
         return dy * fmaf(z * s, sm, s);
     }
+    // As df_tail; near the zero of f' the d alpha term (a product, which does
+    // not cancel) keeps its main-path value.
     template <bool P>
     static __device__ __forceinline__ float df_da_tail(float x, float dy, const Coef &k, float &term)
     {
+        if constexpr (!P && RC) {
+            if (near_root(x, k)) {
+                bool unused = false;
+                (void)df_da<P>(x, dy, k, unused, term);
+                return root_df<SwishT>(root_dx(x, k), dy);
+            }
+        }
         float s64 = tail_s64<P>(x, k);
         float z = fmaxf(k.p * x, -kBig);
         term = (((x * s64) * x) * dy) * kTwoM64;
         return ((dy * s64) * (1.f + z)) * kTwoM64;
     }
 };
+using Swish = SwishT<true>;
 
 }  // namespace mea

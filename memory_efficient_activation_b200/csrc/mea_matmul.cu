@@ -214,7 +214,8 @@ __device__ __forceinline__ void epilogue32(const uint32_t (&acc)[32], const Coef
         if (tail) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (A::is_tail(zr[j], k)) r[j] = A::template df_tail<false>(zr[j], __uint_as_float(acc[j]), k);
+                if (A::template is_tail_bwd<false>(zr[j], k))
+                    r[j] = A::template df_tail<false>(zr[j], __uint_as_float(acc[j]), k);
         }
     }
     uint32_t rb[16];

@@ -12,19 +12,22 @@
 // exits.
 //
 // Host code cannot use the array's name as a device address (on the host it
-// names a host-side stand-in), so the device address is looked up with
-// cudaGetSymbolAddress once per device, with that device current, on the
-// first call made while it is current; that first call should come before
-// any stream capture.  The array is shared by every call on a device and
+// names a host-side stand-in), so every call looks the device address up with
+// cudaGetSymbolAddress on the current device.  Looking it up per call rather
+// than caching it keeps the address right after a device reset (which
+// reloads the library's device code at a new address).  The first call on a
+// device may load that code, so it should come before any stream capture.
+// The array is shared by every call on a device and
 // keeps whatever the last call left in it; the completion counter at its
 // start is cleared (cudaMemsetAsync on the caller's stream) before every
 // launch.  Calls whose kernels overlap on the GPU (different streams, no
 // ordering between them) race on the array and must not be issued.
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdint>
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/mea.h"
 #include "mea_internal.h"
@@ -37,25 +40,13 @@ static __device__ __align__(256) unsigned char g_dalpha_scratch[kNoAllocScratchB
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch on the current device (looked up once).
+// Device address of the scratch on the current device.
 cudaError_t scratch_for_current_device(void **out)
 {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_dalpha_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_dalpha_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -67,10 +58,24 @@ namespace mea {
 void set_last_error_detail(const char *detail);
 }  // namespace mea
 
+static mea_status_t noalloc_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const void *dy, void *dx,
+                                int64_t n, float param, const float *param_dev, float *dparam_dev,
+                                mea_stream_t stream);
+
 extern "C" mea_status_t mea_act_bwd_dparam_noalloc(mea_act_t act, mea_dtype_t dtype, const void *x,
                                                    const void *dy, void *dx, int64_t n, float param,
                                                    const float *param_dev, float *dparam_dev,
                                                    mea_stream_t stream)
+{
+    nvtxRangePushA("mea_act_bwd_dparam_noalloc");
+    const mea_status_t st = noalloc_bwd(act, dtype, x, dy, dx, n, param, param_dev, dparam_dev, stream);
+    nvtxRangePop();
+    return st;
+}
+
+static mea_status_t noalloc_bwd(mea_act_t act, mea_dtype_t dtype, const void *x, const void *dy, void *dx,
+                                int64_t n, float param, const float *param_dev, float *dparam_dev,
+                                mea_stream_t stream)
 {
     // Without d alpha there is no reduction and no scratch: a plain backward.
     if (!dparam_dev)

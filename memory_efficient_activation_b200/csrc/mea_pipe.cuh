@@ -15,6 +15,8 @@ namespace mea {
 
 constexpr uint32_t kMbarSpins = 1u << 22;
 constexpr uint32_t kMbarSuspendNs = 1000;
+// The limit of the bounded-wait self-test (a few milliseconds at most).
+constexpr uint32_t kMbarSpinsSelfTest = 1u << 12;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -34,9 +36,9 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t spins = kMbarSpins)
 {
-    for (uint32_t i = 0; i < kMbarSpins; ++i) {
+    for (uint32_t i = 0; i < spins; ++i) {
         uint32_t done;
         asm volatile(
             "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"

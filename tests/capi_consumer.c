@@ -53,6 +53,34 @@ int main(void)
     CHECK(mea_act_bwd(MEA_RELU, MEA_BF16, x, dy, dx, 1000, 1.0f, NULL, dparam, ws, need, NULL) ==
           MEA_ERR_UNSUPPORTED);
 
+    /* grouped calls: counts, NULL tables, overlapping segments, d alpha in
+     * some segments only, workspace size */
+    {
+        mea_act_segment_t segs[3];
+        memset(segs, 0, sizeof(segs));
+        segs[0].x = x; segs[0].dy = dy; segs[0].out = dx; segs[0].n = 1000; segs[0].param = 1.0f;
+        segs[1].x = y; segs[1].dy = (char *)dy + 8192; segs[1].out = (char *)dx + 8192; segs[1].n = 10;
+        segs[2].x = (char *)x + 8192; segs[2].dy = (char *)dy + 16384; segs[2].out = (char *)dx + 16384;
+        segs[2].n = 0;
+        CHECK(mea_act_fwd_grouped(MEA_SWISH, MEA_BF16, 0, NULL, NULL) == MEA_OK);
+        CHECK(mea_act_fwd_grouped(MEA_SWISH, MEA_BF16, -1, segs, NULL) == MEA_ERR_INVALID_ARG);
+        CHECK(mea_act_fwd_grouped(MEA_SWISH, MEA_BF16, 2, NULL, NULL) == MEA_ERR_INVALID_ARG);
+        CHECK(mea_act_bwd_grouped((mea_act_t)8, MEA_BF16, 2, segs, NULL, 0, NULL) == MEA_ERR_INVALID_ARG);
+        segs[1].out = (char *)dx + 100;   /* overlaps segment 0's dx */
+        CHECK(mea_act_bwd_grouped(MEA_SWISH, MEA_BF16, 2, segs, NULL, 0, NULL) == MEA_ERR_INVALID_ARG);
+        segs[1].out = (char *)dx + 8192;
+        segs[0].dparam_dev = dparam;      /* d alpha in one segment only */
+        CHECK(mea_act_bwd_grouped(MEA_SWISH, MEA_BF16, 2, segs, ws, 1 << 20, NULL) == MEA_ERR_INVALID_ARG);
+        segs[1].dparam_dev = dparam + 1;
+        segs[2].dparam_dev = dparam + 2;
+        need = mea_act_bwd_grouped_workspace_bytes(MEA_SWISH, 3, segs);
+        CHECK(need >= 3 * 256 && need % 256 == 0);
+        CHECK(mea_act_bwd_grouped(MEA_SWISH, MEA_BF16, 3, segs, ws, need - 1, NULL) == MEA_ERR_WORKSPACE);
+        CHECK(mea_act_bwd_grouped(MEA_SWISH, MEA_BF16, 3, segs, (char *)ws + 16, need, NULL) ==
+              MEA_ERR_WORKSPACE);
+        CHECK(mea_act_bwd_grouped(MEA_RELU, MEA_BF16, 3, segs, ws, need, NULL) == MEA_ERR_UNSUPPORTED);
+    }
+
     /* per-channel entry points */
     need = mea_affine_swish_bwd_workspace_bytes(MEA_BF16, MEA_NHWC, shape);
     CHECK(need > 0);

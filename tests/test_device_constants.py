@@ -15,6 +15,7 @@ import os
 import re
 
 import numpy as np
+import pytest
 from scipy.special import erfcx
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -100,3 +101,46 @@ def test_q8_bound_and_fit():
     coef, ferr = mod.fit_q(points=100001, iterations=100)
     assert np.allclose(coef, np.array(c[::-1], dtype=np.float32), rtol=1e-4, atol=1e-6), (coef, c)
     assert ferr < 1e-7                      # a shorter refit, less converged
+
+
+# ------------------------------------------------ zeros of f' (near-root recompute)
+
+def _root_constants(struct: str) -> dict:
+    """kRootD, kRootHi, kRootF2, kRootF3h of `struct` in mea_math.cuh."""
+    text = open(SRC).read()
+    head = f"struct {struct} {{" if struct != "Swish" else "struct SwishT {"
+    body = text[text.index(head):]
+    body = body[:body.index("root_scale")]
+    out = {}
+    for name in ("kRootD", "kRootHi", "kRootF2", "kRootF3h"):
+        m = re.search(name + r" = ([-0-9.eE]+)f?;", body)
+        out[name] = float(m.group(1))
+    return out
+
+
+@pytest.mark.parametrize("struct,act,alpha", [("Swish", "swish", 1.0), ("GeluErf", "gelu_erf", 1.0),
+                                              ("GeluTanh", "gelu_tanh", 1.0)])
+def test_root_constants_against_oracle_derivative(struct, act, alpha):
+    # The zero of f' and the Taylor coefficients there, checked against the
+    # oracle's f' (itself pinned by closed forms, finite differences and
+    # torch autograd): f'(v0) vanishes to double rounding, f'' and f'''/2 by
+    # central differences of f'.
+    import oracle
+    c = _root_constants(struct)
+    v0 = c["kRootD"]
+    assert np.float32(v0) == np.float32(c["kRootHi"])
+    d = lambda v: oracle.act_deriv(act, np.asarray(v, dtype=np.float64), alpha)   # noqa: E731
+    assert abs(d([v0])[0]) < 1e-15
+    h = 1e-4
+    fm, f0, fp = d([v0 - h, v0, v0 + h])
+    f2 = (fp - fm) / (2 * h)
+    f3h = (fp - 2 * f0 + fm) / (h * h) / 2
+    assert abs(c["kRootF2"] - f2) <= 1e-6 * abs(f2)
+    assert abs(c["kRootF3h"] - f3h) <= 1e-5 * abs(f3h)
+
+
+def test_swish_root_is_lambert_w():
+    # v0 = -(1 + W(1/e)) (the zero of s + v s (1 - s))
+    from scipy.special import lambertw
+    c = _root_constants("Swish")
+    assert abs(c["kRootD"] + 1.0 + float(lambertw(np.exp(-1.0)).real)) < 1e-15

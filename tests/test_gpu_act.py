@@ -230,3 +230,78 @@ def test_host_pipelined_matches_device_calls(n, chunks):
     dx = mea.act_bwd("gelu_tanh", x.cuda(), dy.cuda())
     torch.cuda.synchronize()
     assert torch.equal(hy, y.cpu()) and torch.equal(hdx, dx.cpu())
+
+
+# The zero of Swish'(v), v = alpha x: v0 = -(1 + W(1/e)).
+SWISH_V0 = -1.2784645427610737951
+
+
+@pytest.mark.parametrize("x0", [-1.0, -1.5, -0.75, -2.5, -0.3125])
+def test_bf16_swish_alpha_at_zero_of_derivative(x0):
+    # alpha = fp32(v0 / x0) puts alpha x0 within an fp32 rounding of the zero
+    # of f' (|f'| ~ 1e-8 there), and every other bf16 x is swept as well: the
+    # backward must still be within one bf16 ulp of the exact dy f'(x)
+    alpha = float(np.float32(SWISH_V0 / x0))
+    x = synthetic.all_finite_bf16()
+    for g in (1.0, -0.75):
+        dy = torch.full_like(x, g)
+        _check_pair("swish", "bf16", x, dy, alpha, f"swish alpha={alpha} (zero of f' at x={x0}), dy={g}")
+    # the same inputs through the d alpha variant of the backward
+    xs = x.cuda()
+    dy = torch.full_like(xs, -0.75)
+    da = torch.empty(1, dtype=torch.float32, device="cuda")
+    dx = mea.act_bwd("swish", xs, dy, alpha, dparam=da)
+    torch.cuda.synchronize()
+    xd = to_f64(x)
+    gd = np.full(xd.size, -0.75)
+    check("bf16", dx.cpu(), oracle.act_bwd("swish", xd, gd, alpha), what="swish d alpha variant dx")
+
+
+@pytest.mark.parametrize("alpha", [1.0, 0.5, -2.0])
+def test_bf16_swish_exact_scale_forms_agree(alpha):
+    # With alpha = 0 or +-2^k and bf16 x the kernels skip the near-zero test
+    # (alpha x is exact there); a device-side alpha always takes the general
+    # form.  Both must give the same bits on every finite bf16 x, with and
+    # without d alpha.
+    x = synthetic.all_finite_bf16().cuda()
+    dy = torch.full_like(x, -0.75)
+    a_dev = torch.tensor([alpha], dtype=torch.float32, device="cuda")
+    dx_host = mea.act_bwd("swish", x, dy, alpha)
+    dx_dev = mea.act_bwd("swish", x, dy, 0.0, param_dev=a_dev)
+    da_h = torch.empty(1, dtype=torch.float32, device="cuda")
+    da_d = torch.empty(1, dtype=torch.float32, device="cuda")
+    fin = torch.isfinite(x.float()) & (x.float().abs() < 1e4)
+    xs, gs = x[fin].contiguous(), dy[fin].contiguous()
+    dxa_h = mea.act_bwd("swish", xs, gs, alpha, dparam=da_h)
+    dxa_d = mea.act_bwd("swish", xs, gs, 0.0, param_dev=a_dev, dparam=da_d)
+    torch.cuda.synchronize()
+    assert torch.equal(dx_host.view(torch.int16), dx_dev.view(torch.int16))
+    assert torch.equal(dxa_h.view(torch.int16), dxa_d.view(torch.int16))
+    assert torch.equal(da_h, da_d)
+
+
+@pytest.mark.parametrize("alpha", [1.0, 1.3])
+def test_f32_swish_dense_grid_2_26(alpha):
+    # 2^26 evenly spaced fp32 values in [-30, 30] (the sweep the survey plans
+    # for the fp32 path), dy ~ N(0, 1), checked against the oracle in four
+    # chunks of 2^24; the largest errors seen are printed (run with -s)
+    n = 1 << 26
+    x = synthetic.f32_grid(n, -30.0, 30.0)
+    dy = synthetic.normal(n, 1.0, 105, synthetic.STREAM_DY, "f32")
+    xc, dyc = x.cuda(), dy.cuda()
+    y = mea.act_fwd("swish", xc, alpha).cpu()
+    dx = mea.act_bwd("swish", xc, dyc, alpha).cpu()
+    del xc, dyc
+    worst_fwd = worst_bwd = 0.0
+    chunk = 1 << 24
+    for c0 in range(0, n, chunk):
+        sl = slice(c0, c0 + chunk)
+        xd, gd = to_f64(x[sl]), to_f64(dy[sl])
+        a = check("f32", y[sl], oracle.act_fwd("swish", xd, alpha), what=f"fwd chunk {c0}")
+        b = check("f32", dx[sl], oracle.act_bwd("swish", xd, gd, alpha),
+                  scale=oracle.act_bwd_scale("swish", xd, gd, alpha), floor=TINY * np.maximum(1.0, np.abs(gd)),
+                  what=f"bwd chunk {c0}")
+        worst_fwd = max(worst_fwd, a["max_rel"])
+        worst_bwd = max(worst_bwd, b["max_rel"])
+    print(f"swish fp32 alpha={alpha}, 2^26 points in [-30, 30]: forward max relative error {worst_fwd:.3e}, "
+          f"backward max error / condition scale {worst_bwd:.3e}")

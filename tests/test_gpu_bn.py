@@ -2,27 +2,28 @@
 (mea_concat_bn_relu_fwd / _apply / _bwd) against the oracle, through the C
 ABI, and the memory-efficient DenseNet bottleneck built on them.
 
-Rules (tests/_compare.py): y is held to one bf16 ulp or, in fp32, 1e-5 of
-its condition scale (|gamma| r (|x| + |mean|) + |beta|, the terms any
+Rules (tests/_compare.py, check_bn): y is held to one bf16 ulp or, in fp32,
+1e-5 of its condition scale (|gamma| r (|x| + |mean|) + |beta|, the terms any
 evaluation of gamma xhat + beta adds); with bf16 storage a y that misses the
-ulp rule may meet the fp32 rule against that scale.  The statistics: see
+ulp rule may meet the fp32 rule against that scale (the batch statistics are
+fp32 results: where gamma xhat + beta cancels their rounding alone exceeds a
+bf16 ulp), for at most 1e-3 of the elements.  The statistics: see
 _check_stats (fp32 sums of at most 8 shifted values, then fp64).  dx is held to the same rules with
 the oracle's scale |gamma| r (|dz| + sum|dz| / n + |xhat| sum|dz xhat| / n).
 An element whose exact gamma xhat + beta lies within 1e-5 of its scale of
 zero may take either side of the ReLU: its dz may differ by dy, which adds
 |gamma r dy| to its dx allowance and |dy| (|dy xhat|) to its channel's
-dbeta (dgamma) allowance.  dgamma and dbeta: 1e-5 relative plus 1e-5 of
-the sum of their terms' magnitudes.
+dbeta (dgamma) allowance.  dgamma and dbeta: 1e-5 relative plus 1e-8 of the
+sum of their terms' magnitudes for channels of at least 2^16 values (1e-6
+below that: the worst case of the kernels' short fp32 runs).
 """
-import copy
-
 import numpy as np
 import pytest
 import torch
 
 import memory_efficient_activation_b200 as mea
 import oracle
-from _compare import TINY, check, to_f64
+from _compare import TINY, check_bn, to_f64
 from memory_efficient_activation_b200 import synthetic
 
 pytestmark = pytest.mark.gpu
@@ -71,7 +72,7 @@ def _ambiguous(pieces, g, b, rm, rv, ys):
     return np.abs(z) <= 1e-5 * ys.reshape(z.shape), x, r
 
 
-def _run(N, ks, spatial, dtype, seed, accumulate=False):
+def _run(N, ks, spatial, dtype, seed, accumulate=False, cap=1e-3):
     pieces = _pieces(N, ks, spatial, dtype, seed)
     C = sum(ks)
     g, b = _params(C, seed + 1)
@@ -93,7 +94,7 @@ def _run(N, ks, spatial, dtype, seed, accumulate=False):
     assert torch.equal(y, y2)                     # the re-populated output is the forward's, bitwise
     ry, rm, rv, ys = oracle.concat_bn_relu_fwd(_np(pieces), g.double().numpy(), b.double().numpy(), EPS)
     _check_stats(mean, invstd, rm, rv, pieces)
-    check(dtype, y.cpu(), ry.ravel(), scale=ys.ravel(), what="y", bf16_cond=True)
+    check_bn(dtype, y.cpu(), ry.ravel(), scale=ys.ravel(), what="y", cap=cap)
     dyn = dy.double().numpy().reshape(N, C, HW)
     rdp, rdg, rdb, rsc = oracle.concat_bn_relu_bwd(_np(pieces), dyn, g.double().numpy(), b.double().numpy(),
                                                    rm, rv, EPS)
@@ -107,16 +108,21 @@ def _run(N, ks, spatial, dtype, seed, accumulate=False):
         if accumulate:
             ref = ref + prev[i].double().numpy().reshape(ref.shape)
             sc = sc + np.abs(prev[i].double().numpy().reshape(ref.shape))
-        check(dtype, dp.cpu(), ref.ravel(), scale=sc.ravel() + ex.ravel() * 1e5, floor=floor, what=f"dpiece {i}",
-              bf16_cond=True)
+        check_bn(dtype, dp.cpu(), ref.ravel(), scale=sc.ravel() + ex.ravel() * 1e5, floor=floor, what=f"dpiece {i}",
+                 cap=cap)
     xh = (x - rm[None, :, None]) * r[None, :, None]
     dz = np.where(g.double().numpy()[None, :, None] * xh + b.double().numpy()[None, :, None] > 0, dyn, 0.0)
-    tb = np.abs(dz).sum(axis=(0, 2)) + np.where(amb, np.abs(dyn), 0).sum(axis=(0, 2)) * 1e5
-    tg = np.abs(dz * xh).sum(axis=(0, 2)) + np.where(amb, np.abs(dyn * xh), 0).sum(axis=(0, 2)) * 1e5
+    # per-channel sums (the rule of _compare.check_channel_sums), plus |dy|
+    # (|dy xhat|) for every element whose ReLU side is ambiguous
+    c = 1e-8 if N * HW >= (1 << 16) else 1e-6
+    tb = np.abs(dz).sum(axis=(0, 2))
+    tg = np.abs(dz * xh).sum(axis=(0, 2))
+    ab = np.where(amb, np.abs(dyn), 0).sum(axis=(0, 2))
+    ag = np.where(amb, np.abs(dyn * xh), 0).sum(axis=(0, 2))
     eb = np.abs(db.cpu().double().numpy() - rdb)
     eg = np.abs(dg.cpu().double().numpy() - rdg)
-    assert np.all(eb <= 1e-5 * np.abs(rdb) + 1e-5 * tb), eb.max()
-    assert np.all(eg <= 1e-5 * np.abs(rdg) + 1e-5 * tg), eg.max()
+    assert np.all(eb <= 1e-5 * np.abs(rdb) + c * tb + ab), (eb / (1e-5 * np.abs(rdb) + c * tb + ab)).max()
+    assert np.all(eg <= 1e-5 * np.abs(rdg) + c * tg + ag), (eg / (1e-5 * np.abs(rdg) + c * tg + ag)).max()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -154,9 +160,9 @@ def test_concat_bn_relu_running_stats_and_determinism():
     assert torch.equal(y1, y2) and torch.equal(m1, m2) and torch.equal(i1, i2)
     _, rm, rv, _ = oracle.concat_bn_relu_fwd(_np([p.cpu() for p in pieces]), g.cpu().double().numpy(),
                                              b.cpu().double().numpy(), EPS)
-    n = N * 81
-    em = 0.9 * 0.5 + 0.1 * rm
-    ev = 0.9 * 2.0 + 0.1 * rv * n / (n - 1)
+    em, ev = oracle.bn_running_update(np.full(C, 0.5), np.full(C, 2.0), rm, rv, N * 81, 0.1)
+    # the kernel's statistics are fp32 results (see _check_stats); the update
+    # adds one fp64 blend and one rounding to fp32
     assert np.allclose(rmean.cpu().double().numpy(), em, rtol=2e-6, atol=1e-7)
     assert np.allclose(rvar.cpu().double().numpy(), ev, rtol=2e-6, atol=1e-7)
 
@@ -209,8 +215,11 @@ def test_dense_bottleneck_module():
 def test_concat_bn_relu_one_value_per_channel(dtype):
     # N H W = 1: the batch variance is 0 and xhat = 0, so y = max(beta, 0) up
     # to the rounding of the folded gamma' x + beta' (held to the oracle's
-    # rules), invstd = eps^-1/2, and dgamma = 0 exactly (x equals its mean)
-    _run(1, [5, 3], (1, 1), dtype, 69)
+    # rules), invstd = eps^-1/2, and dgamma = 0 exactly (x equals its mean).
+    # The exact dx is 0 for every element (dz - dbeta / n - xhat dgamma / n
+    # cancels completely), so every bf16 dx that is not exactly 0 is held to
+    # the scale rule: no cap on their number here.
+    _run(1, [5, 3], (1, 1), dtype, 69, cap=1.0)
     pieces = [p.cuda() for p in _pieces(1, [5, 3], (1, 1), dtype, 69)]
     g, b = [t.cuda() for t in _params(8, 70)]
     y, mean, invstd = mea.concat_bn_relu_fwd(pieces, g, b, EPS)
@@ -218,60 +227,3 @@ def test_concat_bn_relu_one_value_per_channel(dtype):
     torch.cuda.synchronize()
     assert torch.allclose(invstd.cpu(), torch.full((8,), EPS ** -0.5), rtol=1e-6)
     assert torch.all(dg == 0)
-
-
-def test_densenet_bc_efficient_matches_naive():
-    # the same DenseNet-BC (depth 16: two layers per block), same weights,
-    # fp32: the memory-efficient bottleneck gives the naive network's logits
-    # and gradients up to summation order (batch statistics in fp64 here,
-    # cuDNN's own in the naive layers)
-    import bench
-    tf32 = (torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32)
-    torch.backends.cudnn.allow_tf32 = False      # both networks in plain fp32 convolutions
-    torch.backends.cuda.matmul.allow_tf32 = False
-    try:
-        _densenet_compare(bench)
-    finally:
-        torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32 = tf32
-
-
-def _densenet_compare(bench):
-    # Both fp32 networks against the naive one evaluated in float64: a wiring
-    # fault (a stale shared buffer, a piece gradient lost or counted twice)
-    # moves the logits and gradients by O(1).  The library convolutions both
-    # networks call (cuDNN's algorithm choices) put the naive network's own
-    # fp32 gradients up to ~1e-3 from float64 here, so the bound is 1e-2.
-    torch.manual_seed(0)
-    naive = bench._densenet_bc(False, depth=16).cuda()
-    eff = bench._densenet_bc(True, depth=16).cuda()
-    with torch.no_grad():
-        for bn, be in zip(naive.blocks, eff.blocks):
-            for ln, le in zip(bn, be):
-                le.b1.weight.copy_(ln.c1.weight)
-                le.b1.gamma.copy_(ln.n1.weight)
-                le.b1.beta.copy_(ln.n1.bias)
-                le.n2.load_state_dict(ln.n2.state_dict())
-                le.c2.load_state_dict(ln.c2.state_dict())
-        for name in ("stem", "trans", "final", "fc"):
-            getattr(eff, name).load_state_dict(getattr(naive, name).state_dict())
-    ref = copy.deepcopy(naive).double()
-    x = torch.from_numpy(synthetic.normal_f64(8 * 3 * 32 * 32, 1.0, 81, synthetic.STREAM_X)).view(8, 3, 32, 32)
-    outs = []
-    for net, xx in ((naive, x.float().cuda()), (eff, x.float().cuda()), (ref, x.cuda())):
-        net.train()
-        out = net(xx)
-        out.square().sum().backward()
-        outs.append(out.detach().double())
-    torch.cuda.synchronize()
-
-    def rel(a, b):
-        return float((a.detach().double() - b.detach()).norm() / b.detach().norm())
-
-    assert rel(outs[1], outs[2]) < 1e-3
-    for bn, be, br in zip(naive.blocks, eff.blocks, ref.blocks):
-        for ln, le, lr in zip(bn, be, br):
-            assert rel(le.b1.weight.grad, lr.c1.weight.grad) < 1e-2
-            assert rel(le.b1.gamma.grad, lr.n1.weight.grad) < 1e-2
-            assert rel(le.b1.beta.grad, lr.n1.bias.grad) < 1e-2
-            assert rel(le.c2.weight.grad, lr.c2.weight.grad) < 1e-2
-    assert rel(eff.stem.weight.grad, ref.stem.weight.grad) < 1e-2

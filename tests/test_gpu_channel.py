@@ -6,9 +6,12 @@ alpha per channel (mea_swish_channel_fwd / mea_swish_channel_bwd).
 Small NHWC and NCHW shapes in both dtypes are compared element by element
 (shapes that take the NHWC fast path, shapes that leave it, NCHW planes that
 are and are not multiples of the vector width); per-channel sums are
-compared on every channel.  The full-size workloads ([128, 56, 56, 144] NHWC
-bf16 for the affine family, [64, 144, 56, 56] NCHW fp32 for the channel
-Swish) are compared on every output.  Also: deep tails, alpha of zero and of
+compared on every channel (_compare.check_channel_sums).  The full-size
+workloads ([128, 56, 56, 144] NHWC bf16 for the affine family, [64, 144, 56,
+56] NCHW fp32 for the channel Swish) are compared on every output.  bf16
+outputs are held to one ulp of the oracle; fp32 affine outputs to 1e-5 of
+their condition scale plus the change that rounding z = gamma x + beta to
+fp32 makes to the exact result (oracle.affine_act_zround).  Also: deep tails, alpha of zero and of
 either sign, empty batches, bitwise determinism with the workspace counter
 returned to zero, agreement of the Swish member with the affine + Swish
 entry point, and the autograd modules.
@@ -19,7 +22,7 @@ import torch
 
 import memory_efficient_activation_b200 as mea
 import oracle
-from _compare import TINY, check, to_f64
+from _compare import TINY, check, check_channel_sums, to_f64
 from memory_efficient_activation_b200 import synthetic
 
 pytestmark = pytest.mark.gpu
@@ -59,18 +62,6 @@ def _inputs(shape_mem, layout, dtype, seed, sigma=1.0):
     return x, dy, g, b, a
 
 
-def _check_sums(got, ref, allow_terms):
-    """Per-channel fp32 sums.  Every term may carry the elementwise fp32
-    error (1e-5 of its condition scale), so a channel's sum may differ from
-    the oracle's by 1e-5 of its value plus 1e-5 of the sum of its terms'
-    condition scales (allow_terms), which also covers the rounding of the
-    fp32 per-tile partials."""
-    err = np.abs(got.cpu().double().numpy() - ref)
-    ok = err <= 1e-5 * np.abs(ref) + 1e-5 * allow_terms
-    assert np.all(ok), [(int(c), float(got[c]), float(ref[c]), float(allow_terms[c]))
-                        for c in np.flatnonzero(~ok)[:6]]
-
-
 def _check_sums_against_dx(dx, x, g, dg, db, ch, C):
     """fp32 only: the channel sums agree with the kernel's own dx (dz = dx /
     gamma_c, each dx one fp32 rounding of gamma_c dz), which checks the
@@ -99,20 +90,19 @@ def _affine_compare(act, dtype, layout, shape, x, dy, g, b, y, dx, dg, db):
     gg, bb = g.double().numpy(), b.double().numpy()
     ry = oracle.affine_act_fwd(act, layout, nchw, xd, gg, bb, p)
     rdx, rdg, rdb, scale = oracle.affine_act_bwd(act, layout, nchw, xd, gd, gg, bb, p)
+    # fp32: plus the change of the exact result when z = gamma x + beta is
+    # rounded once to fp32 (the configurations compute z in fp32); bf16: the
+    # plain ulp rule
+    ey, edx = oracle.affine_act_zround(act, layout, nchw, xd, gd, gg, bb, p)
     ch = _channels(xd.size, layout, nchw)
     C = nchw[1]
-    # the oracle at z rounded once to fp32 (the kernel's intermediate); gamma x
-    # and gamma dy are exact in double (products of two 24-bit significands)
-    z32 = oracle.round_f32(gg[ch] * xd + bb[ch])
-    gdy = gg[ch] * gd
-    alt_y = (oracle.act_fwd(act, z32, p), None)
-    alt_dx = (oracle.act_bwd(act, z32, gdy, p), oracle.act_bwd_scale(act, z32, gdy, p))
-    check(dtype, y.cpu(), ry, what=f"affine {act} fwd", alt=alt_y)
+    check(dtype, y.cpu(), ry, what=f"affine {act} fwd", zround=ey)
     check(dtype, dx.cpu(), rdx, scale=scale, floor=TINY * np.maximum(1, np.abs(gd)), what=f"affine {act} dx",
-          bf16_cond=True, alt=alt_dx)
-    dz_scale = scale / np.abs(gg[ch])           # condition scale of each dz term
-    _check_sums(dg, rdg, np.bincount(ch, dz_scale * np.abs(xd), minlength=C))
-    _check_sums(db, rdb, np.bincount(ch, dz_scale, minlength=C))
+          zround=edx)
+    dz = rdx / gg[ch]
+    n_c = xd.size // C if C else 0
+    check_channel_sums(dg, rdg, np.bincount(ch, np.abs(dz * xd), minlength=C), n_c, f"affine {act} dgamma")
+    check_channel_sums(db, rdb, np.bincount(ch, np.abs(dz), minlength=C), n_c, f"affine {act} dbeta")
     if dtype == "f32":
         _check_sums_against_dx(dx, x, g, dg, db, ch, C)
 
@@ -240,14 +230,13 @@ def _channel_compare(dtype, layout, shape, x, dy, a, y, dx, da):
     rdx, rda, scale = oracle.swish_channel_bwd(layout, nchw, xd, gd, aa)
     check(dtype, y.cpu(), ry, what="channel swish fwd")
     check(dtype, dx.cpu(), rdx, scale=scale, floor=TINY * np.maximum(1, np.abs(gd)), what="channel swish dx")
-    # each d alpha term dy x^2 s (1 - s) is a product (no cancellation): its
-    # condition scale is its own magnitude
+    # |terms| of each channel's sum: dy x^2 s (1 - s) = dy x^2 s Sigmoid(-alpha x)
     ch = _channels(xd.size, layout, nchw)
     t = aa[ch] * xd
     with np.errstate(over="ignore"):
-        s = 1.0 / (1.0 + np.exp(-t))
-        terms = np.abs(gd * xd * xd * s * (1.0 - s))
-    _check_sums(da, rda, np.bincount(ch, terms, minlength=nchw[1]))
+        terms = np.abs(gd * xd * xd) / ((1.0 + np.exp(-t)) * (1.0 + np.exp(t)))
+    C = nchw[1]
+    check_channel_sums(da, rda, np.bincount(ch, terms, minlength=C), xd.size // C if C else 0, "dalpha")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -325,3 +314,66 @@ def test_channel_swish_module_autograd():
     y.backward(dy.cuda())
     torch.cuda.synchronize()
     _channel_compare("bf16", "nchw", shape, x, dy, a, y.detach(), xc.grad, m.alpha.grad)
+
+
+# Zeros of f' (v = alpha z for Swish), to double precision.
+ROOTS = {"swish": -1.2784645427610737951, "gelu_erf": -0.75179152469356445746, "gelu_tanh": -0.75246142207101625849}
+
+
+def _near_root_inputs(act, layout, shape, dtype, seed, p):
+    """Per channel c: a bf16 value x0_c and beta_c such that z = gamma_c x0_c +
+    beta_c lies at a chosen offset, anywhere within 2^-10, of the zero of f'
+    (in v = alpha z for Swish); half the positions of every channel hold x0_c,
+    the rest N(0, 1) values."""
+    n = int(np.prod(shape))
+    C = shape[3] if layout == "nhwc" else shape[1]
+    x, dy, g, b, _ = _inputs(shape, layout, dtype, seed)
+    x0 = synthetic.to_storage(synthetic.uniform_f64(C, -2.0, 2.0, seed, synthetic.STREAM_PARAM), dtype)
+    off = synthetic.uniform_f64(C, -2.0 ** -10, 2.0 ** -10, seed + 1, synthetic.STREAM_PARAM)
+    off[: C // 4] = 0.0                      # a quarter of the channels at the zero itself
+    z0 = ROOTS[act] / p
+    gd = g.double().numpy()
+    b = torch.from_numpy(z0 + off / p - gd * x0.double().numpy()).float()
+    ch = _channels(n, layout, _nchw(shape, layout))
+    flat = x.reshape(-1).clone()
+    pos = np.arange(n)
+    sel = torch.from_numpy((pos // C if layout == "nhwc" else pos) % 2 == 0)
+    flat[sel] = x0[torch.from_numpy(ch)][sel]
+    return flat.view(shape), dy, g, b
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("layout,shape", [("nhwc", (4, 6, 6, 144)), ("nhwc", (2, 3, 5, 12)), ("nchw", (4, 16, 9, 9)),
+                                          ("nhwc", (3, 5, 5, 20))])
+@pytest.mark.parametrize("act", ["swish", "gelu_erf", "gelu_tanh"])
+def test_affine_act_near_zero_of_derivative(act, dtype, layout, shape):
+    # z lands within 2^-10 of the zero of f' for half the elements: bf16 dx
+    # stays within one ulp of the exact result (the kernels recompute these
+    # elements from a compensated z), fp32 within its rule
+    p = _param(act)
+    x, dy, g, b = _near_root_inputs(act, layout, shape, dtype, 407, p)
+    y = mea.affine_act_fwd(act, x.cuda(), g.cuda(), b.cuda(), p, layout)
+    dx, dg, db = mea.affine_act_bwd(act, x.cuda(), dy.cuda(), g.cuda(), b.cuda(), p, layout)
+    torch.cuda.synchronize()
+    _affine_compare(act, dtype, layout, shape, x, dy, g, b, y, dx, dg, db)
+
+
+@pytest.mark.parametrize("layout,shape", [("nhwc", (4, 6, 6, 16)), ("nchw", (4, 16, 9, 9))])
+def test_swish_channel_bf16_near_zero_of_derivative(layout, shape):
+    # alpha_c = fp32(v0 / x0_c) for a bf16 x0_c held by half the positions
+    x, dy, _, _, _ = _inputs(shape, layout, "bf16", 415, sigma=1.5)
+    C = shape[3] if layout == "nhwc" else shape[1]
+    n = x.numel()
+    x0 = synthetic.to_storage(synthetic.uniform_f64(C, 0.3, 3.0, 415, synthetic.STREAM_PARAM), "bf16")
+    x0 = x0 * torch.where(torch.arange(C) % 2 == 0, -1.0, 1.0).to(x0.dtype)
+    a = torch.from_numpy(np.float32(ROOTS["swish"] / x0.double().numpy()).astype(np.float32))
+    ch = torch.from_numpy(_channels(n, layout, _nchw(shape, layout)))
+    flat = x.reshape(-1).clone()
+    pos = np.arange(n)
+    sel = torch.from_numpy((pos // C if layout == "nhwc" else pos) % 2 == 0)
+    flat[sel] = x0[ch][sel]
+    x = flat.view(shape)
+    y = mea.swish_channel_fwd(x.cuda(), a.cuda(), layout)
+    dx, da = mea.swish_channel_bwd(x.cuda(), dy.cuda(), a.cuda(), layout)
+    torch.cuda.synchronize()
+    _channel_compare("bf16", layout, shape, x, dy, a, y, dx, da)
