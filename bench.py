@@ -62,7 +62,29 @@ def _dist():
     torch.cuda.set_device(local)
     dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                             device_id=torch.device("cuda", local))
+    if dist.get_world_size() != ws:
+        raise SystemExit(f"process group formed {dist.get_world_size()} ranks, WORLD_SIZE says {ws}")
     return rank, ws, local
+
+
+def _relaunch(nproc: int, argv, script: str | None = None) -> int:
+    """Runs `script` (this file by default) as nproc ranks of one node under
+    torch.distributed.run (rendezvous on 127.0.0.1, a free port), passing
+    argv to every rank; returns the launcher's exit code.  NCCL's init log is
+    switched on (to stderr, so that stdout carries only rank 0's JSON line),
+    which shows how many ranks the communicator formed."""
+    import socket
+    import subprocess
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    env = dict(os.environ)
+    env.setdefault("NCCL_DEBUG", "INFO")
+    env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    env.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nproc}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", script or os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd, env=env).returncode
 
 
 def _barrier(ws):
@@ -218,38 +240,44 @@ def run_ours(args, rank, ws, local):
         step()
     torch.cuda.synchronize()
 
-    # Timed region: K steps.  Every EVERY-th step also brackets each kernel
-    # with CUDA events on the launching stream (for the roofline); an event
-    # between two kernels costs the overlap of the second kernel's launch
-    # with the first one's drain, so the other steps run without them.
-    every = max(1, args.event_every)
-    sampled = [k for k in range(args.steps) if k % every == 0]
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for k in sampled}
+    # Timed region: K steps, no events between the kernels (an event between
+    # two kernels costs the overlap of the second kernel's launch with the
+    # first one's drain).
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     _barrier(ws)
     torch.cuda.synchronize()
     with _ClockSampler(local) as clk:
         start.record(stream)
-        for k in range(args.steps):
-            e3 = ev.get(k)
-            if e3 is None:
-                mea.act_fwd("swish", x, 1.0, out=y)
-                mea.act_bwd("swish", x, dy, 1.0, out=dx)
-                continue
-            e3[0].record(stream)
-            mea.act_fwd("swish", x, 1.0, out=y)
-            e3[1].record(stream)
-            mea.act_bwd("swish", x, dy, 1.0, out=dx)
-            e3[2].record(stream)
+        for _ in range(args.steps):
+            step()
         end.record(stream)
         torch.cuda.synchronize()
+        _barrier(ws)
+        elapsed_ms = _max_over_ranks(start.elapsed_time(end), ws)
+        # Kernel-timing pass (the roofline), right after the timed region:
+        # each kernel timed over back-to-back launches of itself (5 rounds of
+        # `per` forwards, then `per` backwards, CUDA events at the round
+        # boundaries on the launching stream), so that every launch overlaps
+        # its neighbours' ramp and drain as it does in the timed steps; 3
+        # unbracketed steps first refill the launch queue.  Median over rounds.
+        rounds = 5
+        per = max(10, max(50, args.steps) // rounds)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(rounds)]
+        for _ in range(3):
+            step()
+        for e3 in ev:
+            e3[0].record(stream)
+            for _ in range(per):
+                mea.act_fwd("swish", x, 1.0, out=y)
+            e3[1].record(stream)
+            for _ in range(per):
+                mea.act_bwd("swish", x, dy, 1.0, out=dx)
+            e3[2].record(stream)
+        torch.cuda.synchronize()
     _barrier(ws)
-    elapsed_ms = _max_over_ranks(start.elapsed_time(end), ws)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev.values())
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev.values())
-    fwd_ms = _max_over_ranks(fwd_ms, ws)
-    bwd_ms = _max_over_ranks(bwd_ms, ws)
+    fwd_ms = _max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) / per for e in ev), ws)
+    bwd_ms = _max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) / per for e in ev), ws)
 
     step_bytes = accounting.step_bytes(n, DTYPE)
     ms_per_step = elapsed_ms / args.steps
@@ -273,8 +301,11 @@ def run_ours(args, rank, ws, local):
         "algorithmic_bytes_per_launch": bwd_bytes,
         "fwd_ms": round(fwd_ms, 5),
         "bwd_ms": round(bwd_ms, 5),
-        "launches_timed": len(ev),
-        "timing": f"CUDA events around each kernel on every {every}th step of the timed region",
+        "fwd_plus_bwd_ms": round(fwd_ms + bwd_ms, 5),
+        "ms_per_step": round(ms_per_step, 5),
+        "launches_timed": 2 * rounds * per,
+        "timing": f"after the timed region: {rounds} rounds of {per} back-to-back launches of each kernel, CUDA "
+                  "events at the round boundaries on the launching stream; median per launch",
         "fwd_frac": round(accounting.fwd_bytes(n, DTYPE) / (fwd_ms * 1e-3) / 1e9 / peak, 4),
         "step_frac": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
         "step_frac_of_nominal_8tbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
@@ -302,6 +333,7 @@ def run_ours(args, rank, ws, local):
             "x_dist": "N(0,1)", "dy_dist": "N(0,1)",
             "l2": "inputs larger than L2 (536 MB working set per step vs 126 MB L2); no flush",
             "parallelism": f"replicas x{ws} (independent shards, no data-path collective)",
+            "process_group": ({"backend": "nccl", "ranks": ws} if ws > 1 else None),
             "pct_of_hbm_roofline": round(100 * value / ws / peak, 2),
             "saved_bytes_per_layer": accounting.saved_bytes_per_layer(n, DTYPE),
             "saved_bytes_per_layer_naive": accounting.saved_bytes_per_layer(n, DTYPE, naive=True),
@@ -345,6 +377,7 @@ def run_e2e(args, rank, ws, local, w):
     _barrier(ws)
     ms = _max_over_ranks(s.elapsed_time(e), ws)
     nbytes = accounting.step_bytes(w.n, DTYPE)
+    link = _copy_bound(hx, hdy, hy, hdx, dev)
     return {
         "value": round(ws * nbytes * steps / (ms * 1e-3) / 1e9, 2),
         "unit": "GB/s",
@@ -353,7 +386,47 @@ def run_e2e(args, rank, ws, local, w):
         "steps": steps,
         "ms_per_step": round(ms / steps, 4),
         "pipelining": "8 pieces over 3 streams (copy in, kernels, copy out)",
+        "host_link": link,
+        "frac_of_copy_bound": round(link["both_ms"] / (ms / steps), 4),
     }
+
+
+def _copy_bound(hx, hdy, hy, hdx, dev, reps: int = 3):
+    """The host link's floor for one end-to-end step: the time to copy the
+    step's inputs to the device and its results back, pinned host memory,
+    the two directions at once on two streams (no kernels); also each
+    direction alone.  Min over reps."""
+    dx_, ddy = torch.empty_like(hx, device=dev), torch.empty_like(hdy, device=dev)
+    dy_, ddx = torch.empty_like(hy, device=dev), torch.empty_like(hdx, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+    res = {"h2d_ms": [], "d2h_ms": [], "both_ms": []}
+    for _ in range(reps):
+        for key in ("h2d_ms", "d2h_ms", "both_ms"):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(cur)
+            s_in.wait_stream(cur)
+            s_out.wait_stream(cur)
+            if key != "d2h_ms":
+                with torch.cuda.stream(s_in):
+                    dx_.copy_(hx, non_blocking=True)
+                    ddy.copy_(hdy, non_blocking=True)
+            if key != "h2d_ms":
+                with torch.cuda.stream(s_out):
+                    hy.copy_(dy_, non_blocking=True)
+                    hdx.copy_(ddx, non_blocking=True)
+            cur.wait_stream(s_in)
+            cur.wait_stream(s_out)
+            b.record(cur)
+            torch.cuda.synchronize()
+            res[key].append(a.elapsed_time(b))
+    nb = hx.numel() * hx.element_size() + hdy.numel() * hdy.element_size()
+    out = {k: round(min(v), 4) for k, v in res.items()}
+    out["h2d_GB/s"] = round(nb / (out["h2d_ms"] * 1e-3) / 1e9, 1)
+    out["d2h_GB/s"] = round(nb / (out["d2h_ms"] * 1e-3) / 1e9, 1)
+    out["note"] = "pinned copies of the step's 2 input and 2 output tensors, no kernels; both_ms is the floor"
+    return out
 
 
 # ------------------------------------------------- oracle (CPU) baseline
@@ -365,11 +438,23 @@ def _oracle_step(oracle, xd, gd):
     oracle.round_bf16(dx)
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, budget_s: float = 12.0):
     """The double-precision oracle (as it stands, OpenMP over the host cores)
     on the same workload: forward + backward + rounding of y and dx to bf16,
     repeated over the full 67M-element batch until about budget_s seconds of
-    work; GB/s under the same 10 bytes/element accounting."""
+    work; GB/s under the same 10 bytes/element accounting.  Then the same on
+    one core, over the first 1/16 of the batch for about budget_s / 3 s."""
     import oracle
     xd = w.x.reshape(-1).double().numpy()
     gd = w.dy.reshape(-1).double().numpy()
@@ -380,12 +465,28 @@ def cpu_baseline(w, budget_s: float = 12.0):
         t_total += time.perf_counter() - t0
         reps += 1
     n = w.n
+    cores = oracle.num_threads()
+    m = n // 16
+    xs, gs = xd[:m], gd[:m]
+    oracle.set_num_threads(1)
+    try:
+        reps1, t1 = 0, 0.0
+        while t1 < budget_s / 3 and reps1 < 50:
+            t0 = time.perf_counter()
+            _oracle_step(oracle, xs, gs)
+            t1 += time.perf_counter() - t0
+            reps1 += 1
+    finally:
+        oracle.set_num_threads(cores)
     return {
         "value": round(reps * accounting.step_bytes(n, DTYPE) / t_total / 1e9, 3),
         "unit": "GB/s",
-        "cores": oracle.num_threads(),
+        "cores": cores,
         "kind": "oracle",
         "sample": f"{reps} x full {n}-element batch (fwd + bwd + bf16 rounding), {t_total:.1f} s",
+        "cpu_model": _cpu_model(),
+        "single_core": {"value": round(reps1 * accounting.step_bytes(m, DTYPE) / t1 / 1e9, 4), "unit": "GB/s",
+                        "cores": 1, "sample": f"{reps1} x first {m} elements, {t1:.1f} s"},
     }
 
 
@@ -487,19 +588,12 @@ def _sets_for(nbytes: int) -> int:
     return max(2, -(-3 * L2_BYTES // max(nbytes, 1)))
 
 
-def run_secondary(args):
-    """Per-kernel GB/s and roofline fractions for the other configurations
-    (activation family, EfficientNet-like fp32 maps with d alpha, fused
-    affine + Swish NHWC, fused affine + every activation NHWC, Swish with a
-    per-channel alpha on EfficientNet-like maps, the L2-resident 1M fp32
-    case).  Diagnostics: the
-    headline line is the default run."""
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
-    peak, peak_kind = _peaks()
+def _ops_for(wl, dev, args):
+    """The launchers of one workload's kernels, each over buffer sets that
+    together exceed the L2 (the 1M fp32 case excepted): a list of (name,
+    launchers, algorithmic bytes or FLOPs).  Sets args._flop_ops for the
+    workloads whose ops are contractions."""
     ops = []
-    wl = args.workload
 
     def clones(ts, k):
         return [[t.to(dev).clone() for t in ts] for _ in range(k)]
@@ -531,6 +625,23 @@ def run_secondary(args):
                         [lambda b=b, d=d, ws=ws, a=a: mea.act_bwd("swish", b[0], b[1], 0.0, param_dev=a, dparam=d,
                                                                   out=b[3], workspace=ws)
                          for b, d, ws in zip(sets, ds, wss)], accounting.bwd_bytes(w.n, "f32")))
+    elif wl == "effnet_f32_dalpha_grouped":
+        # the same six maps, each direction one grouped launch over all six
+        wls = [synthetic.effnet_swish_f32(i) for i in range(len(synthetic.EFFNET_B0_SHAPES))]
+        fwd_b = sum(accounting.fwd_bytes(w.n, "f32") for w in wls)
+        bwd_b = sum(accounting.bwd_bytes(w.n, "f32") for w in wls)
+        k = _sets_for(bwd_b)
+        alphas = [w.param for w in wls]
+        sets = [[clones([w.x, w.dy, w.x, w.x], 1)[0] for w in wls] for _ in range(k)]
+        ds = [[torch.empty(1, dtype=torch.float32, device=dev) for _ in wls] for _ in range(k)]
+        need = mea.act_bwd_grouped_workspace_bytes("swish", [w.n for w in wls], True)
+        wss = [torch.zeros(need, dtype=torch.uint8, device=dev) for _ in range(k)]
+        ops.append(("grouped_fwd", [lambda b=b: mea.act_fwd_grouped("swish", [t[0] for t in b], alphas,
+                                                                    outs=[t[2] for t in b]) for b in sets], fwd_b))
+        ops.append(("grouped_bwd_dalpha",
+                    [lambda b=b, d=d, w_=w_: mea.act_bwd_grouped("swish", [t[0] for t in b], [t[1] for t in b], alphas,
+                                                                 dparams=d, outs=[t[3] for t in b], workspace=w_)
+                     for b, d, w_ in zip(sets, ds, wss)], bwd_b))
     elif wl == "affine_nhwc_bf16":
         w = synthetic.affine_swish_nhwc()
         C = w.extra["gamma"].numel()
@@ -607,14 +718,6 @@ def run_secondary(args):
                     accounting.bwd_bytes(M * N, "bf16")))
         args._flop_ops = {name for name, _, _ in ops if not name.startswith("act_")}
         args._tf_peak = tf_peak
-    elif wl == "mlp_bf16":
-        return run_mlp(args)
-    elif wl == "densenet_bn_bf16":
-        return run_densenet_bn(args)
-    elif wl == "densenet_bc100":
-        return run_densenet_bc100(args)
-    elif wl == "memory_study":
-        return run_memory_study(args)
     elif wl == "swish_f32_1m":
         w = synthetic.swish_f32_1m()
         sets = clones([w.x, w.dy, w.x, w.x], 1)       # L2-resident on purpose
@@ -623,6 +726,28 @@ def run_secondary(args):
                     accounting.bwd_bytes(w.n, "f32")))
     else:
         raise SystemExit(f"unknown workload {wl}")
+    return ops
+
+
+def run_secondary(args):
+    """Per-kernel GB/s and roofline fractions for the other configurations
+    (activation family, EfficientNet-like fp32 maps with d alpha, fused
+    affine + Swish NHWC, fused affine + every activation NHWC, Swish with a
+    per-channel alpha on EfficientNet-like maps, the L2-resident 1M fp32
+    case, the fused matmul).  Diagnostics: the headline line is the default
+    run, which carries the configurations' figures in its "configs" block."""
+    wl = args.workload
+    if wl == "mlp_bf16":
+        return run_mlp(args)
+    if wl == "densenet_bn_bf16":
+        return run_densenet_bn(args)
+    if wl == "memory_study":
+        return run_memory_study(args)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = _peaks()
+    ops = _ops_for(wl, dev, args)
     # capture on a side stream (graphs cannot be captured on the legacy stream)
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
@@ -652,6 +777,57 @@ def run_secondary(args):
     if wl == "swish_f32_1m":
         out["note"] = "21 MB of traffic per step fits in the 126 MB L2: an L2-resident figure, not HBM bandwidth"
     return out
+
+
+# The other configurations of the metric's workload list, timed in the
+# default run after the headline (N = 1): key -> _ops_for workload.
+CONFIG_WORKLOADS = (
+    ("c1_swish_f32_1m", "swish_f32_1m"),
+    ("c3_family_bf16_8x2048x4096", "family_bf16"),
+    ("c4_effnet_b0_f32_dalpha", "effnet_f32_dalpha"),
+    ("c4_effnet_b0_f32_dalpha_grouped", "effnet_f32_dalpha_grouped"),
+    ("c5_affine_swish_nhwc_bf16_128x56x56x144", "affine_nhwc_bf16"),
+)
+
+
+def run_configs(args):
+    """Per-kernel device time, GB/s and fraction of the HBM peak for
+    configurations 1 and 3-5, each kernel captured in a CUDA graph of 24
+    launches that rotate over buffer sets together larger than 3x the L2
+    (configuration 1, 21 MB of traffic, fits in L2 and is reported as such),
+    replayed args.config_steps times with events around every replay; the
+    configuration's figure is its total algorithmic bytes over the total
+    device time of one launch of each of its kernels."""
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = _peaks()
+    res = {}
+    t0 = time.perf_counter()
+    for key, wl in CONFIG_WORKLOADS:
+        ops = _ops_for(wl, dev, args)
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            per, total = _time_ops(ops, args.config_steps, 3, cap)
+        stream.wait_stream(cap)
+        tot_bytes = sum(b for _, _, b in ops)
+        res[key] = {
+            "GB/s": round(tot_bytes / (total * 1e-3) / 1e9, 1),
+            "frac": round(tot_bytes / (total * 1e-3) / 1e9 / peak, 4),
+            "bytes": tot_bytes,
+            "us": round(total * 1e3, 2),
+            "kernels": {name: {"us": round(per[name] * 1e3, 2), "bytes": b,
+                               "GB/s": round(b / (per[name] * 1e-3) / 1e9, 1),
+                               "frac": round(b / (per[name] * 1e-3) / 1e9 / peak, 4)} for name, _, b in ops},
+        }
+        if wl == "swish_f32_1m":
+            res[key]["note"] = "21 MB of traffic per step stays in the 126 MB L2: an L2 figure, not HBM"
+        del ops
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return {"peak": peak, "peak_kind": peak_kind, "steps": args.config_steps,
+            "timing": "CUDA-graph replays of 24 launches per kernel rotating over buffer sets > 3x L2; mean per launch",
+            "wall_s": round(time.perf_counter() - t0, 1), **res}
 
 
 def run_mlp(args, M: int = 16384, d: int = 4096, h: int = 4096, act: str = "gelu_tanh"):
@@ -781,121 +957,6 @@ def run_densenet_bn(args, N: int = 64, ks=(64, 32, 32, 32, 32, 32), spatial=(56,
             "clocks": clk.summary()}
 
 
-def _densenet_bc(efficient: bool, growth: int = 12, depth: int = 100, classes: int = 10, dtype=torch.float32):
-    """DenseNet-BC (bottleneck + compression 0.5) for 32 x 32 inputs, random
-    weights: three dense blocks of (depth - 4) / 6 layers; a layer is
-    BN-ReLU-conv1x1 (4 growth channels) then BN-ReLU-conv3x3 (growth
-    channels) on the concatenation of every earlier feature map of its block.
-    efficient: the first BN-ReLU-conv1x1 of each layer is the memory-efficient
-    bottleneck (concatenation never formed, normalized tensor in one buffer
-    shared by all layers, re-populated in the backward); otherwise torch.cat
-    + BatchNorm2d + ReLU + Conv2d."""
-    import torch.nn as nn
-    layers_per_block = (depth - 4) // 6
-    shared = mea.SharedBuffer()
-
-    class Layer(nn.Module):
-        def __init__(self, cin):
-            super().__init__()
-            if efficient:
-                self.b1 = mea.MemoryEfficientDenseBottleneck(cin, 4 * growth, shared, dtype=dtype)
-            else:
-                self.n1 = nn.BatchNorm2d(cin)
-                self.c1 = nn.Conv2d(cin, 4 * growth, 1, bias=False)
-            self.n2 = nn.BatchNorm2d(4 * growth)
-            self.c2 = nn.Conv2d(4 * growth, growth, 3, padding=1, bias=False)
-
-        def forward(self, feats):
-            if efficient:
-                h = self.b1(*feats)
-            else:
-                h = self.c1(torch.relu(self.n1(torch.cat(feats, 1))))
-            return self.c2(torch.relu(self.n2(h)))
-
-    class Net(nn.Module):
-        def __init__(self):
-            super().__init__()
-            c = 2 * growth
-            self.stem = nn.Conv2d(3, c, 3, padding=1, bias=False)
-            self.blocks = nn.ModuleList()
-            self.trans = nn.ModuleList()
-            for bi in range(3):
-                blk = nn.ModuleList()
-                for _ in range(layers_per_block):
-                    blk.append(Layer(c))
-                    c += growth
-                self.blocks.append(blk)
-                if bi < 2:
-                    self.trans.append(nn.Sequential(nn.BatchNorm2d(c), nn.ReLU(), nn.Conv2d(c, c // 2, 1, bias=False),
-                                                    nn.AvgPool2d(2)))
-                    c //= 2
-            self.final = nn.BatchNorm2d(c)
-            self.fc = nn.Linear(c, classes)
-
-        def forward(self, x):
-            h = self.stem(x)
-            for bi, blk in enumerate(self.blocks):
-                feats = [h]
-                for layer in blk:
-                    feats.append(layer(feats))
-                h = torch.cat(feats, 1)
-                if bi < 2:
-                    h = self.trans[bi](h)
-            h = torch.relu(self.final(h)).mean(dim=(2, 3))
-            return self.fc(h)
-
-    return Net().to(dtype)
-
-
-def run_densenet_bc100(args, batch: int = 64):
-    """One training step (forward, backward) of DenseNet-BC-100 (growth 12)
-    on a synthetic batch of 64 32 x 32 images, fp32, random weights: the page's
-    "Performance" comparison (naive against memory-efficient implementation,
-    memory per GPU and time per minibatch) re-measured on one B200 with the
-    memory-efficient bottleneck kernels.  No dataset: inputs and the loss
-    weights are synthetic."""
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    torch.backends.cudnn.benchmark = True     # both networks: cuDNN picks its fastest convolution algorithms
-    x = torch.from_numpy(synthetic.normal_f64(batch * 3 * 32 * 32, 1.0, 80, synthetic.STREAM_X)).float()
-    x = x.view(batch, 3, 32, 32).to(dev)
-    wloss = torch.from_numpy(synthetic.normal_f64(batch * 10, 1.0, 80, synthetic.STREAM_DY)).float().view(batch, 10).to(dev)
-    res = {}
-    for name, eff in (("naive", False), ("memory_efficient", True)):
-        torch.manual_seed(0)
-        net = _densenet_bc(eff).to(dev)
-        net.train()
-
-        def step():
-            net.zero_grad(set_to_none=True)
-            (net(x) * wloss).sum().backward()
-
-        for _ in range(max(3, args.warmup)):
-            step()
-        torch.cuda.synchronize()
-        torch.cuda.reset_peak_memory_stats()
-        base = torch.cuda.memory_allocated()
-        step()
-        torch.cuda.synchronize()
-        peak = torch.cuda.max_memory_allocated()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        for _ in range(args.steps):
-            step()
-        e.record()
-        torch.cuda.synchronize()
-        res[name] = {"peak_memory_bytes": int(peak), "peak_above_weights_bytes": int(peak - base),
-                     "ms_per_minibatch": round(s.elapsed_time(e) / args.steps, 3),
-                     "parameters": int(sum(p.numel() for p in net.parameters()))}
-        del net
-        torch.cuda.empty_cache()
-    return {"workload": "densenet_bc100", "batch": batch, "image": [3, 32, 32], "dtype": "fp32",
-            "data": "synthetic (no dataset, random weights)", "steps": args.steps, "warmup": args.warmup,
-            "results": res,
-            "memory_ratio": round(res["memory_efficient"]["peak_memory_bytes"] / res["naive"]["peak_memory_bytes"], 4),
-            "time_ratio": round(res["memory_efficient"]["ms_per_minibatch"] / res["naive"]["ms_per_minibatch"], 4)}
-
-
 class _PlainSwish(torch.nn.Module):
     """The plain autograd Swish of the pages' first listing: x * sigmoid(alpha x)
     built from PyTorch ops, which keeps every intermediate for the backward.
@@ -977,19 +1038,30 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--event-every", type=int, default=16,
-                    help="bracket the kernels of every Nth timed step with CUDA events (roofline)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave out the configs block (configurations 1, 3-5 timed after the headline)")
+    ap.add_argument("--config-steps", type=int, default=10)
     ap.add_argument("--workload", default="swish_bf16",
-                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "affine_nhwc_bf16",
+                    choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "effnet_f32_dalpha_grouped",
+                             "affine_nhwc_bf16",
                              "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "mlp_bf16",
-                             "densenet_bn_bf16", "densenet_bc100", "swish_f32_1m", "memory_study"],
+                             "densenet_bn_bf16", "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    env_ws = os.environ.get("WORLD_SIZE")
+    if env_ws is None:
+        if args.gpus > 1:
+            # one process per GPU: start args.gpus ranks of this script
+            return _relaunch(args.gpus, sys.argv[1:] if argv is None else list(argv))
+    elif int(env_ws) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={env_ws}: launch one rank per GPU")
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -1005,6 +1077,8 @@ def main(argv=None):
 
     rank, ws, local = _dist()
     out = run_ours(args, rank, ws, local)
+    if rank == 0 and ws == 1 and not args.no_configs:
+        out["configs"] = run_configs(args)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:
