@@ -39,6 +39,7 @@
 #include "mea_bn_api.h"
 #include "mea_device.cuh"
 #include "mea_internal.h"
+#include "mea_math.cuh"
 #include "mea_stream.cuh"
 
 namespace mea {
@@ -92,16 +93,50 @@ __device__ __forceinline__ PlaneJob plane_job(const BnPieces &t, int64_t N, int 
 constexpr int kBnUnroll = 4;     // items in flight per thread
 
 // Runs f over the block's planes in items of VL elements (one 16-byte vector,
-// or one element), kBnUnroll items per thread per step: f.template step<U>
-// gets each item's index in the piece (ii) and in the concatenation (io), in
-// item units, and whether it exists (ok).
+// or one element), kBnUnroll items per thread per step: f.step gets each
+// item's index in the piece (ii) and in the concatenation (io), in item
+// units, and whether it exists (ok).  Thread t takes items t, t + bd, t + 2
+// bd, ... of the block's planes laid end to end.
+//
+// When a plane holds at least bd items (and every index fits in 32 bits),
+// one step of bd items crosses at most one plane boundary, so the plane
+// offset and both indices advance by additions alone; otherwise each item's
+// (plane, offset) comes from a multiply-shift division.  Both visit the same
+// items in the same order.
 template <int VL, class F>
 __device__ __forceinline__ void stream_items(const PlaneJob &p, int64_t C, int64_t HW, F &f)
 {
     const uint32_t per = (uint32_t)(HW / VL);
     const uint32_t total = (uint32_t)(p.n1 - p.n0) * per;
-    const DivU32 div(per);
     const uint32_t bd = blockDim.x;
+    const bool fits = (uint64_t)(p.n1 * C) * per < (1ull << 31);
+    if (per >= bd && fits) {
+        uint32_t v = threadIdx.x;
+        uint32_t ii = (uint32_t)((p.n0 * p.k + p.j) * per) + v;
+        uint32_t io = (uint32_t)((p.n0 * C + p.c) * per) + v;
+        const uint32_t ii_skip = (uint32_t)(p.k - 1) * per, io_skip = (uint32_t)(C - 1) * per;
+        for (uint32_t q0 = threadIdx.x; q0 < total; q0 += kBnUnroll * bd) {
+            int64_t iu[kBnUnroll], ou[kBnUnroll];
+            bool ok[kBnUnroll];
+#pragma unroll
+            for (int u = 0; u < kBnUnroll; ++u) {
+                ok[u] = q0 + u * bd < total;
+                iu[u] = ii;
+                ou[u] = io;
+                v += bd;
+                ii += bd;
+                io += bd;
+                if (v >= per) {
+                    v -= per;
+                    ii += ii_skip;
+                    io += io_skip;
+                }
+            }
+            f.step(iu, ou, ok);
+        }
+        return;
+    }
+    const DivU32 div(per);
     for (uint32_t q0 = threadIdx.x; q0 < total; q0 += kBnUnroll * bd) {
         int64_t ii[kBnUnroll], io[kBnUnroll];
         bool ok[kBnUnroll];
@@ -117,6 +152,57 @@ __device__ __forceinline__ void stream_items(const PlaneJob &p, int64_t C, int64
         }
         f.step(ii, io, ok);
     }
+}
+
+// One 16-byte item as packed .f32x2 pairs (4 for bf16, 2 for fp32), so the
+// per-element arithmetic of the vector path takes half the instructions.
+template <typename T>
+struct Pairs;
+template <>
+struct Pairs<Bf16> {
+    static constexpr int N = 4;
+    static __device__ __forceinline__ void unpack(const uint4 &w, F2 (&p)[N])
+    {
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) p[q] = pk(__uint_as_float(u[q] << 16), __uint_as_float(u[q] & 0xffff0000u));
+    }
+    static __device__ __forceinline__ uint4 pack(const F2 (&p)[N])
+    {
+        uint32_t u[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float lo, hi;
+            upk(p[q], lo, hi);
+            u[q] = pack_bf16x2(lo, hi);
+        }
+        return make_uint4(u[0], u[1], u[2], u[3]);
+    }
+};
+template <>
+struct Pairs<float> {
+    static constexpr int N = 2;
+    static __device__ __forceinline__ void unpack(const uint4 &w, F2 (&p)[N])
+    {
+        p[0] = pk(__uint_as_float(w.x), __uint_as_float(w.y));
+        p[1] = pk(__uint_as_float(w.z), __uint_as_float(w.w));
+    }
+    static __device__ __forceinline__ uint4 pack(const F2 (&p)[N])
+    {
+        float a, b, c, d;
+        upk(p[0], a, b);
+        upk(p[1], c, d);
+        return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c), __float_as_uint(d));
+    }
+};
+
+// A ReLU mask on two elements: d where z > 0, else 0 (the forward's test).
+__device__ __forceinline__ F2 relu_pass2(F2 z, F2 d)
+{
+    float z0, z1, d0, d1;
+    upk(z, z0, z1);
+    upk(d, d0, d1);
+    return pk(z0 > 0.f ? d0 : 0.f, z1 > 0.f ? d1 : 0.f);
 }
 
 template <typename T, class F>
@@ -158,14 +244,27 @@ struct StatsF {
 #pragma unroll
             for (int u = 0; u < kBnUnroll; ++u) {
                 if (!ok[u]) continue;
-                float xf[VL];
-                Item<T, VL>::unpack(xr[u], xf);
                 float a = 0.f, b = 0.f;
+                if constexpr (VL == 1) {
+                    const float d = xr[u] - shift;
+                    a = d;
+                    b = d * d;
+                } else {
+                    // fp32 within the item: each lane sums every other element
+                    F2 xp[Pairs<T>::N];
+                    Pairs<T>::unpack(xr[u], xp);
+                    F2 a2 = sp2(0.f), b2 = sp2(0.f);
 #pragma unroll
-                for (int j = 0; j < VL; ++j) {
-                    const float d = xf[j] - shift;
-                    a += d;
-                    b = fmaf(d, d, b);
+                    for (int q = 0; q < Pairs<T>::N; ++q) {
+                        const F2 d = add2(xp[q], sp2(-shift));
+                        a2 = add2(a2, d);
+                        b2 = fma2(d, d, b2);
+                    }
+                    float a0, a1, b0, b1;
+                    upk(a2, a0, a1);
+                    upk(b2, b0, b1);
+                    a = a0 + a1;
+                    b = b0 + b1;
                 }
                 s1 += (double)a;
                 s2 += (double)b;
@@ -192,7 +291,7 @@ __device__ __forceinline__ int64_t first_of_channel(const BnPieces &t, const Pla
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads, 3)
+__global__ void __launch_bounds__(kBnThreads, 6)
 bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, double *__restrict__ partials)
 {
     pdl_wait();
@@ -259,11 +358,20 @@ struct ApplyF {
 #pragma unroll
             for (int u = 0; u < kBnUnroll; ++u) {
                 if (!ok[u]) continue;
-                float xf[VL], of[VL];
-                Item<T, VL>::unpack(xr[u], xf);
+                if constexpr (VL == 1) {
+                    const float of[1] = {fmaxf(fmaf(g, xr[u], b), 0.f)};
+                    Item<T, VL>::store(y, io[u], of);
+                } else {
+                    F2 xp[Pairs<T>::N];
+                    Pairs<T>::unpack(xr[u], xp);
 #pragma unroll
-                for (int j = 0; j < VL; ++j) of[j] = fmaxf(fmaf(g, xf[j], b), 0.f);
-                Item<T, VL>::store(y, io[u], of);
+                    for (int q = 0; q < Pairs<T>::N; ++q) {
+                        float z0, z1;
+                        upk(fma2(sp2(g), xp[q], sp2(b)), z0, z1);
+                        xp[q] = pk(fmaxf(z0, 0.f), fmaxf(z1, 0.f));
+                    }
+                    st_v4(static_cast<uint4 *>(y) + io[u], Pairs<T>::pack(xp));
+                }
             }
         }
     };
@@ -279,7 +387,7 @@ struct ApplyF {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads, 3)
+__global__ void __launch_bounds__(kBnThreads, 6)
 bn_apply_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, const float *__restrict__ gamma,
                 const float *__restrict__ beta, const float *__restrict__ mean, const float *__restrict__ invstd,
                 void *__restrict__ y)
@@ -336,15 +444,27 @@ struct ReduceF {
 #pragma unroll
             for (int u = 0; u < kBnUnroll; ++u) {
                 if (!ok[u]) continue;
-                float xf[VL], gf[VL];
-                Item<T, VL>::unpack(xr[u], xf);
-                Item<T, VL>::unpack(gr[u], gf);
                 float a = 0.f, b = 0.f;
+                if constexpr (VL == 1) {
+                    const float dz = fmaf(k.gp, xr[u], k.bp) > 0.f ? gr[u] : 0.f;
+                    a = dz;
+                    b = dz * ((xr[u] - k.mu) * k.r);
+                } else {
+                    F2 xp[Pairs<T>::N], gp[Pairs<T>::N];
+                    Pairs<T>::unpack(xr[u], xp);
+                    Pairs<T>::unpack(gr[u], gp);
+                    F2 a2 = sp2(0.f), b2 = sp2(0.f);
 #pragma unroll
-                for (int j = 0; j < VL; ++j) {
-                    const float dz = fmaf(k.gp, xf[j], k.bp) > 0.f ? gf[j] : 0.f;
-                    a += dz;
-                    b = fmaf(dz, (xf[j] - k.mu) * k.r, b);
+                    for (int q = 0; q < Pairs<T>::N; ++q) {
+                        const F2 dz = relu_pass2(fma2(sp2(k.gp), xp[q], sp2(k.bp)), gp[q]);
+                        a2 = add2(a2, dz);
+                        b2 = fma2(dz, mul2(add2(xp[q], sp2(-k.mu)), sp2(k.r)), b2);
+                    }
+                    float a0, a1, b0, b1;
+                    upk(a2, a0, a1);
+                    upk(b2, b0, b1);
+                    a = a0 + a1;
+                    b = b0 + b1;
                 }
                 s1 += (double)a;
                 s2 += (double)b;
@@ -365,7 +485,7 @@ struct ReduceF {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kBnThreads, 3)
+__global__ void __launch_bounds__(kBnThreads, 4)
 bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices, int vec,
                      const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
                      const float *__restrict__ invstd, double *__restrict__ partials)
@@ -408,14 +528,15 @@ bn_bwd_finalize_kernel(const double *__restrict__ partials, int64_t C, int slice
     coef[3 * c + 2] = (float)(-a * s2 / n);
 }
 
-template <typename T>
+// ACC: add d to what dx already holds (a fixed choice per launch, so the
+// plain instance carries no read of dx).
+template <typename T, bool ACC>
 struct DxF {
     const void *x;
     const void *dy;
     void *dx;
     BwdCoef k;
     float a, b, cc;
-    bool acc;
     template <int VL>
     struct It {
         const void *x;
@@ -423,7 +544,6 @@ struct DxF {
         void *dx;
         BwdCoef k;
         float a, b, cc;
-        bool acc;
         __device__ __forceinline__ void step(const int64_t (&ii)[kBnUnroll], const int64_t (&io)[kBnUnroll],
                                              const bool (&ok)[kBnUnroll])
         {
@@ -437,24 +557,33 @@ struct DxF {
 #pragma unroll
             for (int u = 0; u < kBnUnroll; ++u) {
                 if (!ok[u]) continue;
-                float xf[VL], gf[VL], pf[VL], of[VL];
-                Item<T, VL>::unpack(xr[u], xf);
-                Item<T, VL>::unpack(gr[u], gf);
-                if (acc) Item<T, VL>::unpack(Item<T, VL>::load_rw(dx, ii[u]), pf);
+                if constexpr (VL == 1) {
+                    const float dz = fmaf(k.gp, xr[u], k.bp) > 0.f ? gr[u] : 0.f;
+                    const float d = fmaf(a, dz, fmaf(cc, (xr[u] - k.mu) * k.r, b));
+                    const float of[1] = {ACC ? Item<T, VL>::load_rw(dx, ii[u]) + d : d};
+                    Item<T, VL>::store(dx, ii[u], of);
+                } else {
+                    F2 xp[Pairs<T>::N], gp[Pairs<T>::N], pp[Pairs<T>::N];
+                    Pairs<T>::unpack(xr[u], xp);
+                    Pairs<T>::unpack(gr[u], gp);
+                    if constexpr (ACC) Pairs<T>::unpack(Item<T, VL>::load_rw(dx, ii[u]), pp);
 #pragma unroll
-                for (int j = 0; j < VL; ++j) {
-                    const float dz = fmaf(k.gp, xf[j], k.bp) > 0.f ? gf[j] : 0.f;
-                    const float d = fmaf(a, dz, fmaf(cc, (xf[j] - k.mu) * k.r, b));
-                    of[j] = acc ? pf[j] + d : d;
+                    for (int q = 0; q < Pairs<T>::N; ++q) {
+                        const F2 dz = relu_pass2(fma2(sp2(k.gp), xp[q], sp2(k.bp)), gp[q]);
+                        const F2 xh = mul2(add2(xp[q], sp2(-k.mu)), sp2(k.r));
+                        const F2 d = fma2(sp2(a), dz, fma2(sp2(cc), xh, sp2(b)));
+                        if constexpr (ACC) xp[q] = add2(pp[q], d);
+                        else xp[q] = d;
+                    }
+                    st_v4(static_cast<uint4 *>(dx) + ii[u], Pairs<T>::pack(xp));
                 }
-                Item<T, VL>::store(dx, ii[u], of);
             }
         }
     };
     template <int VL>
     __device__ __forceinline__ It<VL> items() const
     {
-        return It<VL>{x, dy, dx, k, a, b, cc, acc};
+        return It<VL>{x, dy, dx, k, a, b, cc};
     }
     template <class I>
     __device__ __forceinline__ void absorb(const I &)
@@ -462,16 +591,16 @@ struct DxF {
     }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kBnThreads, 3)
+template <typename T, bool ACC>
+__global__ void __launch_bounds__(kBnThreads, 4)
 bn_dx_kernel(BnPieces t, BnOutPieces d, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices,
              int vec, const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
-             const float *__restrict__ invstd, const float *__restrict__ coef, int accumulate)
+             const float *__restrict__ invstd, const float *__restrict__ coef)
 {
     pdl_wait();
     const PlaneJob p = plane_job(t, N, slices);
-    DxF<T> f{t.ptr[p.piece], dy, d.ptr[p.piece], bwd_coef(gamma, beta, mean, invstd, p.c), coef[3 * p.c],
-             coef[3 * p.c + 1], coef[3 * p.c + 2], accumulate != 0};
+    DxF<T, ACC> f{t.ptr[p.piece], dy, d.ptr[p.piece], bwd_coef(gamma, beta, mean, invstd, p.c), coef[3 * p.c],
+                  coef[3 * p.c + 1], coef[3 * p.c + 2]};
     for_planes<T>(p, C, HW, vec, f);
     pdl_trigger();
 }
@@ -532,9 +661,10 @@ cudaError_t bwd_t(const BnLaunch &a)
                    static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.gamma,
                    static_cast<const float *>(a.invstd), a.dgamma, a.dbeta, coef);
     if (e != cudaSuccess) return e;
-    return launch_pdl(bn_dx_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.din, a.dy, a.N,
-                      a.C, a.HW, slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
-                      static_cast<const float *>(a.invstd), static_cast<const float *>(coef), a.accumulate);
+    auto dx_kernel = a.accumulate ? bn_dx_kernel<T, true> : bn_dx_kernel<T, false>;
+    return launch_pdl(dx_kernel, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.din, a.dy, a.N, a.C,
+                      a.HW, slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
+                      static_cast<const float *>(a.invstd), static_cast<const float *>(coef));
 }
 
 }  // namespace

@@ -104,12 +104,6 @@ inline int plane_slices(int64_t N, int64_t C)
     return (int)s;
 }
 
-__device__ __forceinline__ F2 add2(F2 a, F2 b)
-{
-    F2 r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
-    return r;
-}
 
 // ------------------------------------------------------------ load units
 

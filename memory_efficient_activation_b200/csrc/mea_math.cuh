@@ -95,6 +95,12 @@ __device__ __forceinline__ F2 mul2(F2 a, F2 b)
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
     return r;
 }
+__device__ __forceinline__ F2 add2(F2 a, F2 b)
+{
+    F2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
 
 // Multiplicative correction 2^t_lo ~ 1 + t_lo ln 2 for a float-float t.
 __device__ __forceinline__ float corr(float t_hi, float t_lo)
