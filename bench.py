@@ -692,6 +692,31 @@ def _ops_for(wl, dev, args):
                         [lambda b=b, d=d, ws=ws, a=a: mea.swish_channel_bwd(b[0], b[1], a, "nchw", out=b[3], dalpha=d,
                                                                             workspace=ws)
                          for b, d, ws in zip(sets, ds, wss)], accounting.channel_swish_bwd_bytes(w.n, "f32", C)))
+    elif wl == "swish_channel_f32_grouped":
+        # Swish with alpha per channel on the six maps: the three small stages
+        # (28 x 28, 14 x 14, 7 x 7) as one grouped launch per direction, then
+        # all six in one grouped call (the three large maps are launched alone
+        # inside it)
+        all_ws = [synthetic.swish_channel_nchw(seed=8 + i, shape=synthetic.EFFNET_B0_SHAPES[i])
+                  for i in range(len(synthetic.EFFNET_B0_SHAPES))]
+        for tag, wls in (("small3", all_ws[3:]), ("all6", all_ws)):
+            fwd_b = sum(accounting.channel_swish_fwd_bytes(w.n, "f32", w.extra["alpha"].numel()) for w in wls)
+            bwd_b = sum(accounting.channel_swish_bwd_bytes(w.n, "f32", w.extra["alpha"].numel()) for w in wls)
+            k = _sets_for(bwd_b)
+            alphas = [w.extra["alpha"].to(dev) for w in wls]
+            sets = [[clones([w.x, w.dy, w.x, w.x], 1)[0] for w in wls] for _ in range(k)]
+            ds = [[torch.empty(a.numel(), dtype=torch.float32, device=dev) for a in alphas] for _ in range(k)]
+            need = mea.swish_channel_bwd_grouped_workspace_bytes(torch.float32, [tuple(w.x.shape) for w in wls])
+            wss = [torch.zeros(need, dtype=torch.uint8, device=dev) for _ in range(k)]
+            ops.append((f"{tag}_grouped_fwd",
+                        [lambda b=b, a=alphas: mea.swish_channel_fwd_grouped([t[0] for t in b], a,
+                                                                             outs=[t[2] for t in b])
+                         for b in sets], fwd_b))
+            ops.append((f"{tag}_grouped_bwd_dalpha",
+                        [lambda b=b, d=d, w_=w_, a=alphas: mea.swish_channel_bwd_grouped(
+                            [t[0] for t in b], [t[1] for t in b], a, outs=[t[3] for t in b], dalphas=d, workspace=w_)
+                         for b, d, w_ in zip(sets, ds, wss)], bwd_b))
+            del sets
     elif wl == "matmul_act_bf16":
         # the d x d matmul of problem B07 ([8 x 2048, 4096] x [4096, 4096]) with
         # the activation in its epilogue, and the same work unfused (cuBLAS
@@ -1047,7 +1072,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="swish_bf16",
                     choices=["swish_bf16", "family_bf16", "effnet_f32_dalpha", "effnet_f32_dalpha_grouped",
                              "affine_nhwc_bf16",
-                             "affine_family_nhwc_bf16", "swish_channel_f32", "matmul_act_bf16", "mlp_bf16",
+                             "affine_family_nhwc_bf16", "swish_channel_f32", "swish_channel_f32_grouped",
+                             "matmul_act_bf16", "mlp_bf16",
                              "densenet_bn_bf16", "swish_f32_1m", "memory_study"],
                     help="swish_bf16 (default) is the headline; the others print per-kernel diagnostics")
     args = ap.parse_args(argv)

@@ -324,6 +324,58 @@ MEA_API mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layou
                                            const float *alpha, void *dx, float *dalpha,
                                            void *workspace, size_t ws_bytes, mea_stream_t stream);
 
+/* One NCHW tensor of a grouped per-channel Swish call
+ * (mea_swish_channel_fwd_grouped / mea_swish_channel_bwd_grouped). */
+typedef struct {
+    const void *x;            /* device, [N, C, H, W] NCHW, read only (the saved tensor) */
+    const void *dy;           /* backward: device, same shape; ignored by the forward */
+    void *out;                /* device, same shape: y (forward) or dx (backward) */
+    const float *alpha;       /* device fp32[C], read only */
+    float *dalpha;            /* backward: device fp32[C], OVERWRITTEN; ignored by the forward */
+    int64_t shape[4];         /* N, C, H, W (each >= 0) */
+} mea_channel_segment_t;
+
+/* Forward of Swish with a per-channel alpha over several independent NCHW
+ * tensors: for every segment s, out_s = x_s Sigmoid(alpha_s,c x_s), each
+ * bitwise what mea_swish_channel_fwd (MEA_NCHW) gives on that segment alone.
+ * Segments whose planes take the library's row path (H W <= 1024 elements,
+ * 16-byte aligned tensors: EfficientNet's 28 x 28 to 1 x 1 stages) run in
+ * one grid, up to 32 per kernel; any other segment is launched alone.
+ *   segs         host array of nseg (>= 0) segments; read during the call only.
+ *   Every segment is validated as mea_swish_channel_fwd validates its
+ *   tensors, and no segment's output may overlap any other segment's input
+ *   or output (MEA_ERR_INVALID_ARG, nothing launched).
+ * Source: as mea_swish_channel_fwd; one launch for many layers' tensors is
+ * this library's (the pages call the activation once per layer). */
+MEA_API mea_status_t mea_swish_channel_fwd_grouped(mea_dtype_t dtype, int nseg,
+                                                   const mea_channel_segment_t *segs, mea_stream_t stream);
+
+/* Bytes of device workspace mea_swish_channel_bwd_grouped needs: the sum over
+ * segments of mea_swish_channel_bwd_workspace_bytes (MEA_NCHW) rounded up to
+ * 256 bytes.  Pure host arithmetic; 0 for an invalid request. */
+MEA_API size_t mea_swish_channel_bwd_grouped_workspace_bytes(mea_dtype_t dtype, int nseg,
+                                                             const mea_channel_segment_t *segs);
+
+/* Backward of Swish with a per-channel alpha over several independent NCHW
+ * tensors: dx_s and dalpha_s for every segment, each bitwise what
+ * mea_swish_channel_bwd (MEA_NCHW) gives on that segment alone (same blocks,
+ * same summation order).  The row-path segments run in one grid and their
+ * dalpha sums in a second, small kernel on the same stream.
+ *   segs         as in mea_swish_channel_fwd_grouped; dx may alias that
+ *                segment's dy or x exactly, no other overlap with any
+ *                segment; dalpha of different segments must not overlap.
+ *                A segment with C > 0 and no elements gets dalpha = 0.
+ *   workspace,
+ *   ws_bytes     device scratch of at least
+ *                mea_swish_channel_bwd_grouped_workspace_bytes(), 256-byte
+ *                aligned, any contents (the call clears what it needs).
+ *                Calls sharing a workspace must not run concurrently on the
+ *                GPU.
+ * Source: as mea_swish_channel_bwd. */
+MEA_API mea_status_t mea_swish_channel_bwd_grouped(mea_dtype_t dtype, int nseg,
+                                                   const mea_channel_segment_t *segs, void *workspace,
+                                                   size_t ws_bytes, mea_stream_t stream);
+
 /* Matrix multiply with the activation fused into its epilogue, forward:
  *   Z = X W^T  (bf16 inputs, fp32 accumulation on the tensor cores),
  *   z = Z rounded to bf16 (written when z is non-NULL),

@@ -37,6 +37,7 @@ from ._capi import ACT_IDS, LAYOUT_IDS, MeaError
 __all__ = [
     "act_fwd", "act_bwd", "act_fwd_grouped", "act_bwd_grouped", "affine_swish_fwd", "affine_swish_bwd",
     "affine_act_fwd", "affine_act_bwd", "swish_channel_fwd", "swish_channel_bwd",
+    "swish_channel_fwd_grouped", "swish_channel_bwd_grouped", "swish_channel_bwd_grouped_workspace_bytes",
     "matmul_act_fwd", "matmul_act_bwd",
     "concat_bn_relu_fwd", "concat_bn_relu_apply", "concat_bn_relu_bwd",
     "act_fwd_bwd_host",
@@ -419,6 +420,82 @@ def swish_channel_bwd(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, la
                                             ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x))
     _capi.check("mea_swish_channel_bwd", st)
     return dx, da
+
+
+def _channel_group_args(xs, alphas, name, dys=None, dalphas=None, outs=None):
+    """Checks a grouped per-channel call's lists (NCHW, one device and dtype,
+    alpha fp32 [C] per tensor) and builds its mea_channel_segment_t array;
+    returns (segments, outputs, d alphas)."""
+    xs, alphas = list(xs), list(alphas)
+    k = len(xs)
+    if len(alphas) != k or (dys is not None and len(dys) != k) or (outs is not None and len(outs) != k) \
+            or (dalphas is not None and len(dalphas) != k):
+        raise ValueError(f"{name}: every list must have one entry per tensor")
+    if k == 0:
+        return (_capi.ChannelSegment * 0)(), [], []
+    _need_cuda(*xs)
+    ref = xs[0]
+    for x in xs:
+        if x.device != ref.device or x.dtype != ref.dtype:
+            raise ValueError(f"{name}: every tensor must share the first one's device and dtype")
+    outs = [torch.empty_like(x) for x in xs] if outs is None else [_like(x, o, "out") for x, o in zip(xs, outs)]
+    das = []
+    segs = (_capi.ChannelSegment * k)()
+    for i, x in enumerate(xs):
+        shape = _affine_shape(x, "nchw")
+        C = shape[1]
+        _chan_params(C, alphas[i], device=x.device)
+        dy = _like(x, dys[i], "dy") if dys is not None else None
+        da = None
+        if dys is not None:
+            da = torch.empty(C, dtype=torch.float32, device=x.device) if dalphas is None else dalphas[i]
+            _chan_params(C, da, device=x.device)
+            das.append(da)
+        segs[i] = _capi.ChannelSegment(x.data_ptr(), dy.data_ptr() if dy is not None else None, outs[i].data_ptr(),
+                                       alphas[i].data_ptr(), da.data_ptr() if da is not None else None,
+                                       (ctypes.c_int64 * 4)(*shape))
+    return segs, outs, das
+
+
+def swish_channel_fwd_grouped(xs, alphas, outs=None) -> list:
+    """y_i = x_i Sigmoid(alpha_i,c x_i) for every NCHW tensor of xs in one
+    launch where the planes allow it (H W <= 1024 and 16-byte aligned); each
+    y_i is bitwise what swish_channel_fwd gives for x_i."""
+    segs, outs, _ = _channel_group_args(xs, alphas, "swish_channel_fwd_grouped", outs=outs)
+    if not outs:
+        return []
+    st = _capi.lib().mea_swish_channel_fwd_grouped(_dtype_id(outs[0]), len(outs), segs, _stream(outs[0]))
+    _capi.check("mea_swish_channel_fwd_grouped", st)
+    return outs
+
+
+def swish_channel_bwd_grouped_workspace_bytes(dtype: torch.dtype, shapes) -> int:
+    """Workspace bytes of a grouped per-channel backward over NCHW tensors of
+    these (N, C, H, W) shapes."""
+    shapes = [tuple(int(v) for v in sh) for sh in shapes]
+    if not shapes:
+        return 0
+    segs = (_capi.ChannelSegment * len(shapes))()
+    for i, sh in enumerate(shapes):
+        segs[i].shape = (ctypes.c_int64 * 4)(*sh)
+    return int(_capi.lib().mea_swish_channel_bwd_grouped_workspace_bytes(_DTYPES[dtype], len(shapes), segs))
+
+
+def swish_channel_bwd_grouped(xs, dys, alphas, outs=None, dalphas=None,
+                              workspace: torch.Tensor | None = None):
+    """Returns (dxs, dalphas) for every NCHW tensor of xs in one launch where
+    the planes allow it; each pair is bitwise what swish_channel_bwd gives."""
+    segs, outs, das = _channel_group_args(xs, alphas, "swish_channel_bwd_grouped", dys=dys, dalphas=dalphas,
+                                          outs=outs)
+    if not outs:
+        return [], []
+    x0 = outs[0]
+    need = int(_capi.lib().mea_swish_channel_bwd_grouped_workspace_bytes(_dtype_id(x0), len(outs), segs))
+    ws = _on_device(x0, workspace, "workspace") if workspace is not None else _pool.get(x0.device, _stream(x0), need)
+    st = _capi.lib().mea_swish_channel_bwd_grouped(_dtype_id(x0), len(outs), segs, ws.data_ptr(),
+                                                    ws.numel() * ws.element_size(), _stream(x0))
+    _capi.check("mea_swish_channel_bwd_grouped", st)
+    return outs, das
 
 
 def _mat2d(t: torch.Tensor, name: str) -> torch.Tensor:

@@ -44,7 +44,14 @@ class ActSegment(ctypes.Structure):
                 ("dparam_dev", _vp)]
 
 
+class ChannelSegment(ctypes.Structure):
+    """mea_channel_segment_t: one NCHW tensor of a grouped per-channel Swish call."""
+    _fields_ = [("x", _vp), ("dy", _vp), ("out", _vp), ("alpha", _vp), ("dalpha", _vp),
+                ("shape", ctypes.c_int64 * 4)]
+
+
 _segs = ctypes.POINTER(ActSegment)
+_csegs = ctypes.POINTER(ChannelSegment)
 SIGNATURES = {
     "mea_act_fwd": (_i, [_i, _i, _vp, _vp, _i64, _f, _vp, _vp]),
     "mea_act_bwd_workspace_bytes": (_sz, [_i, _i64, _i]),
@@ -52,6 +59,9 @@ SIGNATURES = {
     "mea_act_fwd_grouped": (_i, [_i, _i, _i, _segs, _vp]),
     "mea_act_bwd_grouped_workspace_bytes": (_sz, [_i, _i, _segs]),
     "mea_act_bwd_grouped": (_i, [_i, _i, _i, _segs, _vp, _sz, _vp]),
+    "mea_swish_channel_fwd_grouped": (_i, [_i, _i, _csegs, _vp]),
+    "mea_swish_channel_bwd_grouped_workspace_bytes": (_sz, [_i, _i, _csegs]),
+    "mea_swish_channel_bwd_grouped": (_i, [_i, _i, _csegs, _vp, _sz, _vp]),
     "mea_affine_swish_bwd_workspace_bytes": (_sz, [_i, _i, _shape]),
     "mea_affine_swish_fwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp]),
     "mea_affine_swish_bwd": (_i, [_i, _i, _shape, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),

@@ -510,6 +510,125 @@ mea_status_t mea_swish_channel_bwd(mea_dtype_t dtype, mea_layout_t layout, const
                     dalpha, nullptr, workspace, ws_bytes, stream);
 }
 
+// Validates a grouped per-channel Swish call and converts its segments.
+static mea_status_t channel_segments(const char *name, int nseg, const mea_channel_segment_t *segs, int dtype,
+                                     bool bwd, std::vector<mea::ChanSeg> &out)
+{
+    if (!valid_dtype(dtype)) return fail(MEA_ERR_INVALID_ARG, "dtype = %d is not a mea_dtype_t", dtype);
+    if (nseg < 0) return fail(MEA_ERR_INVALID_ARG, "%s: nseg = %d", name, nseg);
+    if (nseg > 0 && !segs) return fail(MEA_ERR_INVALID_ARG, "%s: segs is NULL", name);
+    const size_t es = dtype_bytes(dtype);
+    std::vector<size_t> bytes((size_t)nseg, 0);
+    for (int i = 0; i < nseg; ++i) {
+        const mea_channel_segment_t &g = segs[i];
+        int64_t n = 0;
+        mea_status_t st = check_shape(g.shape, &n);
+        if (st != MEA_OK) {
+            char why[256];
+            snprintf(why, sizeof(why), "%s", mea_last_error());
+            return fail(st, "%s: segment %d: %s", name, i, why);
+        }
+        bytes[(size_t)i] = (size_t)n * es;
+        const int64_t C = g.shape[1];
+        if (C > 0 && (!g.alpha || (bwd && !g.dalpha)))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: alpha%s is NULL", name, i, bwd ? " or dalpha" : "");
+        if (n == 0) continue;
+        if (!g.x || !g.out || (bwd && !g.dy))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: a tensor pointer is NULL", name, i);
+        const size_t b = bytes[(size_t)i];
+        if (!bwd && overlaps(g.x, b, g.out, b))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: y overlaps x", name, i);
+        if (bwd && (partial_overlap(g.out, g.dy, b) || partial_overlap(g.out, g.x, b)))
+            return fail(MEA_ERR_INVALID_ARG, "%s: segment %d: dx partially overlaps x or dy", name, i);
+    }
+    for (int i = 0; i < nseg; ++i) {
+        const size_t bi = bytes[(size_t)i], ci = (size_t)segs[i].shape[1] * sizeof(float);
+        for (int j = 0; j < nseg; ++j) {
+            if (j == i) continue;
+            const size_t bj = bytes[(size_t)j], cj = (size_t)segs[j].shape[1] * sizeof(float);
+            if (bi > 0 && bj > 0 &&
+                (overlaps(segs[i].out, bi, segs[j].x, bj) || overlaps(segs[i].out, bi, segs[j].out, bj) ||
+                 (bwd && overlaps(segs[i].out, bi, segs[j].dy, bj))))
+                return fail(MEA_ERR_INVALID_ARG, "%s: the output of segment %d overlaps a tensor of segment %d",
+                            name, i, j);
+            if (bwd && ci > 0 && cj > 0 && overlaps(segs[i].dalpha, ci, segs[j].dalpha, cj))
+                return fail(MEA_ERR_INVALID_ARG, "%s: dalpha of segments %d and %d overlap", name, i, j);
+        }
+    }
+    out.resize((size_t)nseg);
+    for (int i = 0; i < nseg; ++i) {
+        const mea_channel_segment_t &g = segs[i];
+        mea::ChanSeg c{};
+        c.x = g.x;
+        c.dy = bwd ? g.dy : nullptr;
+        c.out = g.out;
+        c.alpha = g.alpha;
+        c.dalpha = bwd ? g.dalpha : nullptr;
+        c.N = g.shape[0];
+        c.C = g.shape[1];
+        c.H = g.shape[2];
+        c.W = g.shape[3];
+        out[(size_t)i] = c;
+    }
+    return MEA_OK;
+}
+
+mea_status_t mea_swish_channel_fwd_grouped(mea_dtype_t dtype, int nseg, const mea_channel_segment_t *segs,
+                                           mea_stream_t stream)
+{
+    Range range_("mea_swish_channel_fwd_grouped");
+    clear_error();
+    std::vector<mea::ChanSeg> tab;
+    mea_status_t st = channel_segments("mea_swish_channel_fwd_grouped", nseg, segs, dtype, false, tab);
+    if (st != MEA_OK) return st;
+    if (nseg == 0) return MEA_OK;
+    cudaError_t e = mea::launch_channel_swish_fwd_grouped(dtype, nseg, tab.data(), reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_swish_channel_fwd_grouped launch");
+}
+
+size_t mea_swish_channel_bwd_grouped_workspace_bytes(mea_dtype_t dtype, int nseg, const mea_channel_segment_t *segs)
+{
+    if (nseg <= 0 || !segs) return 0;
+    size_t total = 0;
+    for (int i = 0; i < nseg; ++i) {
+        const size_t b = chan_ws_bytes(1, dtype, MEA_NCHW, segs[i].shape);
+        if (b == 0) return 0;
+        total += round256(b);
+    }
+    return total;
+}
+
+mea_status_t mea_swish_channel_bwd_grouped(mea_dtype_t dtype, int nseg, const mea_channel_segment_t *segs,
+                                           void *workspace, size_t ws_bytes, mea_stream_t stream)
+{
+    Range range_("mea_swish_channel_bwd_grouped");
+    clear_error();
+    std::vector<mea::ChanSeg> tab;
+    mea_status_t st = channel_segments("mea_swish_channel_bwd_grouped", nseg, segs, dtype, true, tab);
+    if (st != MEA_OK) return st;
+    if (nseg == 0) return MEA_OK;
+    const size_t need = mea_swish_channel_bwd_grouped_workspace_bytes(dtype, nseg, segs);
+    if (!workspace || ws_bytes < need)
+        return fail(MEA_ERR_WORKSPACE, "mea_swish_channel_bwd_grouped needs %zu bytes of workspace, got %zu%s", need,
+                    ws_bytes, workspace ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(MEA_ERR_WORKSPACE, "grouped workspace must be 256-byte aligned");
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    size_t off = 0;
+    for (int i = 0; i < nseg; ++i) {
+        tab[(size_t)i].ws = static_cast<char *>(workspace) + off;
+        off += round256(chan_ws_bytes(1, dtype, MEA_NCHW, segs[i].shape));
+        // An empty batch still defines d alpha: zero.
+        const mea::ChanSeg &g = tab[(size_t)i];
+        if (g.C > 0 && g.N * g.H * g.W == 0) {
+            cudaError_t e = cudaMemsetAsync(g.dalpha, 0, (size_t)g.C * sizeof(float), s);
+            if (e != cudaSuccess) return cuda_fail(e, "mea_swish_channel_bwd_grouped");
+        }
+    }
+    cudaError_t e = mea::launch_channel_swish_bwd_grouped(dtype, nseg, tab.data(), s);
+    return e == cudaSuccess ? MEA_OK : cuda_fail(e, "mea_swish_channel_bwd_grouped launch");
+}
+
 static mea_status_t check_matmul(const char *name, int act, int64_t M, int64_t N, int64_t K)
 {
     (void)name;

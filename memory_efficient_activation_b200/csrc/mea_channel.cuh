@@ -32,11 +32,17 @@
 // block; a second kernel adds each channel's column in block order.  So the
 // reductions are bitwise reproducible on any device.
 //
-// Plane path (NCHW, and NHWC shapes the fast path does not take): block
-// (c, s) owns channel c and the s-th slice of the batch; for NCHW it streams
-// the contiguous H W planes of that channel (16-byte vectors when H W is a
-// multiple of the vector width and the pointers are aligned), and the last
-// block to finish (atomic ticket) adds the per-block partials in order.
+// Row path (NCHW with planes of at most kRowMaxHW elements, aligned
+// pointers): a block streams a contiguous run of whole planes in 16-byte
+// vectors whatever H W is, finds each element's channel from its position,
+// and sums each plane's reduction terms in fixed order (chan_row_kernel).
+//
+// Plane path (larger NCHW planes, unaligned NCHW tensors, and NHWC shapes the
+// fast path does not take): block (c, s) owns channel c and the s-th slice
+// of the batch; for NCHW it streams the contiguous H W planes of that
+// channel (16-byte vectors when H W is a multiple of the vector width and
+// the pointers are aligned), and the last block to finish (atomic ticket)
+// adds the per-block partials in order.
 #pragma once
 
 #include <cstdint>
@@ -687,6 +693,281 @@ chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanA
     }
 }
 
+// ------------------------------------------------------------ row path
+// NCHW with small planes (EfficientNet's 7 x 7 to 28 x 28 stages): the
+// tensor read as N C planes of H W contiguous elements.  Block b owns the
+// whole planes [b P, b P + P), a contiguous range of P H W elements that it
+// streams in 16-byte vectors, so a plane of 49 elements costs no scalar
+// loads and no stride.  P is a multiple of the vector width over
+// gcd(H W, vector width), so every block starts on a 16-byte boundary; only
+// the last block can end inside a vector (its ragged end goes element by
+// element).  The constants of the block's planes sit in shared memory and
+// each element finds its plane by counting positions within the vector.
+//
+// Backward: each element's reduction terms (fp32) are staged in shared
+// memory; once the block's elements are done, warp w adds up planes w,
+// w + 8, ... in fp64 (lane l takes positions l, l + 32, ...; then a fixed
+// shuffle tree) and writes one value per plane and reduction to row n,
+// column r C + c of the partials; a second kernel adds each column over the
+// N rows in fixed order, one warp per column.  P depends only on the shape,
+// so the sums are bitwise reproducible on any device.
+constexpr int kRowThreads = 256;
+constexpr int kRowUnroll = 4;            // vectors in flight per thread
+constexpr int kRowBlocksTarget = 1184;   // 148 SMs x 8
+constexpr int kRowTerms = 8192;          // fp32 terms staged per block (32 KB)
+constexpr int kRowMaxPlanes = 256;
+#ifndef MEA_ROW_MAX_HW
+#define MEA_ROW_MAX_HW 1024
+#endif
+constexpr int64_t kRowMaxHW = MEA_ROW_MAX_HW;   // larger planes take the plane path
+
+struct RowShape {
+    int planes;          // P; 0: the row path is not taken
+    int64_t grid;
+};
+
+// P for nr reductions and vl elements per 16-byte vector: about
+// N C / kRowBlocksTarget planes, rounded up to the alignment multiple, at
+// most what the staging buffer and the constants table hold.
+inline RowShape row_shape(int nr, int vl, int64_t N, int64_t C, int64_t HW)
+{
+    const int64_t np = N * C;
+    if (np < 1 || HW < 1 || HW > kRowMaxHW) return RowShape{0, 0};
+    int64_t a = HW % vl, b = vl;
+    while (a) {
+        const int64_t t = b % a;
+        b = a;
+        a = t;
+    }
+    const int64_t m = vl / b;                 // planes per 16-byte-aligned step
+    int64_t pmax = kRowMaxPlanes;
+    if (nr > 0 && kRowTerms / (HW * nr) < pmax) pmax = kRowTerms / (HW * nr);
+    pmax -= pmax % m;
+    if (pmax < m) return RowShape{0, 0};
+    int64_t p = (np + kRowBlocksTarget - 1) / kRowBlocksTarget;
+    p = (p + m - 1) / m * m;
+    if (p > pmax) p = pmax;
+    return RowShape{(int)p, (np + p - 1) / p};
+}
+
+// Block `blk` of the row path over one tensor (the single-tensor kernel and
+// every segment of the grouped one run this).  Dynamic shared memory: NR P
+// H W floats in the backward.  The first vectors are requested before the
+// constants table is filled, so the two memory round trips overlap.
+template <class Op, typename T, int MODE>
+__device__ __forceinline__ void row_body(const void *__restrict__ x, const void *__restrict__ dy, const ChanArgs &ca,
+                                         void *__restrict__ out, int64_t C, int64_t HW, int64_t nplanes, int P,
+                                         double *__restrict__ partials, int64_t blk)
+{
+    constexpr bool Pk = Store<T>::P;
+    constexpr int NR = Op::NR;
+    constexpr int VL = Store<T>::V;
+    using I = Item<T, VL>;
+    using I1 = Item<T, 1>;
+    using Ch = typename Op::Ch;
+    extern __shared__ float terms[];   // [NR][P H W], MODE 1 only
+    __shared__ Ch chs[kRowMaxPlanes];
+    const int64_t g0 = blk * P;
+    const uint32_t np = (uint32_t)(nplanes - g0 < P ? nplanes - g0 : P);
+    const uint32_t hw = (uint32_t)HW;
+    const uint32_t L = np * hw;               // elements of the block
+    const uint32_t ld = (uint32_t)P * hw;     // stride of terms between reductions
+    const int64_t e0 = g0 * HW;
+    const uint32_t nv = L / VL;
+    const int64_t v0g = e0 / VL;
+    typename I::Raw xr[kRowUnroll], gr[kRowUnroll];
+    auto load_batch = [&](uint32_t q0) {
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+            const uint32_t q = q0 + u * kRowThreads;
+            if (q < nv) {
+                xr[u] = I::load(x, v0g + q);
+                if constexpr (MODE == 1) gr[u] = I::load(dy, v0g + q);
+            }
+        }
+    };
+    pdl_wait();
+    load_batch(threadIdx.x);
+    const typename Op::K k = Op::kcoef(ca);
+    for (uint32_t i = threadIdx.x; i < np; i += kRowThreads) chs[i] = Op::load(ca, (int)((g0 + i) % C));
+    __syncthreads();
+    const DivU32 div(hw);
+
+    // One element of plane lp: the value (MODE 0) or dx and its reduction
+    // terms, written to tm[NR].
+    auto elem = [&](float xv, float gv, uint32_t lp, float (&tm)[NR]) -> float {
+        const Ch h = chs[lp];
+        bool tail = false;
+        if constexpr (MODE == 0) {
+            const float y = Op::template f<Pk>(xv, k, h, tail);
+            return tail && Op::is_tail(xv, k, h) ? Op::template f_tail<Pk>(xv, k, h) : y;
+        } else {
+            float o, t;
+            Op::template bwd<Pk>(xv, gv, k, h, tail, o, t);
+            if (tail && Op::template flag_bwd<Pk>(xv, k, h)) Op::template bwd_tail<Pk>(xv, gv, k, h, o, t);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) tm[r] = 0.f;
+            return Op::finish(xv, o, t, h, tm);
+        }
+    };
+
+    for (uint32_t q0 = threadIdx.x; q0 < nv; q0 += kRowUnroll * kRowThreads) {
+        if (q0 != threadIdx.x) load_batch(q0);
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+            const uint32_t q = q0 + u * kRowThreads;
+            if (q >= nv) continue;
+            float xf[VL], gf[VL], of[VL], tv[NR][VL];
+            I::unpack(xr[u], xf);
+            if constexpr (MODE == 1) I::unpack(gr[u], gf);
+            uint32_t lp, pos;
+            div.divmod(q * VL, lp, pos);
+#pragma unroll
+            for (int j = 0; j < VL; ++j) {
+                float tm[NR];
+                of[j] = elem(xf[j], MODE == 1 ? gf[j] : 0.f, lp, tm);
+                if constexpr (MODE == 1) {
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) tv[r][j] = tm[r];
+                }
+                if (++pos == hw) {
+                    pos = 0;
+                    ++lp;
+                }
+            }
+            I::store(out, v0g + q, of);
+            if constexpr (MODE == 1) {
+#pragma unroll
+                for (int r = 0; r < NR; ++r)
+#pragma unroll
+                    for (int j = 0; j < VL; j += 4)
+                        *reinterpret_cast<float4 *>(terms + r * ld + q * VL + j) =
+                            make_float4(tv[r][j], tv[r][j + 1], tv[r][j + 2], tv[r][j + 3]);
+            }
+        }
+    }
+    // The ragged end of the last block (fewer than VL elements).
+    for (uint32_t l = nv * VL + threadIdx.x; l < L; l += kRowThreads) {
+        float tm[NR];
+        const float xv = I1::load(x, e0 + l);
+        const float gv = MODE == 1 ? (float)I1::load(dy, e0 + l) : 0.f;
+        const float of[1] = {elem(xv, gv, l / hw, tm)};
+        I1::store(out, e0 + l, of);
+        if constexpr (MODE == 1) {
+#pragma unroll
+            for (int r = 0; r < NR; ++r) terms[r * ld + l] = tm[r];
+        }
+    }
+    pdl_trigger();
+    if constexpr (MODE == 1) {
+        __syncthreads();
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        for (uint32_t lp = w; lp < np; lp += kRowThreads / 32) {
+            const int64_t g = g0 + lp;
+            const int64_t n = g / C, c = g - n * C;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                double v = 0.0;
+                for (uint32_t i = lane; i < hw; i += 32) v += (double)terms[r * ld + lp * hw + i];
+                v = warp_sum(v);
+                if (lane == 0) partials[(n * NR + r) * C + c] = v;
+            }
+        }
+    }
+}
+
+// Column o of the row path's [N][NR C] partials: lane l adds rows l, l + 32,
+// ... in order, then a fixed shuffle tree (one warp per column).
+__device__ __forceinline__ double row_colsum(const double *__restrict__ partials, int64_t N, int64_t ld, int64_t o)
+{
+    double v = 0.0;
+    for (int64_t n = threadIdx.x & 31; n < N; n += 32) v += partials[n * ld + o];
+    return warp_sum(v);
+}
+
+template <class Op, typename T, int MODE>
+__global__ void __launch_bounds__(kRowThreads)
+chan_row_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanArgs ca, void *__restrict__ out,
+                int64_t C, int64_t HW, int64_t nplanes, int P, double *__restrict__ partials)
+{
+    row_body<Op, T, MODE>(x, dy, ca, out, C, HW, nplanes, P, partials, blockIdx.x);
+}
+
+// Output o (r C + c) of the row path: r = 0 to out0, r = 1 to out1.
+template <int NR>
+__global__ void __launch_bounds__(kRowThreads)
+chan_row_colsum_kernel(const double *__restrict__ partials, int64_t N, int64_t C, float *__restrict__ out0,
+                       float *__restrict__ out1)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t o = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    if (o >= NR * C) return;
+    const double v = row_colsum(partials, N, NR * C, o);
+    if ((threadIdx.x & 31) == 0) {
+        if (o < C) out0[o] = (float)v;
+        else out1[o - C] = (float)v;
+    }
+}
+
+// Grouped row path: segments laid end to end in one grid (block ranges
+// start[s] .. start[s + 1]); the column sums of segment s are outputs
+// ostart[s] .. ostart[s + 1] of the second kernel.  Each segment's blocks
+// and sums are those of its single-tensor launch, so its results are
+// bitwise the same.
+constexpr int kMaxRowSegs = 32;
+struct RowSeg {
+    const void *x;
+    const void *dy;
+    void *out;
+    const float *p0;
+    const float *p1;
+    double *partials;
+    float *out0;
+    float *out1;
+    int64_t N, C, HW;
+    int P;
+};
+struct RowSegTable {
+    RowSeg seg[kMaxRowSegs];
+    int start[kMaxRowSegs + 1];
+    int ostart[kMaxRowSegs + 1];
+    int nseg;
+    float scalar;
+};
+static_assert(sizeof(RowSegTable) < 4000, "kernel parameter space");
+
+template <class Op, typename T, int MODE>
+__global__ void __launch_bounds__(kRowThreads)
+chan_row_group_kernel(const __grid_constant__ RowSegTable tab)
+{
+    int s = 0;
+    while (s + 1 < tab.nseg && (int)blockIdx.x >= tab.start[s + 1]) ++s;
+    const RowSeg &g = tab.seg[s];
+    const ChanArgs ca{g.p0, g.p1, tab.scalar};
+    row_body<Op, T, MODE>(g.x, g.dy, ca, g.out, g.C, g.HW, g.N * g.C, g.P, g.partials,
+                          (int64_t)blockIdx.x - tab.start[s]);
+}
+
+template <int NR>
+__global__ void __launch_bounds__(kRowThreads)
+chan_row_group_colsum_kernel(const __grid_constant__ RowSegTable tab)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t og = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    if (og >= tab.ostart[tab.nseg]) return;
+    int s = 0;
+    while (s + 1 < tab.nseg && og >= tab.ostart[s + 1]) ++s;
+    const RowSeg &g = tab.seg[s];
+    const int64_t o = og - tab.ostart[s];
+    const double v = row_colsum(g.partials, g.N, NR * g.C, o);
+    if ((threadIdx.x & 31) == 0) {
+        if (o < g.C) g.out0[o] = (float)v;
+        else g.out1[o - g.C] = (float)v;
+    }
+}
+
 // ------------------------------------------------------------ launchers
 
 inline int64_t nhwc_blocks(int64_t nunits, int threads, int U)
@@ -757,6 +1038,10 @@ inline size_t chan_bwd_workspace_bytes(int nr, int dtype, int layout, int64_t N,
     const int VE = dtype == kBF16 ? NhwcCfg<Bf16>::VE : NhwcCfg<float>::VE;
     const int U = dtype == kBF16 ? NhwcCfg<Bf16>::U_BWD : NhwcCfg<float>::U_BWD;
     size_t plane = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)plane_slices(N, C);
+    if (layout == 0 && row_shape(nr, dtype == kBF16 ? Store<Bf16>::V : Store<float>::V, N, C, H * W).planes > 0) {
+        const size_t row = kWsHeader + sizeof(double) * nr * (size_t)C * (size_t)N;
+        if (row > plane) plane = row;
+    }
     if (layout == 1 && C % VE == 0 && nhwc_threads((int)(C / VE)) > 0) {
         const int threads = nhwc_threads((int)(C / VE));
         const int64_t nunits = N * C * H * W / VE;
@@ -824,6 +1109,18 @@ cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out
     }
     uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
     if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
+    const RowShape rs = a.layout == 0 ? row_shape(NR, V, a.N, a.C, HW) : RowShape{0, 0};
+    if (rs.planes > 0 && (al & 15u) == 0) {
+        if (rs.grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+        double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
+        const size_t smem = MODE == 1 ? sizeof(float) * NR * (size_t)rs.planes * (size_t)HW : 0;
+        cudaError_t e = launch_pdl(chan_row_kernel<Op, T, MODE>, dim3((unsigned)rs.grid), dim3(kRowThreads), smem,
+                                   a.stream, a.x, a.dy, ca, a.out, a.C, HW, a.N * a.C, rs.planes, partials);
+        if (e != cudaSuccess || MODE == 0) return e;
+        const int64_t cb = (NR * a.C + kRowThreads / 32 - 1) / (kRowThreads / 32);
+        return launch_pdl(chan_row_colsum_kernel<NR>, dim3((unsigned)cb), dim3(kRowThreads), 0, a.stream,
+                          static_cast<const double *>(partials), a.N, a.C, out0, out1);
+    }
     const int vec_ok = a.layout == 0 && HW % V == 0 && (al & 15u) == 0;
     const int slices = plane_slices(a.N, a.C);
     const int64_t grid = a.C * slices;

@@ -113,4 +113,110 @@ cudaError_t launch_channel_swish_bwd(const AffineLaunch &a)
                             : launch_channel<ChannelSwishOp, float, 1>(a, ca, a.dgamma, nullptr);
 }
 
+namespace {
+
+// Segments the row path takes go into one grid (kMaxRowSegs at a time),
+// each with the block partition and partials of its single-tensor launch;
+// any other segment is launched alone on its usual path.
+template <typename T, int MODE>
+cudaError_t launch_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_t stream)
+{
+    constexpr int NR = ChannelSwishOp::NR, V = Store<T>::V;
+    RowSegTable tab{};
+    tab.scalar = 1.f;
+    int k = 0;
+    int64_t blocks = 0, outs = 0;
+    size_t smem = 0;
+    auto flush = [&]() -> cudaError_t {
+        if (k == 0) return cudaSuccess;
+        tab.nseg = k;
+        tab.start[k] = (int)blocks;
+        tab.ostart[k] = (int)outs;
+        cudaError_t e = launch_pdl(chan_row_group_kernel<ChannelSwishOp, T, MODE>, dim3((unsigned)blocks),
+                                   dim3(kRowThreads), smem, stream, tab);
+        if (e == cudaSuccess && MODE == 1) {
+            const int64_t cb = (outs + kRowThreads / 32 - 1) / (kRowThreads / 32);
+            e = launch_pdl(chan_row_group_colsum_kernel<NR>, dim3((unsigned)cb), dim3(kRowThreads), 0, stream, tab);
+        }
+        k = 0;
+        blocks = outs = 0;
+        smem = 0;
+        return e;
+    };
+    for (int i = 0; i < nseg; ++i) {
+        const ChanSeg &g = segs[i];
+        const int64_t HW = g.H * g.W;
+        if (g.N * g.C * HW == 0) continue;
+        uintptr_t al = reinterpret_cast<uintptr_t>(g.x) | reinterpret_cast<uintptr_t>(g.out);
+        if (MODE == 1) al |= reinterpret_cast<uintptr_t>(g.dy);
+        const RowShape rs = row_shape(NR, V, g.N, g.C, HW);
+        cudaError_t e = cudaSuccess;
+        if (rs.planes == 0 || (al & 15u) || rs.grid > 0x7fffffff || NR * g.C > 0x7fffffff) {
+            AffineLaunch a{};
+            a.act = 6;
+            a.param = 1.f;
+            a.dtype = dtype;
+            a.layout = 0;
+            a.N = g.N;
+            a.C = g.C;
+            a.H = g.H;
+            a.W = g.W;
+            a.x = g.x;
+            a.dy = g.dy;
+            a.gamma = g.alpha;
+            a.out = g.out;
+            a.dgamma = g.dalpha;
+            a.workspace = g.ws;
+            a.stream = stream;
+            if (MODE == 1) e = cudaMemsetAsync(g.ws, 0, kWsHeader, stream);
+            if (e == cudaSuccess)
+                e = launch_channel<ChannelSwishOp, T, MODE>(a, ChanArgs{g.alpha, nullptr, 1.f},
+                                                            MODE == 1 ? g.dalpha : nullptr, nullptr);
+            if (e != cudaSuccess) return e;
+            continue;
+        }
+        if (k == kMaxRowSegs || blocks + rs.grid > 0x7fffffff || outs + NR * g.C > 0x7fffffff) {
+            e = flush();
+            if (e != cudaSuccess) return e;
+        }
+        RowSeg &r = tab.seg[k];
+        r.x = g.x;
+        r.dy = MODE == 1 ? g.dy : nullptr;
+        r.out = g.out;
+        r.p0 = g.alpha;
+        r.p1 = nullptr;
+        r.partials = MODE == 1 ? reinterpret_cast<double *>(static_cast<char *>(g.ws) + kWsHeader) : nullptr;
+        r.out0 = MODE == 1 ? g.dalpha : nullptr;
+        r.out1 = nullptr;
+        r.N = g.N;
+        r.C = g.C;
+        r.HW = HW;
+        r.P = rs.planes;
+        tab.start[k] = (int)blocks;
+        tab.ostart[k] = (int)outs;
+        blocks += rs.grid;
+        outs += NR * g.C;
+        if (MODE == 1) {
+            const size_t b = sizeof(float) * NR * (size_t)rs.planes * (size_t)HW;
+            if (b > smem) smem = b;
+        }
+        ++k;
+    }
+    return flush();
+}
+
+}  // namespace
+
+cudaError_t launch_channel_swish_fwd_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_t stream)
+{
+    return dtype == kBF16 ? launch_grouped<Bf16, 0>(dtype, nseg, segs, stream)
+                          : launch_grouped<float, 0>(dtype, nseg, segs, stream);
+}
+
+cudaError_t launch_channel_swish_bwd_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_t stream)
+{
+    return dtype == kBF16 ? launch_grouped<Bf16, 1>(dtype, nseg, segs, stream)
+                          : launch_grouped<float, 1>(dtype, nseg, segs, stream);
+}
+
 }  // namespace mea

@@ -38,4 +38,20 @@ size_t channel_swish_bwd_workspace_bytes(int dtype, int layout, int64_t N, int64
 cudaError_t launch_channel_swish_fwd(const AffineLaunch &a);
 cudaError_t launch_channel_swish_bwd(const AffineLaunch &a);
 
+// One NCHW tensor of a grouped Swish launch with a per-channel alpha.
+struct ChanSeg {
+    const void *x;
+    const void *dy;          // backward only
+    void *out;               // y or dx
+    const float *alpha;      // [C]
+    float *dalpha;           // [C], backward only
+    int64_t N, C, H, W;
+    void *ws;                // backward: this segment's workspace (channel_swish_bwd_workspace_bytes)
+};
+// Segments whose planes take the row path run in one grid (up to 32 per
+// launch, their d alpha sums in a second one); any other segment runs alone
+// on its usual path (its workspace counter cleared first).
+cudaError_t launch_channel_swish_fwd_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_t stream);
+cudaError_t launch_channel_swish_bwd_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_t stream);
+
 }  // namespace mea

@@ -34,7 +34,7 @@ def _header_enum(name):
 
 def test_every_declared_symbol_is_exported(lib):
     declared = _header_functions()
-    assert len(declared) == 27, declared
+    assert len(declared) == 30, declared
     for fn in declared:
         assert hasattr(lib, fn), fn
         assert fn in _capi.SIGNATURES, fn
@@ -361,3 +361,50 @@ def test_binding_matmul_and_bn_patterns_with_stand_in_library(monkeypatch):
         with pytest.raises(ValueError):
             call()
     assert len(fake.calls) == n
+
+
+def _chan_segs(specs):
+    segs = (_capi.ChannelSegment * len(specs))()
+    for i, (x, dy, out, alpha, dalpha, shape) in enumerate(specs):
+        segs[i] = _capi.ChannelSegment(x, dy, out, alpha, dalpha, (_capi.ctypes.c_int64 * 4)(*shape))
+    return segs
+
+
+def test_channel_grouped_validation(lib):
+    # grouped Swish with a per-channel alpha: every refusal happens before a
+    # launch (fake addresses), and the workspace is the per-segment sizes,
+    # each rounded up to 256 bytes
+    sh_a, sh_b = (2, 16, 7, 7), (3, 40, 14, 14)
+    f = lib.mea_swish_channel_fwd_grouped
+    b = lib.mea_swish_channel_bwd_grouped
+    ok2 = _chan_segs([(X, None, Y, G, None, sh_a), (0x500000, None, 0x600000, 0x310000, None, sh_b)])
+    assert f(1, 0, None, None) == _capi.MEA_OK
+    assert f(1, -1, ok2, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(1, 2, None, None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(7, 2, ok2, None) == _capi.MEA_ERR_INVALID_ARG
+    neg = _chan_segs([(X, None, Y, G, None, sh_a), (X, None, Y, G, None, (1, -4, 2, 2))])
+    assert f(1, 2, neg, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b"segment 1" in lib.mea_last_error() and b"negative" in lib.mea_last_error()
+    assert f(1, 1, _chan_segs([(X, None, Y, None, None, sh_a)]), None) == _capi.MEA_ERR_INVALID_ARG
+    assert f(1, 1, _chan_segs([(X, None, X + 64, G, None, sh_a)]), None) == _capi.MEA_ERR_INVALID_ARG
+    # segment 1's output lands on segment 0's input
+    cross = _chan_segs([(X, None, Y, G, None, sh_a), (0x500000, None, X + 128, 0x310000, None, sh_b)])
+    assert f(1, 2, cross, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b"overlaps" in lib.mea_last_error()
+    wq = lib.mea_swish_channel_bwd_grouped_workspace_bytes
+    per = [lib.mea_swish_channel_bwd_workspace_bytes(1, _capi.MEA_NCHW, _capi.shape4(s)) for s in (sh_a, sh_b)]
+    need = wq(1, 2, ok2)
+    assert need == sum((p + 255) // 256 * 256 for p in per)
+    assert wq(1, 0, ok2) == 0 and wq(1, 2, neg) == 0 and wq(9, 2, ok2) == 0
+    bsegs = _chan_segs([(X, D, Y, G, 0x700000, sh_a), (0x500000, 0x580000, 0x600000, 0x310000, 0x710000, sh_b)])
+    assert b(1, 2, bsegs, 0x800000, need - 1, None) == _capi.MEA_ERR_WORKSPACE
+    assert b(1, 2, bsegs, None, need, None) == _capi.MEA_ERR_WORKSPACE
+    assert b(1, 2, bsegs, 0x800010, need, None) == _capi.MEA_ERR_WORKSPACE
+    assert b"256-byte" in lib.mea_last_error()
+    nod = _chan_segs([(X, D, Y, G, None, sh_a)])
+    assert b(1, 1, nod, 0x800000, need, None) == _capi.MEA_ERR_INVALID_ARG
+    shared_da = _chan_segs([(X, D, Y, G, 0x700000, sh_a), (0x500000, 0x580000, 0x600000, 0x310000, 0x700020, sh_b)])
+    assert b(1, 2, shared_da, 0x800000, need, None) == _capi.MEA_ERR_INVALID_ARG
+    assert b"dalpha" in lib.mea_last_error()
+    part = _chan_segs([(X, D, X + 2, G, 0x700000, sh_a)])
+    assert b(1, 1, part, 0x800000, need, None) == _capi.MEA_ERR_INVALID_ARG

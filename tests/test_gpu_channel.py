@@ -31,6 +31,10 @@ ACTS = ["relu", "leaky_relu", "sigmoid", "tanh", "gelu_erf", "gelu_tanh", "swish
 SHAPES = [
     ("nhwc", (2, 5, 7, 144)), ("nhwc", (2, 3, 5, 12)), ("nhwc", (2, 2, 3, 5)), ("nhwc", (2, 3, 3, 1152)),
     ("nchw", (2, 16, 7, 7)), ("nchw", (2, 8, 4, 8)), ("nchw", (3, 5, 3, 3)), ("nchw", (2, 96, 14, 14)),
+    # row path: several planes per vector (1 x 1, 1 x 3), a ragged last block
+    ("nchw", (5, 37, 1, 1)), ("nchw", (3, 7, 1, 3)), ("nchw", (3, 201, 7, 7)),
+    # plane path (planes above the row path's size): scalar and vector loads
+    ("nchw", (2, 3, 33, 33)), ("nchw", (2, 4, 40, 40)),
 ]
 
 
@@ -273,7 +277,41 @@ def test_swish_channel_full_workload():
     _channel_compare("f32", "nchw", tuple(w.x.shape), w.x, w.dy, w.extra["alpha"], y, dx, da)
 
 
-@pytest.mark.parametrize("layout,shape", [("nhwc", (16, 14, 14, 144)), ("nchw", (16, 40, 14, 14))])
+@pytest.mark.parametrize("shape", [(64, 480, 14, 14), (64, 1152, 7, 7), (64, 240, 28, 28)])
+def test_swish_channel_effnet_small_planes(shape):
+    # EfficientNet-B0's 28 x 28, 14 x 14 and 7 x 7 stages at batch 64 (the
+    # row path: hundreds of blocks of whole planes), every output
+    x, dy, _, _, a = _inputs(shape, "nchw", "f32", 416, sigma=1.5)
+    y = mea.swish_channel_fwd(x.cuda(), a.cuda(), "nchw")
+    dx, da = mea.swish_channel_bwd(x.cuda(), dy.cuda(), a.cuda(), "nchw")
+    torch.cuda.synchronize()
+    _channel_compare("f32", "nchw", shape, x, dy, a, y, dx, da)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(3, 40, 7, 7), (2, 24, 14, 14)])
+def test_channel_ops_nchw_unaligned(dtype, shape):
+    # tensors starting one element past a 16-byte boundary leave the row path
+    # for the plane path; both must match the oracle
+    x, dy, g, b, a = _inputs(shape, "nchw", dtype, 417, sigma=1.5)
+    n = x.numel()
+    xb = torch.empty(n + 1, dtype=x.dtype, device="cuda")
+    gb = torch.empty(n + 1, dtype=x.dtype, device="cuda")
+    xs, gs = xb[1:].view(shape), gb[1:].view(shape)
+    xs.copy_(x.cuda())
+    gs.copy_(dy.cuda())
+    assert xs.data_ptr() % 16 != 0 and gs.data_ptr() % 16 != 0
+    y = mea.swish_channel_fwd(xs, a.cuda(), "nchw")
+    dx, da = mea.swish_channel_bwd(xs, gs, a.cuda(), "nchw")
+    ya = mea.affine_act_fwd("gelu_erf", xs, g.cuda(), b.cuda(), 1.0, "nchw")
+    dxa, dg, db = mea.affine_act_bwd("gelu_erf", xs, gs, g.cuda(), b.cuda(), 1.0, "nchw")
+    torch.cuda.synchronize()
+    _channel_compare(dtype, "nchw", shape, x, dy, a, y, dx, da)
+    _affine_compare("gelu_erf", dtype, "nchw", shape, x, dy, g, b, ya, dxa, dg, db)
+
+
+@pytest.mark.parametrize("layout,shape", [("nhwc", (16, 14, 14, 144)), ("nchw", (16, 40, 14, 14)),
+                                          ("nchw", (16, 40, 33, 33))])
 def test_swish_channel_deterministic_and_counter_reset(layout, shape):
     x, dy, _, _, a = _inputs(shape, layout, "f32", 413, sigma=1.5)
     x, dy, a = x.cuda(), dy.cuda(), a.cuda()

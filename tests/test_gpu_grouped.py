@@ -1,5 +1,6 @@
 """GPU tests of the grouped entry points (mea_act_fwd_grouped /
-mea_act_bwd_grouped) through the C ABI.
+mea_act_bwd_grouped, mea_swish_channel_fwd_grouped /
+mea_swish_channel_bwd_grouped) through the C ABI.
 
 Each segment of a grouped launch runs exactly the work of its own single
 launch (same block count, element assignment and summation order), so the
@@ -8,7 +9,12 @@ tensor bit for bit: checked for every activation and both dtypes over
 segments of ragged sizes (0, 1, 7, 4097, 100003, 2^20 + 3), a view that is
 not 16-byte aligned, more than 32 segments (several launches), host and
 device alphas.  The EfficientNet-B0 shapes of the fp32 learnable-alpha
-workload are also compared with the oracle directly.
+workload are also compared with the oracle directly.  The grouped
+per-channel calls are held to the same rule against mea_swish_channel_fwd /
+mea_swish_channel_bwd (NCHW) on every segment, including the segments they
+launch alone (large planes, unaligned tensors), an empty batch, more than
+32 segments and a workspace of arbitrary contents; the EfficientNet-B0 small
+stages with alpha per channel are compared with the oracle.
 """
 import numpy as np
 import pytest
@@ -16,7 +22,7 @@ import torch
 
 import memory_efficient_activation_b200 as mea
 import oracle
-from _compare import TINY, check, to_f64
+from _compare import TINY, check, check_channel_sums, to_f64
 from memory_efficient_activation_b200 import synthetic
 
 pytestmark = pytest.mark.gpu
@@ -131,3 +137,106 @@ def test_grouped_rejects_overlap_and_partial_dparam():
     with pytest.raises(mea.MeaError):
         mea.act_bwd_grouped("swish", [x, x.clone()], [x.clone(), x.clone()],
                             dparams=[torch.empty(1, device="cuda"), None])
+
+
+# ------------------------------------------------- Swish with alpha per channel
+
+# Row-path shapes (several planes per vector, a ragged last block, EfficientNet
+# stages), an empty batch, and a plane-path shape (40 x 40 planes) that the
+# grouped call launches alone.
+CHANNEL_SHAPES = [(2, 16, 7, 7), (3, 201, 7, 7), (5, 37, 1, 1), (3, 7, 1, 3), (0, 16, 7, 7), (2, 4, 40, 40),
+                  (4, 96, 14, 14), (2, 24, 28, 28)]
+
+
+def _channel_tensors(shapes, dtype, seed, misaligned=True):
+    xs, dys, alphas = [], [], []
+    for i, shape in enumerate(shapes):
+        w = synthetic.swish_channel_nchw(seed + i, shape, dtype)
+        xs.append(w.x.cuda())
+        dys.append(w.dy.cuda())
+        alphas.append(w.extra["alpha"].cuda())
+    if misaligned:
+        # tensors one element past a 16-byte boundary: launched alone on the plane path
+        shape = (2, 24, 14, 14)
+        w = synthetic.swish_channel_nchw(seed + 99, shape, dtype)
+        n = w.x.numel()
+        bx = torch.empty(n + 1, dtype=w.x.dtype, device="cuda")
+        bg = torch.empty(n + 1, dtype=w.x.dtype, device="cuda")
+        bx[1:].copy_(w.x.reshape(-1).cuda())
+        bg[1:].copy_(w.dy.reshape(-1).cuda())
+        xs.append(bx[1:].view(shape))
+        dys.append(bg[1:].view(shape))
+        alphas.append(w.extra["alpha"].cuda())
+    return xs, dys, alphas
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_channel_grouped_equals_single_launches(dtype):
+    xs, dys, alphas = _channel_tensors(CHANNEL_SHAPES, dtype, 511)
+    ys = mea.swish_channel_fwd_grouped(xs, alphas)
+    dxs, das = mea.swish_channel_bwd_grouped(xs, dys, alphas)
+    ref_y = [mea.swish_channel_fwd(x, a, "nchw") for x, a in zip(xs, alphas)]
+    ref = [mea.swish_channel_bwd(x, g, a, "nchw") for x, g, a in zip(xs, dys, alphas)]
+    torch.cuda.synchronize()
+    for a, b in zip(ys, ref_y):
+        assert torch.equal(_bits(a), _bits(b))
+    for dx, da, (rdx, rda) in zip(dxs, das, ref):
+        assert torch.equal(_bits(dx), _bits(rdx))
+        assert torch.equal(da.view(torch.int32), rda.view(torch.int32))
+    assert torch.all(das[CHANNEL_SHAPES.index((0, 16, 7, 7))] == 0)
+
+
+def test_channel_grouped_many_segments_and_dirty_workspace():
+    # 40 row-path segments (two grids of at most 32), a workspace filled with
+    # garbage before each call: the same bits every time
+    shapes = [(1 + i % 3, 8 + 4 * (i % 5), 7, 7) if i % 2 else (2, 12 + i, 14, 14) for i in range(40)]
+    xs, dys, alphas = _channel_tensors(shapes, "f32", 521, misaligned=False)
+    need = mea.swish_channel_bwd_grouped_workspace_bytes(torch.float32, [tuple(x.shape) for x in xs])
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    for fill in (0, 255, 77):
+        ws.fill_(fill)
+        outs.append(mea.swish_channel_bwd_grouped(xs, dys, alphas, workspace=ws))
+    ref = [mea.swish_channel_bwd(x, g, a, "nchw") for x, g, a in zip(xs, dys, alphas)]
+    torch.cuda.synchronize()
+    for dxs, das in outs:
+        for dx, da, (rdx, rda) in zip(dxs, das, ref):
+            assert torch.equal(dx.view(torch.int32), rdx.view(torch.int32))
+            assert torch.equal(da.view(torch.int32), rda.view(torch.int32))
+
+
+def test_channel_grouped_effnet_small_planes_against_oracle():
+    # EfficientNet-B0's 28 x 28, 14 x 14 and 7 x 7 stages with alpha per
+    # channel, batch 64, fp32, in one grouped forward and backward: every
+    # output against the oracle
+    shapes = [(64, 240, 28, 28), (64, 480, 14, 14), (64, 1152, 7, 7)]
+    ws = [synthetic.swish_channel_nchw(531 + i, s) for i, s in enumerate(shapes)]
+    xs = [w.x.cuda() for w in ws]
+    ys = mea.swish_channel_fwd_grouped(xs, [w.extra["alpha"].cuda() for w in ws])
+    dxs, das = mea.swish_channel_bwd_grouped(xs, [w.dy.cuda() for w in ws], [w.extra["alpha"].cuda() for w in ws])
+    torch.cuda.synchronize()
+    del xs
+    for w, y, dx, da in zip(ws, ys, dxs, das):
+        xd, gd = to_f64(w.x), to_f64(w.dy)
+        aa = w.extra["alpha"].double().numpy()
+        N, C, H, W = w.extra["nchw_shape"]
+        ry = oracle.swish_channel_fwd("nchw", (N, C, H, W), xd, aa)
+        rdx, rda, scale = oracle.swish_channel_bwd("nchw", (N, C, H, W), xd, gd, aa)
+        check("f32", y.cpu(), ry, what="grouped channel fwd")
+        check("f32", dx.cpu(), rdx, scale=scale, floor=TINY * np.maximum(1, np.abs(gd)), what="grouped channel dx")
+        ch = (np.arange(xd.size) // (H * W)) % C
+        t = aa[ch] * xd
+        terms = np.abs(gd * xd * xd) / ((1.0 + np.exp(-t)) * (1.0 + np.exp(t)))
+        check_channel_sums(da, rda, np.bincount(ch, terms, minlength=C), xd.size // C, "grouped dalpha")
+
+
+def test_channel_grouped_rejects_overlap():
+    x = torch.zeros(2, 16, 7, 7, device="cuda")
+    a = torch.ones(16, device="cuda")
+    out = torch.empty(2 * 16 * 49 + 10, device="cuda")
+    with pytest.raises(mea.MeaError):
+        mea.swish_channel_fwd_grouped([x, x.clone()], [a, a], outs=[out[:1568].view(2, 16, 7, 7),
+                                                                   out[10:1578].view(2, 16, 7, 7)])
+    with pytest.raises(mea.MeaError):
+        da = torch.empty(16, device="cuda")
+        mea.swish_channel_bwd_grouped([x, x.clone()], [x.clone(), x.clone()], [a, a], dalphas=[da, da])
