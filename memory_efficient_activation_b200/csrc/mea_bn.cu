@@ -15,18 +15,20 @@
 //                                  x - shift and d^2 (shift: one element of
 //                                  the channel), fp32 within a 16-byte
 //                                  vector, fp64 across -> partials
-//             bn_finalize_kernel   per channel, slices in order: mean,
-//                                  invstd = 1 / sqrt(var + eps), running
-//                                  statistics (momentum; unbiased variance)
-//             bn_apply_kernel      y = max(gamma' x + beta', 0), gamma' =
-//                                  gamma invstd, beta' = beta - mean gamma'
+//             bn_apply_kernel      in its prologue, per channel, slices in
+//                                  order: mean, invstd = 1 / sqrt(var +
+//                                  eps), running statistics (momentum;
+//                                  unbiased variance); then y = max(gamma' x
+//                                  + beta', 0), gamma' = gamma invstd, beta'
+//                                  = beta - mean gamma'
 //   backward  bn_bwd_reduce_kernel per (channel, slice): recompute the ReLU
 //                                  mask from x; sums of dz and dz xhat
 //                                  (fp32 within a vector, fp64 across)
-//             bn_bwd_finalize      dbeta, dgamma and the coefficients of dx
-//             bn_dx_kernel         dx = gamma invstd (dz - dbeta / n -
-//                                  xhat dgamma / n), written or added into
-//                                  the pieces' gradients
+//             bn_dx_kernel         in its prologue dbeta, dgamma and the
+//                                  coefficients of dx; then dx = gamma invstd
+//                                  (dz - dbeta / n - xhat dgamma / n),
+//                                  written or added into the pieces'
+//                                  gradients
 // Blocks own (channel c, slice s of the batch) and stream the contiguous
 // H W planes of that channel (16-byte vectors when a plane is a multiple of
 // 16 bytes and the pieces are aligned), four items in flight per thread,
@@ -47,7 +49,6 @@ namespace {
 
 constexpr int kBnThreads = 256;
 constexpr int kBnBlocksTarget = 1184;     // C * S is sized to about this many blocks (148 x 8)
-constexpr int kBnFinThreads = 128;
 
 int bn_slices(int64_t N, int64_t C)
 {
@@ -310,31 +311,38 @@ bn_stats_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int ve
     }
 }
 
-__global__ void __launch_bounds__(kBnFinThreads)
-bn_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n, float eps, float momentum,
-                   float *__restrict__ mean, float *__restrict__ invstd, float *__restrict__ running_mean,
-                   float *__restrict__ running_var)
+// Batch statistics of channel c from its slices' partials, slices in order:
+// mean, invstd = 1 / sqrt(var + eps) (rounded to fp32), and with `write` the
+// stored mean, invstd and running statistics (momentum; unbiased variance).
+struct BnFin {
+    double n;
+    float eps, momentum;
+    float *running_mean, *running_var;
+};
+
+__device__ __forceinline__ void bn_finalize(const double *__restrict__ partials, int64_t c, int slices, const BnFin &f,
+                                         bool write, float *__restrict__ mean, float *__restrict__ invstd,
+                                         float &mu_out, float &r_out)
 {
-    pdl_wait();
-    pdl_trigger();
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= C) return;
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < slices; ++s) {
-        s1 += partials[3 * (c * slices + s)];
-        s2 += partials[3 * (c * slices + s) + 1];
+        s1 += __ldcg(partials + 3 * (c * slices + s));
+        s2 += __ldcg(partials + 3 * (c * slices + s) + 1);
     }
-    const double shift = partials[3 * c * slices + 2];
-    const double md = s1 / n;                 // mean of d = x - shift
-    double var = s2 / n - md * md;
+    const double shift = __ldcg(partials + 3 * c * slices + 2);
+    const double md = s1 / f.n;               // mean of d = x - shift
+    double var = s2 / f.n - md * md;
     if (var < 0.0) var = 0.0;
     const double mu = shift + md;
-    mean[c] = (float)mu;
-    invstd[c] = (float)(1.0 / sqrt(var + (double)eps));
-    if (running_mean) {
-        const double unbiased = n > 1.0 ? var * n / (n - 1.0) : var;
-        running_mean[c] = (float)((1.0 - momentum) * running_mean[c] + momentum * mu);
-        running_var[c] = (float)((1.0 - momentum) * running_var[c] + momentum * unbiased);
+    mu_out = (float)mu;
+    r_out = (float)(1.0 / sqrt(var + (double)f.eps));
+    if (!write) return;
+    mean[c] = mu_out;
+    invstd[c] = r_out;
+    if (f.running_mean) {
+        const double unbiased = f.n > 1.0 ? var * f.n / (f.n - 1.0) : var;
+        f.running_mean[c] = (float)((1.0 - f.momentum) * f.running_mean[c] + f.momentum * mu);
+        f.running_var[c] = (float)((1.0 - f.momentum) * f.running_var[c] + f.momentum * unbiased);
     }
 }
 
@@ -386,16 +394,32 @@ struct ApplyF {
     }
 };
 
+// With partials (the forward): the block's thread 0 first forms the
+// channel's statistics from them (bn_finalize), and the slice-0 block of
+// each channel stores them; without (the re-population): mean and invstd
+// are read.  Either way the same fp32 values enter the same arithmetic.
 template <typename T>
 __global__ void __launch_bounds__(kBnThreads, 6)
 bn_apply_kernel(BnPieces t, int64_t N, int64_t C, int64_t HW, int slices, int vec, const float *__restrict__ gamma,
-                const float *__restrict__ beta, const float *__restrict__ mean, const float *__restrict__ invstd,
-                void *__restrict__ y)
+                const float *__restrict__ beta, float *__restrict__ mean, float *__restrict__ invstd,
+                void *__restrict__ y, const double *__restrict__ partials, BnFin fin)
 {
+    __shared__ float stat[2];
     pdl_wait();
     const PlaneJob p = plane_job(t, N, slices);
-    const float gp = gamma[p.c] * invstd[p.c];
-    ApplyF<T> f{t.ptr[p.piece], y, gp, fmaf(-mean[p.c], gp, beta[p.c])};
+    float mu, r;
+    if (partials) {
+        if (threadIdx.x == 0)
+            bn_finalize(partials, p.c, slices, fin, blockIdx.x % slices == 0, mean, invstd, stat[0], stat[1]);
+        __syncthreads();
+        mu = stat[0];
+        r = stat[1];
+    } else {
+        mu = mean[p.c];
+        r = invstd[p.c];
+    }
+    const float gp = gamma[p.c] * r;
+    ApplyF<T> f{t.ptr[p.piece], y, gp, fmaf(-mu, gp, beta[p.c])};
     for_planes<T>(p, C, HW, vec, f);
     pdl_trigger();
 }
@@ -504,28 +528,27 @@ bn_bwd_reduce_kernel(BnPieces t, const void *__restrict__ dy, int64_t N, int64_t
     }
 }
 
-// dbeta, dgamma, and dx = a dz + b + c xhat with a = gamma r, b = -a dbeta / n,
-// c = -a dgamma / n (coef[3 ch + 0..2]).
-__global__ void __launch_bounds__(kBnFinThreads)
-bn_bwd_finalize_kernel(const double *__restrict__ partials, int64_t C, int slices, double n,
-                       const float *__restrict__ gamma, const float *__restrict__ invstd, float *__restrict__ dgamma,
-                       float *__restrict__ dbeta, float *__restrict__ coef)
+// dbeta, dgamma (stored with `write`), and the coefficients of dx = a dz + b +
+// c xhat: a = gamma r, b = -a dbeta / n, c = -a dgamma / n, from channel c's
+// slices in order.
+__device__ __forceinline__ void bn_bwd_finalize(const double *__restrict__ partials, int64_t c, int slices, double n,
+                                             const float *__restrict__ gamma, const float *__restrict__ invstd,
+                                             bool write, float *__restrict__ dgamma, float *__restrict__ dbeta,
+                                             float (&coef)[3])
 {
-    pdl_wait();
-    pdl_trigger();
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= C) return;
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < slices; ++s) {
-        s1 += partials[3 * (c * slices + s)];
-        s2 += partials[3 * (c * slices + s) + 1];
+        s1 += __ldcg(partials + 3 * (c * slices + s));
+        s2 += __ldcg(partials + 3 * (c * slices + s) + 1);
     }
-    dbeta[c] = (float)s1;
-    dgamma[c] = (float)s2;
+    if (write) {
+        dbeta[c] = (float)s1;
+        dgamma[c] = (float)s2;
+    }
     const double a = (double)gamma[c] * (double)invstd[c];
-    coef[3 * c] = (float)a;
-    coef[3 * c + 1] = (float)(-a * s1 / n);
-    coef[3 * c + 2] = (float)(-a * s2 / n);
+    coef[0] = (float)a;
+    coef[1] = (float)(-a * s1 / n);
+    coef[2] = (float)(-a * s2 / n);
 }
 
 // ACC: add d to what dx already holds (a fixed choice per launch, so the
@@ -591,16 +614,29 @@ struct DxF {
     }
 };
 
+// The block's thread 0 first forms the channel's coefficients from the
+// reduce kernel's partials (bn_bwd_finalize); the slice-0 block of each
+// channel stores dgamma and dbeta.
 template <typename T, bool ACC>
 __global__ void __launch_bounds__(kBnThreads, 4)
 bn_dx_kernel(BnPieces t, BnOutPieces d, const void *__restrict__ dy, int64_t N, int64_t C, int64_t HW, int slices,
              int vec, const float *__restrict__ gamma, const float *__restrict__ beta, const float *__restrict__ mean,
-             const float *__restrict__ invstd, const float *__restrict__ coef)
+             const float *__restrict__ invstd, const double *__restrict__ partials, float *__restrict__ dgamma,
+             float *__restrict__ dbeta)
 {
+    __shared__ float cf[3];
     pdl_wait();
     const PlaneJob p = plane_job(t, N, slices);
-    DxF<T, ACC> f{t.ptr[p.piece], dy, d.ptr[p.piece], bwd_coef(gamma, beta, mean, invstd, p.c), coef[3 * p.c],
-                  coef[3 * p.c + 1], coef[3 * p.c + 2]};
+    if (threadIdx.x == 0) {
+        float k3[3];
+        bn_bwd_finalize(partials, p.c, slices, (double)(N * HW), gamma, invstd, blockIdx.x % slices == 0, dgamma,
+                        dbeta, k3);
+        cf[0] = k3[0];
+        cf[1] = k3[1];
+        cf[2] = k3[2];
+    }
+    __syncthreads();
+    DxF<T, ACC> f{t.ptr[p.piece], dy, d.ptr[p.piece], bwd_coef(gamma, beta, mean, invstd, p.c), cf[0], cf[1], cf[2]};
     for_planes<T>(p, C, HW, vec, f);
     pdl_trigger();
 }
@@ -627,20 +663,15 @@ cudaError_t fwd_t(const BnLaunch &a, bool stats)
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const int vec = vec_ok(a, Store<T>::kBytes, false);
     double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
-    cudaError_t e = cudaSuccess;
     if (stats) {
-        e = launch_pdl(bn_stats_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
-                       slices, vec, partials);
-        if (e != cudaSuccess) return e;
-        const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
-        e = launch_pdl(bn_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
-                       static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.eps, a.momentum,
-                       a.mean, a.invstd, a.running_mean, a.running_var);
+        cudaError_t e = launch_pdl(bn_stats_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in,
+                                   a.N, a.C, a.HW, slices, vec, partials);
         if (e != cudaSuccess) return e;
     }
+    const BnFin fin{(double)(a.N * a.HW), a.eps, a.momentum, a.running_mean, a.running_var};
     return launch_pdl(bn_apply_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.N, a.C, a.HW,
-                      slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
-                      static_cast<const float *>(a.invstd), a.y);
+                      slices, vec, a.gamma, a.beta, a.mean, a.invstd, a.y,
+                      stats ? static_cast<const double *>(partials) : nullptr, fin);
 }
 
 template <typename T>
@@ -651,20 +682,15 @@ cudaError_t bwd_t(const BnLaunch &a)
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const int vec = vec_ok(a, Store<T>::kBytes, true);
     double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);
-    float *coef = reinterpret_cast<float *>(partials + 3 * grid);
     cudaError_t e = launch_pdl(bn_bwd_reduce_kernel<T>, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in,
                                a.dy, a.N, a.C, a.HW, slices, vec, a.gamma, a.beta,
                                static_cast<const float *>(a.mean), static_cast<const float *>(a.invstd), partials);
     if (e != cudaSuccess) return e;
-    const unsigned fg = (unsigned)((a.C + kBnFinThreads - 1) / kBnFinThreads);
-    e = launch_pdl(bn_bwd_finalize_kernel, dim3(fg), dim3(kBnFinThreads), 0, a.stream,
-                   static_cast<const double *>(partials), a.C, slices, (double)(a.N * a.HW), a.gamma,
-                   static_cast<const float *>(a.invstd), a.dgamma, a.dbeta, coef);
-    if (e != cudaSuccess) return e;
     auto dx_kernel = a.accumulate ? bn_dx_kernel<T, true> : bn_dx_kernel<T, false>;
     return launch_pdl(dx_kernel, dim3((unsigned)grid), dim3(kBnThreads), 0, a.stream, a.in, a.din, a.dy, a.N, a.C,
                       a.HW, slices, vec, a.gamma, a.beta, static_cast<const float *>(a.mean),
-                      static_cast<const float *>(a.invstd), static_cast<const float *>(coef));
+                      static_cast<const float *>(a.invstd), static_cast<const double *>(partials), a.dgamma,
+                      a.dbeta);
 }
 
 }  // namespace
