@@ -726,6 +726,20 @@ struct RowShape {
     int64_t grid;
 };
 
+// Lanes that add up one plane's terms: the largest power of two at most
+// H W / 16, within 1 .. 32.
+__device__ __forceinline__ uint32_t row_team(uint32_t hw)
+{
+    uint32_t ts = 1;
+    while (ts < 32 && ts * 2 * 16 <= hw) ts *= 2;
+    return ts;
+}
+// The lanes of lane's team of ts (a power of two) within its warp.
+__device__ __forceinline__ unsigned row_team_mask(uint32_t lane, uint32_t ts)
+{
+    return ts == 32 ? 0xffffffffu : ((1u << ts) - 1u) << (lane & ~(ts - 1u));
+}
+
 // P for nr reductions and vl elements per 16-byte vector: about
 // N C / kRowBlocksTarget planes, rounded up to the alignment multiple, at
 // most what the staging buffer and the constants table hold.
@@ -861,17 +875,33 @@ __device__ __forceinline__ void row_body(const void *__restrict__ x, const void 
     pdl_trigger();
     if constexpr (MODE == 1) {
         __syncthreads();
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-        for (uint32_t lp = w; lp < np; lp += kRowThreads / 32) {
-            const int64_t g = g0 + lp;
-            const int64_t n = g / C, c = g - n * C;
+        // A team of ts lanes per plane (about 16 terms per lane; a power of
+        // two from 1 to 32, fixed by H W): lane i of a team adds positions
+        // i, i + ts, ... in fp64, then a fixed shuffle tree within the team.
+        auto sums = [&](auto tsc) {
+            constexpr uint32_t TS = decltype(tsc)::value;
+            const uint32_t lane = threadIdx.x & 31, sub = lane & (TS - 1);
+            const unsigned mask = row_team_mask(lane, TS);
+            for (uint32_t lp = threadIdx.x / TS; lp < np; lp += kRowThreads / TS) {
+                const int64_t g = g0 + lp;
+                const int64_t n = g / C, c = g - n * C;
 #pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                double v = 0.0;
-                for (uint32_t i = lane; i < hw; i += 32) v += (double)terms[r * ld + lp * hw + i];
-                v = warp_sum(v);
-                if (lane == 0) partials[(n * NR + r) * C + c] = v;
+                for (int r = 0; r < NR; ++r) {
+                    double v = 0.0;
+                    for (uint32_t i = sub; i < hw; i += TS) v += (double)terms[r * ld + lp * hw + i];
+#pragma unroll
+                    for (uint32_t off = TS >> 1; off >= 1; off >>= 1) v += __shfl_xor_sync(mask, v, off);
+                    if (sub == 0) partials[(n * NR + r) * C + c] = v;
+                }
             }
+        };
+        switch (row_team(hw)) {
+        case 1: sums(std::integral_constant<uint32_t, 1>{}); break;
+        case 2: sums(std::integral_constant<uint32_t, 2>{}); break;
+        case 4: sums(std::integral_constant<uint32_t, 4>{}); break;
+        case 8: sums(std::integral_constant<uint32_t, 8>{}); break;
+        case 16: sums(std::integral_constant<uint32_t, 16>{}); break;
+        default: sums(std::integral_constant<uint32_t, 32>{}); break;
         }
     }
 }

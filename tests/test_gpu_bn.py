@@ -132,6 +132,15 @@ def _run(N, ks, spatial, dtype, seed, accumulate=False, cap=1e-3):
     (2, [1] * 7, (3, 5)),            # many one-channel pieces
     (3, [24], (8, 8)),               # a single piece
     (16, [64, 32, 32], (14, 14)),    # 196-element planes: vectors for fp32 only
+    # the pipelined path (planes of 16-byte multiples up to 16 KB): one sample
+    # and 300 channels (blocks span three channels), 300 samples of two
+    # channels (16-byte planes, 300 planes per stage), 16 KB fp32 planes,
+    # one-channel pieces, pieces that end inside a block
+    (1, [300], (8, 8)),
+    (300, [2], (2, 4)),
+    (4, [8, 8], (64, 64)),
+    (2, [1] * 7, (2, 4)),
+    (5, [17, 40], (4, 6)),
 ])
 def test_concat_bn_relu(dtype, N, ks, spatial):
     _run(N, ks, spatial, dtype, 61)
@@ -147,8 +156,9 @@ def test_concat_bn_relu_densenet_block_size():
     _run(64, [64, 32, 32, 32, 32, 32], (56, 56), "bf16", 63)
 
 
-def test_concat_bn_relu_running_stats_and_determinism():
-    N, ks, spatial = 8, [12, 20], (9, 9)
+@pytest.mark.parametrize("spatial", [(9, 9), (8, 8)])   # plane path, pipelined path
+def test_concat_bn_relu_running_stats_and_determinism(spatial):
+    N, ks = 8, [12, 20]
     pieces = [p.cuda() for p in _pieces(N, ks, spatial, "f32", 64)]
     C = sum(ks)
     g, b = [t.cuda() for t in _params(C, 65)]
@@ -160,7 +170,7 @@ def test_concat_bn_relu_running_stats_and_determinism():
     assert torch.equal(y1, y2) and torch.equal(m1, m2) and torch.equal(i1, i2)
     _, rm, rv, _ = oracle.concat_bn_relu_fwd(_np([p.cpu() for p in pieces]), g.cpu().double().numpy(),
                                              b.cpu().double().numpy(), EPS)
-    em, ev = oracle.bn_running_update(np.full(C, 0.5), np.full(C, 2.0), rm, rv, N * 81, 0.1)
+    em, ev = oracle.bn_running_update(np.full(C, 0.5), np.full(C, 2.0), rm, rv, N * spatial[0] * spatial[1], 0.1)
     # the kernel's statistics are fp32 results (see _check_stats); the update
     # adds one fp64 blend and one rounding to fp32
     assert np.allclose(rmean.cpu().double().numpy(), em, rtol=2e-6, atol=1e-7)
