@@ -410,63 +410,72 @@ struct GeluErf {
     static constexpr float kTwoRsqrtPi = 1.12837916709551257f;     // 2 / sqrt(pi)
     static constexpr float kRsqrt2Pi = 0.398942280401432678f;      // 1 / sqrt(2 pi)
     static constexpr float kLog2ef = 1.44269504088896340736f;
-    // Backward: erfc(a) = t e^(-a^2) Q(t), t = 1 / (1 + a / 2), with
-    // Q(t) = erfcx(a) / t fitted directly (degree 8, coefficients of t^0 ..
-    // t^8; csrc/fit_erfc_bf16.py), so that the one exponential e^(-a^2)
-    // serves both erfc and the Gaussian of f' (q8, q8_2).
-    static __device__ __forceinline__ float q8(float t)
+    // The bf16 forms use t = 1 / (1 + a / 2) (Press et al., "Numerical
+    // Recipes in C", 6.2) through h = t / 2 = 1 / (2 + a): each polynomial in
+    // t is evaluated in h with coefficient k scaled by 2^k, which leaves every
+    // Horner step the t-form's value times a power of two, so the polynomial's
+    // value is bitwise the same, and a product with h is half the product
+    // with t, exactly.  That half is the 1/2 of Phi = erfc / 2, which then
+    // costs no multiply.
+    //
+    // Backward: erfc(a) = t e^(-a^2) Q(t) with Q(t) = erfcx(a) / t fitted
+    // directly (degree 8, coefficients of t^8 .. t^0, each times 2^k below;
+    // csrc/fit_erfc_bf16.py), so that the one exponential e^(-a^2) serves
+    // both erfc and the Gaussian of f' (q8, q8_2); h e^(-a^2) Q = erfc / 2.
+    static __device__ __forceinline__ float q8(float h)
     {
-        float q = -0.058932472f;
-        q = fmaf(q, t, 0.283905655f);
-        q = fmaf(q, t, -0.485806316f);
-        q = fmaf(q, t, 0.276463121f);
-        q = fmaf(q, t, -0.0255132243f);
-        q = fmaf(q, t, 0.202212647f);
-        q = fmaf(q, t, 0.243224636f);
-        q = fmaf(q, t, 0.282358527f);
-        return fmaf(q, t, 0.282087386f);
+        float q = -0.058932472f * 256.f;
+        q = fmaf(q, h, 0.283905655f * 128.f);
+        q = fmaf(q, h, -0.485806316f * 64.f);
+        q = fmaf(q, h, 0.276463121f * 32.f);
+        q = fmaf(q, h, -0.0255132243f * 16.f);
+        q = fmaf(q, h, 0.202212647f * 8.f);
+        q = fmaf(q, h, 0.243224636f * 4.f);
+        q = fmaf(q, h, 0.282358527f * 2.f);
+        return fmaf(q, h, 0.282087386f);
     }
-    static __device__ __forceinline__ F2 q8_2(F2 t)
+    static __device__ __forceinline__ F2 q8_2(F2 h)
     {
-        F2 q = sp2(-0.058932472f);
-        q = fma2(q, t, sp2(0.283905655f));
-        q = fma2(q, t, sp2(-0.485806316f));
-        q = fma2(q, t, sp2(0.276463121f));
-        q = fma2(q, t, sp2(-0.0255132243f));
-        q = fma2(q, t, sp2(0.202212647f));
-        q = fma2(q, t, sp2(0.243224636f));
-        q = fma2(q, t, sp2(0.282358527f));
-        return fma2(q, t, sp2(0.282087386f));
+        F2 q = sp2(-0.058932472f * 256.f);
+        q = fma2(q, h, sp2(0.283905655f * 128.f));
+        q = fma2(q, h, sp2(-0.485806316f * 64.f));
+        q = fma2(q, h, sp2(0.276463121f * 32.f));
+        q = fma2(q, h, sp2(-0.0255132243f * 16.f));
+        q = fma2(q, h, sp2(0.202212647f * 8.f));
+        q = fma2(q, h, sp2(0.243224636f * 4.f));
+        q = fma2(q, h, sp2(0.282358527f * 2.f));
+        return fma2(q, h, sp2(0.282087386f));
     }
 
     static __device__ __forceinline__ Coef coef(float) { return Coef{1.f, 0.f, 0.f}; }
 
-    // Chebyshev approximation pieces for a = |w|: t, and u = (-a^2 + P(t)) log2 e.
-    static __device__ __forceinline__ float nr_parts(float a, float &t)
+    // Chebyshev approximation pieces for a = |w| (Press et al.'s degree-9
+    // erfc): h, and u = (-a^2 + P(t)) log2 e, so that erfc(a) = 2 h 2^u.
+    static __device__ __forceinline__ float nr_parts(float a, float &h)
     {
-        t = rcp_ftz(fmaf(0.5f, a, 1.0f));
-        float p = 0.17087277f;
-        p = fmaf(p, t, -0.82215223f);
-        p = fmaf(p, t, 1.48851587f);
-        p = fmaf(p, t, -1.13520398f);
-        p = fmaf(p, t, 0.27886807f);
-        p = fmaf(p, t, -0.18628806f);
-        p = fmaf(p, t, 0.09678418f);
-        p = fmaf(p, t, 0.37409196f);
-        p = fmaf(p, t, 1.00002368f);
-        p = fmaf(p, t, -1.26551223f);
+        h = rcp_ftz(a + 2.0f);
+        float p = 0.17087277f * 512.f;
+        p = fmaf(p, h, -0.82215223f * 256.f);
+        p = fmaf(p, h, 1.48851587f * 128.f);
+        p = fmaf(p, h, -1.13520398f * 64.f);
+        p = fmaf(p, h, 0.27886807f * 32.f);
+        p = fmaf(p, h, -0.18628806f * 16.f);
+        p = fmaf(p, h, 0.09678418f * 8.f);
+        p = fmaf(p, h, 0.37409196f * 4.f);
+        p = fmaf(p, h, 1.00002368f * 2.f);
+        p = fmaf(p, h, -1.26551223f);
         return fmaf(-a, a, p) * kLog2ef;
     }
     // Degree-5 form of nr_parts for the bf16 forward.
-    static __device__ __forceinline__ float nr5_parts(float a, float &t)
+    static __device__ __forceinline__ float nr5_parts(float a, float &h)
     {
-        t = rcp_ftz(fmaf(0.5f, a, 1.0f));
-        float p = 0.228795588f;
-        p = fmaf(p, t, -0.709205508f);
-        p = fmaf(p, t, 0.474508315f);
-        p = fmaf(p, t, 0.254436046f);
-        p = fmaf(p, t, 1.01801503f);
-        p = fmaf(p, t, -1.26654184f);
+        h = rcp_ftz(a + 2.0f);
+        float p = 0.228795588f * 32.f;
+        p = fmaf(p, h, -0.709205508f * 16.f);
+        p = fmaf(p, h, 0.474508315f * 8.f);
+        p = fmaf(p, h, 0.254436046f * 4.f);
+        p = fmaf(p, h, 1.01801503f * 2.f);
+        p = fmaf(p, h, -1.26654184f);
         return fmaf(-a, a, p) * kLog2ef;
     }
     // The bf16 main paths serve x >= kTailX, where every exponential they take
@@ -502,57 +511,38 @@ struct GeluErf {
     // Pairwise bf16-mode forward and backward: the same operations in the
     // same order as f / df below (bitwise the same results), with the
     // multiply-add chains on packed pairs and the two MUFU operations scalar.
-    static __device__ __forceinline__ void nr_parts2(F2 x, float &w0, float &w1, F2 &t, F2 &u)
+    static __device__ __forceinline__ void nr5_parts2(F2 x, float &w0, float &w1, F2 &h, F2 &u)
     {
         const F2 w = mul2(x, sp2(kNegRsqrt2Hi));
         upk(w, w0, w1);
         const F2 a = pk(fabsf(w0), fabsf(w1));
         float d0, d1;
-        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
-        t = pk(rcp_ftz(d0), rcp_ftz(d1));
-        F2 p = sp2(0.17087277f);
-        p = fma2(p, t, sp2(-0.82215223f));
-        p = fma2(p, t, sp2(1.48851587f));
-        p = fma2(p, t, sp2(-1.13520398f));
-        p = fma2(p, t, sp2(0.27886807f));
-        p = fma2(p, t, sp2(-0.18628806f));
-        p = fma2(p, t, sp2(0.09678418f));
-        p = fma2(p, t, sp2(0.37409196f));
-        p = fma2(p, t, sp2(1.00002368f));
-        p = fma2(p, t, sp2(-1.26551223f));
+        upk(add2(a, sp2(2.0f)), d0, d1);
+        h = pk(rcp_ftz(d0), rcp_ftz(d1));
+        F2 p = sp2(0.228795588f * 32.f);
+        p = fma2(p, h, sp2(-0.709205508f * 16.f));
+        p = fma2(p, h, sp2(0.474508315f * 8.f));
+        p = fma2(p, h, sp2(0.254436046f * 4.f));
+        p = fma2(p, h, sp2(1.01801503f * 2.f));
+        p = fma2(p, h, sp2(-1.26654184f));
         u = mul2(fma2(pk(-fabsf(w0), -fabsf(w1)), a, p), sp2(kLog2ef));
     }
-    static __device__ __forceinline__ void nr5_parts2(F2 x, float &w0, float &w1, F2 &t, F2 &u)
-    {
-        const F2 w = mul2(x, sp2(kNegRsqrt2Hi));
-        upk(w, w0, w1);
-        const F2 a = pk(fabsf(w0), fabsf(w1));
-        float d0, d1;
-        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
-        t = pk(rcp_ftz(d0), rcp_ftz(d1));
-        F2 p = sp2(0.228795588f);
-        p = fma2(p, t, sp2(-0.709205508f));
-        p = fma2(p, t, sp2(0.474508315f));
-        p = fma2(p, t, sp2(0.254436046f));
-        p = fma2(p, t, sp2(1.01801503f));
-        p = fma2(p, t, sp2(-1.26654184f));
-        u = mul2(fma2(pk(-fabsf(w0), -fabsf(w1)), a, p), sp2(kLog2ef));
-    }
-    static __device__ __forceinline__ F2 erfc2(float w0, float w1, F2 t, float u0, float u1)
+    // Phi(x) = erfc(w) / 2 for w = -x / sqrt 2: h 2^u for w >= 0, else 1 - h 2^u.
+    static __device__ __forceinline__ F2 half_erfc2(float w0, float w1, F2 h, float u0, float u1)
     {
         float a0, a1;
-        upk(mul2(t, pk(ex2_ftz(u0), ex2_ftz(u1))), a0, a1);
-        return pk(w0 >= 0.f ? a0 : 2.f - a0, w1 >= 0.f ? a1 : 2.f - a1);
+        upk(mul2(h, pk(ex2_ftz(u0), ex2_ftz(u1))), a0, a1);
+        return pk(w0 >= 0.f ? a0 : 1.f - a0, w1 >= 0.f ? a1 : 1.f - a1);
     }
     static __device__ __forceinline__ void f2(float x0, float x1, const Coef &, bool &tail, float &o0, float &o1)
     {
         const F2 x = pk(x0, x1);
         float w0, w1, u0, u1;
-        F2 t, u;
-        nr5_parts2(x, w0, w1, t, u);
+        F2 h, u;
+        nr5_parts2(x, w0, w1, h, u);
         upk(u, u0, u1);
         tail |= (x0 < kTailX) | (x1 < kTailX);
-        upk(mul2(mul2(sp2(0.5f), x), erfc2(w0, w1, t, u0, u1)), o0, o1);
+        upk(mul2(x, half_erfc2(w0, w1, h, u0, u1)), o0, o1);
     }
     static __device__ __forceinline__ void df2(float x0, float x1, float dy0, float dy1, const Coef &, bool &tail,
                                                float &o0, float &o1)
@@ -563,17 +553,17 @@ struct GeluErf {
         upk(w, w0, w1);
         const F2 a = pk(fabsf(w0), fabsf(w1));
         float d0, d1;
-        upk(fma2(sp2(0.5f), a, sp2(1.0f)), d0, d1);
-        const F2 t = pk(rcp_ftz(d0), rcp_ftz(d1));
-        const F2 q = q8_2(t);
+        upk(add2(a, sp2(2.0f)), d0, d1);
+        const F2 h = pk(rcp_ftz(d0), rcp_ftz(d1));
+        const F2 q = q8_2(h);
         float v0, v1;
         upk(mul2(mul2(w, w), sp2(-kLog2ef)), v0, v1);
         tail |= (x0 < kTailX) | (x1 < kTailX);
         const F2 g = pk(ex2_ftz(v0), ex2_ftz(v1));
         float a0, a1;
-        upk(mul2(mul2(t, q), g), a0, a1);
-        const F2 ec = pk(w0 >= 0.f ? a0 : 2.f - a0, w1 >= 0.f ? a1 : 2.f - a1);
-        const F2 d = fma2(mul2(x, sp2(kRsqrt2Pi)), g, mul2(sp2(0.5f), ec));
+        upk(mul2(mul2(h, q), g), a0, a1);
+        const F2 phi = pk(w0 >= 0.f ? a0 : 1.f - a0, w1 >= 0.f ? a1 : 1.f - a1);   // Phi(x)
+        const F2 d = fma2(mul2(x, sp2(kRsqrt2Pi)), g, phi);
         upk(mul2(pk(dy0, dy1), d), o0, o1);
     }
 
@@ -586,12 +576,11 @@ struct GeluErf {
             return (0.5f * x) * ec;
         } else {
             const float w = x * kNegRsqrt2Hi;
-            float t;
-            const float u = nr5_parts(fabsf(w), t);
+            float h;
+            const float u = nr5_parts(fabsf(w), h);
             tail |= x < kTailX;
-            const float ans = t * ex2_ftz(u);
-            const float ec = w >= 0.f ? ans : 2.f - ans;
-            return (0.5f * x) * ec;
+            const float half = h * ex2_ftz(u);                  // erfc(|w|) / 2
+            return x * (w >= 0.f ? half : 1.f - half);          // x Phi(x)
         }
     }
     template <bool P>
@@ -601,11 +590,11 @@ struct GeluErf {
             bool t = false;
             return f<P>(x, k, t);
         } else {
-            // x << 0: w > 0, erfc(w) = t 2^u with u < -124; scale by 2^64
+            // x << 0: w > 0, erfc(w) / 2 = h 2^u with u < -124; scale by 2^64
             const float w = x * kNegRsqrt2Hi;
-            float t;
-            const float u = nr_parts(w, t);
-            return (((0.5f * x) * t) * ex2_ftz(u + 64.f)) * kTwoM64;
+            float h;
+            const float u = nr_parts(w, h);
+            return ((x * h) * ex2_ftz(u + 64.f)) * kTwoM64;
         }
     }
     template <bool P>
@@ -617,14 +606,13 @@ struct GeluErf {
             return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
         } else {
             const float w = x * kNegRsqrt2Hi;
-            const float t = rcp_ftz(fmaf(0.5f, fabsf(w), 1.0f));
-            const float q = q8(t);
+            const float h = rcp_ftz(fabsf(w) + 2.0f);
+            const float q = q8(h);
             const float v = (w * w) * -kLog2ef;
             tail |= x < kTailX;
             const float g = ex2_ftz(v);
-            const float ans = (t * q) * g;
-            const float ec = w >= 0.f ? ans : 2.f - ans;
-            return dy * fmaf(x * kRsqrt2Pi, g, 0.5f * ec);
+            const float half = (h * q) * g;                     // erfc(|w|) / 2
+            return dy * fmaf(x * kRsqrt2Pi, g, w >= 0.f ? half : 1.f - half);
         }
     }
     template <bool P>
@@ -635,11 +623,11 @@ struct GeluErf {
             return df<P>(x, dy, k, t);
         } else {
             const float w = x * kNegRsqrt2Hi;
-            float t;
-            const float u = nr_parts(w, t);
-            const float e64 = ex2_ftz(u + 64.f);                       // erfc(w) / t, scaled
+            float h;
+            const float u = nr_parts(w, h);
+            const float e64 = ex2_ftz(u + 64.f);                       // erfc(w) / (2 h), scaled
             const float g64 = ex2_ftz(fmaf(-(w * w), kLog2ef, 64.f));  // e^(-w^2), scaled
-            return (dy * fmaf(x * kRsqrt2Pi, g64, (0.5f * t) * e64)) * kTwoM64;
+            return (dy * fmaf(x * kRsqrt2Pi, g64, h * e64)) * kTwoM64;
         }
     }
 };

@@ -2,7 +2,8 @@
 (mea_math.cuh, GeluErf::nr_parts, nr5_parts and q8), read from the source
 text and evaluated in float64 against scipy's scaled complementary error
 function.  All are polynomials in t = 1 / (1 + a / 2) (Press et al.,
-"Numerical Recipes in C", 2nd ed., section 6.2).  nr_parts and nr5_parts
+"Numerical Recipes in C", 2nd ed., section 6.2); the kernels evaluate them in
+h = t / 2 with coefficient k times 2^k, which the parser checks and undoes.  nr_parts and nr5_parts
 approximate log(erfc(a) / t) + a^2; q8 approximates erfcx(a) / t.  The
 claims checked are the fractional error bounds that the kernel comments and
 the design notes state, over the range each is used on (a up to 9.6, where
@@ -22,26 +23,61 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                    "memory_efficient_activation_b200", "csrc", "mea_math.cuh")
 
 
+# One Horner term of the kernels' h-form (h = t / 2): a coefficient literal,
+# optionally times its power of two.
+_TERM = r"([-0-9.eE]+)f(?: \* ([0-9.]+)f)?"
+
+
+def _unscale(terms) -> list[float]:
+    """The published coefficients (highest degree first) from the kernel's
+    h-form terms: the coefficient of degree k must carry exactly 2^k, so that
+    the polynomial in h = t / 2 is the published polynomial in t."""
+    deg = len(terms) - 1
+    out = []
+    for i, (lit, scale) in enumerate(terms):
+        assert float(scale or 1) == 2.0 ** (deg - i), (i, lit, scale)
+        out.append(float(lit))
+    return out
+
+
 def _horner_coefficients(func: str) -> list[float]:
-    """The Horner chain of `func` in GeluErf, highest degree first."""
+    """The Horner chain of `func` in GeluErf, highest degree first, in t."""
     text = open(SRC).read()
     start = text.index("struct GeluErf")
-    body = text[text.index(f"float {func}(float a, float &t)", start):]
+    body = text[text.index(f"float {func}(float a, float &h)", start):]
     body = body[:body.index("return")]
-    first = float(re.search(r"float p = ([-0-9.eE]+)f;", body).group(1))
-    rest = [float(v) for v in re.findall(r"p = fmaf\(p, t, ([-0-9.eE]+)f\);", body)]
-    return [first] + rest
+    first = re.search(r"float p = " + _TERM + ";", body).groups()
+    rest = re.findall(r"p = fmaf\(p, h, " + _TERM + r"\);", body)
+    return _unscale([first] + rest)
 
 
 def _q8_coefficients() -> list[float]:
-    """q8's Horner chain, highest degree first."""
+    """q8's Horner chain, highest degree first, in t."""
     text = open(SRC).read()
     start = text.index("struct GeluErf")
-    body = text[text.index("float q8(float t)", start):]
+    body = text[text.index("float q8(float h)", start):]
     body = body[:body.index("}")]
-    first = float(re.search(r"float q = ([-0-9.eE]+)f;", body).group(1))
-    rest = [float(v) for v in re.findall(r"fmaf\(q, t, ([-0-9.eE]+)f\)", body)]
-    return [first] + rest
+    first = re.search(r"float q = " + _TERM + ";", body).groups()
+    rest = re.findall(r"fmaf\(q, h, " + _TERM + r"\)", body)
+    return _unscale([first] + rest)
+
+
+def test_h_form_is_the_t_form_bitwise():
+    # Horner in h = t / 2 with coefficient k times 2^k: every step is the
+    # t-form's step times a power of two, so the float32 results agree bit
+    # for bit (checked here with separately rounded multiply and add)
+    rng = np.random.default_rng(5)
+    t = np.float32(1.0) / (np.float32(1.0) + rng.uniform(0, 4.8, 100001).astype(np.float32))
+    h = (t * np.float32(0.5)).astype(np.float32)
+    for c in (_horner_coefficients("nr_parts"), _horner_coefficients("nr5_parts"), _q8_coefficients()):
+        c32 = np.array(c, dtype=np.float32)
+        deg = len(c32) - 1
+        pt = np.full_like(t, c32[0])
+        ph = np.full_like(t, np.float32(c32[0] * np.float32(2.0 ** deg)))
+        for i in range(1, len(c32)):
+            pt = (pt * t + c32[i]).astype(np.float32)
+            ph = (ph * h + np.float32(c32[i] * np.float32(2.0 ** (deg - i)))).astype(np.float32)
+        assert np.array_equal(pt.view(np.int32), ph.view(np.int32))
 
 
 def _max_fractional_error(coef_high_first, a_max=9.6, points=200001):
