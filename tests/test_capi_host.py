@@ -408,3 +408,62 @@ def test_channel_grouped_validation(lib):
     assert b"dalpha" in lib.mea_last_error()
     part = _chan_segs([(X, D, X + 2, G, 0x700000, sh_a)])
     assert b(1, 1, part, 0x800000, need, None) == _capi.MEA_ERR_INVALID_ARG
+
+
+class _RecordingLib(_FakeLib):
+    """_FakeLib that also keeps each call's arguments."""
+
+    def __init__(self):
+        super().__init__()
+        self.args = {}
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append(name)
+            self.args[name] = args
+            return 0
+        return fn
+
+
+def test_binding_channel_grouped_marshalling(monkeypatch):
+    # swish_channel_*_grouped build one mea_channel_segment_t per tensor with
+    # its pointers and (N, C, H, W); mismatched lists and companions are
+    # refused before the library is reached
+    import torch
+    import memory_efficient_activation_b200 as mea
+    from memory_efficient_activation_b200 import _capi
+    fake = _RecordingLib()
+    monkeypatch.setattr(_capi, "lib", lambda: fake)
+    monkeypatch.setattr(mea, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(mea, "_stream", lambda t: 0)
+    shapes = [(2, 16, 7, 7), (3, 40, 14, 14), (1, 8, 1, 1)]
+    xs = [torch.randn(s) for s in shapes]
+    dys = [torch.randn(s) for s in shapes]
+    alphas = [torch.ones(s[1]) for s in shapes]
+    ys = mea.swish_channel_fwd_grouped(xs, alphas)
+    nseg, segs = fake.args["mea_swish_channel_fwd_grouped"][1:3]
+    assert nseg == 3
+    for i, (x, y, a, s) in enumerate(zip(xs, ys, alphas, shapes)):
+        g = segs[i]
+        assert (g.x, g.out, g.alpha) == (x.data_ptr(), y.data_ptr(), a.data_ptr())
+        assert not g.dy and not g.dalpha and tuple(g.shape) == s
+    dxs, das = mea.swish_channel_bwd_grouped(xs, dys, alphas, workspace=torch.zeros(1 << 16, dtype=torch.uint8))
+    nseg, segs = fake.args["mea_swish_channel_bwd_grouped"][1:3]
+    assert nseg == 3 and "mea_swish_channel_bwd_grouped_workspace_bytes" in fake.calls
+    for i, (x, dy, dx, da, s) in enumerate(zip(xs, dys, dxs, das, shapes)):
+        g = segs[i]
+        assert (g.x, g.dy, g.out, g.dalpha) == (x.data_ptr(), dy.data_ptr(), dx.data_ptr(), da.data_ptr())
+        assert da.numel() == s[1] and da.dtype == torch.float32 and tuple(g.shape) == s
+    assert mea.swish_channel_fwd_grouped([], []) == []
+    n = len(fake.calls)
+    for call in (
+        lambda: mea.swish_channel_fwd_grouped(xs, alphas[:2]),                          # list lengths
+        lambda: mea.swish_channel_fwd_grouped(xs, [torch.ones(3)] * 3),                  # alpha size
+        lambda: mea.swish_channel_fwd_grouped([xs[0], xs[1].double()], alphas[:2]),      # dtype mix
+        lambda: mea.swish_channel_bwd_grouped(xs, dys[:2], alphas),                     # dy list
+        lambda: mea.swish_channel_bwd_grouped(xs, [torch.randn(2, 16, 7, 8)] + dys[1:], alphas),  # dy shape
+        lambda: mea.swish_channel_fwd_grouped([torch.randn(4, 4)], [torch.ones(4)]),      # not 4-D
+    ):
+        with pytest.raises(ValueError):
+            call()
+    assert len(fake.calls) == n
