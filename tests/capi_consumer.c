@@ -91,6 +91,27 @@ int main(void)
                              NULL) == MEA_ERR_INVALID_ARG);
     CHECK(mea_swish_channel_fwd(MEA_F32, (mea_layout_t)3, shape, x, (float *)dy, y, NULL) ==
           MEA_ERR_INVALID_ARG);
+    {
+        /* grouped per-channel Swish: the C struct, the size query, refusals */
+        mea_channel_segment_t cs[2];
+        memset(cs, 0, sizeof(cs));
+        cs[0].x = x;
+        cs[0].out = y;
+        cs[0].alpha = (float *)dy;
+        cs[0].shape[0] = 2;
+        cs[0].shape[1] = 16;
+        cs[0].shape[2] = 7;
+        cs[0].shape[3] = 7;
+        cs[1] = cs[0];
+        cs[1].shape[1] = -1;
+        CHECK(mea_swish_channel_fwd_grouped(MEA_BF16, 0, NULL, NULL) == MEA_OK);
+        CHECK(mea_swish_channel_fwd_grouped(MEA_BF16, 2, cs, NULL) == MEA_ERR_INVALID_ARG);
+        CHECK(mea_swish_channel_bwd_grouped_workspace_bytes(MEA_BF16, 2, cs) == 0);
+        CHECK(mea_swish_channel_bwd_grouped_workspace_bytes(MEA_BF16, 1, cs) % 256 == 0);
+        CHECK(mea_swish_channel_bwd_grouped_workspace_bytes(MEA_BF16, 1, cs) >=
+              mea_swish_channel_bwd_workspace_bytes(MEA_BF16, MEA_NCHW, cs[0].shape));
+        CHECK(mea_swish_channel_bwd_grouped(MEA_BF16, 1, cs, ws, 1 << 20, NULL) == MEA_ERR_INVALID_ARG);
+    }
 
     /* matmul: K = 0 is not served, N must be a multiple of 8 */
     CHECK(mea_matmul_act_fwd(MEA_SWISH, 256, 256, 0, x, y, 1.0f, dy, dx, NULL) == MEA_ERR_UNSUPPORTED);
