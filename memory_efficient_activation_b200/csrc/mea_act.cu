@@ -106,7 +106,8 @@ __device__ __forceinline__ void act_body(const void *__restrict__ x, const void 
                 S::unpack(xv[u], xf);
                 if constexpr (MODE != 0) S::unpack(gv[u], gf);
                 bool tail = false;
-                if constexpr (HasPairs<A, P>::value) {
+                constexpr bool kPairs = MODE == 0 ? HasPairs<A, P>::value : HasPairsBwd<A, P>::value;
+                if constexpr (kPairs) {
 #pragma unroll
                     for (int j = 0; j < V; j += 2) {
                         if constexpr (MODE == 0)

@@ -121,6 +121,12 @@ template <class A, bool P>
 struct HasPairs {
     static constexpr bool value = false;
 };
+// Activations whose plain (not per-channel) backward also has a pairwise df2
+// (a superset of HasPairs).
+template <class A, bool P>
+struct HasPairsBwd {
+    static constexpr bool value = HasPairs<A, P>::value;
+};
 
 // Per-launch constants, built on the device from the scalar parameter.
 struct Coef {
@@ -690,8 +696,18 @@ struct GeluTanh {
         float tl;
         return expo_arg<false>(x, tl) > kTailT;
     }
+    // The plain bf16 backward's packed form (df2) also flags t < -kHugeT
+    // (x beyond about 2e10, where x v' could overflow); df_tail gives those
+    // the scalar form.
+    static constexpr float kHugeT = 1e30f;
     template <bool P>
-    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k) { return is_tail(x, k); }
+    static __device__ __forceinline__ bool is_tail_bwd(float x, const Coef &k)
+    {
+        if constexpr (P) return is_tail(x, k);
+        float tl;
+        const float t = expo_arg<false>(x, tl);
+        return t > kTailT || t < -kHugeT;
+    }
     // Every element a backward main path flags: t > kTailT (scalar form);
     // for bf16, |u| < kRootWinT or |u| > kTailU, u = t - kRootT (the packed
     // form of the per-channel kernels, which contains the scalar one's).
@@ -747,13 +763,45 @@ struct GeluTanh {
         float q = xdv(x);
         return dy * fmaf(q * s, sm, s);
     }
-    // v << 0: Sigmoid(-v) = 1, f' = s (1 + x v')
+    // v << 0: Sigmoid(-v) = 1, f' = s (1 + x v'); huge positive x (flagged by
+    // df2 only): the scalar form, whose x v' is clamped.
     template <bool P>
-    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &)
+    static __device__ __forceinline__ float df_tail(float x, float dy, const Coef &k)
     {
+        if constexpr (!P) {
+            if (x > 0.f) {
+                bool unused = false;
+                return df<false>(x, dy, k, unused);
+            }
+        }
         float q = xdv(x);
         return ((dy * s64_tail<P>(x)) * (1.f + q)) * kTwoM64;
     }
+    // Two elements, bf16 storage (the plain backward): t as in expo_arg, E =
+    // 2^t, s = 1 / (1 + E), and f' = s (1 + x v' E s) with E s = Sigmoid(-v);
+    // flags t > kTailT (deep negative x) and t < -kHugeT.
+    static __device__ __forceinline__ void df2(float x0, float x1, float dy0, float dy1, const Coef &, bool &tail,
+                                               float &o0, float &o1)
+    {
+        const F2 x = pk(x0, x1);
+        const F2 x2 = mul2(x, x);
+        float t0, t1;
+        upk(mul2(x, fma2(sp2(kC3f), x2, sp2(kC1f))), t0, t1);
+        const float e0 = ex2_ftz(t0), e1 = ex2_ftz(t1);
+        tail |= (t0 > kTailT) | (t1 > kTailT) | (t0 < -kHugeT) | (t1 < -kHugeT);
+        const F2 E = pk(e0, e1);
+        float a0, a1;
+        upk(add2(sp2(1.f), E), a0, a1);
+        const F2 s = pk(rcp_ftz(a0), rcp_ftz(a1));
+        const F2 q = mul2(x, fma2(sp2(kK3x3f), x2, sp2(kK1f)));
+        const F2 r = fma2(q, mul2(E, s), sp2(1.f));
+        upk(mul2(pk(dy0, dy1), mul2(s, r)), o0, o1);
+    }
+};
+
+template <>
+struct HasPairsBwd<GeluTanh, false> {
+    static constexpr bool value = true;
 };
 
 // ---------------------------------------------------------------- Swish
