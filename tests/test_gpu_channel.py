@@ -35,6 +35,8 @@ SHAPES = [
     ("nchw", (5, 37, 1, 1)), ("nchw", (3, 7, 1, 3)), ("nchw", (3, 201, 7, 7)),
     # plane path (planes above the row path's size): scalar and vector loads
     ("nchw", (2, 3, 33, 33)), ("nchw", (2, 4, 40, 40)),
+    # the boundary between them: 1024 elements (row path), 1025 (plane path)
+    ("nchw", (2, 5, 32, 32)), ("nchw", (2, 3, 41, 25)),
 ]
 
 

@@ -142,10 +142,10 @@ def test_grouped_rejects_overlap_and_partial_dparam():
 # ------------------------------------------------- Swish with alpha per channel
 
 # Row-path shapes (several planes per vector, a ragged last block, EfficientNet
-# stages), an empty batch, and a plane-path shape (40 x 40 planes) that the
-# grouped call launches alone.
+# stages, 1024-element planes), an empty batch, and plane-path shapes (40 x 40
+# and 41 x 25 planes) that the grouped call launches alone.
 CHANNEL_SHAPES = [(2, 16, 7, 7), (3, 201, 7, 7), (5, 37, 1, 1), (3, 7, 1, 3), (0, 16, 7, 7), (2, 4, 40, 40),
-                  (4, 96, 14, 14), (2, 24, 28, 28)]
+                  (4, 96, 14, 14), (2, 24, 28, 28), (2, 5, 32, 32), (2, 3, 41, 25)]
 
 
 def _channel_tensors(shapes, dtype, seed, misaligned=True):
