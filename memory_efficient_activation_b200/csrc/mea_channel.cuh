@@ -346,19 +346,23 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
     }
 }
 
-// Backward, pipelined: the same work split and summation order as
-// chan_nhwc_bwd_kernel (block b owns tiles b, b + grid, ...; fp32 sums per
-// tile, fp64 per thread, one row of fp64 partials per block), but the x and
-// dy tiles reach shared memory by 1-D bulk copies (cp.async.bulk) that one
-// producer thread keeps `stages` tiles ahead, so the bytes in flight no
-// longer cost registers.  Warp 0 is the producer; warps 1.. are consumers
-// (blockDim.x - 32 of them, a multiple of the G = C / VE channel groups, so
-// every consumer thread keeps the same VE channels).  A consumer copies its
-// UT units of the tile from shared memory to registers, releases the stage
-// (one arrival per warp on the stage's `empty` barrier), computes, and
-// stores dx to global memory directly.  The partial tile at the end (fewer
-// than a tile's units) is done with plain loads by the block that owns its
-// index.  Waits are bounded: one that expires sets err[0] and the kernel
+// Backward, pipelined: a fixed work split (a function of the shape and the
+// grid only; fp32 sums per few tiles, fp64 per thread, one row of fp64
+// partials per block) in which the x and dy tiles reach shared memory by
+// 1-D bulk copies (cp.async.bulk) that one producer thread keeps `stages`
+// tiles ahead, so the bytes in flight cost no registers.  Warp 0 is the
+// producer; warps 1.. are consumers (blockDim.x - 32 of them, a multiple of
+// the G = C / VE channel groups, so every consumer thread keeps the same VE
+// channels).  Block b owns tiles b, b + grid, ... below the last whole round
+// of the grid (rounds * grid tiles).  A consumer copies its UT units of a
+// tile from shared memory to registers, releases the stage (one arrival per
+// warp on the stage's `empty` barrier), computes, and stores dx to global
+// memory directly.  What is left after the whole rounds (the last
+// ntiles % grid tiles and the partial tile) is cut into rows of `consumers`
+// units, row r going to block r % grid, so that every block ends within a
+// row of the others instead of a third of the blocks taking one more tile;
+// the consumers load their rows before the producer's first copies and
+// compute them while the first stages are in flight.  Waits are bounded: one that expires sets err[0] and the kernel
 // finishes without computing further tiles.
 //
 // Shared memory: [0, 256) barriers; then NR VE * consumers fp64 running sums;
@@ -403,7 +407,8 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     unsigned char *buf = smem + kPipeHeader + acc_bytes;
     const int64_t tile_units = (int64_t)consumers * UT;
     const uint32_t tile_bytes = (uint32_t)(tile_units * UB);
-    const int64_t ntiles = nunits / tile_units;
+    // tiles of the whole rounds, which go through the stages
+    const int64_t piped = nunits / tile_units / gridDim.x * gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t spins = kWaitOut ? kMbarSpinsSelfTest : kMbarSpins;
 
@@ -416,6 +421,25 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     }
     __syncthreads();
     pdl_wait();
+    // The consumers' rows of the remainder are loaded before the producer
+    // issues its first copies, so that they are not queued behind them.  The
+    // remainder is under grid whole tiles (ntiles - piped < grid, plus a
+    // partial tile), i.e. at most grid * UT rows: at most UT per block.
+    constexpr int kLeft = UT;
+    const int64_t r0 = piped * tile_units;
+    const int ct = threadIdx.x - 32;
+    W lx[kLeft], lg[kLeft];
+    if (!kWaitOut && warp != 0) {
+#pragma unroll
+        for (int q = 0; q < kLeft; ++q) {
+            const int64_t i = r0 + (blockIdx.x + (int64_t)q * gridDim.x) * consumers + ct;
+            if (i < nunits) {
+                lx[q] = L::load(x, i);
+                lg[q] = L::load(dy, i);
+            }
+        }
+    }
+    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -423,7 +447,7 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
             // without a division
             int it = 0, s = 0;
             uint32_t phase = 0;
-            for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+            for (int64_t t = blockIdx.x; t < piped; t += gridDim.x, ++it) {
                 if (it >= stages && !mbar_wait(smem_addr(empty + s), (phase & 1) ^ 1, spins)) {
                     atomicExch(err, 1u);
                     break;
@@ -448,7 +472,6 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
         return;
     }
 
-    const int ct = threadIdx.x - 32;
     const int g = ct % groups;
     const typename Op::K k = Op::kcoef(ca);
     typename Op::Ch ch[VE];
@@ -515,9 +538,19 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
     };
     clear();
 
+    // This block's rows of the remainder, while the first stages are in
+    // flight; none in the self-test, which writes no dx.
+    if constexpr (!kWaitOut) {
+#pragma unroll
+        for (int q = 0; q < kLeft; ++q) {
+            const int64_t i = r0 + (blockIdx.x + (int64_t)q * gridDim.x) * consumers + ct;
+            if (i < nunits) L::store(dx, i, unit(lx[q], lg[q]));
+        }
+    }
+
     int it = 0, s = 0;
     uint32_t phase = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    for (int64_t t = blockIdx.x; t < piped; t += gridDim.x, ++it) {
         if (!mbar_wait(smem_addr(full + s), phase & 1, spins)) {
             atomicExch(err, 1u);
             break;
@@ -540,15 +573,6 @@ chan_nhwc_bwd_pipe_kernel(const void *__restrict__ x, const void *__restrict__ d
         if (++s == stages) {
             s = 0;
             ++phase;
-        }
-    }
-    // The partial tile at the end, if any, belongs to block ntiles % grid.
-    if (ntiles * tile_units < nunits && blockIdx.x == ntiles % gridDim.x) {
-        const int64_t base = ntiles * tile_units + ct;
-#pragma unroll
-        for (int u = 0; u < UT; ++u) {
-            const int64_t i = base + (int64_t)u * consumers;
-            if (i < nunits) L::store(dx, i, unit(L::load(x, i), L::load(dy, i)));
         }
     }
     flush();
