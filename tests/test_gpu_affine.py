@@ -40,6 +40,9 @@ def _nchw(shape_mem, layout):
 @pytest.mark.parametrize("layout,shape", [
     ("nhwc", (2, 5, 7, 144)), ("nhwc", (3, 4, 4, 16)), ("nhwc", (1, 3, 3, 8)),
     ("nhwc", (2, 3, 5, 12)), ("nhwc", (2, 2, 3, 5)), ("nhwc", (4, 9, 9, 1152)),
+    # pipelined backward: more tiles than its 296 blocks, not a multiple of
+    # them, and a partial tile (a remainder of 441 rows of 288 units)
+    ("nhwc", (4, 57, 57, 144)),
     ("nchw", (2, 16, 7, 7)), ("nchw", (2, 8, 4, 8)), ("nchw", (3, 5, 3, 3)),
     ("nchw", (4, 32, 28, 28)), ("nchw", (2, 1152, 7, 7)),
 ])
