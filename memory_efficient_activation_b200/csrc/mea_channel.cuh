@@ -362,8 +362,9 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
 // units, row r going to block r % grid, so that every block ends within a
 // row of the others instead of a third of the blocks taking one more tile;
 // the consumers load their rows before the producer's first copies and
-// compute them while the first stages are in flight.  Waits are bounded: one that expires sets err[0] and the kernel
-// finishes without computing further tiles.
+// compute them while the first stages are in flight.  Waits are bounded:
+// one that expires sets err[0] and the kernel finishes without computing
+// further tiles.
 //
 // Shared memory: [0, 256) barriers; then NR VE * consumers fp64 running sums;
 // then `stages` x {x tile, dy tile}.

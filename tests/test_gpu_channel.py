@@ -208,7 +208,9 @@ def test_affine_act_swish_matches_affine_swish(dtype, layout, shape):
 
 
 @pytest.mark.parametrize("act", ["sigmoid", "gelu_tanh"])
-@pytest.mark.parametrize("layout,shape", [("nhwc", (16, 14, 14, 144)), ("nchw", (16, 40, 14, 14))])
+@pytest.mark.parametrize("layout,shape", [("nhwc", (16, 14, 14, 144)), ("nchw", (16, 40, 14, 14)),
+                                          # remainder rows after whole rounds of the pipelined grid
+                                          ("nhwc", (4, 57, 57, 144))])
 def test_affine_act_deterministic_and_counter_reset(act, layout, shape):
     x, dy, g, b, _ = _inputs(shape, layout, "bf16", 404)
     x, dy, g, b = x.cuda(), dy.cuda(), g.cuda(), b.cuda()
