@@ -831,6 +831,7 @@ __device__ __forceinline__ void row_body(const void *__restrict__ x, const void 
     for (uint32_t i = threadIdx.x; i < np; i += kRowThreads) chs[i] = Op::load(ca, (int)((g0 + i) % C));
     __syncthreads();
     const DivU32 div(hw);
+    const bool in_plane = hw % VL == 0;
 
     // One element of a plane whose constants are h: the value (MODE 0) or
     // dx and its reduction terms, written to tm[NR].
@@ -862,24 +863,37 @@ __device__ __forceinline__ void row_body(const void *__restrict__ x, const void 
             div.divmod(q * VL, lp, pos);
             // the backward reads the plane's constants again only where the
             // vector crosses into the next plane (measured: backward 28^2
-            // 0.649 -> 0.659 of copy bandwidth); the forward reads them per
+            // 0.649 -> 0.659 of copy bandwidth), and when H W is a multiple
+            // of VL (every vector then lies in one plane; the choice is the
+            // same for the whole block, so no warp runs both forms) counts
+            // no positions (28^2 0.646 -> 0.690); the forward reads them per
             // element, which measured faster there
             Ch h = chs[lp];
+            if (MODE == 1 && in_plane) {
 #pragma unroll
-            for (int j = 0; j < VL; ++j) {
-                float tm[NR];
-                if constexpr (MODE == 0) {
-                    if (j > 0) h = chs[lp];
-                }
-                of[j] = elem(xf[j], MODE == 1 ? gf[j] : 0.f, h, tm);
-                if constexpr (MODE == 1) {
+                for (int j = 0; j < VL; ++j) {
+                    float tm[NR];
+                    of[j] = elem(xf[j], MODE == 1 ? gf[j] : 0.f, h, tm);
 #pragma unroll
                     for (int r = 0; r < NR; ++r) tv[r][j] = tm[r];
                 }
-                if (j + 1 < VL && ++pos == hw) {
-                    pos = 0;
-                    ++lp;
-                    if constexpr (MODE == 1) h = chs[lp];
+            } else {
+#pragma unroll
+                for (int j = 0; j < VL; ++j) {
+                    float tm[NR];
+                    if constexpr (MODE == 0) {
+                        if (j > 0) h = chs[lp];
+                    }
+                    of[j] = elem(xf[j], MODE == 1 ? gf[j] : 0.f, h, tm);
+                    if constexpr (MODE == 1) {
+#pragma unroll
+                        for (int r = 0; r < NR; ++r) tv[r][j] = tm[r];
+                    }
+                    if (j + 1 < VL && ++pos == hw) {
+                        pos = 0;
+                        ++lp;
+                        if constexpr (MODE == 1) h = chs[lp];
+                    }
                 }
             }
             I::store(out, v0g + q, of);
@@ -921,7 +935,9 @@ __device__ __forceinline__ void row_body(const void *__restrict__ x, const void 
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
                     double v = 0.0;
-                    for (uint32_t i = sub; i < hw; i += TS) v += (double)terms[r * ld + lp * hw + i];
+                    const float *tp = terms + r * ld + lp * hw;
+#pragma unroll 4
+                    for (uint32_t i = sub; i < hw; i += TS) v += (double)tp[i];
 #pragma unroll
                     for (uint32_t off = TS >> 1; off >= 1; off >>= 1) v += __shfl_xor_sync(mask, v, off);
                     if (sub == 0) partials[(n * NR + r) * C + c] = v;
