@@ -73,7 +73,12 @@ constexpr int kNhwcBwdMaxRegs = MEA_NHWC_BWD_MAXREGS;
 #endif
 constexpr int kNhwcFwdMaxRegs = MEA_NHWC_FWD_MAXREGS;
 constexpr int kPlaneThreads = 256;
-constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks
+constexpr int kPlaneBlocksTarget = 1184; // C * S is sized to about this many blocks (backward)
+// The forward, with no reduction at its end, measured best with twice as many
+// (NCHW fp32, Swish with alpha per channel: [64, 96, 112, 112] 0.834 -> 0.901
+// of copy bandwidth, [64, 144, 56, 56] 0.797 -> 0.835, [64, 32, 112, 112]
+// 0.837 -> 0.851); the backward lost 3-7% there and more with fewer.
+constexpr int kPlaneBlocksTargetFwd = 2368;
 
 // Parameter arrays and scalar of a per-channel operation (device pointers).
 struct ChanArgs {
@@ -102,9 +107,11 @@ inline int nhwc_threads(int groups)
     return (int)(lcm * m);
 }
 
-inline int plane_slices(int64_t N, int64_t C)
+// Slices of N per channel, so that C S is about `target` blocks: the
+// backward's kPlaneBlocksTarget, or kPlaneBlocksTargetFwd for the forward.
+inline int plane_slices(int64_t N, int64_t C, int64_t target = kPlaneBlocksTarget)
 {
-    int64_t s = (kPlaneBlocksTarget + C - 1) / C;
+    int64_t s = (target + C - 1) / C;
     if (s > N) s = N;
     if (s < 1) s = 1;
     return (int)s;
@@ -1201,7 +1208,7 @@ cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out
                           static_cast<const double *>(partials), a.N, a.C, out0, out1);
     }
     const int vec_ok = a.layout == 0 && HW % V == 0 && (al & 15u) == 0;
-    const int slices = plane_slices(a.N, a.C);
+    const int slices = plane_slices(a.N, a.C, MODE == 0 ? kPlaneBlocksTargetFwd : kPlaneBlocksTarget);
     const int64_t grid = a.C * slices;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     if (a.layout == 1)
