@@ -745,16 +745,15 @@ chan_plane_kernel(const void *__restrict__ x, const void *__restrict__ dy, ChanA
 // so the sums are bitwise reproducible on any device.
 constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;            // vectors in flight per thread
-constexpr int kRowBlocksTarget = 1184;   // 148 SMs x 8
-// The forward (no staging, no sums) measured best with half as many blocks,
-// each of twice the planes: NCHW fp32, Swish with alpha per channel, batch
-// 64, forward at 14^2 0.603 -> 0.649 of copy bandwidth, 7^2 0.510 -> 0.539,
-// 28^2 level, the three small stages grouped 0.840 -> 0.857 (targets 296,
-// 444, 592, 1184, 2368 and 4736 measured; more blocks lost up to 40%).
-#ifndef MEA_ROW_FWD_TARGET
-#define MEA_ROW_FWD_TARGET 592
-#endif
-constexpr int kRowBlocksTargetFwd = MEA_ROW_FWD_TARGET;
+// Blocks the row path aims at (148 SMs x 4), each of about N C / 592 planes.
+// Measured on NCHW fp32, Swish with alpha per channel, batch 64, against
+// 1184: forward at 14^2 0.603 -> 0.649 of copy bandwidth, 7^2 0.510 ->
+// 0.539; backward at 14^2 0.524 -> 0.531, 7^2 0.412 -> 0.427; the three
+// small stages grouped 0.840 -> 0.857 forward and 0.707 -> 0.734 backward;
+// 28^2 level (its backward is held by the staging buffer).  Targets of 296
+// to 4736 were measured; more blocks lost up to 40% in the forward, and 888
+// lost 8% in the 7^2 backward.
+constexpr int kRowBlocksTarget = 592;
 constexpr int kRowTerms = 8192;          // fp32 terms staged per block (32 KB)
 constexpr int kRowMaxPlanes = 256;
 #ifndef MEA_ROW_MAX_HW
@@ -784,7 +783,7 @@ __device__ __forceinline__ unsigned row_team_mask(uint32_t lane, uint32_t ts)
 // P for nr reductions and vl elements per 16-byte vector: about
 // N C / kRowBlocksTarget planes, rounded up to the alignment multiple, at
 // most what the staging buffer and the constants table hold.
-inline RowShape row_shape(int nr, int vl, int64_t N, int64_t C, int64_t HW, int64_t target = kRowBlocksTarget)
+inline RowShape row_shape(int nr, int vl, int64_t N, int64_t C, int64_t HW)
 {
     const int64_t np = N * C;
     if (np < 1 || HW < 1 || HW > kRowMaxHW) return RowShape{0, 0};
@@ -799,7 +798,7 @@ inline RowShape row_shape(int nr, int vl, int64_t N, int64_t C, int64_t HW, int6
     if (nr > 0 && kRowTerms / (HW * nr) < pmax) pmax = kRowTerms / (HW * nr);
     pmax -= pmax % m;
     if (pmax < m) return RowShape{0, 0};
-    int64_t p = (np + target - 1) / target;
+    int64_t p = (np + kRowBlocksTarget - 1) / kRowBlocksTarget;
     p = (p + m - 1) / m * m;
     if (p > pmax) p = pmax;
     return RowShape{(int)p, (np + p - 1) / p};
@@ -1204,9 +1203,7 @@ cudaError_t launch_channel(const AffineLaunch &a, const ChanArgs &ca, float *out
     }
     uintptr_t al = reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.out);
     if (a.dy) al |= reinterpret_cast<uintptr_t>(a.dy);
-    const RowShape rs =
-        a.layout == 0 ? row_shape(NR, V, a.N, a.C, HW, MODE == 0 ? kRowBlocksTargetFwd : kRowBlocksTarget)
-                      : RowShape{0, 0};
+    const RowShape rs = a.layout == 0 ? row_shape(NR, V, a.N, a.C, HW) : RowShape{0, 0};
     if (rs.planes > 0 && (al & 15u) == 0) {
         if (rs.grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
         double *partials = reinterpret_cast<double *>(static_cast<char *>(a.workspace) + kWsHeader);

@@ -149,7 +149,7 @@ cudaError_t launch_grouped(int dtype, int nseg, const ChanSeg *segs, cudaStream_
         if (g.N * g.C * HW == 0) continue;
         uintptr_t al = reinterpret_cast<uintptr_t>(g.x) | reinterpret_cast<uintptr_t>(g.out);
         if (MODE == 1) al |= reinterpret_cast<uintptr_t>(g.dy);
-        const RowShape rs = row_shape(NR, V, g.N, g.C, HW, MODE == 0 ? kRowBlocksTargetFwd : kRowBlocksTarget);
+        const RowShape rs = row_shape(NR, V, g.N, g.C, HW);
         cudaError_t e = cudaSuccess;
         if (rs.planes == 0 || (al & 15u) || rs.grid > 0x7fffffff || NR * g.C > 0x7fffffff) {
             AffineLaunch a{};
