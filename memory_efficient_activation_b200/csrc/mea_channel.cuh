@@ -367,7 +367,7 @@ chan_nhwc_bwd_kernel(const void *__restrict__ x, const void *__restrict__ dy, Ch
 // memory directly.  What is left after the whole rounds (the last
 // ntiles % grid tiles and the partial tile) is cut into rows of `consumers`
 // units, row r going to block r % grid, so that every block ends within a
-// row of the others instead of a third of the blocks taking one more tile;
+// row of the others instead of ntiles % grid blocks taking one more tile;
 // the consumers load their rows before the producer's first copies and
 // compute them while the first stages are in flight.  Waits are bounded:
 // one that expires sets err[0] and the kernel finishes without computing
